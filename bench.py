@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA NF4 linear hot path on B200.
+
+Workload (one step): for each of the two LLaMA-7B-shaped linears -- W
+4096x4096 and 11008x4096 fp32 ~N(0, 0.02) with 0.1% of entries x8, X 4096
+tokens x 4096 bf16, rank r = 64, alpha = 16 -- quantize W to NF4 with double
+quantization, run the forward Y = X W'^T + s (X A^T) B^T, and the backward
+(dX, dA, dB).  Synthetic, seeded inputs (synth.py).  The metric is the
+algorithmic fwd+bwd FLOP rate, 4MNK + 6Mr(N+K) per linear, over the whole
+step (quantization included).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Under torchrun each rank runs its own token batch against replicated frozen
+weights (weak scaling) and the adapter gradients are all-reduced every step.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s & NF4 quant/dequant GB/s, % of roofline"
+WORKLOAD = "llama7b_linears_w4096x4096_w11008x4096_m4096_r64_alpha16_quantize_fwd_bwd"
+M_TOKENS, RANK, ALPHA = 4096, 64, 16.0
+L2_FLUSH_BYTES = 256 << 20
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def linear_flops(M, N, K, r):
+    return 4 * M * N * K + 6 * M * r * (N + K)
+
+
+def fwd_flops(M, N, K, r):
+    return 2 * M * N * K + 2 * M * r * (N + K)
+
+
+def quant_bytes(numel):
+    nb = -(-numel // 64)
+    return 4 * numel + (numel + 1) // 2 + nb + 4 * (-(-nb // 256)) + 4
+
+
+def dequant_bytes(numel, out_bytes):
+    nb = -(-numel // 64)
+    return (numel + 1) // 2 + nb + 4 * (-(-nb // 256)) + 4 + out_bytes * numel
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a window."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, interval_ms: int = 50):
+        self.lines = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(device_index), "-lms", str(interval_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        if self.proc is None:
+            return None
+        rows = [l for (t, l) in self.lines if t0 <= t <= t1] or [l for (_, l) in self.lines]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in rows:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                sm.append(float(parts[2]))
+                mx.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------- oracle arm
+
+def oracle_weight_bf16(case):
+    """The bf16 weight the linear consumes, from the oracle's own NF4 round
+    trip (computed once per linear, outside any timing)."""
+    import oracle
+    W = case.W.reshape(-1)
+    d = oracle.quantize_nf4_dq(W)
+    return oracle.bf16_rne(oracle.dequantize(d["codes"], d["c2_fp8"], d["c1"], d["mean"],
+                                             W.size)).reshape(case.N, case.K)
+
+
+def oracle_sample(case, Wb, rows_m: int, quant_elems: int):
+    """Time the CPU oracle on a bounded sample of one linear: quantization of
+    the first `quant_elems` weights, and fwd+bwd on the first `rows_m`
+    tokens against the full weight.  Returns (t_quant, t_linear, flops, bytes)."""
+    import oracle
+    W = case.W.reshape(-1)
+    t0 = time.perf_counter()
+    oracle.quantize_nf4_dq(W[:quant_elems])
+    tq = time.perf_counter() - t0
+    X, dY = case.X[:rows_m], case.dY[:rows_m]
+    t1 = time.perf_counter()
+    oracle.linear_fwd(X, Wb, case.A, case.B, case.s)
+    oracle.linear_bwd(dY, X, Wb, case.A, case.B, case.s)
+    tl = time.perf_counter() - t1
+    return tq, tl, linear_flops(rows_m, case.N, case.K, case.r), quant_bytes(quant_elems)
+
+
+def oracle_baseline(cases, wbs, rows_m=4, quant_elems=1 << 22):
+    import oracle
+    tq_tot = tl_tot = fl_tot = qb_tot = 0.0
+    for c, wb in zip(cases, wbs):
+        tq, tl, fl, qb = oracle_sample(c, wb, rows_m, quant_elems)
+        tq_tot += tq
+        tl_tot += tl
+        fl_tot += fl
+        qb_tot += qb
+    return {"value": fl_tot / tl_tot / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": (f"fwd+bwd of {rows_m} tokens per linear (full N, K, r=64) and quantization of "
+                       f"the first {quant_elems} weights per linear, both linears"),
+            "quant_gbs": qb_tot / tq_tot / 1e9, "seconds": tl_tot + tq_tot}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    cases = [synth.llama7b_linear(i, seed=0, M=M_TOKENS) for i in range(2)]
+    wbs = [oracle_weight_bf16(c) for c in cases]
+    for _ in range(args.warmup):
+        oracle_baseline(cases, wbs, rows_m=1, quant_elems=1 << 16)
+    vals = []
+    t_all = 0.0
+    for _ in range(args.steps):
+        b = oracle_baseline(cases, wbs, rows_m=2, quant_elems=1 << 20)
+        vals.append(b["value"])
+        t_all += b["seconds"]
+    value = statistics.mean(vals)
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_all / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "sample": "2 tokens per linear"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": b["cores"], "kind": "oracle",
+                             "sample": "fwd+bwd of 2 tokens per linear and quantization of 2^20 weights "
+                                       "per linear, per step"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- native arm
+
+def run_native(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    import bit_nf4_quantized_13_b200 as q
+    from bit_nf4_quantized_13_b200.dp import allreduce_adapter_grads
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def to_bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    cases = []
+    for i in range(2):
+        c = synth.llama7b_linear(i, seed=0, M=M_TOKENS)
+        if world > 1:  # every rank its own tokens, the same frozen weight and adapters
+            xc = synth.linear_case("x", M_TOKENS, c.N, c.K, RANK, ALPHA, seed=1000 + rank,
+                                   wid=i)
+            c.X, c.dY = xc.X, xc.dY
+        cases.append(c)
+
+    bufs = []
+    for c in cases:
+        b = {"case": c}
+        b["W"] = torch.from_numpy(c.W).to(dev)
+        b["X"], b["A"], b["B"], b["dY"] = to_bf16(c.X), to_bf16(c.A), to_bf16(c.B), to_bf16(c.dY)
+        b["wq"] = q.alloc_nf4_weight((c.N, c.K), dev)
+        b["qws"] = torch.empty(q.qlora_quantize_workspace_size(c.W.size), dtype=torch.uint8, device=dev)
+        b["Y"] = torch.empty((c.M, c.N), dtype=torch.bfloat16, device=dev)
+        b["T"] = torch.empty((c.M, c.r), dtype=torch.bfloat16, device=dev)
+        b["dX"] = torch.empty((c.M, c.K), dtype=torch.bfloat16, device=dev)
+        b["dA"] = torch.empty((c.r, c.K), dtype=torch.bfloat16, device=dev)
+        b["dB"] = torch.empty((c.N, c.r), dtype=torch.bfloat16, device=dev)
+        b["bws"] = torch.empty(q.qlora_linear_bwd_workspace_size(c.M, c.N, c.K, c.r), dtype=torch.uint8,
+                               device=dev)
+        b["Wdq"] = torch.empty((c.N, c.K), dtype=torch.bfloat16, device=dev)
+        bufs.append(b)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        for i, b in enumerate(bufs):
+            c = b["case"]
+            if ev is not None:
+                ev[i][0].record(stream)
+            q.qlora_quantize_nf4_dq(b["W"], out=b["wq"], ws=b["qws"])
+            if ev is not None:
+                ev[i][1].record(stream)
+            q.qlora_linear_fwd(b["X"], b["wq"], b["A"], b["B"], c.s, Y=b["Y"], T_save=b["T"])
+            if ev is not None:
+                ev[i][2].record(stream)
+            q.qlora_linear_bwd(b["dY"], b["X"], b["wq"], b["A"], b["B"], c.s, T=b["T"], dX=b["dX"],
+                               dA=b["dA"], dB=b["dB"], ws=b["bws"])
+            if world > 1:
+                allreduce_adapter_grads(b["dA"], b["dB"])
+            if ev is not None:
+                ev[i][3].record(stream)
+
+    def new_events():
+        return [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in bufs]
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    launches0 = q.qlora_kernel_launch_count()
+    steps_ev, phase_ev = [], []
+    t_wall0 = time.time()
+    for _ in range(args.steps):
+        flush.zero_()  # L2 flush between timed steps (outside the step's events)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pe = new_events()
+        s0.record(stream)
+        step(pe)
+        s1.record(stream)
+        steps_ev.append((s0, s1))
+        phase_ev.append(pe)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    launches = q.qlora_kernel_launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.stop()
+
+    step_ms = [a.elapsed_time(b) for a, b in steps_ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    flops_step = sum(linear_flops(c.M, c.N, c.K, c.r) for c in cases)
+    value = flops_step * world / (ms_per_step * 1e-3) / 1e12
+
+    # per-phase breakdown (rank-local)
+    qt = sum(pe[i][0].elapsed_time(pe[i][1]) for pe in phase_ev for i in range(2))
+    ft = sum(pe[i][1].elapsed_time(pe[i][2]) for pe in phase_ev for i in range(2))
+    bt = sum(pe[i][2].elapsed_time(pe[i][3]) for pe in phase_ev for i in range(2))
+    qbytes = sum(quant_bytes(c.W.size) for c in cases) * args.steps
+    fflops = sum(fwd_flops(c.M, c.N, c.K, c.r) for c in cases) * args.steps
+    bflops = sum(linear_flops(c.M, c.N, c.K, c.r) - fwd_flops(c.M, c.N, c.K, c.r) for c in cases) * args.steps
+
+    # standalone dequantization (row a7), timed separately after the steps
+    dq_ms, dq_bytes = 0.0, 0
+    for _ in range(3):
+        for b in bufs:
+            q.qlora_dequantize(b["wq"], torch.bfloat16, out=b["Wdq"])
+    for _ in range(max(3, args.steps // 4)):
+        for b in bufs:
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            q.qlora_dequantize(b["wq"], torch.bfloat16, out=b["Wdq"])
+            e1.record(stream)
+            torch.cuda.synchronize()
+            dq_ms += e0.elapsed_time(e1)
+            dq_bytes += dequant_bytes(b["case"].W.size, 2)
+
+    peaks, peak_src = load_peaks()
+    # the GEMM is timed in short bursts between L2 flushes: the burst peak
+    tc_peak = peaks["bf16_tflops"]
+    fwd_tflops = fflops / (ft * 1e-3) / 1e12
+    roofline = {"kernel": "qlora_linear_fwd (T = X A^T, then the NF4-dequant GEMM with the LoRA slab)",
+                "bound": "tensor", "achieved": fwd_tflops, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": fwd_tflops / tc_peak, "traffic": None, "peak_source": peak_src,
+                "algorithmic": "2MNK + 2Mr(N+K) per launch"}
+
+    # end to end through the C ABI with host buffers: H2D of the step's
+    # inputs from pinned memory, the step, D2H of its outputs
+    e2e = None
+    if not args.no_e2e:
+        hin, hout = [], []
+        for b in bufs:
+            hin.append({k: b[k].cpu().pin_memory() for k in ("W", "X", "A", "B", "dY")})
+            hout.append({k: torch.empty_like(b[k], device="cpu").pin_memory() for k in ("Y", "dX", "dA", "dB")})
+        h2d = sum(t.numel() * t.element_size() for h in hin for t in h.values())
+        d2h = sum(t.numel() * t.element_size() for h in hout for t in h.values())
+
+        def e2e_step():
+            for b, hi, ho in zip(bufs, hin, hout):
+                for k, t in hi.items():
+                    b[k].copy_(t, non_blocking=True)
+            step()
+            for b, ho in zip(bufs, hout):
+                for k, t in ho.items():
+                    t.copy_(b[k], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        ee = []
+        for _ in range(max(3, args.steps // 2)):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            e2e_step()
+            e1.record(stream)
+            ee.append((e0, e1))
+        torch.cuda.synchronize()
+        e_ms = statistics.mean(a.elapsed_time(b) for a, b in ee)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": flops_step * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_baseline(cases, [oracle_weight_bf16(c) for c in cases])
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "linears": ["4096x4096", "11008x4096"], "tokens_per_gpu": M_TOKENS,
+                       "rank": RANK, "alpha": ALPHA, "block": 64, "block2": 256,
+                       "l2": "flushed between timed steps (256 MiB write); inputs also exceed L2",
+                       "parallelism": f"dp{world}"},
+            "gpu_launches": int(launches),
+            "roofline": roofline,
+            "components": {
+                "quantize_gbs": qbytes / (qt * 1e-3) / 1e9,
+                "quantize_frac_hbm": qbytes / (qt * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "dequant_bf16_gbs": dq_bytes / (dq_ms * 1e-3) / 1e9 if dq_ms else None,
+                "dequant_bf16_frac_hbm": (dq_bytes / (dq_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]) if dq_ms else None,
+                "fwd_tflops": fwd_tflops, "bwd_tflops": bflops / (bt * 1e-3) / 1e12,
+                "ms": {"quantize": qt / args.steps, "fwd": ft / args.steps, "bwd": bt / args.steps},
+                "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": tc_peak, "source": peak_src}},
+            "clocks": clocks.summary(t_wall0, t_wall1),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_native(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

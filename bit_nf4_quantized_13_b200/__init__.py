@@ -1,0 +1,246 @@
+"""B200-native QLoRA NF4 linear layer: Python binding of ``libqlora_nf4.so``.
+
+The QLoRA hot path (Dettmers et al., arXiv:2305.14314) for one frozen linear
+layer with a LoRA side path, as hand-written sm_100a CUDA kernels behind the
+C ABI of ``include/qlora.h``.  This module only marshals arguments: it turns
+torch CUDA tensors into device pointers, allocates outputs and workspaces
+with torch, passes torch's current stream, and raises on a non-OK status.
+Every step of the computation runs in the library's kernels; there is no
+fallback.  The library must have been built (``python -m
+bit_nf4_quantized_13_b200.build``); importing without it raises.
+
+Entry points (same names as the C ABI):
+    qlora_nf4_codebook()                         -> numpy float32[16]
+    qlora_quantize_nf4_dq(W)                     -> Nf4Weight
+    qlora_dequantize(w, out_dtype)               -> tensor (N x K)
+    qlora_linear_fwd(X, w, A, B, s)              -> (Y, T)
+    qlora_linear_bwd(dY, X, w, A, B, s, T=None)  -> (dX, dA, dB)
+    qlora_fp8_e4m3_encode(x)                     -> uint8 tensor
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
+
+QLORA_OK = 0
+STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED",
+                3: "QLORA_ERR_WORKSPACE", 4: "QLORA_ERR_CUDA", 5: "QLORA_ERR_NONFINITE",
+                6: "QLORA_ERR_TIMEOUT"}
+BLOCK, BLOCK2, MAX_RANK = 64, 256, 256
+
+
+class QloraError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m bit_nf4_quantized_13_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    i64, i32, vp, sz, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
+    sig = {
+        "qlora_nf4_codebook": (i32, [vp]),
+        "qlora_quantize_workspace_size": (sz, [i64]),
+        "qlora_quantize_nf4_dq": (i32, [vp, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp]),
+        "qlora_dequantize": (i32, [vp, vp, vp, vp, i64, i32, i32, vp, i32, vp]),
+        "qlora_linear_fwd_workspace_size": (sz, [i64, i64, i64, i32]),
+        "qlora_linear_bwd_workspace_size": (sz, [i64, i64, i64, i32]),
+        "qlora_linear_fwd": (i32, [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp, vp,
+                                   sz, vp]),
+        "qlora_linear_bwd": (i32, [vp, vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp,
+                                   vp, vp, vp, sz, vp]),
+        "qlora_fp8_e4m3_encode": (i32, [vp, vp, i64, vp]),
+        "qlora_kernel_launch_count": (ctypes.c_uint64, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype, fn.argtypes = res, args
+    return L
+
+
+lib = _load()
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, st: int) -> None:
+    if st != QLORA_OK:
+        raise QloraError(fn, st)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def _workspace(nbytes: int, device):
+    torch = _torch()
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+# ----------------------------------------------------------------- codebook
+
+def qlora_nf4_codebook() -> np.ndarray:
+    out = np.zeros(16, np.float32)
+    _check("qlora_nf4_codebook", lib.qlora_nf4_codebook(out.ctypes.data_as(ctypes.c_void_p)))
+    return out
+
+
+# ----------------------------------------------------------------- quantize
+
+@dataclass
+class Nf4Weight:
+    """A frozen weight in the library's storage format (4 device buffers)."""
+    codes: object   # uint8 [ceil(numel/2)]
+    c2_fp8: object  # uint8 [ceil(numel/64)]
+    c1: object      # float32 [ceil(numel/16384)]
+    mean: object    # float32 [1]
+    shape: tuple
+
+    @property
+    def numel(self) -> int:
+        n = 1
+        for d in self.shape:
+            n *= int(d)
+        return n
+
+    def nbytes(self) -> int:
+        return sum(int(t.numel() * t.element_size()) for t in (self.codes, self.c2_fp8, self.c1, self.mean))
+
+
+def qlora_quantize_workspace_size(numel: int) -> int:
+    return int(lib.qlora_quantize_workspace_size(int(numel)))
+
+
+def alloc_nf4_weight(shape, device) -> Nf4Weight:
+    torch = _torch()
+    n = 1
+    for d in shape:
+        n *= int(d)
+    nb = -(-n // BLOCK)
+    return Nf4Weight(torch.empty((n + 1) // 2, dtype=torch.uint8, device=device),
+                     torch.empty(max(nb, 1), dtype=torch.uint8, device=device),
+                     torch.empty(max(-(-nb // BLOCK2), 1), dtype=torch.float32, device=device),
+                     torch.zeros(1, dtype=torch.float32, device=device), tuple(int(d) for d in shape))
+
+
+def qlora_quantize_nf4_dq(W, out: Nf4Weight | None = None, ws=None, status=None,
+                          stream=None) -> Nf4Weight:
+    """NF4 + double quantization of an fp32 CUDA tensor (any shape, flattened)."""
+    torch = _torch()
+    _need_cuda(W)
+    if W.dtype != torch.float32:
+        raise ValueError("W must be float32")
+    n = W.numel()
+    w = out if out is not None else alloc_nf4_weight(tuple(W.shape), W.device)
+    if ws is None:
+        ws = _workspace(qlora_quantize_workspace_size(n), W.device)
+    st = lib.qlora_quantize_nf4_dq(_ptr(W), n, BLOCK, BLOCK2, _ptr(w.codes), _ptr(w.c2_fp8),
+                                   _ptr(w.c1), _ptr(w.mean), _ptr(ws), ws.numel(), _ptr(status),
+                                   _stream(stream))
+    _check("qlora_quantize_nf4_dq", st)
+    return w
+
+
+def qlora_dequantize(w: Nf4Weight, out_dtype=None, out=None, stream=None):
+    torch = _torch()
+    out_dtype = out_dtype or torch.float32
+    code = {torch.float32: 0, torch.bfloat16: 1}[out_dtype]
+    if out is None:
+        out = torch.empty(w.shape, dtype=out_dtype, device=w.codes.device)
+    st = lib.qlora_dequantize(_ptr(w.codes), _ptr(w.c2_fp8), _ptr(w.c1), _ptr(w.mean), w.numel,
+                              BLOCK, BLOCK2, _ptr(out), code, _stream(stream))
+    _check("qlora_dequantize", st)
+    return out
+
+
+# ------------------------------------------------------------------- linear
+
+def qlora_linear_fwd_workspace_size(M, N, K, r) -> int:
+    return int(lib.qlora_linear_fwd_workspace_size(int(M), int(N), int(K), int(r)))
+
+
+def qlora_linear_bwd_workspace_size(M, N, K, r) -> int:
+    return int(lib.qlora_linear_bwd_workspace_size(int(M), int(N), int(K), int(r)))
+
+
+def qlora_linear_fwd(X, w: Nf4Weight, A, B, s: float, Y=None, T_save=None, ws=None, stream=None):
+    """Y = X W'^T + s (X A^T) B^T; returns (Y, T) with T = bf16(s X A^T)."""
+    torch = _torch()
+    _need_cuda(X, A, B)
+    M, K = X.shape
+    N = w.shape[0]
+    r = A.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    if T_save is None:
+        T_save = torch.empty((M, r), dtype=torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = _workspace(16, X.device)
+    st = lib.qlora_linear_fwd(_ptr(X), M, N, K, _ptr(w.codes), _ptr(w.c2_fp8), _ptr(w.c1),
+                              _ptr(w.mean), _ptr(A), _ptr(B), r, float(s), _ptr(Y), _ptr(T_save),
+                              _ptr(ws), ws.numel(), _stream(stream))
+    _check("qlora_linear_fwd", st)
+    return Y, T_save
+
+
+def qlora_linear_bwd(dY, X, w: Nf4Weight, A, B, s: float, T=None, dX=None, dA=None, dB=None,
+                     ws=None, want_dx: bool = True, stream=None):
+    """Adapter gradients and the input gradient; no gradient for W."""
+    torch = _torch()
+    _need_cuda(dY, X, A, B, T)
+    M, K = X.shape
+    N = w.shape[0]
+    r = A.shape[0]
+    if want_dx and dX is None:
+        dX = torch.empty((M, K), dtype=torch.bfloat16, device=X.device)
+    if dA is None:
+        dA = torch.empty((r, K), dtype=torch.bfloat16, device=X.device)
+    if dB is None:
+        dB = torch.empty((N, r), dtype=torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = _workspace(qlora_linear_bwd_workspace_size(M, N, K, r), X.device)
+    st = lib.qlora_linear_bwd(_ptr(dY), _ptr(X), M, N, K, _ptr(w.codes), _ptr(w.c2_fp8),
+                              _ptr(w.c1), _ptr(w.mean), _ptr(A), _ptr(B), r, float(s), _ptr(T),
+                              _ptr(dX if want_dx else None), _ptr(dA), _ptr(dB), _ptr(ws),
+                              ws.numel(), _stream(stream))
+    _check("qlora_linear_bwd", st)
+    return dX, dA, dB
+
+
+def qlora_fp8_e4m3_encode(x, out=None, stream=None):
+    torch = _torch()
+    _need_cuda(x)
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check("qlora_fp8_e4m3_encode",
+           lib.qlora_fp8_e4m3_encode(_ptr(x), _ptr(out), x.numel(), _stream(stream)))
+    return out
+
+
+def qlora_kernel_launch_count() -> int:
+    """Kernels this library has launched in this process so far."""
+    return int(lib.qlora_kernel_launch_count())

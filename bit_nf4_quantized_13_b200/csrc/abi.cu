@@ -1,0 +1,181 @@
+// abi.cu -- the extern "C" entry points declared in include/qlora.h:
+// argument validation on the host, then kernel launches on the caller's
+// stream.  Nothing here allocates device memory or synchronizes.
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qlora {
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+
+void note_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+cudaError_t launch_fwd_gemm(const uint16_t* X, const Nf4Weight& w, const uint16_t* T,
+                            const uint16_t* B, int64_t M, int r, uint16_t* Y, cudaStream_t st) {
+    return launch_fwd_gemm_simt(X, w, T, B, M, r, Y, st);
+}
+
+cudaError_t launch_bwd_dx_gemm(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U,
+                               const uint16_t* A, int64_t M, int r, uint16_t* dX, cudaStream_t st) {
+    return launch_bwd_dx_gemm_simt(dY, w, U, A, M, r, dX, st);
+}
+
+}  // namespace qlora
+
+using namespace qlora;
+
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+
+inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+
+constexpr int64_t kMaxNumel = int64_t(1) << 46;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int check_weight(const uint8_t* codes, const uint8_t* c2_fp8, const float* c1, const float* mean) {
+    if (!ok_ptr(codes) || !ok_ptr(c2_fp8) || !ok_ptr(c1) || !ok_ptr(mean)) return QLORA_ERR_INVALID_ARG;
+    return QLORA_OK;
+}
+
+int check_linear(int64_t M, int64_t N, int64_t K, int r) {
+    if (M < 0 || N < 1 || K < 1 || r < 1) return QLORA_ERR_INVALID_ARG;
+    if (K % QLORA_BLOCK != 0 || r > QLORA_MAX_RANK) return QLORA_ERR_UNSUPPORTED;
+    if (N * K >= kMaxNumel || M > (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
+    return QLORA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t qlora_quantize_workspace_size(int64_t numel) {
+    if (numel < 0) return 0;
+    const int64_t nb = ceil_div(numel, QLORA_BLOCK);
+    return static_cast<size_t>(kBinBytes + kFlagBytes + round_up(nb * 4, 16));
+}
+
+int qlora_quantize_nf4_dq(const float* W, int64_t numel, int block, int block2, uint8_t* codes,
+                          uint8_t* c2_fp8, float* c1, float* mean, void* ws, size_t ws_bytes,
+                          int32_t* status, void* stream) {
+    if (numel < 0) return QLORA_ERR_INVALID_ARG;
+    if (block != QLORA_BLOCK || block2 != QLORA_BLOCK2) return QLORA_ERR_UNSUPPORTED;
+    if (numel >= kMaxNumel) return QLORA_ERR_UNSUPPORTED;
+    if (numel == 0) return QLORA_OK;
+    if (!ok_ptr(W) || !ok_ptr(codes) || !ok_ptr(c2_fp8) || !ok_ptr(c1) || !ok_ptr(mean))
+        return QLORA_ERR_INVALID_ARG;
+    if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return QLORA_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws) || ws_bytes < qlora_quantize_workspace_size(numel)) return QLORA_ERR_WORKSPACE;
+    return cuda_status(launch_quantize_nf4_dq(W, numel, codes, c2_fp8, c1, mean, ws, status, as_stream(stream)));
+}
+
+int qlora_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c1, const float* mean,
+                     int64_t numel, int block, int block2, void* out, int out_dtype, void* stream) {
+    if (numel < 0 || (out_dtype != 0 && out_dtype != 1)) return QLORA_ERR_INVALID_ARG;
+    if (block != QLORA_BLOCK || block2 != QLORA_BLOCK2) return QLORA_ERR_UNSUPPORTED;
+    if (numel >= kMaxNumel) return QLORA_ERR_UNSUPPORTED;
+    if (numel == 0) return QLORA_OK;
+    if (check_weight(codes, c2_fp8, c1, mean) != QLORA_OK || !ok_ptr(out)) return QLORA_ERR_INVALID_ARG;
+    return cuda_status(launch_dequantize(codes, c2_fp8, c1, mean, numel, out, out_dtype, as_stream(stream)));
+}
+
+size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
+    if (check_linear(M, N, K, r) != QLORA_OK) return 0;
+    return align256(static_cast<size_t>(M) * r * 2);  // T when T_save is NULL
+}
+
+size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
+    if (check_linear(M, N, K, r) != QLORA_OK) return 0;
+    const size_t mr = align256(static_cast<size_t>(M) * r * 2);
+    return 2 * mr + align256(lora_grad_workspace(M, N, K, r));  // U, T (when T is NULL), grads
+}
+
+int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
+                     const uint8_t* c2_fp8, const float* c1, const float* mean, const uint16_t* A,
+                     const uint16_t* B, int r, float s, uint16_t* Y, uint16_t* T_save, void* ws,
+                     size_t ws_bytes, void* stream) {
+    int st = check_linear(M, N, K, r);
+    if (st != QLORA_OK) return st;
+    if (check_weight(codes, c2_fp8, c1, mean) != QLORA_OK) return QLORA_ERR_INVALID_ARG;
+    if (!ok_ptr(A) || !ok_ptr(B) || (M > 0 && (!ok_ptr(X) || !ok_ptr(Y)))) return QLORA_ERR_INVALID_ARG;
+    if (T_save && !aligned16(T_save)) return QLORA_ERR_INVALID_ARG;
+    if (M == 0) return QLORA_OK;
+    uint16_t* T = T_save;
+    if (!T) {
+        if (!ws || !aligned16(ws) || ws_bytes < qlora_linear_fwd_workspace_size(M, N, K, r))
+            return QLORA_ERR_WORKSPACE;
+        T = reinterpret_cast<uint16_t*>(ws);
+    }
+    cudaStream_t cs = as_stream(stream);
+    Nf4Weight w{codes, c2_fp8, c1, mean, N, K};
+    cudaError_t e = launch_lora_xat(X, A, M, K, r, s, T, cs);
+    if (e == cudaSuccess) e = launch_fwd_gemm(X, w, T, B, M, r, Y, cs);
+    return cuda_status(e);
+}
+
+int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                     const uint8_t* codes, const uint8_t* c2_fp8, const float* c1, const float* mean,
+                     const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* T,
+                     uint16_t* dX, uint16_t* dA, uint16_t* dB, void* ws, size_t ws_bytes,
+                     void* stream) {
+    int st = check_linear(M, N, K, r);
+    if (st != QLORA_OK) return st;
+    if (check_weight(codes, c2_fp8, c1, mean) != QLORA_OK) return QLORA_ERR_INVALID_ARG;
+    if (!ok_ptr(A) || !ok_ptr(B) || !ok_ptr(dA) || !ok_ptr(dB)) return QLORA_ERR_INVALID_ARG;
+    if (M > 0 && (!ok_ptr(dY) || !ok_ptr(X))) return QLORA_ERR_INVALID_ARG;
+    if ((T && !aligned16(T)) || (dX && !aligned16(dX))) return QLORA_ERR_INVALID_ARG;
+    cudaStream_t cs = as_stream(stream);
+    if (M == 0) {  // empty batch: the adapter gradients are zero
+        cudaError_t e = cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 2, cs);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, cs);
+        return cuda_status(e);
+    }
+    if (!ws || !aligned16(ws) || ws_bytes < qlora_linear_bwd_workspace_size(M, N, K, r))
+        return QLORA_ERR_WORKSPACE;
+    const size_t mr = align256(static_cast<size_t>(M) * r * 2);
+    uint16_t* U = reinterpret_cast<uint16_t*>(ws);
+    uint16_t* Tw = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + mr);
+    void* gws = reinterpret_cast<char*>(ws) + 2 * mr;
+    Nf4Weight w{codes, c2_fp8, c1, mean, N, K};
+    cudaError_t e = cudaSuccess;
+    if (!T) {
+        e = launch_lora_xat(X, A, M, K, r, s, Tw, cs);
+        T = Tw;
+    }
+    if (e == cudaSuccess) e = launch_lora_dyb(dY, B, M, N, r, s, U, cs);
+    if (e == cudaSuccess && dX) e = launch_bwd_dx_gemm(dY, w, U, A, M, r, dX, cs);
+    if (e == cudaSuccess) e = launch_lora_grads(dY, X, T, U, M, N, K, r, dA, dB, gws, cs);
+    return cuda_status(e);
+}
+
+uint64_t qlora_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int qlora_fp8_e4m3_encode(const float* x, uint8_t* out, int64_t n, void* stream) {
+    if (n < 0) return QLORA_ERR_INVALID_ARG;
+    if (n == 0) return QLORA_OK;
+    if (!ok_ptr(x) || !ok_ptr(out)) return QLORA_ERR_INVALID_ARG;
+    return cuda_status(launch_e4m3_encode(x, out, n, as_stream(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,61 @@
+// kernels.h -- internal launch interface between the C ABI (abi.cu) and the
+// kernel files.  All launches are asynchronous on `stream` and return the
+// CUDA error of the launch.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qlora {
+
+// quantize.cu
+cudaError_t launch_quantize_nf4_dq(const float* W, int64_t numel, uint8_t* codes, uint8_t* c2_fp8,
+                                   float* c1, float* mean, void* ws, int32_t* status,
+                                   cudaStream_t stream);
+cudaError_t launch_e4m3_encode(const float* x, uint8_t* out, int64_t n, cudaStream_t stream);
+
+// dequant.cu
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,
+                              const float* mean, int64_t numel, void* out, int out_dtype,
+                              cudaStream_t stream);
+
+// The frozen NF4 weight W (N x K row-major) as the GEMM kernels see it.
+struct Nf4Weight {
+    const uint8_t* codes;   // N*K/2 bytes
+    const uint8_t* c2_fp8;  // N*K/64 bytes
+    const float* c1;        // N*K/16384 floats (rounded up)
+    const float* mean;      // 1 float
+    int64_t N, K;
+};
+
+// lora.cu -- the skinny rank-r products of the LoRA path
+//   T  = bf16(s * X A^T)   (M x r)
+//   U  = bf16(s * dY B)    (M x r)
+//   dA = bf16(U^T X)       (r x K)
+//   dB = bf16(dY^T T)      (N x r)
+cudaError_t launch_lora_xat(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r,
+                            float s, uint16_t* T, cudaStream_t stream);
+cudaError_t launch_lora_dyb(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t N, int r,
+                            float s, uint16_t* U, cudaStream_t stream);
+size_t lora_grad_workspace(int64_t M, int64_t N, int64_t K, int r);
+cudaError_t launch_lora_grads(const uint16_t* dY, const uint16_t* X, const uint16_t* T,
+                              const uint16_t* U, int64_t M, int64_t N, int64_t K, int r,
+                              uint16_t* dA, uint16_t* dB, void* ws, cudaStream_t stream);
+
+// gemm_simt.cu -- CUDA-core versions of the frozen-weight GEMMs below
+cudaError_t launch_fwd_gemm_simt(const uint16_t* X, const Nf4Weight& w, const uint16_t* T,
+                                 const uint16_t* B, int64_t M, int r, uint16_t* Y, cudaStream_t stream);
+cudaError_t launch_bwd_dx_gemm_simt(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U,
+                                    const uint16_t* A, int64_t M, int r, uint16_t* dX,
+                                    cudaStream_t stream);
+
+// gemm_*.cu -- the frozen-weight GEMMs with the LoRA slab fused in
+//   Y  = bf16(X W'^T + T B^T)      (M x N)
+//   dX = bf16(dY W' + U A)         (M x K)
+cudaError_t launch_fwd_gemm(const uint16_t* X, const Nf4Weight& w, const uint16_t* T,
+                            const uint16_t* B, int64_t M, int r, uint16_t* Y, cudaStream_t stream);
+cudaError_t launch_bwd_dx_gemm(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U,
+                               const uint16_t* A, int64_t M, int r, uint16_t* dX,
+                               cudaStream_t stream);
+
+}  // namespace qlora

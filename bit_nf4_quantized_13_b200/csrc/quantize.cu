@@ -1,0 +1,284 @@
+// quantize.cu -- NF4 block-wise quantization fused with the exact-sum pass of
+// the double quantization, and the FP8 double-quantization pass itself.
+//
+// QLoRA study notes (gitcode.csdn.net): section 3.1 (block-wise absmax
+// quantization, blocks of 64 consecutive elements of the flattened tensor),
+// section 3.2 step 3 (normalise by absmax, then quantize to the nearest NF4
+// value), section 3.3 (double quantization: the fp32 constants c2 minus
+// their mean, quantized to 8-bit floats in blocks of 256).
+//
+// Kernel 1 (k_nf4_quantize) streams W once: HBM-bound at 4 B read + 0.5 B
+// written per weight.  A warp takes 512 consecutive weights per step: in
+// load i (0..3) lane l holds weights 4(32i + l) .. +3, so every load is one
+// fully coalesced 512-byte row and lanes 0-15 / 16-31 hold the two 64-blocks
+// of that row.  The block absmax is a 16-lane shuffle reduction.  Each
+// constant c2 is also added, exactly, into 256 integer bins (one per fp32
+// exponent) so that the mean of all c2 is exact and independent of the
+// order in which blocks finish.
+//
+// Kernel 2 (k_double_quant) turns the bins into the mean, then per group of
+// 256 constants computes c1 = max|c2 - mean| / 448 and the E4M3 bytes.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qlora {
+namespace {
+
+struct EncTab {
+    float thr;
+    int base;
+};
+
+// Nearest NF4 code of n in [-1, 1] (exact fp32 nearest-value rule, ties to
+// the lower code): a 33-bin table built on the host gives the code at the
+// bin's lower end and the one threshold that may lie inside the bin.
+__device__ __forceinline__ int nf4_code(float n, const EncTab* tab) {
+    const float v = __fadd_rn(n, 3.0f);
+    unsigned b = (__float_as_uint(v) >> 18) - 0x1000u;
+    b = b > 32u ? 32u : b;  // NaN / out-of-range guard (status is flagged)
+    const EncTab e = tab[b];
+    return e.base + (n >= e.thr ? 1 : 0);
+}
+
+__device__ __forceinline__ float4 ld_stream(const float* p) {
+    float4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ bool finite4(const float4& v) {
+    return isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
+}
+
+constexpr int kQuantThreads = 256;
+constexpr int kChunk = 512;  // weights per warp step
+
+__global__ void __launch_bounds__(kQuantThreads)
+k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__ codes,
+               float* __restrict__ c2, unsigned long long* __restrict__ bins,
+               int* __restrict__ flag, Nf4Tables tabs) {
+    __shared__ EncTab tab[33];
+    __shared__ unsigned long long sbins[256];
+    __shared__ int sbad;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
+    if (threadIdx.x < 33) tab[threadIdx.x] = EncTab{tabs.thr[threadIdx.x], tabs.base[threadIdx.x]};
+    if (threadIdx.x == 0) sbad = 0;
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int64_t nb = ceil_div(numel, kBlock);
+    const int64_t nchunks = ceil_div(numel, kChunk);
+    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    bool bad = false;
+
+    for (int64_t c = warp0; c < nchunks; c += nwarps) {
+        const int64_t base = c * kChunk;
+        const bool full = base + kChunk <= numel;
+        float4 v[4];
+        if (full) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[i] = ld_stream(W + base + 4 * (32 * i + lane));
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int64_t e = base + 4 * (32 * i + lane);
+                v[i].x = e + 0 < numel ? W[e + 0] : 0.0f;
+                v[i].y = e + 1 < numel ? W[e + 1] : 0.0f;
+                v[i].z = e + 2 < numel ? W[e + 2] : 0.0f;
+                v[i].w = e + 3 < numel ? W[e + 3] : 0.0f;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            bad |= !finite4(v[i]);
+            float m = fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w)));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            int q0 = 7, q1 = 7, q2 = 7, q3 = 7;
+            if (m > 0.0f) {
+                q0 = nf4_code(__fdiv_rn(v[i].x, m), tab);
+                q1 = nf4_code(__fdiv_rn(v[i].y, m), tab);
+                q2 = nf4_code(__fdiv_rn(v[i].z, m), tab);
+                q3 = nf4_code(__fdiv_rn(v[i].w, m), tab);
+            }
+            const int64_t e = base + 4 * (32 * i + lane);  // first weight of this lane
+            // byte e/2 = (code e << 4) | code e+1; byte e/2+1 likewise
+            const uint32_t b01 = static_cast<uint32_t>((q0 << 4) | q1) |
+                                 (static_cast<uint32_t>((q2 << 4) | q3) << 8);
+            if (full) {
+                *reinterpret_cast<uint16_t*>(codes + (e >> 1)) = static_cast<uint16_t>(b01);
+            } else {
+                if (e < numel) codes[e >> 1] = static_cast<uint8_t>(e + 1 < numel ? (b01 & 0xff) : (b01 & 0xf0));
+                if (e + 2 < numel) codes[(e >> 1) + 1] = static_cast<uint8_t>(e + 3 < numel ? (b01 >> 8) : ((b01 >> 8) & 0xf0));
+            }
+            if ((lane & 15) == 0) {
+                const int64_t blk = (base >> 6) + 2 * i + (lane >> 4);
+                if (blk < nb) {
+                    c2[blk] = m;
+                    const uint32_t u = __float_as_uint(m);
+                    const uint32_t ex = u >> 23;
+                    const unsigned long long mant = ex ? ((u & 0x7fffffu) | 0x800000u) : (u & 0x7fffffu);
+                    if (mant) atomicAdd(&sbins[ex & 255u], mant);
+                }
+            }
+        }
+    }
+    if (bad) sbad = 1;
+    __syncthreads();
+    for (int i = threadIdx.x; i < 256; i += blockDim.x)
+        if (sbins[i]) atomicAdd(&bins[i], sbins[i]);
+    if (threadIdx.x == 0 && sbad) atomicOr(flag, 1);
+}
+
+// ------------------------------------------------------------------------
+// Exact mean from the exponent bins.  Bin E holds the integer sum of the
+// 24-bit significands of all c2 with exponent field E; its value is
+// bins[E] * 2^(max(E,1) - 150).  The total, as an integer multiple of
+// 2^-149, is accumulated in 32-bit digits (carries deferred), rounded once
+// to the nearest double, divided by nb and rounded to fp32.
+constexpr int kDigits = 12;
+
+__device__ float mean_from_bins(const unsigned long long* __restrict__ bins, int64_t nb,
+                                unsigned long long* sdig /* shared, kDigits */) {
+    const int lane = threadIdx.x & 31;
+    if (lane < kDigits) sdig[lane] = 0ull;
+    __syncwarp();
+    for (int e = lane; e < 256; e += 32) {
+        const unsigned long long v = bins[e];
+        if (!v) continue;
+        const int sh = (e ? e : 1) - 1;
+        const int d0 = sh >> 5, off = sh & 31;
+        const unsigned long long lo = (v << off) & 0xffffffffull;
+        const unsigned long long mid = (off ? (v >> (32 - off)) : (v >> 32)) & 0xffffffffull;
+        const unsigned long long hi = off ? (v >> (64 - off)) : 0ull;
+        atomicAdd(&sdig[d0], lo);
+        atomicAdd(&sdig[d0 + 1], mid);
+        if (hi) atomicAdd(&sdig[d0 + 2], hi);
+    }
+    __syncwarp();
+    float mu = 0.0f;
+    if (lane == 0) {
+        unsigned long long d[kDigits + 1];
+        unsigned long long carry = 0;
+        for (int i = 0; i < kDigits; ++i) {
+            const unsigned long long t = sdig[i] + carry;
+            d[i] = t & 0xffffffffull;
+            carry = t >> 32;
+        }
+        d[kDigits] = carry;
+        int top = -1;
+        for (int i = kDigits; i >= 0; --i)
+            if (d[i]) { top = i; break; }
+        double sum = 0.0;
+        if (top >= 0) {
+            const int msb = 32 * top + 31 - __clzll(d[top]);  // bit index of the leading 1
+            auto bit = [&](int k) -> unsigned long long {
+                return k < 0 ? 0ull : (d[k >> 5] >> (k & 31)) & 1ull;
+            };
+            // the 53 bits [msb-52, msb], the round bit below them, and a
+            // sticky bit for everything further down
+            const int lsb = msb - 52;
+            unsigned long long m = 0;
+            for (int k = msb; k >= (lsb > 0 ? lsb : 0); --k) m = (m << 1) | bit(k);
+            if (lsb > 0) {
+                const unsigned long long rnd = bit(lsb - 1);
+                const int below = lsb - 1;  // bits [0, below) feed the sticky bit
+                bool sticky = false;
+                for (int i = 0; i < (below >> 5) && !sticky; ++i) sticky = d[i] != 0;
+                if (!sticky && (below & 31))
+                    sticky = (d[below >> 5] & ((1ull << (below & 31)) - 1ull)) != 0;
+                if (rnd && (sticky || (m & 1ull))) m += 1ull;  // 2^53 stays exact
+                sum = ldexp(static_cast<double>(m), lsb - 149);
+            } else {
+                sum = ldexp(static_cast<double>(m), -149);
+            }
+        }
+        mu = __double2float_rn(__ddiv_rn(sum, static_cast<double>(nb)));
+    }
+    return __shfl_sync(0xffffffffu, mu, 0);
+}
+
+constexpr int kDqThreads = 256;  // one thread per constant of a 256-group
+
+__global__ void __launch_bounds__(kDqThreads)
+k_double_quant(const float* __restrict__ c2, int64_t nb, const unsigned long long* __restrict__ bins,
+               const int* __restrict__ flag, uint8_t* __restrict__ c2_fp8, float* __restrict__ c1,
+               float* __restrict__ mean_out, int32_t* __restrict__ status) {
+    __shared__ unsigned long long sdig[kDigits];
+    __shared__ float smu;
+    __shared__ float sred[kDqThreads / 32];
+    if (threadIdx.x < 32) {
+        const float mu = mean_from_bins(bins, nb, sdig);
+        if (threadIdx.x == 0) smu = mu;
+    }
+    __syncthreads();
+    const float mu = smu;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *mean_out = mu;
+        if (status) *status = (*flag) ? QLORA_ERR_NONFINITE : QLORA_OK;
+    }
+    const int64_t ng = ceil_div(nb, kBlock2);
+    for (int64_t g = blockIdx.x; g < ng; g += gridDim.x) {
+        const int64_t j = g * kBlock2 + threadIdx.x;
+        const bool valid = j < nb;
+        const float y = valid ? __fsub_rn(c2[j], mu) : 0.0f;
+        float a = fabsf(y);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        if ((threadIdx.x & 31) == 0) sred[threadIdx.x >> 5] = a;
+        __syncthreads();
+        float amax = sred[0];
+#pragma unroll
+        for (int w = 1; w < kDqThreads / 32; ++w) amax = fmaxf(amax, sred[w]);
+        __syncthreads();  // sred is reused by the next group
+        const float c = __fdiv_rn(amax, 448.0f);
+        if (threadIdx.x == 0) c1[g] = c;
+        if (valid) c2_fp8[j] = (c == 0.0f) ? static_cast<uint8_t>(0) : f32_to_e4m3(__fdiv_rn(y, c));
+    }
+}
+
+__global__ void k_e4m3_encode(const float* __restrict__ x, uint8_t* __restrict__ out, int64_t n) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        out[i] = f32_to_e4m3(x[i]);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_nf4_dq(const float* W, int64_t numel, uint8_t* codes, uint8_t* c2_fp8,
+                                   float* c1, float* mean, void* ws, int32_t* status,
+                                   cudaStream_t stream) {
+    const int64_t nb = ceil_div(numel, kBlock);
+    auto* bins = reinterpret_cast<unsigned long long*>(ws);
+    int* flag = reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + kBinBytes);
+    float* c2 = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kBinBytes + kFlagBytes);
+    cudaError_t err = cudaMemsetAsync(ws, 0, kBinBytes + kFlagBytes, stream);
+    if (err != cudaSuccess) return err;
+    const int64_t nchunks = ceil_div(numel, kChunk);
+    const int64_t want = ceil_div(nchunks, kQuantThreads / 32);
+    const int grid1 = static_cast<int>(want < num_sms() * 8LL ? want : num_sms() * 8LL);
+    k_nf4_quantize<<<grid1, kQuantThreads, 0, stream>>>(W, numel, codes, c2, bins, flag, tables());
+    note_launches(1);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    const int64_t ng = ceil_div(nb, kBlock2);
+    const int grid2 = static_cast<int>(ng < num_sms() * 4LL ? ng : num_sms() * 4LL);
+    k_double_quant<<<grid2, kDqThreads, 0, stream>>>(c2, nb, bins, flag, c2_fp8, c1, mean, status);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_e4m3_encode(const float* x, uint8_t* out, int64_t n, cudaStream_t stream) {
+    const int64_t want = ceil_div(n, 256);
+    const int grid = static_cast<int>(want < num_sms() * 16LL ? want : num_sms() * 16LL);
+    k_e4m3_encode<<<grid, 256, 0, stream>>>(x, out, n);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace qlora

@@ -1,0 +1,171 @@
+/*
+ * qlora.h -- C ABI of the B200 (sm_100a) QLoRA NF4 linear-layer library.
+ *
+ * The hot path of QLoRA (Dettmers et al., "QLoRA: Efficient Finetuning of
+ * Quantized LLMs", arXiv:2305.14314) for one frozen linear layer with a LoRA
+ * side path.  Citations name the QLoRA study-notes page (gitcode.csdn.net) by
+ * section and equation.
+ *
+ * Notation (row-major, "out x in" like torch.nn.Linear):
+ *   W  N x K   frozen weight, stored as NF4 codes + double-quantized constants
+ *   X  M x K   input activations (bf16)
+ *   A  r x K   LoRA down projection (the pages' L1 = A^T)
+ *   B  N x r   LoRA up projection   (the pages' L2 = B^T)
+ *   s          the LoRA scalar of eq. (3) (usually alpha / r)
+ *   Y  M x N   output; dY, dX, dA, dB the matching gradients
+ *
+ * Conventions for every entry point:
+ *   - Array pointers are DEVICE pointers owned by the caller, except the one
+ *     host array of qlora_nf4_codebook.  The library never allocates or frees
+ *     memory; scratch space is passed in as a workspace (ws, ws_bytes).
+ *   - Every device pointer must be 16-byte aligned; tensors are contiguous.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued asynchronously; no call synchronizes the device.
+ *   - Every call returns a qlora_status.  Argument errors are detected on
+ *     the host before anything is enqueued.  QLORA_ERR_CUDA means a launch
+ *     failed (the CUDA error was consumed with cudaGetLastError).
+ *   - Calls that share a workspace must be ordered on one stream.
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qlora_status {
+    QLORA_OK = 0,
+    QLORA_ERR_INVALID_ARG = 1, /* null / negative / misaligned / bad dtype          */
+    QLORA_ERR_UNSUPPORTED = 2, /* block sizes other than 64/256, K % 64 != 0, r > 256 */
+    QLORA_ERR_WORKSPACE = 3,   /* ws NULL or ws_bytes below the documented size       */
+    QLORA_ERR_CUDA = 4,        /* a kernel launch or CUDA runtime call failed          */
+    QLORA_ERR_NONFINITE = 5,   /* written to the device status word: NaN/Inf in W      */
+    QLORA_ERR_TIMEOUT = 6      /* reserved: a bounded device wait gave up              */
+} qlora_status;
+
+#define QLORA_BLOCK 64       /* first-level block: elements per absmax constant  */
+#define QLORA_BLOCK2 256     /* second-level block: constants per FP8 scale       */
+#define QLORA_MAX_RANK 256   /* largest LoRA rank r                              */
+
+/*
+ * qlora_nf4_codebook -- the 16 values of the 4-bit NormalFloat type
+ * (section 3.2, eq. 4 and the asymmetric construction that keeps an exact
+ * zero): 7 negative quantiles of N(0,1), one 0 and 8 positive quantiles,
+ * normalised into [-1, 1].  Each half places its points at evenly spaced
+ * probabilities from 1/2 out to delta = ((1 - 1/30) + (1 - 1/32)) / 2.
+ * out_host: HOST array of 16 floats, sorted ascending (out[7] == 0,
+ * out[0] == -1, out[15] == +1).  Pure host function; never touches the GPU.
+ * Returns QLORA_INVALID_ARG for a NULL pointer.
+ */
+int qlora_nf4_codebook(float out_host[16]);
+
+/*
+ * Workspace bytes that qlora_quantize_nf4_dq needs for `numel` weights:
+ *   2048 (exact-sum bins) + 16 (flags) + round_up_16(4 * ceil(numel / 64)).
+ */
+size_t qlora_quantize_workspace_size(int64_t numel);
+
+/*
+ * qlora_quantize_nf4_dq -- block-wise NF4 quantization of a frozen weight
+ * with double quantization of its constants (sections 3.1-3.3, 3.5).
+ *
+ *   W       in : numel fp32 values (the flattened tensor).
+ *   block   in : must be 64 (QLORA_BLOCK); block2 must be 256 (QLORA_BLOCK2).
+ *   codes   out: ceil(numel/2) bytes; element 2t in the high nibble, 2t+1 in
+ *                the low nibble; an odd tail leaves a zero low nibble.
+ *   c2_fp8  out: nb = ceil(numel/64) bytes, the per-block absmax c2 after
+ *                double quantization, as OCP E4M3 codes.
+ *   c1      out: ceil(nb/256) fp32 second-level scales.
+ *   mean    out: 1 fp32, the mean of all c2, subtracted before the FP8 pass.
+ *   ws           scratch of qlora_quantize_workspace_size(numel) bytes.
+ *   status  out: nullable device int32; receives QLORA_OK, or
+ *                QLORA_ERR_NONFINITE if W holds a NaN or Inf (outputs then
+ *                unspecified).
+ *
+ * Definition (all steps IEEE fp32, round to nearest even, unfused):
+ *   c2[j]  = max |w| over the 64 consecutive elements of block j
+ *   code   = argmin_i |w / c2[j] - q_i| (ties to the lower i); c2 = 0 -> 7
+ *   mean   = RN32(RN64(S) / nb), S the exact sum of all c2
+ *   c1[g]  = max_{j in g} |c2[j] - mean| / 448
+ *   c2_fp8 = E4M3_rne_satfinite((c2[j] - mean) / c1[g]); 0 where c1[g] == 0
+ * numel == 0 enqueues nothing.  numel must be below 2^46.
+ */
+int qlora_quantize_nf4_dq(const float* W, int64_t numel, int block, int block2,
+                          uint8_t* codes, uint8_t* c2_fp8, float* c1, float* mean,
+                          void* ws, size_t ws_bytes, int32_t* status, void* stream);
+
+/*
+ * qlora_dequantize -- double dequantization (section 3.5, eq. 6):
+ *   c2' = RN32(RN32(E4M3(c2_fp8[j]) * c1[j / 256]) + mean)
+ *   w   = RN32(q[code] * c2')                 (out_dtype 0: fp32)
+ *   w   = bf16_rne(RN32(q[code] * c2'))       (out_dtype 1: bf16 bits)
+ * Inputs as written by qlora_quantize_nf4_dq; `mean` is a device pointer.
+ * out: numel elements of the chosen dtype.
+ */
+int qlora_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,
+                     const float* mean, int64_t numel, int block, int block2,
+                     void* out, int out_dtype, void* stream);
+
+/*
+ * Workspace bytes for qlora_linear_fwd / qlora_linear_bwd.  Both are safe to
+ * call with the maximum of the two.
+ */
+size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int r);
+size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r);
+
+/*
+ * qlora_linear_fwd -- the QLoRA linear (section 3.5 eq. 5 with the LoRA
+ * scalar of section 4 eq. 3):
+ *   T = bf16(s * X A^T)                       (M x r; saved to T_save if given)
+ *   Y = bf16(X W'^T + T B^T)                  fp32 accumulation
+ * where W' = bf16 of the double-dequantized weight (eq. 6).  W is given by
+ * the four buffers of qlora_quantize_nf4_dq for an N x K row-major weight.
+ * Requires K % 64 == 0, 1 <= r <= 256, M >= 0, N >= 1.
+ */
+int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                     const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,
+                     const float* mean, const uint16_t* A, const uint16_t* B, int r,
+                     float s, uint16_t* Y, uint16_t* T_save, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/*
+ * qlora_linear_bwd -- gradients of the QLoRA linear (section 3.5: gradients
+ * only for the adapters; the input gradient flows through the dequantized
+ * frozen weight in bf16; there is no gradient for W):
+ *   U  = bf16(s * dY B)                       (M x r)
+ *   dX = bf16(dY W' + U A)                    (nullable: skipped)
+ *   dA = bf16(U^T X)                          (r x K)
+ *   dB = bf16(dY^T T)                         (N x r), T = bf16(s X A^T)
+ * T: the T_save of the forward, or NULL to recompute it.  fp32 accumulation
+ * throughout.  Same shape rules as qlora_linear_fwd.
+ */
+int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N,
+                     int64_t K, const uint8_t* codes, const uint8_t* c2_fp8,
+                     const float* c1, const float* mean, const uint16_t* A,
+                     const uint16_t* B, int r, float s, const uint16_t* T,
+                     uint16_t* dX, uint16_t* dA, uint16_t* dB, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/*
+ * qlora_fp8_e4m3_encode -- the FP8 encoder the double quantization uses
+ * (section 3.3 names 8-bit floats; read as OCP E4M3): out[i] =
+ * E4M3_rne_satfinite(x[i]), NaN -> 0x7f.  n elements, device pointers.
+ */
+int qlora_fp8_e4m3_encode(const float* x, uint8_t* out, int64_t n, void* stream);
+
+/*
+ * qlora_kernel_launch_count -- number of kernels this library has launched
+ * in the calling process since it was loaded (all devices, all streams).
+ * A diagnostic for benchmarks that report how many kernels ran.
+ */
+uint64_t qlora_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H */
