@@ -176,7 +176,7 @@ __device__ float mean_from_bins(const unsigned long long* __restrict__ bins, int
             if (d[i]) { top = i; break; }
         double sum = 0.0;
         if (top >= 0) {
-            const int msb = 32 * top + 31 - __clzll(d[top]);  // bit index of the leading 1
+            const int msb = 32 * top + 63 - __clzll(d[top]);  // bit index of the leading 1 (digits are < 2^32)
             auto bit = [&](int k) -> unsigned long long {
                 return k < 0 ? 0ull : (d[k >> 5] >> (k & 31)) & 1ull;
             };

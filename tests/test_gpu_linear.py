@@ -34,13 +34,17 @@ def _run_case(case, rows=None, want_dx=True, pass_T=True):
     torch.cuda.synchronize()
     # the quantized weight is the oracle's, bit for bit
     np.testing.assert_array_equal(wq.codes.cpu().numpy(), d_ref["codes"])
+    np.testing.assert_array_equal(wq.c2_fp8.cpu().numpy(), d_ref["c2_fp8"])
+    assert wq.mean.cpu().numpy().view(np.uint32)[0] == np.float32(d_ref["mean"]).view(np.uint32)
+    np.testing.assert_array_equal(bits_of(q.qlora_dequantize(wq, torch.bfloat16)).reshape(-1),
+                                  Wb.reshape(-1))
 
     Yr, T0 = oracle.linear_fwd(case.X, Wb, case.A, case.B, case.s, rows=rows)
     dXr, dAr, dBr = oracle.linear_bwd(case.dY, case.X, Wb, case.A, case.B, case.s, rows=rows,
                                       want_dx=want_dx)
     sel = slice(None) if rows is None else rows
-    check_close(host_f64(Y)[sel], Yr, "Y")
     check_close(host_f64(T)[sel], case.s * T0, "T")
+    check_close(host_f64(Y)[sel], Yr, "Y")
     if want_dx:
         check_close(host_f64(dX)[sel], dXr, "dX")
     check_close(host_f64(dA), dAr, "dA")
