@@ -382,7 +382,7 @@ def run_native(args, world, rank, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_baseline(cases, [oracle_weight_bf16(c) for c in cases])
+        cpu = oracle_baseline(cases, [oracle_weight_bf16(c) for c in cases], rows_m=256, quant_elems=1 << 24)
 
     if rank == 0:
         line = {
