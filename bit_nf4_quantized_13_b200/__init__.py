@@ -7,7 +7,8 @@ torch CUDA tensors into device pointers, allocates outputs and workspaces
 with torch, passes torch's current stream, and raises on a non-OK status.
 Every step of the computation runs in the library's kernels; there is no
 fallback.  The library must have been built (``python -m
-bit_nf4_quantized_13_b200.build``); importing without it raises.
+bit_nf4_quantized_13_b200.build``); it is loaded on first use, and a missing
+or stale library raises ImportError there.
 
 Entry points (same names as the C ABI):
     qlora_nf4_codebook()                         -> numpy float32[16]
@@ -60,6 +61,7 @@ def _load() -> ctypes.CDLL:
                                    vp, vp, vp, sz, vp]),
         "qlora_fp8_e4m3_encode": (i32, [vp, vp, i64, vp]),
         "qlora_kernel_launch_count": (ctypes.c_uint64, []),
+        "qlora_quantize_nf4_dq_noalloc": (i32, [vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -67,7 +69,23 @@ def _load() -> ctypes.CDLL:
     return L
 
 
-lib = _load()
+_lib_handle = None
+
+
+def _get_lib() -> ctypes.CDLL:
+    global _lib_handle
+    if _lib_handle is None:
+        try:
+            _lib_handle = _load()
+        except AttributeError as e:  # a library built from older sources
+            raise ImportError(f"{LIB_PATH} is stale ({e}); rebuild it") from e
+    return _lib_handle
+
+
+def __getattr__(name):
+    if name == "lib":
+        return _get_lib()
+    raise AttributeError(name)
 
 
 def _torch():
@@ -105,7 +123,7 @@ def _workspace(nbytes: int, device):
 
 def qlora_nf4_codebook() -> np.ndarray:
     out = np.zeros(16, np.float32)
-    _check("qlora_nf4_codebook", lib.qlora_nf4_codebook(out.ctypes.data_as(ctypes.c_void_p)))
+    _check("qlora_nf4_codebook", _get_lib().qlora_nf4_codebook(out.ctypes.data_as(ctypes.c_void_p)))
     return out
 
 
@@ -132,7 +150,7 @@ class Nf4Weight:
 
 
 def qlora_quantize_workspace_size(numel: int) -> int:
-    return int(lib.qlora_quantize_workspace_size(int(numel)))
+    return int(_get_lib().qlora_quantize_workspace_size(int(numel)))
 
 
 def alloc_nf4_weight(shape, device) -> Nf4Weight:
@@ -158,7 +176,7 @@ def qlora_quantize_nf4_dq(W, out: Nf4Weight | None = None, ws=None, status=None,
     w = out if out is not None else alloc_nf4_weight(tuple(W.shape), W.device)
     if ws is None:
         ws = _workspace(qlora_quantize_workspace_size(n), W.device)
-    st = lib.qlora_quantize_nf4_dq(_ptr(W), n, BLOCK, BLOCK2, _ptr(w.codes), _ptr(w.c2_fp8),
+    st = _get_lib().qlora_quantize_nf4_dq(_ptr(W), n, BLOCK, BLOCK2, _ptr(w.codes), _ptr(w.c2_fp8),
                                    _ptr(w.c1), _ptr(w.mean), _ptr(ws), ws.numel(), _ptr(status),
                                    _stream(stream))
     _check("qlora_quantize_nf4_dq", st)
@@ -171,7 +189,7 @@ def qlora_dequantize(w: Nf4Weight, out_dtype=None, out=None, stream=None):
     code = {torch.float32: 0, torch.bfloat16: 1}[out_dtype]
     if out is None:
         out = torch.empty(w.shape, dtype=out_dtype, device=w.codes.device)
-    st = lib.qlora_dequantize(_ptr(w.codes), _ptr(w.c2_fp8), _ptr(w.c1), _ptr(w.mean), w.numel,
+    st = _get_lib().qlora_dequantize(_ptr(w.codes), _ptr(w.c2_fp8), _ptr(w.c1), _ptr(w.mean), w.numel,
                               BLOCK, BLOCK2, _ptr(out), code, _stream(stream))
     _check("qlora_dequantize", st)
     return out
@@ -180,11 +198,11 @@ def qlora_dequantize(w: Nf4Weight, out_dtype=None, out=None, stream=None):
 # ------------------------------------------------------------------- linear
 
 def qlora_linear_fwd_workspace_size(M, N, K, r) -> int:
-    return int(lib.qlora_linear_fwd_workspace_size(int(M), int(N), int(K), int(r)))
+    return int(_get_lib().qlora_linear_fwd_workspace_size(int(M), int(N), int(K), int(r)))
 
 
 def qlora_linear_bwd_workspace_size(M, N, K, r) -> int:
-    return int(lib.qlora_linear_bwd_workspace_size(int(M), int(N), int(K), int(r)))
+    return int(_get_lib().qlora_linear_bwd_workspace_size(int(M), int(N), int(K), int(r)))
 
 
 def qlora_linear_fwd(X, w: Nf4Weight, A, B, s: float, Y=None, T_save=None, ws=None, stream=None):
@@ -200,7 +218,7 @@ def qlora_linear_fwd(X, w: Nf4Weight, A, B, s: float, Y=None, T_save=None, ws=No
         T_save = torch.empty((M, r), dtype=torch.bfloat16, device=X.device)
     if ws is None:
         ws = _workspace(16, X.device)
-    st = lib.qlora_linear_fwd(_ptr(X), M, N, K, _ptr(w.codes), _ptr(w.c2_fp8), _ptr(w.c1),
+    st = _get_lib().qlora_linear_fwd(_ptr(X), M, N, K, _ptr(w.codes), _ptr(w.c2_fp8), _ptr(w.c1),
                               _ptr(w.mean), _ptr(A), _ptr(B), r, float(s), _ptr(Y), _ptr(T_save),
                               _ptr(ws), ws.numel(), _stream(stream))
     _check("qlora_linear_fwd", st)
@@ -223,7 +241,7 @@ def qlora_linear_bwd(dY, X, w: Nf4Weight, A, B, s: float, T=None, dX=None, dA=No
         dB = torch.empty((N, r), dtype=torch.bfloat16, device=X.device)
     if ws is None:
         ws = _workspace(qlora_linear_bwd_workspace_size(M, N, K, r), X.device)
-    st = lib.qlora_linear_bwd(_ptr(dY), _ptr(X), M, N, K, _ptr(w.codes), _ptr(w.c2_fp8),
+    st = _get_lib().qlora_linear_bwd(_ptr(dY), _ptr(X), M, N, K, _ptr(w.codes), _ptr(w.c2_fp8),
                               _ptr(w.c1), _ptr(w.mean), _ptr(A), _ptr(B), r, float(s), _ptr(T),
                               _ptr(dX if want_dx else None), _ptr(dA), _ptr(dB), _ptr(ws),
                               ws.numel(), _stream(stream))
@@ -237,10 +255,29 @@ def qlora_fp8_e4m3_encode(x, out=None, stream=None):
     if out is None:
         out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     _check("qlora_fp8_e4m3_encode",
-           lib.qlora_fp8_e4m3_encode(_ptr(x), _ptr(out), x.numel(), _stream(stream)))
+           _get_lib().qlora_fp8_e4m3_encode(_ptr(x), _ptr(out), x.numel(), _stream(stream)))
     return out
 
 
 def qlora_kernel_launch_count() -> int:
     """Kernels this library has launched in this process so far."""
-    return int(lib.qlora_kernel_launch_count())
+    return int(_get_lib().qlora_kernel_launch_count())
+
+
+NOALLOC_MAX_NUMEL = 1 << 28
+
+
+def qlora_quantize_nf4_dq_noalloc(W, out: Nf4Weight | None = None, status=None,
+                                  stream=None) -> Nf4Weight:
+    """qlora_quantize_nf4_dq without a workspace: the library's built-in
+    device scratch is used instead (numel <= 2^28; calls must not overlap)."""
+    torch = _torch()
+    _need_cuda(W)
+    if W.dtype != torch.float32:
+        raise ValueError("W must be float32")
+    w = out if out is not None else alloc_nf4_weight(tuple(W.shape), W.device)
+    st = _get_lib().qlora_quantize_nf4_dq_noalloc(_ptr(W), W.numel(), BLOCK, BLOCK2, _ptr(w.codes),
+                                           _ptr(w.c2_fp8), _ptr(w.c1), _ptr(w.mean), _ptr(status),
+                                           _stream(stream))
+    _check("qlora_quantize_nf4_dq_noalloc", st)
+    return w

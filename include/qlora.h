@@ -99,6 +99,32 @@ int qlora_quantize_nf4_dq(const float* W, int64_t numel, int block, int block2,
                           void* ws, size_t ws_bytes, int32_t* status, void* stream);
 
 /*
+ * qlora_quantize_nf4_dq_noalloc -- the same quantization as
+ * qlora_quantize_nf4_dq (same arguments minus ws / ws_bytes, same outputs,
+ * bit for bit), for callers that cannot give the library a workspace: for
+ * example a plugin whose host program owns all device memory and offers no
+ * allocator, or a loop that cannot afford cudaMalloc's implicit
+ * synchronisation.  The paper has no counterpart; this is a library
+ * convenience.
+ *
+ * Its scratch is one fixed device array inside the library, reserved on
+ * every GPU that loads it until the process exits: 2064 bytes plus 4 bytes
+ * per 64-block, sized for numel <= QLORA_NOALLOC_MAX_NUMEL (2^28 weights,
+ * about 16 MiB).  Larger numel returns QLORA_ERR_WORKSPACE without
+ * launching anything.  The call allocates nothing (no cudaMalloc/cudaFree).
+ * The first call on each device, made with that device current, looks up
+ * the array's device address once (cudaGetSymbolAddress); make that first
+ * call before any stream capture.  All calls share the one array: calls
+ * whose kernels overlap on the GPU (different streams without ordering,
+ * or several host threads) race on it and must be serialised by the
+ * caller.  Each call clears the parts that must start at zero.
+ */
+#define QLORA_NOALLOC_MAX_NUMEL (1LL << 28)
+int qlora_quantize_nf4_dq_noalloc(const float* W, int64_t numel, int block, int block2,
+                                  uint8_t* codes, uint8_t* c2_fp8, float* c1, float* mean,
+                                  int32_t* status, void* stream);
+
+/*
  * qlora_dequantize -- double dequantization (section 3.5, eq. 6):
  *   c2' = RN32(RN32(E4M3(c2_fp8[j]) * c1[j / 256]) + mean)
  *   w   = RN32(q[code] * c2')                 (out_dtype 0: fp32)
