@@ -61,6 +61,7 @@ def _load() -> ctypes.CDLL:
                                    vp, vp, vp, sz, vp]),
         "qlora_fp8_e4m3_encode": (i32, [vp, vp, i64, vp]),
         "qlora_kernel_launch_count": (ctypes.c_uint64, []),
+        "qlora_device_error": (i32, [i32]),
         "qlora_quantize_nf4_dq_noalloc": (i32, [vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
@@ -257,6 +258,12 @@ def qlora_fp8_e4m3_encode(x, out=None, stream=None):
     _check("qlora_fp8_e4m3_encode",
            _get_lib().qlora_fp8_e4m3_encode(_ptr(x), _ptr(out), x.numel(), _stream(stream)))
     return out
+
+
+def qlora_device_error(reset: bool = False) -> int:
+    """Sticky error word of the tensor-core kernels (0 = none, 6 = a bounded
+    in-kernel wait timed out)."""
+    return int(_get_lib().qlora_device_error(1 if reset else 0))
 
 
 def qlora_kernel_launch_count() -> int:

@@ -30,6 +30,7 @@ int num_sms() {
 
 cudaError_t launch_fwd_gemm(const uint16_t* X, const Nf4Weight& w, const uint16_t* T,
                             const uint16_t* B, int64_t M, int r, uint16_t* Y, cudaStream_t st) {
+    if (fwd_tc_supported(M, w, r)) return launch_fwd_gemm_tc(X, w, T, B, M, r, Y, st);
     return launch_fwd_gemm_simt(X, w, T, B, M, r, Y, st);
 }
 

@@ -184,6 +184,15 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N
 int qlora_fp8_e4m3_encode(const float* x, uint8_t* out, int64_t n, void* stream);
 
 /*
+ * qlora_device_error -- the sticky error word of the tensor-core kernels on
+ * the current device: QLORA_OK, or QLORA_ERR_TIMEOUT if a pipeline wait
+ * inside a kernel gave up (the kernel then ended early and its outputs are
+ * invalid).  Synchronizes with the device to read it; reset != 0 clears it.
+ * Returns QLORA_ERR_CUDA if the word cannot be read.
+ */
+int qlora_device_error(int reset);
+
+/*
  * qlora_kernel_launch_count -- number of kernels this library has launched
  * in the calling process since it was loaded (all devices, all streams).
  * A diagnostic for benchmarks that report how many kernels ran.

@@ -42,6 +42,7 @@ def _run_case(case, rows=None, want_dx=True, pass_T=True):
     Yr, T0 = oracle.linear_fwd(case.X, Wb, case.A, case.B, case.s, rows=rows)
     dXr, dAr, dBr = oracle.linear_bwd(case.dY, case.X, Wb, case.A, case.B, case.s, rows=rows,
                                       want_dx=want_dx)
+    assert q.qlora_device_error(reset=True) == 0
     sel = slice(None) if rows is None else rows
     check_close(host_f64(T)[sel], case.s * T0, "T")
     check_close(host_f64(Y)[sel], Yr, "Y")
