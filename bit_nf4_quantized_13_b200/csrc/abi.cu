@@ -36,6 +36,7 @@ cudaError_t launch_fwd_gemm(const uint16_t* X, const Nf4Weight& w, const uint16_
 
 cudaError_t launch_bwd_dx_gemm(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U,
                                const uint16_t* A, int64_t M, int r, uint16_t* dX, cudaStream_t st) {
+    if (dx_tc_supported(M, w, r)) return launch_bwd_dx_gemm_tc(dY, w, U, A, M, r, dX, st);
     return launch_bwd_dx_gemm_simt(dY, w, U, A, M, r, dX, st);
 }
 

@@ -49,10 +49,14 @@ cudaError_t launch_bwd_dx_gemm_simt(const uint16_t* dY, const Nf4Weight& w, cons
                                     const uint16_t* A, int64_t M, int r, uint16_t* dX,
                                     cudaStream_t stream);
 
-// gemm_fwd_sm100.cu -- tcgen05 forward (r % 8 == 0)
+// gemm_nf4_sm100.cu -- tcgen05 forward and backward-dX (r % 8 == 0; the
+// backward also needs N % 8 == 0)
 bool fwd_tc_supported(int64_t M, const Nf4Weight& w, int r);
+bool dx_tc_supported(int64_t M, const Nf4Weight& w, int r);
 cudaError_t launch_fwd_gemm_tc(const uint16_t* X, const Nf4Weight& w, const uint16_t* T, const uint16_t* B,
                                int64_t M, int r, uint16_t* Y, cudaStream_t stream);
+cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U, const uint16_t* A,
+                                  int64_t M, int r, uint16_t* dX, cudaStream_t stream);
 
 // gemm_*.cu -- the frozen-weight GEMMs with the LoRA slab fused in
 //   Y  = bf16(X W'^T + T B^T)      (M x N)

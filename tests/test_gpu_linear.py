@@ -60,7 +60,8 @@ def test_tiny_config():
 
 @pytest.mark.parametrize("M,N,K,r", [(1, 64, 64, 1), (3, 100, 192, 8), (17, 513, 128, 16),
                                      (130, 257, 320, 64), (64, 128, 256, 256), (200, 96, 512, 3),
-                                     (129, 200, 64, 33)])
+                                     (129, 200, 64, 33), (300, 520, 192, 16), (257, 1000, 256, 72),
+                                     (77, 136, 448, 24)])
 def test_ragged_shapes(M, N, K, r):
     case = synth.linear_case(f"m{M}n{N}k{K}r{r}", M, N, K, r, 16.0, seed=1, outlier_frac=0.001)
     _run_case(case)
