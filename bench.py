@@ -256,7 +256,7 @@ def run_native(args, world, rank, local):
             q.qlora_quantize_nf4_dq(b["W"], out=b["wq"], ws=b["qws"])
             if ev is not None:
                 ev[i][1].record(stream)
-            q.qlora_linear_fwd(b["X"], b["wq"], b["A"], b["B"], c.s, Y=b["Y"], T_save=b["T"])
+            q.qlora_linear_fwd(b["X"], b["wq"], b["A"], b["B"], c.s, Y=b["Y"], T_save=b["T"], ws=b["bws"])
             if ev is not None:
                 ev[i][2].record(stream)
             q.qlora_linear_bwd(b["dY"], b["X"], b["wq"], b["A"], b["B"], c.s, T=b["T"], dX=b["dX"],

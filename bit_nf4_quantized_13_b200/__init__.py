@@ -218,7 +218,7 @@ def qlora_linear_fwd(X, w: Nf4Weight, A, B, s: float, Y=None, T_save=None, ws=No
     if T_save is None:
         T_save = torch.empty((M, r), dtype=torch.bfloat16, device=X.device)
     if ws is None:
-        ws = _workspace(16, X.device)
+        ws = _workspace(qlora_linear_fwd_workspace_size(M, N, K, r), X.device)
     st = _get_lib().qlora_linear_fwd(_ptr(X), M, N, K, _ptr(w.codes), _ptr(w.c2_fp8), _ptr(w.c1),
                               _ptr(w.mean), _ptr(A), _ptr(B), r, float(s), _ptr(Y), _ptr(T_save),
                               _ptr(ws), ws.numel(), _stream(stream))

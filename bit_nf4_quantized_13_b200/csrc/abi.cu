@@ -40,6 +40,28 @@ cudaError_t launch_bwd_dx_gemm(const uint16_t* dY, const Nf4Weight& w, const uin
     return launch_bwd_dx_gemm_simt(dY, w, U, A, M, r, dX, st);
 }
 
+// The rank-r products: tensor cores where the shapes allow TMA (r % 8 == 0,
+// N % 8 == 0), CUDA cores otherwise.
+cudaError_t lora_xat(const uint16_t* X, const uint16_t* A, int64_t M, int64_t N, int64_t K, int r, float s,
+                     uint16_t* T, float* part, cudaStream_t st) {
+    if (lora_tc_supported(M, N, K, r)) return launch_lora_xat_tc(X, A, M, K, r, s, T, part, st);
+    return launch_lora_xat_simt(X, A, M, K, r, s, T, st);
+}
+
+cudaError_t lora_dyb(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t N, int64_t K, int r, float s,
+                     uint16_t* U, float* part, cudaStream_t st) {
+    if (lora_tc_supported(M, N, K, r)) return launch_lora_dyb_tc(dY, B, M, N, r, s, U, part, st);
+    return launch_lora_dyb_simt(dY, B, M, N, r, s, U, st);
+}
+
+cudaError_t lora_grads(const uint16_t* dY, const uint16_t* X, const uint16_t* T, const uint16_t* U, int64_t M,
+                       int64_t N, int64_t K, int r, uint16_t* dA, uint16_t* dB, float* part, cudaStream_t st) {
+    if (!lora_tc_supported(M, N, K, r)) return launch_lora_grads_simt(dY, X, T, U, M, N, K, r, dA, dB, st);
+    cudaError_t e = launch_lora_da_tc(X, U, M, K, r, dA, part, st);
+    if (e != cudaSuccess) return e;
+    return launch_lora_db_tc(dY, T, M, N, r, dB, part, st);
+}
+
 }  // namespace qlora
 
 using namespace qlora;
@@ -104,13 +126,14 @@ int qlora_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c
 
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
     if (check_linear(M, N, K, r) != QLORA_OK) return 0;
-    return align256(static_cast<size_t>(M) * r * 2);  // T when T_save is NULL
+    // T (used when T_save is NULL), then the split-K partials of the rank-r products
+    return align256(static_cast<size_t>(M) * r * 2) + align256(lora_tc_workspace(M, N, K, r));
 }
 
 size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
     if (check_linear(M, N, K, r) != QLORA_OK) return 0;
     const size_t mr = align256(static_cast<size_t>(M) * r * 2);
-    return 2 * mr + align256(lora_grad_workspace(M, N, K, r));  // U, T (when T is NULL), grads
+    return 2 * mr + align256(lora_tc_workspace(M, N, K, r));  // U, T (when T is NULL), partials
 }
 
 int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
@@ -123,15 +146,13 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     if (!ok_ptr(A) || !ok_ptr(B) || (M > 0 && (!ok_ptr(X) || !ok_ptr(Y)))) return QLORA_ERR_INVALID_ARG;
     if (T_save && !aligned16(T_save)) return QLORA_ERR_INVALID_ARG;
     if (M == 0) return QLORA_OK;
-    uint16_t* T = T_save;
-    if (!T) {
-        if (!ws || !aligned16(ws) || ws_bytes < qlora_linear_fwd_workspace_size(M, N, K, r))
-            return QLORA_ERR_WORKSPACE;
-        T = reinterpret_cast<uint16_t*>(ws);
-    }
+    if (!ws || !aligned16(ws) || ws_bytes < qlora_linear_fwd_workspace_size(M, N, K, r))
+        return QLORA_ERR_WORKSPACE;
+    uint16_t* T = T_save ? T_save : reinterpret_cast<uint16_t*>(ws);
+    float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + align256(static_cast<size_t>(M) * r * 2));
     cudaStream_t cs = as_stream(stream);
     Nf4Weight w{codes, c2_fp8, c1, mean, N, K};
-    cudaError_t e = launch_lora_xat(X, A, M, K, r, s, T, cs);
+    cudaError_t e = lora_xat(X, A, M, N, K, r, s, T, part, cs);
     if (e == cudaSuccess) e = launch_fwd_gemm(X, w, T, B, M, r, Y, cs);
     return cuda_status(e);
 }
@@ -158,17 +179,23 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N
     const size_t mr = align256(static_cast<size_t>(M) * r * 2);
     uint16_t* U = reinterpret_cast<uint16_t*>(ws);
     uint16_t* Tw = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + mr);
-    void* gws = reinterpret_cast<char*>(ws) + 2 * mr;
+    float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 2 * mr);
     Nf4Weight w{codes, c2_fp8, c1, mean, N, K};
     cudaError_t e = cudaSuccess;
     if (!T) {
-        e = launch_lora_xat(X, A, M, K, r, s, Tw, cs);
+        e = lora_xat(X, A, M, N, K, r, s, Tw, part, cs);
         T = Tw;
     }
-    if (e == cudaSuccess) e = launch_lora_dyb(dY, B, M, N, r, s, U, cs);
+    if (e == cudaSuccess) e = lora_dyb(dY, B, M, N, K, r, s, U, part, cs);
     if (e == cudaSuccess && dX) e = launch_bwd_dx_gemm(dY, w, U, A, M, r, dX, cs);
-    if (e == cudaSuccess) e = launch_lora_grads(dY, X, T, U, M, N, K, r, dA, dB, gws, cs);
+    if (e == cudaSuccess) e = lora_grads(dY, X, T, U, M, N, K, r, dA, dB, part, cs);
     return cuda_status(e);
+}
+
+int qlora_device_error(int reset) {
+    const int a = gemm_device_error(reset);
+    const int b = lora_device_error(reset);
+    return a != QLORA_OK ? a : b;
 }
 
 uint64_t qlora_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -465,12 +465,16 @@ cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const 
 
 }  // namespace qlora
 
-extern "C" int qlora_device_error(int reset) {
+namespace qlora {
+
+int gemm_device_error(int reset) {
     int v = 0;
-    if (cudaMemcpyFromSymbol(&v, qlora::g_tc_error, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, g_tc_error, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
     if (reset && v) {
         const int zero = 0;
-        if (cudaMemcpyToSymbol(qlora::g_tc_error, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+        if (cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
     }
     return v;
 }
+
+}  // namespace qlora

@@ -111,23 +111,21 @@ cudaError_t gemm(int64_t Mo, int64_t No, const Opnd& a1, const Opnd& b1, int64_t
 
 }  // namespace
 
-cudaError_t launch_lora_xat(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r,
+cudaError_t launch_lora_xat_simt(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r,
                             float s, uint16_t* T, cudaStream_t st) {
     // T(m, j) = s * sum_k X[m][k] A[j][k]
     return gemm(M, r, bf16_op(X, K, 1), bf16_op(A, K, 1), K, Opnd{}, Opnd{}, 0, s, T, r, st);
 }
 
-cudaError_t launch_lora_dyb(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t N, int r,
+cudaError_t launch_lora_dyb_simt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t N, int r,
                             float s, uint16_t* U, cudaStream_t st) {
     // U(m, j) = s * sum_n dY[m][n] B[n][j]
     return gemm(M, r, bf16_op(dY, N, 1), bf16_op(B, 1, r), N, Opnd{}, Opnd{}, 0, s, U, r, st);
 }
 
-size_t lora_grad_workspace(int64_t, int64_t, int64_t, int) { return 0; }
-
-cudaError_t launch_lora_grads(const uint16_t* dY, const uint16_t* X, const uint16_t* T,
+cudaError_t launch_lora_grads_simt(const uint16_t* dY, const uint16_t* X, const uint16_t* T,
                               const uint16_t* U, int64_t M, int64_t N, int64_t K, int r,
-                              uint16_t* dA, uint16_t* dB, void*, cudaStream_t st) {
+                              uint16_t* dA, uint16_t* dB, cudaStream_t st) {
     // dA(j, k) = sum_m U[m][j] X[m][k];  dB(n, j) = sum_m dY[m][n] T[m][j]
     cudaError_t e = gemm(r, K, bf16_op(U, 1, r), bf16_op(X, 1, K), M, Opnd{}, Opnd{}, 0, 1.0f, dA, K, st);
     if (e != cudaSuccess) return e;

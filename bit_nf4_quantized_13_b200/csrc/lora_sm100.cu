@@ -1,0 +1,340 @@
+// lora_sm100.cu -- the rank-r products of the LoRA path (QLoRA study notes,
+// gitcode.csdn.net, section 4 eq. 3 and the adapter gradients of section
+// 3.5) on the 5th-generation tensor cores:
+//
+//   T  = bf16(s X A^T)      (M x r)   contraction over K
+//   U  = bf16(s dY B)       (M x r)   contraction over N
+//   dA = bf16(U^T X)        (r x K)   contraction over the M tokens
+//   dB = bf16(dY^T T)       (N x r)   contraction over the M tokens
+//
+// Each is a skinny GEMM C[rows x r] = sum_k Aop[row][k] Bop[j][k] whose
+// operands are row-major bf16 matrices read either along their contiguous
+// dimension (K-major) or across it (MN-major); TMA loads both in the
+// 128-byte swizzled layout and tcgen05.mma takes either major-ness.  The
+// outputs have only r columns, so the contraction is split across CTAs
+// (split-K) to fill the GPU; each split writes fp32 partials that a second
+// kernel sums in a fixed order (deterministic), scales and rounds to bf16.
+//
+// One CTA = one 128-row tile x one contraction split: warp 0 issues TMA,
+// warp 1 the MMAs (M = 128, N = r rounded up to 16), then all four warps
+// read the accumulator from tensor memory and store the partials.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace qlora {
+
+__device__ int g_lora_error = 0;  // sticky: QLORA_ERR_TIMEOUT if a wait gave up
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kRows = 128;   // output rows per tile (MMA M)
+constexpr int kBK = 64;      // contraction per stage
+constexpr int kThreads = 128;
+constexpr int kABytes = kRows * kBK * 2;  // 16 KiB
+constexpr int kMaxSmem = 200 * 1024;
+
+struct SkinnyParams {
+    float* part;   // [splits][rows][nt] fp32
+    int rows;      // output rows
+    int nt;        // r rounded up to 16 (MMA N)
+    int kb_total;  // 64-wide contraction blocks
+    int kb_per_split;
+    int stages;
+    int b_bytes;   // bytes of one B stage
+    uint32_t tmem_cols;
+};
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kThreads)
+k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, const SkinnyParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int stage_bytes = kABytes + p.b_bytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.stages * stage_bytes);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * p.stages + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t bar0 = smem_u32(bars);
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (p.stages + s); };
+    const uint32_t done = bar0 + 8u * (2 * p.stages);
+
+    const int row0 = blockIdx.x * kRows;
+    const int split = blockIdx.y;
+    const int kb_begin = split * p.kb_per_split;
+    const int kb_end = min(p.kb_total, kb_begin + p.kb_per_split);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(done, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    int* err = &g_lora_error;
+    bool ok = true;
+
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&ta);
+        tma_prefetch_desc(&tb);
+        for (int kb = kb_begin, it = 0; kb < kb_end; ++kb, ++it) {
+            const int s = it % p.stages;
+            const uint32_t ph = (it / p.stages) & 1u;
+            if (!mbar_wait(empty(s), ph ^ 1u, err)) break;
+            mbar_arrive_expect_tx(full(s), kABytes + p.b_bytes);
+            const uint32_t sa = smem_u32(smem + s * stage_bytes);
+            const uint32_t sb = sa + kABytes;
+            if (A_MN) {  // 128 MN-contiguous rows as two 64-wide boxes, 64 contraction rows each
+                tma_load_2d(sa, &ta, full(s), row0, kb * kBK);
+                tma_load_2d(sa + 8192, &ta, full(s), row0 + 64, kb * kBK);
+            } else {
+                tma_load_2d(sa, &ta, full(s), kb * kBK, row0);
+            }
+            if (B_MN) {
+                for (int b = 0; b * 64 < p.nt; ++b) tma_load_2d(sb + b * 8192, &tb, full(s), b * 64, kb * kBK);
+            } else {
+                tma_load_2d(sb, &tb, full(s), kb * kBK, 0);
+            }
+        }
+    } else if (warp == 1 && lane == 0) {
+        const uint32_t idesc = idesc_bf16(kRows, p.nt, A_MN ? 1 : 0, B_MN ? 1 : 0);
+        for (int kb = kb_begin, it = 0; kb < kb_end; ++kb, ++it) {
+            const int s = it % p.stages;
+            const uint32_t ph = (it / p.stages) & 1u;
+            if (!mbar_wait(full(s), ph, err)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + s * stage_bytes);
+            const uint32_t sb = sa + kABytes;
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+                // 16 contraction steps: +32 bytes along a K-major row, +16 rows of 128 bytes MN-major
+                const uint64_t ad = A_MN ? sdesc_mnmajor_sw128(sa + kk * 2048, 8192)
+                                         : sdesc_kmajor_sw128(sa) + static_cast<uint64_t>(kk * 2);
+                const uint64_t bd = B_MN ? sdesc_mnmajor_sw128(sb + kk * 2048, 8192)
+                                         : sdesc_kmajor_sw128(sb) + static_cast<uint64_t>(kk * 2);
+                mma_bf16_ss(tmem, ad, bd, idesc, (kb > kb_begin || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(empty(s));
+        }
+        if (ok) tc_commit(done);
+    }
+    __syncwarp();
+    // epilogue: lane quarter of each warp = 32 output rows, 16 columns at a time
+    const bool fin = __all_sync(0xffffffffu, mbar_wait(done, 0, err));
+    if (fin) {
+        tc_fence_after();
+        const int row = row0 + warp * 32 + lane;
+        float* dst = p.part + (static_cast<int64_t>(split) * p.rows + row) * p.nt;
+        for (int c0 = 0; c0 < p.nt; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
+            tmem_wait_ld();
+            if (row < p.rows) {
+#pragma unroll
+                for (int t = 0; t < 16; t += 4)
+                    *reinterpret_cast<float4*>(dst + c0 + t) = make_float4(
+                        __uint_as_float(v[t]), __uint_as_float(v[t + 1]), __uint_as_float(v[t + 2]),
+                        __uint_as_float(v[t + 3]));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, p.tmem_cols);
+    }
+}
+
+// out = bf16(scale * sum_s part[s]) in a fixed order; `transposed` writes
+// out[j][i] (dA) instead of out[i][j].
+__global__ void k_lora_reduce(const float* __restrict__ part, int splits, int rows, int nt, int r, float scale,
+                              uint16_t* __restrict__ out, int transposed) {
+    const int64_t total = static_cast<int64_t>(rows) * r;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        int64_t i, j;
+        if (transposed) {  // consecutive threads walk i so the stores are contiguous
+            j = idx / rows;
+            i = idx % rows;
+        } else {
+            i = idx / r;
+            j = idx % r;
+        }
+        float acc = 0.0f;
+        for (int s = 0; s < splits; ++s) acc += part[(static_cast<int64_t>(s) * rows + i) * nt + j];
+        const uint16_t b = f32_to_bf16_bits(scale * acc);
+        if (transposed)
+            out[j * rows + i] = b;
+        else
+            out[i * r + j] = b;
+    }
+}
+
+// ------------------------------------------------------------------ host
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+              uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Plan {
+    int nt, kb_total, kb_per_split, splits, stages, b_bytes, smem;
+    uint32_t tmem_cols;
+    int64_t tiles;
+};
+
+Plan plan(int64_t rows, int64_t ctr, int r, bool b_mn) {
+    Plan pl;
+    pl.nt = static_cast<int>(round_up(r, 16));
+    pl.kb_total = static_cast<int>(ceil_div(ctr, kBK));
+    pl.tiles = ceil_div(rows, kRows);
+    const int64_t target = 2LL * num_sms();
+    int64_t splits = ceil_div(target, pl.tiles);
+    splits = splits < 1 ? 1 : (splits > pl.kb_total ? pl.kb_total : splits);
+    pl.kb_per_split = static_cast<int>(ceil_div(pl.kb_total, splits));
+    pl.splits = static_cast<int>(ceil_div(pl.kb_total, pl.kb_per_split));  // no empty split
+    pl.b_bytes = b_mn ? static_cast<int>(ceil_div(pl.nt, 64)) * 8192 : pl.nt * kBK * 2;
+    const int stage = kABytes + pl.b_bytes;
+    pl.stages = (kMaxSmem - 2048) / stage;
+    pl.stages = pl.stages > 4 ? 4 : pl.stages;  // keeps two CTAs per SM for r <= 64
+    pl.smem = pl.stages * stage + 1024 + 1024;
+    uint32_t c = 32;
+    while (c < static_cast<uint32_t>(pl.nt)) c <<= 1;
+    pl.tmem_cols = c;
+    return pl;
+}
+
+size_t partial_bytes(const Plan& pl, int64_t rows) {
+    return static_cast<size_t>(pl.splits) * static_cast<size_t>(rows) * pl.nt * 4;
+}
+
+template <bool A_MN, bool B_MN>
+cudaError_t run(const Plan& pl, const CUtensorMap& ma, const CUtensorMap& mb, int64_t rows, int r, float scale,
+                float* part, uint16_t* out, bool transposed, cudaStream_t st) {
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    std::call_once(once, [] {
+        attr = cudaFuncSetAttribute(k_lora_tc<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem + 2048);
+    });
+    if (attr != cudaSuccess) return attr;
+    SkinnyParams p;
+    p.part = part;
+    p.rows = static_cast<int>(rows);
+    p.nt = pl.nt;
+    p.kb_total = pl.kb_total;
+    p.kb_per_split = pl.kb_per_split;
+    p.stages = pl.stages;
+    p.b_bytes = pl.b_bytes;
+    p.tmem_cols = pl.tmem_cols;
+    dim3 grid(static_cast<unsigned>(pl.tiles), static_cast<unsigned>(pl.splits));
+    k_lora_tc<A_MN, B_MN><<<grid, kThreads, pl.smem, st>>>(ma, mb, p);
+    note_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t total = rows * r;
+    const int64_t want = ceil_div(total, 256);
+    const int g2 = static_cast<int>(want < num_sms() * 8LL ? want : num_sms() * 8LL);
+    k_lora_reduce<<<g2, 256, 0, st>>>(part, pl.splits, static_cast<int>(rows), pl.nt, r, scale, out, transposed ? 1 : 0);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool lora_tc_supported(int64_t M, int64_t N, int64_t K, int r) {
+    return r % 8 == 0 && r >= 8 && r <= 256 && N % 8 == 0 && K % 64 == 0 && M >= 1 && M < (int64_t(1) << 31) &&
+           N < (int64_t(1) << 31) && encode_fn() != nullptr;
+}
+
+size_t lora_tc_workspace(int64_t M, int64_t N, int64_t K, int r) {
+    size_t b = partial_bytes(plan(M, K, r, false), M);                    // T
+    b = std::max(b, partial_bytes(plan(M, N, r, true), M));               // U
+    b = std::max(b, partial_bytes(plan(K, M, r, true), K));               // dA^T
+    b = std::max(b, partial_bytes(plan(N, M, r, true), N));               // dB
+    return b;
+}
+
+// T = bf16(s X A^T): A operand X (K-major), B operand A (K-major).
+cudaError_t launch_lora_xat_tc(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, float s,
+                               uint16_t* T, float* part, cudaStream_t st) {
+    const Plan pl = plan(M, K, r, false);
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, X, K, M, kBK, kRows) || !make_map(&mb, A, K, r, kBK, pl.nt)) return cudaErrorInvalidValue;
+    return run<false, false>(pl, ma, mb, M, r, s, part, T, false, st);
+}
+
+// U = bf16(s dY B): A operand dY (K-major over n), B operand B^T (MN-major).
+cudaError_t launch_lora_dyb_tc(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t N, int r, float s,
+                               uint16_t* U, float* part, cudaStream_t st) {
+    const Plan pl = plan(M, N, r, true);
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, dY, N, M, kBK, kRows) || !make_map(&mb, B, r, N, 64, kBK)) return cudaErrorInvalidValue;
+    return run<false, true>(pl, ma, mb, M, r, s, part, U, false, st);
+}
+
+// dA = bf16(U^T X) computed as dA^T[k][j] = sum_m X[m][k] U[m][j]: both MN-major.
+cudaError_t launch_lora_da_tc(const uint16_t* X, const uint16_t* U, int64_t M, int64_t K, int r, uint16_t* dA,
+                              float* part, cudaStream_t st) {
+    const Plan pl = plan(K, M, r, true);
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, X, K, M, 64, kBK) || !make_map(&mb, U, r, M, 64, kBK)) return cudaErrorInvalidValue;
+    return run<true, true>(pl, ma, mb, K, r, 1.0f, part, dA, true, st);
+}
+
+// dB = bf16(dY^T T), dB[n][j] = sum_m dY[m][n] T[m][j]: both MN-major.
+cudaError_t launch_lora_db_tc(const uint16_t* dY, const uint16_t* T, int64_t M, int64_t N, int r, uint16_t* dB,
+                              float* part, cudaStream_t st) {
+    const Plan pl = plan(N, M, r, true);
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, dY, N, M, 64, kBK) || !make_map(&mb, T, r, M, 64, kBK)) return cudaErrorInvalidValue;
+    return run<true, true>(pl, ma, mb, N, r, 1.0f, part, dB, false, st);
+}
+
+int lora_device_error(int reset) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_lora_error, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (reset && v) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_lora_error, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    }
+    return v;
+}
+
+}  // namespace qlora
