@@ -223,8 +223,8 @@ struct Plan {
 Plan plan(int64_t rows, int64_t ctr, int r, bool b_mn) {
     Plan pl;
     pl.nt = static_cast<int>(round_up(r, 16));
-    pl.kb_total = static_cast<int>(ceil_div(ctr, kBK));
-    pl.tiles = ceil_div(rows, kRows);
+    pl.kb_total = static_cast<int>(ceil_div(ctr > 0 ? ctr : 1, kBK));
+    pl.tiles = ceil_div(rows > 0 ? rows : 1, kRows);
     const int64_t target = 2LL * num_sms();
     int64_t splits = ceil_div(target, pl.tiles);
     splits = splits < 1 ? 1 : (splits > pl.kb_total ? pl.kb_total : splits);
@@ -284,6 +284,7 @@ bool lora_tc_supported(int64_t M, int64_t N, int64_t K, int r) {
 }
 
 size_t lora_tc_workspace(int64_t M, int64_t N, int64_t K, int r) {
+    if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return 0;
     size_t b = partial_bytes(plan(M, K, r, false), M);                    // T
     b = std::max(b, partial_bytes(plan(M, N, r, true), M));               // U
     b = std::max(b, partial_bytes(plan(K, M, r, true), K));               // dA^T
