@@ -34,6 +34,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -56,10 +57,12 @@ constexpr int kXStageBytes = kTileT * kBK * 2;  // 32 KiB
 constexpr int kAccCols = kTileT;                // fp32 accumulator columns
 constexpr int kAStageCols = kBK / 2;            // bf16 pairs per TMEM column
 constexpr uint32_t kTmemCols = 512;
-constexpr int kDqWarps = 8;
-constexpr int kPrefetch = 4;   // k-blocks of codes in flight per dequant thread
-constexpr int kThreads = 32 * (2 + kDqWarps);
-constexpr int kStageWords = 4 * 36 + 32;        // backward transpose staging per warp
+constexpr int kDqWarps = 16;                    // four per TMEM lane quarter
+constexpr int kParts = kDqWarps / 4;            // each takes 16 of a stage's 64 contraction values
+constexpr int kPartK = kBK / kParts;            // 16
+constexpr int kPrefetch = 4;                    // stages of codes in flight per dequant thread
+constexpr int kThreads = 32 * (2 + kDqWarps);   // 576
+constexpr int kStageWords = 4 * 20 + 16;        // backward transpose staging per warp
 constexpr uint32_t kNoRow = 0x100u;             // prefetch slot holds no weights
 constexpr int kSmemBytes = kStages * kXStageBytes + 1024 /* align */ + 1024 /* barriers etc. */ +
                            kDqWarps * kStageWords * 4;
@@ -79,6 +82,11 @@ struct GemmParams {
     float q[16];
 };
 
+__device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
     uint4 v;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -148,56 +156,91 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* er
     return __all_sync(0xffffffffu, ok);
 }
 
-// Forward operand: lane = weight row n, the 32 contraction values k of this
-// warp's half-stage come from one 16-byte run of codes and share one block
-// constant.  Element 2t (high nibble) lands in the low half of column t.
-__device__ __forceinline__ void convert_row(const uint4& cw, float sc, const float* lut, uint32_t (&v)[16]) {
-    const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+// q[code] read from the 16-entry table by a byte offset (code * 4).
+__device__ __forceinline__ float lut_at(const float* lut, uint32_t byte_off) {
+    return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(lut) + byte_off);
+}
+
+// Two weights scaled by the block constant and packed as bf16x2 (first in
+// the low half).
+__device__ __forceinline__ uint32_t scale_pack(float a, float b, float sc) {
+    const float2 x = __fmul2_rn(make_float2(a, b), make_float2(sc, sc));
+    return pack_bf16x2(x.x, x.y);
+}
+
+// Forward operand: lane = weight row n; its 16 contraction values of this
+// stage are one 8-byte run of codes under one block constant.  In each code
+// byte the high nibble is the even element, which lands in the low half of
+// its TMEM column.
+__device__ __forceinline__ void convert_row(const uint2& cw, float sc, const float* lut, uint32_t (&v)[8]) {
+    const uint32_t w2[2] = {cw.x, cw.y};
 #pragma unroll
-    for (int t = 0; t < 16; ++t) {
-        const uint32_t byte = (w4[t >> 2] >> (8 * (t & 3))) & 0xffu;
-        v[t] = pack_bf16x2(__fmul_rn(lut[byte >> 4], sc), __fmul_rn(lut[byte & 15u], sc));
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t hi4 = (w2[h] >> 2) & 0x3C3C3C3Cu;  // even-element code * 4, per byte
+        const uint32_t lo4 = (w2[h] << 2) & 0x3C3C3C3Cu;  // odd-element code * 4, per byte
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float a = lut_at(lut, __byte_perm(hi4, 0u, 0x4440u | j));
+            const float b = lut_at(lut, __byte_perm(lo4, 0u, 0x4440u | j));
+            v[4 * h + j] = scale_pack(a, b, sc);
+        }
     }
 }
 
-// Backward operand: lane = weight column k, the 32 contraction values are 32
-// weight rows n.  Lane l loads row n0 + l's 16-byte run of codes (the 32
-// columns of this warp) and its block constant; the warp then exchanges
-// them through a small shared buffer so that each lane reads the nibble of
-// its own column from every row.
+// Backward operand: lane = weight column k; its 16 contraction values are
+// 16 weight rows n.  Lanes 0..15 each load one row's 16-byte run of codes
+// (the 32 columns of this warp) and its block constant; the warp exchanges
+// them through a small shared buffer and each lane rotates its own nibble
+// out of every row's word.
 __device__ __forceinline__ void convert_cols(const uint4& cw, float sc, const float* lut, uint32_t* wsm, int lane,
-                                             uint32_t (&v)[16]) {
-    float* ssm = reinterpret_cast<float*>(wsm + 4 * 36);
-    wsm[0 * 36 + lane] = cw.x;
-    wsm[1 * 36 + lane] = cw.y;
-    wsm[2 * 36 + lane] = cw.z;
-    wsm[3 * 36 + lane] = cw.w;
-    ssm[lane] = sc;
+                                             uint32_t (&v)[8]) {
+    float* ssm = reinterpret_cast<float*>(wsm + 4 * 20);
+    if (lane < 16) {
+        wsm[0 * 20 + lane] = cw.x;
+        wsm[1 * 20 + lane] = cw.y;
+        wsm[2 * 20 + lane] = cw.z;
+        wsm[3 * 20 + lane] = cw.w;
+        ssm[lane] = sc;
+    }
     __syncwarp();
     const int wi = lane >> 3;  // the 32-bit word holding this column's nibbles
     const int shift = ((lane & 7) >> 1) * 8 + ((lane & 1) ? 0 : 4);
+    const uint32_t rot = static_cast<uint32_t>(shift + 30) & 31u;  // nibble -> bits [2, 6)
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-        const uint4 c4 = *reinterpret_cast<const uint4*>(wsm + wi * 36 + 4 * g);
+    for (int g = 0; g < 4; ++g) {
+        const uint4 c4 = *reinterpret_cast<const uint4*>(wsm + wi * 20 + 4 * g);
         const float4 s4 = *reinterpret_cast<const float4*>(ssm + 4 * g);
-        const float x0 = __fmul_rn(lut[(c4.x >> shift) & 15u], s4.x);
-        const float x1 = __fmul_rn(lut[(c4.y >> shift) & 15u], s4.y);
-        const float x2 = __fmul_rn(lut[(c4.z >> shift) & 15u], s4.z);
-        const float x3 = __fmul_rn(lut[(c4.w >> shift) & 15u], s4.w);
-        v[2 * g] = pack_bf16x2(x0, x1);
-        v[2 * g + 1] = pack_bf16x2(x2, x3);
+        const float x0 = lut_at(lut, __funnelshift_r(c4.x, c4.x, rot) & 0x3Cu);
+        const float x1 = lut_at(lut, __funnelshift_r(c4.y, c4.y, rot) & 0x3Cu);
+        const float x2 = lut_at(lut, __funnelshift_r(c4.z, c4.z, rot) & 0x3Cu);
+        const float x3 = lut_at(lut, __funnelshift_r(c4.w, c4.w, rot) & 0x3Cu);
+        const float2 y01 = __fmul2_rn(make_float2(x0, x1), make_float2(s4.x, s4.y));
+        const float2 y23 = __fmul2_rn(make_float2(x2, x3), make_float2(s4.z, s4.w));
+        v[2 * g] = pack_bf16x2(y01.x, y01.y);
+        v[2 * g + 1] = pack_bf16x2(y23.x, y23.y);
     }
     __syncwarp();
 }
 
-// warps 2..9: dequantize the weight tile into TMEM stage by stage, then
+__device__ __forceinline__ void load_codes(uint2& c, const uint8_t* p) { c = ldg_nc_v2(p); }
+__device__ __forceinline__ void load_codes(uint4& c, const uint8_t* p) { c = ldg_nc_v4(p); }
+__device__ __forceinline__ void convert(const uint2& cw, float sc, const float* lut, uint32_t*, int,
+                                        uint32_t (&v)[8]) {
+    convert_row(cw, sc, lut, v);
+}
+__device__ __forceinline__ void convert(const uint4& cw, float sc, const float* lut, uint32_t* wsm, int lane,
+                                        uint32_t (&v)[8]) {
+    convert_cols(cw, sc, lut, wsm, lane, v);
+}
+
+// warps 2..17: dequantize the weight tile into TMEM stage by stage, then
 // write this tile's outputs.
 template <bool kBwd>
-__device__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const float* lut, uint32_t* wsm,
-                                      int warp, int lane, int* err) {
+__device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const float* lut,
+                                                      uint32_t* wsm, int warp, int lane, int* err) {
     const int dq = warp - 2;
     const int quarter = warp & 3;  // the TMEM lanes this warp may touch
-    const int half = dq >> 2;      // 32-wide half of each 64-wide stage
+    const int part = dq >> 2;      // 16-wide part of each 64-wide stage
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float mu = *p.mean;
@@ -211,25 +254,26 @@ __device__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const 
         const bool warp_cols_ok = wcol0 < p.rows;
 
         // codes, FP8 constant and c1 of the next kPrefetch stages in flight
-        uint4 cbuf[kPrefetch];
+        using Codes = typename std::conditional<kBwd, uint4, uint2>::type;
+        Codes cbuf[kPrefetch];
         uint32_t sbuf[kPrefetch];
         float c1buf[kPrefetch];
         auto issue = [&](int kb, int slot) {
-            cbuf[slot] = make_uint4(0u, 0u, 0u, 0u);
+            cbuf[slot] = Codes{};
             sbuf[slot] = kNoRow;  // no weights here: the block constant reads as 0
             c1buf[slot] = 0.0f;
             if (kb >= P.kb_w) return;
-            int64_t e0;  // flat index of the first weight of this lane's 16-byte code run
+            int64_t e0;  // flat index of the first weight of this lane's run of codes
             if (kBwd) {
-                const int n = kb * kBK + half * 32 + lane;
-                if (!warp_cols_ok || n >= p.N) return;
+                const int n = kb * kBK + part * kPartK + lane;
+                if (lane >= kPartK || !warp_cols_ok || n >= p.N) return;
                 e0 = static_cast<int64_t>(n) * p.K + wcol0;
             } else {
                 if (!lane_ok) return;
-                e0 = static_cast<int64_t>(grow) * p.K + kb * kBK + half * 32;
+                e0 = static_cast<int64_t>(grow) * p.K + kb * kBK + part * kPartK;
             }
+            load_codes(cbuf[slot], p.codes + (e0 >> 1));
             const int64_t blk = e0 >> 6;
-            cbuf[slot] = ldg_nc_v4(p.codes + (e0 >> 1));
             sbuf[slot] = __ldg(p.c2_fp8 + blk);
             c1buf[slot] = __ldg(p.c1 + (blk >> 8));
         };
@@ -240,23 +284,16 @@ __device__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const 
             for (int u = 0; u < kPrefetch; ++u) {
                 const int kb = kb0 + u;
                 if (kb >= P.kb_total) break;
-                uint32_t v[16];
+                uint32_t v[8];
                 if (kb < P.kb_w) {
                     const float sc =
                         sbuf[u] == kNoRow ? 0.0f : dq_constant(static_cast<uint8_t>(sbuf[u]), c1buf[u], mu);
-                    if (kBwd)
-                        convert_cols(cbuf[u], sc, lut, wsm, lane, v);
-                    else
-                        convert_row(cbuf[u], sc, lut, v);
-                    if (!kBwd && !lane_ok) {
-#pragma unroll
-                        for (int t = 0; t < 16; ++t) v[t] = 0u;
-                    }
+                    convert(cbuf[u], sc, lut, wsm, lane, v);
                 } else {
-                    const int j0 = (kb - P.kb_w) * kBK + half * 32;
+                    const int j0 = (kb - P.kb_w) * kBK + part * kPartK;
                     if (kBwd) {  // A^T: lane = column k of A (r x K)
 #pragma unroll
-                        for (int t = 0; t < 16; ++t) {
+                        for (int t = 0; t < 8; ++t) {
                             const int j = j0 + 2 * t;
                             const uint32_t a = (lane_ok && j < p.r) ? p.lora[static_cast<int64_t>(j) * p.K + grow] : 0u;
                             const uint32_t b =
@@ -266,7 +303,7 @@ __device__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const 
                     } else {  // B: lane = row n of B (N x r)
                         const uint16_t* brow = p.lora + static_cast<int64_t>(grow) * p.r + j0;
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
+                        for (int c = 0; c < 2; ++c) {
                             uint4 w = make_uint4(0u, 0u, 0u, 0u);
                             if (lane_ok && j0 + 8 * c < p.r) w = *reinterpret_cast<const uint4*>(brow + 8 * c);
                             v[4 * c + 0] = w.x;
@@ -276,26 +313,30 @@ __device__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const 
                         }
                     }
                 }
+                if (!kBwd && !lane_ok) {
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) v[t] = 0u;
+                }
                 issue(kb + kPrefetch, u);
                 const int s = static_cast<int>(it % kStages);
                 const uint32_t ph = (it / kStages) & 1u;
                 ++it;
                 if (!warp_wait(P.empty(s), ph ^ 1u, err)) return;
-                tmem_st_32x32b_x16(P.tmem + lane_base + kAccCols + s * kAStageCols + half * 16, v);
+                tmem_st_32x32b_x8(P.tmem + lane_base + kAccCols + s * kAStageCols + part * (kPartK / 2), v);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(P.full_a(s));
             }
         }
-        // epilogue: this warp's lane quarter, columns [128 half, 128 half + 128)
+        // epilogue: this warp's lane quarter, columns [64 part, 64 part + 64)
         if (!warp_wait(P.acc_full(), tcount & 1u, err)) return;
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-            const int col = half * 128 + c * 32;
-            uint32_t acc[32];
-            tmem_ld_32x32b_x32(P.tmem + lane_base + col, acc);
+            const int col = part * 64 + c * 16;
+            uint32_t acc[16];
+            tmem_ld_32x32b_x16(P.tmem + lane_base + col, acc);
             tmem_wait_ld();
             if (c == 3) {
                 tc_fence_before();
@@ -303,12 +344,10 @@ __device__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const 
                 if (lane == 0) mbar_arrive(P.acc_empty());
             }
             if (lane_ok) {
+                uint16_t* o = p.out + static_cast<int64_t>(t0 + col) * p.rows + grow;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int m = t0 + col + j;
-                    if (m < p.M)
-                        p.out[static_cast<int64_t>(m) * p.rows + grow] = f32_to_bf16_bits(__uint_as_float(acc[j]));
-                }
+                for (int j = 0; j < 16; ++j)
+                    if (t0 + col + j < p.M) o[static_cast<int64_t>(j) * p.rows] = f32_to_bf16_bits(__uint_as_float(acc[j]));
             }
         }
     }
@@ -319,10 +358,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_lora,
               const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
+    __shared__ float s_lut[16];  // static, so table reads use an immediate address
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kXStageBytes);
-    float* lut = reinterpret_cast<float*>(bars + 3 * kStages + 2);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lut + 16);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 2);
     uint32_t* stage_words = reinterpret_cast<uint32_t*>(smem + kStages * kXStageBytes + 1024);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -339,7 +378,7 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
         mbar_init(P.acc_empty(), kDqWarps);
         fence_barrier_init();
     }
-    if (threadIdx.x < 16) lut[threadIdx.x] = p.q[threadIdx.x];
+    if (threadIdx.x < 16) s_lut[threadIdx.x] = p.q[threadIdx.x];
     if (warp == 0) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
@@ -365,7 +404,7 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
         if (lane == 0) role_mma(P, err);
         __syncwarp();
     } else {
-        role_dequant_epilogue<kBwd>(P, p, lut, stage_words + (warp - 2) * kStageWords, warp, lane, err);
+        role_dequant_epilogue<kBwd>(P, p, s_lut, stage_words + (warp - 2) * kStageWords, warp, lane, err);
     }
     tc_fence_before();
     __syncthreads();
