@@ -58,11 +58,13 @@ constexpr int kAccCols = kTileT;                // fp32 accumulator columns
 constexpr int kAStageCols = kBK / 2;            // bf16 pairs per TMEM column
 constexpr uint32_t kTmemCols = 512;
 constexpr int kDqWarps = 16;                    // four per TMEM lane quarter
-constexpr int kParts = kDqWarps / 4;            // each takes 16 of a stage's 64 contraction values
-constexpr int kPartK = kBK / kParts;            // 16
-constexpr int kPrefetch = 4;                    // stages of codes in flight per dequant thread
+constexpr int kParts = kDqWarps / 4;            // stage kb is converted by the warps with part == kb % 4
+template <bool kBwd>
+struct Prefetch {  // own stages of codes in flight per dequant thread
+    static constexpr int value = kBwd ? 1 : 2;
+};
 constexpr int kThreads = 32 * (2 + kDqWarps);   // 576
-constexpr int kStageWords = 4 * 20 + 16;        // backward transpose staging per warp
+constexpr int kStageWords = 4 * 68 + 64;        // backward transpose staging per warp (64 rows)
 constexpr uint32_t kNoRow = 0x100u;             // prefetch slot holds no weights
 constexpr int kSmemBytes = kStages * kXStageBytes + 1024 /* align */ + 1024 /* barriers etc. */ +
                            kDqWarps * kStageWords * 4;
@@ -150,10 +152,15 @@ __device__ void role_mma(const Pipe& P, int* err) {
     }
 }
 
-// All lanes of the calling warp wait; the warp gives up together.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* err) {
-    const bool ok = mbar_wait(bar, parity, err);
-    return __all_sync(0xffffffffu, ok);
+// Lane 0 of the calling warp waits; the result is broadcast so the warp
+// proceeds (or gives up) together.  __syncwarp orders the other lanes
+// after the observed phase.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* err, int lane) {
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(bar, parity, err) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
 }
 
 // q[code] read from the 16-entry table by a byte offset (code * 4).
@@ -161,23 +168,32 @@ __device__ __forceinline__ float lut_at(const float* lut, uint32_t byte_off) {
     return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(lut) + byte_off);
 }
 
-// Two weights scaled by the block constant and packed as bf16x2 (first in
-// the low half).
 __device__ __forceinline__ uint32_t scale_pack(float a, float b, float sc) {
     const float2 x = __fmul2_rn(make_float2(a, b), make_float2(sc, sc));
     return pack_bf16x2(x.x, x.y);
 }
 
-// Forward operand: lane = weight row n; its 16 contraction values of this
-// stage are one 8-byte run of codes under one block constant.  In each code
-// byte the high nibble is the even element, which lands in the low half of
-// its TMEM column.
-__device__ __forceinline__ void convert_row(const uint2& cw, float sc, const float* lut, uint32_t (&v)[8]) {
-    const uint32_t w2[2] = {cw.x, cw.y};
+// Per-lane, per-stage inputs of the dequantization, loaded kPrefetch
+// stages ahead.  Forward: the lane's weight row, 64 consecutive codes (32
+// bytes, one sector) under one block constant.  Backward: weight rows
+// n0 + lane and n0 + 32 + lane, the 32 columns of this warp (16 bytes
+// each), each row with its own block constant.
+struct StageIn {
+    uint4 c0, c1v;      // forward: codes bytes 0..15, 16..31; backward: row lane, row 32+lane
+    uint32_t b0, b1;    // FP8 constant byte(s) (kNoRow: no weights)
+    float s0, s1;       // c1 of the block(s)
+};
+
+// Forward: 32 TMEM columns = 64 contraction values of one row.  In each
+// code byte the high nibble is the even element, which lands in the low
+// half of its column.
+__device__ __forceinline__ void convert_row(const StageIn& in, float mu, const float* lut, uint32_t (&v)[32]) {
+    const float sc = in.b0 == kNoRow ? 0.0f : dq_constant(static_cast<uint8_t>(in.b0), in.s0, mu);
+    const uint32_t w8[8] = {in.c0.x, in.c0.y, in.c0.z, in.c0.w, in.c1v.x, in.c1v.y, in.c1v.z, in.c1v.w};
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const uint32_t hi4 = (w2[h] >> 2) & 0x3C3C3C3Cu;  // even-element code * 4, per byte
-        const uint32_t lo4 = (w2[h] << 2) & 0x3C3C3C3Cu;  // odd-element code * 4, per byte
+    for (int h = 0; h < 8; ++h) {
+        const uint32_t hi4 = (w8[h] >> 2) & 0x3C3C3C3Cu;  // even-element code * 4, per byte
+        const uint32_t lo4 = (w8[h] << 2) & 0x3C3C3C3Cu;  // odd-element code * 4, per byte
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const float a = lut_at(lut, __byte_perm(hi4, 0u, 0x4440u | j));
@@ -187,28 +203,31 @@ __device__ __forceinline__ void convert_row(const uint2& cw, float sc, const flo
     }
 }
 
-// Backward operand: lane = weight column k; its 16 contraction values are
-// 16 weight rows n.  Lanes 0..15 each load one row's 16-byte run of codes
-// (the 32 columns of this warp) and its block constant; the warp exchanges
-// them through a small shared buffer and each lane rotates its own nibble
-// out of every row's word.
-__device__ __forceinline__ void convert_cols(const uint4& cw, float sc, const float* lut, uint32_t* wsm, int lane,
-                                             uint32_t (&v)[8]) {
-    float* ssm = reinterpret_cast<float*>(wsm + 4 * 20);
-    if (lane < 16) {
-        wsm[0 * 20 + lane] = cw.x;
-        wsm[1 * 20 + lane] = cw.y;
-        wsm[2 * 20 + lane] = cw.z;
-        wsm[3 * 20 + lane] = cw.w;
-        ssm[lane] = sc;
-    }
+// Backward: lane = weight column k; its 64 contraction values are 64 weight
+// rows n.  The warp exchanges the rows' code words and constants through a
+// small shared buffer; each lane rotates its own nibble out of each word.
+__device__ __forceinline__ void convert_cols(const StageIn& in, float mu, const float* lut, uint32_t* wsm,
+                                             int lane, uint32_t (&v)[32]) {
+    float* ssm = reinterpret_cast<float*>(wsm + 4 * 68);
+    const float sc0 = in.b0 == kNoRow ? 0.0f : dq_constant(static_cast<uint8_t>(in.b0), in.s0, mu);
+    const float sc1 = in.b1 == kNoRow ? 0.0f : dq_constant(static_cast<uint8_t>(in.b1), in.s1, mu);
+    wsm[0 * 68 + lane] = in.c0.x;
+    wsm[1 * 68 + lane] = in.c0.y;
+    wsm[2 * 68 + lane] = in.c0.z;
+    wsm[3 * 68 + lane] = in.c0.w;
+    wsm[0 * 68 + 32 + lane] = in.c1v.x;
+    wsm[1 * 68 + 32 + lane] = in.c1v.y;
+    wsm[2 * 68 + 32 + lane] = in.c1v.z;
+    wsm[3 * 68 + 32 + lane] = in.c1v.w;
+    ssm[lane] = sc0;
+    ssm[32 + lane] = sc1;
     __syncwarp();
     const int wi = lane >> 3;  // the 32-bit word holding this column's nibbles
     const int shift = ((lane & 7) >> 1) * 8 + ((lane & 1) ? 0 : 4);
     const uint32_t rot = static_cast<uint32_t>(shift + 30) & 31u;  // nibble -> bits [2, 6)
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-        const uint4 c4 = *reinterpret_cast<const uint4*>(wsm + wi * 20 + 4 * g);
+    for (int g = 0; g < 16; ++g) {
+        const uint4 c4 = *reinterpret_cast<const uint4*>(wsm + wi * 68 + 4 * g);
         const float4 s4 = *reinterpret_cast<const float4*>(ssm + 4 * g);
         const float x0 = lut_at(lut, __funnelshift_r(c4.x, c4.x, rot) & 0x3Cu);
         const float x1 = lut_at(lut, __funnelshift_r(c4.y, c4.y, rot) & 0x3Cu);
@@ -222,29 +241,19 @@ __device__ __forceinline__ void convert_cols(const uint4& cw, float sc, const fl
     __syncwarp();
 }
 
-__device__ __forceinline__ void load_codes(uint2& c, const uint8_t* p) { c = ldg_nc_v2(p); }
-__device__ __forceinline__ void load_codes(uint4& c, const uint8_t* p) { c = ldg_nc_v4(p); }
-__device__ __forceinline__ void convert(const uint2& cw, float sc, const float* lut, uint32_t*, int,
-                                        uint32_t (&v)[8]) {
-    convert_row(cw, sc, lut, v);
-}
-__device__ __forceinline__ void convert(const uint4& cw, float sc, const float* lut, uint32_t* wsm, int lane,
-                                        uint32_t (&v)[8]) {
-    convert_cols(cw, sc, lut, wsm, lane, v);
-}
-
-// warps 2..17: dequantize the weight tile into TMEM stage by stage, then
-// write this tile's outputs.
+// warps 2..17: each converts every fourth stage of the weight tile into
+// TMEM (quarter = its TMEM lanes, part = which stages), then writes a
+// quarter of this tile's outputs.
 template <bool kBwd>
 __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const float* lut,
                                                       uint32_t* wsm, int warp, int lane, int* err) {
     const int dq = warp - 2;
     const int quarter = warp & 3;  // the TMEM lanes this warp may touch
-    const int part = dq >> 2;      // 16-wide part of each 64-wide stage
+    const int part = dq >> 2;      // converts the stages kb with kb % 4 == part
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float mu = *p.mean;
-    uint32_t it = 0, tcount = 0;
+    uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x, ++tcount) {
         const int t0 = (tile % P.num_t) * kTileT;
         const int row0 = (tile / P.num_t) * kTileW;
@@ -252,58 +261,70 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
         const bool lane_ok = grow < p.rows;
         const int wcol0 = row0 + quarter * 32;   // backward: first weight column of this warp
         const bool warp_cols_ok = wcol0 < p.rows;
+        const uint32_t g0 = tcount * static_cast<uint32_t>(P.kb_total);  // ring index of stage 0
 
-        // codes, FP8 constant and c1 of the next kPrefetch stages in flight
-        using Codes = typename std::conditional<kBwd, uint4, uint2>::type;
-        Codes cbuf[kPrefetch];
-        uint32_t sbuf[kPrefetch];
-        float c1buf[kPrefetch];
-        auto issue = [&](int kb, int slot) {
-            cbuf[slot] = Codes{};
-            sbuf[slot] = kNoRow;  // no weights here: the block constant reads as 0
-            c1buf[slot] = 0.0f;
+        constexpr int kPrefetch = Prefetch<kBwd>::value;
+        StageIn buf[kPrefetch];
+        auto issue = [&](int kb, StageIn& in) {
+            in.c0 = make_uint4(0u, 0u, 0u, 0u);
+            in.c1v = make_uint4(0u, 0u, 0u, 0u);
+            in.b0 = kNoRow;
+            in.b1 = kNoRow;
+            in.s0 = in.s1 = 0.0f;
             if (kb >= P.kb_w) return;
-            int64_t e0;  // flat index of the first weight of this lane's run of codes
             if (kBwd) {
-                const int n = kb * kBK + part * kPartK + lane;
-                if (lane >= kPartK || !warp_cols_ok || n >= p.N) return;
-                e0 = static_cast<int64_t>(n) * p.K + wcol0;
+                if (!warp_cols_ok) return;
+                const int n0 = kb * kBK + lane;
+                if (n0 < p.N) {
+                    const int64_t e = static_cast<int64_t>(n0) * p.K + wcol0;
+                    in.c0 = ldg_nc_v4(p.codes + (e >> 1));
+                    in.b0 = __ldg(p.c2_fp8 + (e >> 6));
+                    in.s0 = __ldg(p.c1 + (e >> 14));
+                }
+                if (n0 + 32 < p.N) {
+                    const int64_t e = static_cast<int64_t>(n0 + 32) * p.K + wcol0;
+                    in.c1v = ldg_nc_v4(p.codes + (e >> 1));
+                    in.b1 = __ldg(p.c2_fp8 + (e >> 6));
+                    in.s1 = __ldg(p.c1 + (e >> 14));
+                }
             } else {
                 if (!lane_ok) return;
-                e0 = static_cast<int64_t>(grow) * p.K + kb * kBK + part * kPartK;
+                const int64_t e = static_cast<int64_t>(grow) * p.K + kb * kBK;
+                in.c0 = ldg_nc_v4(p.codes + (e >> 1));
+                in.c1v = ldg_nc_v4(p.codes + (e >> 1) + 16);
+                in.b0 = __ldg(p.c2_fp8 + (e >> 6));
+                in.s0 = __ldg(p.c1 + (e >> 14));
             }
-            load_codes(cbuf[slot], p.codes + (e0 >> 1));
-            const int64_t blk = e0 >> 6;
-            sbuf[slot] = __ldg(p.c2_fp8 + blk);
-            c1buf[slot] = __ldg(p.c1 + (blk >> 8));
         };
 #pragma unroll
-        for (int u = 0; u < kPrefetch; ++u) issue(u, u);
-        for (int kb0 = 0; kb0 < P.kb_total; kb0 += kPrefetch) {
+        for (int u = 0; u < kPrefetch; ++u) issue(part + kParts * u, buf[u]);
+        for (int i0 = 0; part + kParts * i0 < P.kb_total; i0 += kPrefetch) {
 #pragma unroll
             for (int u = 0; u < kPrefetch; ++u) {
-                const int kb = kb0 + u;
+                const int kb = part + kParts * (i0 + u);
                 if (kb >= P.kb_total) break;
-                uint32_t v[8];
+                uint32_t v[32];
                 if (kb < P.kb_w) {
-                    const float sc =
-                        sbuf[u] == kNoRow ? 0.0f : dq_constant(static_cast<uint8_t>(sbuf[u]), c1buf[u], mu);
-                    convert(cbuf[u], sc, lut, wsm, lane, v);
+                    if (kBwd)
+                        convert_cols(buf[u], mu, lut, wsm, lane, v);
+                    else
+                        convert_row(buf[u], mu, lut, v);
                 } else {
-                    const int j0 = (kb - P.kb_w) * kBK + part * kPartK;
-                    if (kBwd) {  // A^T: lane = column k of A (r x K)
+                    const int j0 = (kb - P.kb_w) * kBK;
+                    if (kBwd) {  // A^T: lane = column k of A (r x K), in groups of 16 loads
 #pragma unroll
-                        for (int t = 0; t < 8; ++t) {
+                        for (int t = 0; t < 32; ++t) {
                             const int j = j0 + 2 * t;
                             const uint32_t a = (lane_ok && j < p.r) ? p.lora[static_cast<int64_t>(j) * p.K + grow] : 0u;
                             const uint32_t b =
                                 (lane_ok && j + 1 < p.r) ? p.lora[static_cast<int64_t>(j + 1) * p.K + grow] : 0u;
                             v[t] = a | (b << 16);
+                            if ((t & 7) == 7) asm volatile("" ::: "memory");  // bound loads in flight
                         }
                     } else {  // B: lane = row n of B (N x r)
                         const uint16_t* brow = p.lora + static_cast<int64_t>(grow) * p.r + j0;
 #pragma unroll
-                        for (int c = 0; c < 2; ++c) {
+                        for (int c = 0; c < 8; ++c) {
                             uint4 w = make_uint4(0u, 0u, 0u, 0u);
                             if (lane_ok && j0 + 8 * c < p.r) w = *reinterpret_cast<const uint4*>(brow + 8 * c);
                             v[4 * c + 0] = w.x;
@@ -315,14 +336,14 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
                 }
                 if (!kBwd && !lane_ok) {
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) v[t] = 0u;
+                    for (int t = 0; t < 32; ++t) v[t] = 0u;
                 }
-                issue(kb + kPrefetch, u);
-                const int s = static_cast<int>(it % kStages);
-                const uint32_t ph = (it / kStages) & 1u;
-                ++it;
-                if (!warp_wait(P.empty(s), ph ^ 1u, err)) return;
-                tmem_st_32x32b_x8(P.tmem + lane_base + kAccCols + s * kAStageCols + part * (kPartK / 2), v);
+                issue(kb + kParts * kPrefetch, buf[u]);
+                const uint32_t g = g0 + static_cast<uint32_t>(kb);
+                const int s = static_cast<int>(g % kStages);
+                const uint32_t ph = (g / kStages) & 1u;
+                if (!warp_wait(P.empty(s), ph ^ 1u, err, lane)) return;
+                tmem_st_32x32b_x32(P.tmem + lane_base + kAccCols + s * kAStageCols, v);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -330,7 +351,7 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
             }
         }
         // epilogue: this warp's lane quarter, columns [64 part, 64 part + 64)
-        if (!warp_wait(P.acc_full(), tcount & 1u, err)) return;
+        if (!warp_wait(P.acc_full(), tcount & 1u, err, lane)) return;
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -371,7 +392,7 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(P.full_b(s), 1);
-            mbar_init(P.full_a(s), kDqWarps);
+            mbar_init(P.full_a(s), 4);  // one converting warp per TMEM lane quarter
             mbar_init(P.empty(s), 1);
         }
         mbar_init(P.acc_full(), 1);
