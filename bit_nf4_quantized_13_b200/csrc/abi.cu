@@ -35,8 +35,8 @@ cudaError_t launch_fwd_gemm(const uint16_t* X, const Nf4Weight& w, const uint16_
 }
 
 cudaError_t launch_bwd_dx_gemm(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U,
-                               const uint16_t* A, int64_t M, int r, uint16_t* dX, cudaStream_t st) {
-    if (dx_tc_supported(M, w, r)) return launch_bwd_dx_gemm_tc(dY, w, U, A, M, r, dX, st);
+                               const uint16_t* A, int64_t M, int r, uint16_t* dX, void* ws, cudaStream_t st) {
+    if (dx_tc_supported(M, w, r)) return launch_bwd_dx_gemm_tc(dY, w, U, A, M, r, dX, ws, st);
     return launch_bwd_dx_gemm_simt(dY, w, U, A, M, r, dX, st);
 }
 
@@ -133,7 +133,9 @@ size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
 size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
     if (check_linear(M, N, K, r) != QLORA_OK) return 0;
     const size_t mr = align256(static_cast<size_t>(M) * r * 2);
-    return 2 * mr + align256(lora_tc_workspace(M, N, K, r));  // U, T (when T is NULL), partials
+    // U, T (when T is NULL), the rank-r partials, the transposed weight of the dX GEMM
+    Nf4Weight w{nullptr, nullptr, nullptr, nullptr, N, K};
+    return 2 * mr + align256(lora_tc_workspace(M, N, K, r)) + align256(dx_tc_workspace(w, r));
 }
 
 int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
@@ -181,13 +183,14 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N
     uint16_t* Tw = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + mr);
     float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 2 * mr);
     Nf4Weight w{codes, c2_fp8, c1, mean, N, K};
+    void* dxws = reinterpret_cast<char*>(ws) + 2 * mr + align256(lora_tc_workspace(M, N, K, r));
     cudaError_t e = cudaSuccess;
     if (!T) {
         e = lora_xat(X, A, M, N, K, r, s, Tw, part, cs);
         T = Tw;
     }
     if (e == cudaSuccess) e = lora_dyb(dY, B, M, N, K, r, s, U, part, cs);
-    if (e == cudaSuccess && dX) e = launch_bwd_dx_gemm(dY, w, U, A, M, r, dX, cs);
+    if (e == cudaSuccess && dX) e = launch_bwd_dx_gemm(dY, w, U, A, M, r, dX, dxws, cs);
     if (e == cudaSuccess) e = lora_grads(dY, X, T, U, M, N, K, r, dA, dB, part, cs);
     return cuda_status(e);
 }

@@ -10,8 +10,8 @@
 // Both compute the transposed product tile by tile with the weight as the
 // MMA's A operand held in tensor memory:
 //
-//   forward:  D[n][m]     += W'[n][k]     * X[m][k]     (contract over k)
-//   backward: D[k][m]     += W'[n][k]     * dY[m][n]    (contract over n)
+//   forward:  D[n][m] += W'[n][k]   * X[m][k]     (contract over k)
+//   backward: D[k][m] += W'^T[k][n] * dY[m][n]    (contract over n)
 //
 // so a dequantized tile goes from registers straight into tensor memory
 // (tcgen05.st) and costs no shared-memory bandwidth; only the activation
@@ -20,21 +20,27 @@
 // continued over ceil(r/64) extra 64-wide slabs whose A operand is B (or
 // A^T) copied into tensor memory and whose B operand is T (or U) by TMA.
 //
+// The backward reads the weight through a transposed copy made per call by
+// k_prep_bwd: codes of W^T (two consecutive n per byte), the block
+// constants c2' in fp32 laid out [k/64][n], and A^T.  A lane then owns one
+// weight column k and converts 64 consecutive contraction values from one
+// 32-byte run of codes, exactly like the forward owns a row n; the
+// constants of a stage (2 x 64 floats) arrive by TMA with the dY tile.
+//
 // Tile: 128 weight rows (n forward, k backward) x 256 tokens x 64; fp32
-// accumulator in 256 TMEM columns; 6 pipeline stages.  Warp roles (320
+// accumulator in 256 TMEM columns; 6 pipeline stages.  Warp roles (576
 // threads, persistent over tiles, one CTA per SM):
-//   warp 0       TMA producer for the activation tiles
-//   warp 1       MMA issuer (one thread)
-//   warps 2..9   dequant producers (each a TMEM lane quarter and a 32-wide
-//                half of every 64-wide stage), then the epilogue of the
-//                same tile: tcgen05.ld, bf16, stores coalesced along the
-//                weight-row index
+//   warp 0        TMA producer for the activation tiles (and constants)
+//   warp 1        MMA issuer (one thread)
+//   warps 2..17   dequant producers: warp w converts the stages kb with
+//                 kb % 4 == (w - 2) / 4 for the TMEM lane quarter w % 4, then
+//                 the epilogue of the tile: tcgen05.ld, bf16, stores
+//                 coalesced along the weight-row index
 // Every wait is bounded; a timeout records QLORA_ERR_TIMEOUT in a sticky
 // device word (qlora_device_error) and ends the kernel.
 #include <cudaTypedefs.h>
 
 #include <mutex>
-#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -54,41 +60,33 @@ constexpr int kTileT = 256;   // tokens per tile (MMA N)
 constexpr int kBK = 64;       // contraction per stage
 constexpr int kStages = 6;
 constexpr int kXStageBytes = kTileT * kBK * 2;  // 32 KiB
+constexpr int kScaleStageBytes = 2 * kBK * 4;   // backward: c2' of 2 column groups x 64 rows
 constexpr int kAccCols = kTileT;                // fp32 accumulator columns
 constexpr int kAStageCols = kBK / 2;            // bf16 pairs per TMEM column
 constexpr uint32_t kTmemCols = 512;
 constexpr int kDqWarps = 16;                    // four per TMEM lane quarter
 constexpr int kParts = kDqWarps / 4;            // stage kb is converted by the warps with part == kb % 4
-template <bool kBwd>
-struct Prefetch {  // own stages of codes in flight per dequant thread
-    static constexpr int value = kBwd ? 1 : 2;
-};
+constexpr int kPrefetch = 2;                    // own stages of codes in flight per dequant thread
 constexpr int kThreads = 32 * (2 + kDqWarps);   // 576
-constexpr int kStageWords = 4 * 68 + 64;        // backward transpose staging per warp (64 rows)
-constexpr uint32_t kNoRow = 0x100u;             // prefetch slot holds no weights
 constexpr int kSmemBytes = kStages * kXStageBytes + 1024 /* align */ + 1024 /* barriers etc. */ +
-                           kDqWarps * kStageWords * 4;
+                           kStages * kScaleStageBytes;
 static_assert(kAccCols + kStages * kAStageCols <= static_cast<int>(kTmemCols), "TMEM budget");
 
 struct GemmParams {
-    const uint8_t* codes;
-    const uint8_t* c2_fp8;
-    const float* c1;
-    const float* mean;
-    const uint16_t* lora;  // forward: B (N x r); backward: A (r x K)
+    const uint8_t* codes;  // forward: W codes (N x K/2); backward: W^T codes (K x ldT)
+    const uint8_t* c2_fp8; // forward only
+    const float* c1;       // forward only
+    const float* mean;     // forward only
+    const uint16_t* lora;  // forward: B (N x r); backward: A^T (K x r)
     uint16_t* out;         // forward: Y (M x N); backward: dX (M x K)
+    int64_t ld_codes;      // bytes per weight row of `codes`
     int M;                 // tokens
     int rows;              // weight rows of the product: N forward, K backward
     int ctr;               // contraction over the weight: K forward, N backward
-    int N, K, r;
+    int K, r;
     float q[16];
 };
 
-__device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
-    uint2 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-    return v;
-}
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
     uint4 v;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -99,6 +97,7 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
 
 struct Pipe {
     uint8_t* sA;       // kStages x 32 KiB of activation tiles
+    float* sS;         // backward: kStages x [2][64] block constants
     uint32_t bar0;     // full_b[S], full_a[S], empty[S], acc_full, acc_empty
     uint32_t tmem;     // accumulator at columns [0, 256), A stages after it
     int num_t, num_tiles, kb_w, kb_total;
@@ -109,21 +108,30 @@ struct Pipe {
     __device__ uint32_t acc_empty() const { return bar0 + 8u * (3 * kStages + 1); }
 };
 
-// warp 0, one thread: activation tiles, then the LoRA slabs, into the ring.
-__device__ void role_tma(const Pipe& P, const CUtensorMap* tmap_act, const CUtensorMap* tmap_lora, int* err) {
+// warp 0, one thread: activation tiles (backward: with the stage's block
+// constants), then the LoRA slabs, into the ring.
+template <bool kBwd>
+__device__ void role_tma(const Pipe& P, const CUtensorMap* tmap_act, const CUtensorMap* tmap_lora,
+                         const CUtensorMap* tmap_scale, int* err) {
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x) {
         const int t0 = (tile % P.num_t) * kTileT;
+        const int row0 = (tile / P.num_t) * kTileW;
         for (int kb = 0; kb < P.kb_total; ++kb, ++it) {
             const int s = static_cast<int>(it % kStages);
             const uint32_t ph = (it / kStages) & 1u;
             if (!mbar_wait(P.empty(s), ph ^ 1u, err)) return;
-            mbar_arrive_expect_tx(P.full_b(s), kXStageBytes);
             const uint32_t dst = smem_u32(P.sA + s * kXStageBytes);
-            if (kb < P.kb_w)
+            if (kb < P.kb_w) {
+                mbar_arrive_expect_tx(P.full_b(s), kXStageBytes + (kBwd ? kScaleStageBytes : 0));
                 tma_load_2d(dst, tmap_act, P.full_b(s), kb * kBK, t0);
-            else
+                if (kBwd)
+                    tma_load_2d(smem_u32(P.sS + s * (kScaleStageBytes / 4)), tmap_scale, P.full_b(s), kb * kBK,
+                                row0 / kBK);
+            } else {
+                mbar_arrive_expect_tx(P.full_b(s), kXStageBytes);
                 tma_load_2d(dst, tmap_lora, P.full_b(s), (kb - P.kb_w) * kBK, t0);
+            }
         }
     }
 }
@@ -168,77 +176,36 @@ __device__ __forceinline__ float lut_at(const float* lut, uint32_t byte_off) {
     return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(lut) + byte_off);
 }
 
-__device__ __forceinline__ uint32_t scale_pack(float a, float b, float sc) {
-    const float2 x = __fmul2_rn(make_float2(a, b), make_float2(sc, sc));
-    return pack_bf16x2(x.x, x.y);
-}
-
-// Per-lane, per-stage inputs of the dequantization, loaded kPrefetch
-// stages ahead.  Forward: the lane's weight row, 64 consecutive codes (32
-// bytes, one sector) under one block constant.  Backward: weight rows
-// n0 + lane and n0 + 32 + lane, the 32 columns of this warp (16 bytes
-// each), each row with its own block constant.
-struct StageIn {
-    uint4 c0, c1v;      // forward: codes bytes 0..15, 16..31; backward: row lane, row 32+lane
-    uint32_t b0, b1;    // FP8 constant byte(s) (kNoRow: no weights)
-    float s0, s1;       // c1 of the block(s)
-};
-
-// Forward: 32 TMEM columns = 64 contraction values of one row.  In each
-// code byte the high nibble is the even element, which lands in the low
-// half of its column.
-__device__ __forceinline__ void convert_row(const StageIn& in, float mu, const float* lut, uint32_t (&v)[32]) {
-    const float sc = in.b0 == kNoRow ? 0.0f : dq_constant(static_cast<uint8_t>(in.b0), in.s0, mu);
-    const uint32_t w8[8] = {in.c0.x, in.c0.y, in.c0.z, in.c0.w, in.c1v.x, in.c1v.y, in.c1v.z, in.c1v.w};
+// 64 contraction values of one weight row (forward) or column (backward):
+// 32 code bytes, the high nibble of each byte the even element, which lands
+// in the low half of its TMEM column.  The block constant is one value for
+// the whole run (forward) or one per contraction value (backward, read from
+// shared memory).
+template <bool kPerElem>
+__device__ __forceinline__ void convert_run(const uint4& c0, const uint4& c1, float sc, const float* sp,
+                                            const float* lut, uint32_t (&v)[32]) {
+    const uint32_t w8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
         const uint32_t hi4 = (w8[h] >> 2) & 0x3C3C3C3Cu;  // even-element code * 4, per byte
         const uint32_t lo4 = (w8[h] << 2) & 0x3C3C3C3Cu;  // odd-element code * 4, per byte
+        float4 s01 = make_float4(sc, sc, sc, sc), s23 = s01;
+        if (kPerElem) {
+            s01 = *reinterpret_cast<const float4*>(sp + 8 * h);
+            s23 = *reinterpret_cast<const float4*>(sp + 8 * h + 4);
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const float a = lut_at(lut, __byte_perm(hi4, 0u, 0x4440u | j));
             const float b = lut_at(lut, __byte_perm(lo4, 0u, 0x4440u | j));
-            v[4 * h + j] = scale_pack(a, b, sc);
+            const float2 s2 = j == 0 ? make_float2(s01.x, s01.y)
+                            : j == 1 ? make_float2(s01.z, s01.w)
+                            : j == 2 ? make_float2(s23.x, s23.y)
+                                     : make_float2(s23.z, s23.w);
+            const float2 x = __fmul2_rn(make_float2(a, b), s2);
+            v[4 * h + j] = pack_bf16x2(x.x, x.y);
         }
     }
-}
-
-// Backward: lane = weight column k; its 64 contraction values are 64 weight
-// rows n.  The warp exchanges the rows' code words and constants through a
-// small shared buffer; each lane rotates its own nibble out of each word.
-__device__ __forceinline__ void convert_cols(const StageIn& in, float mu, const float* lut, uint32_t* wsm,
-                                             int lane, uint32_t (&v)[32]) {
-    float* ssm = reinterpret_cast<float*>(wsm + 4 * 68);
-    const float sc0 = in.b0 == kNoRow ? 0.0f : dq_constant(static_cast<uint8_t>(in.b0), in.s0, mu);
-    const float sc1 = in.b1 == kNoRow ? 0.0f : dq_constant(static_cast<uint8_t>(in.b1), in.s1, mu);
-    wsm[0 * 68 + lane] = in.c0.x;
-    wsm[1 * 68 + lane] = in.c0.y;
-    wsm[2 * 68 + lane] = in.c0.z;
-    wsm[3 * 68 + lane] = in.c0.w;
-    wsm[0 * 68 + 32 + lane] = in.c1v.x;
-    wsm[1 * 68 + 32 + lane] = in.c1v.y;
-    wsm[2 * 68 + 32 + lane] = in.c1v.z;
-    wsm[3 * 68 + 32 + lane] = in.c1v.w;
-    ssm[lane] = sc0;
-    ssm[32 + lane] = sc1;
-    __syncwarp();
-    const int wi = lane >> 3;  // the 32-bit word holding this column's nibbles
-    const int shift = ((lane & 7) >> 1) * 8 + ((lane & 1) ? 0 : 4);
-    const uint32_t rot = static_cast<uint32_t>(shift + 30) & 31u;  // nibble -> bits [2, 6)
-#pragma unroll
-    for (int g = 0; g < 16; ++g) {
-        const uint4 c4 = *reinterpret_cast<const uint4*>(wsm + wi * 68 + 4 * g);
-        const float4 s4 = *reinterpret_cast<const float4*>(ssm + 4 * g);
-        const float x0 = lut_at(lut, __funnelshift_r(c4.x, c4.x, rot) & 0x3Cu);
-        const float x1 = lut_at(lut, __funnelshift_r(c4.y, c4.y, rot) & 0x3Cu);
-        const float x2 = lut_at(lut, __funnelshift_r(c4.z, c4.z, rot) & 0x3Cu);
-        const float x3 = lut_at(lut, __funnelshift_r(c4.w, c4.w, rot) & 0x3Cu);
-        const float2 y01 = __fmul2_rn(make_float2(x0, x1), make_float2(s4.x, s4.y));
-        const float2 y23 = __fmul2_rn(make_float2(x2, x3), make_float2(s4.z, s4.w));
-        v[2 * g] = pack_bf16x2(y01.x, y01.y);
-        v[2 * g + 1] = pack_bf16x2(y23.x, y23.y);
-    }
-    __syncwarp();
 }
 
 // warps 2..17: each converts every fourth stage of the weight tile into
@@ -246,103 +213,73 @@ __device__ __forceinline__ void convert_cols(const StageIn& in, float mu, const 
 // quarter of this tile's outputs.
 template <bool kBwd>
 __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const float* lut,
-                                                      uint32_t* wsm, int warp, int lane, int* err) {
+                                                      int warp, int lane, int* err) {
     const int dq = warp - 2;
     const int quarter = warp & 3;  // the TMEM lanes this warp may touch
     const int part = dq >> 2;      // converts the stages kb with kb % 4 == part
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const float mu = *p.mean;
+    const float mu = kBwd ? 0.0f : *p.mean;
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x, ++tcount) {
         const int t0 = (tile % P.num_t) * kTileT;
         const int row0 = (tile / P.num_t) * kTileW;
         const int grow = row0 + row;             // this lane's weight row of the product
         const bool lane_ok = grow < p.rows;
-        const int wcol0 = row0 + quarter * 32;   // backward: first weight column of this warp
-        const bool warp_cols_ok = wcol0 < p.rows;
         const uint32_t g0 = tcount * static_cast<uint32_t>(P.kb_total);  // ring index of stage 0
+        const uint8_t* crow = p.codes + static_cast<int64_t>(grow) * p.ld_codes;
 
-        constexpr int kPrefetch = Prefetch<kBwd>::value;
-        StageIn buf[kPrefetch];
-        auto issue = [&](int kb, StageIn& in) {
-            in.c0 = make_uint4(0u, 0u, 0u, 0u);
-            in.c1v = make_uint4(0u, 0u, 0u, 0u);
-            in.b0 = kNoRow;
-            in.b1 = kNoRow;
-            in.s0 = in.s1 = 0.0f;
-            if (kb >= P.kb_w) return;
-            if (kBwd) {
-                if (!warp_cols_ok) return;
-                const int n0 = kb * kBK + lane;
-                if (n0 < p.N) {
-                    const int64_t e = static_cast<int64_t>(n0) * p.K + wcol0;
-                    in.c0 = ldg_nc_v4(p.codes + (e >> 1));
-                    in.b0 = __ldg(p.c2_fp8 + (e >> 6));
-                    in.s0 = __ldg(p.c1 + (e >> 14));
-                }
-                if (n0 + 32 < p.N) {
-                    const int64_t e = static_cast<int64_t>(n0 + 32) * p.K + wcol0;
-                    in.c1v = ldg_nc_v4(p.codes + (e >> 1));
-                    in.b1 = __ldg(p.c2_fp8 + (e >> 6));
-                    in.s1 = __ldg(p.c1 + (e >> 14));
-                }
-            } else {
-                if (!lane_ok) return;
-                const int64_t e = static_cast<int64_t>(grow) * p.K + kb * kBK;
-                in.c0 = ldg_nc_v4(p.codes + (e >> 1));
-                in.c1v = ldg_nc_v4(p.codes + (e >> 1) + 16);
-                in.b0 = __ldg(p.c2_fp8 + (e >> 6));
-                in.s0 = __ldg(p.c1 + (e >> 14));
+        // codes (and, forward, the block constant) of the next kPrefetch own stages
+        uint4 cb0[kPrefetch], cb1[kPrefetch];
+        float scb[kPrefetch];
+        auto issue = [&](int kb, int u) {
+            cb0[u] = make_uint4(0u, 0u, 0u, 0u);
+            cb1[u] = cb0[u];
+            scb[u] = 0.0f;
+            if (kb >= P.kb_w || !lane_ok) return;
+            cb0[u] = ldg_nc_v4(crow + kb * (kBK / 2));
+            cb1[u] = ldg_nc_v4(crow + kb * (kBK / 2) + 16);
+            if (!kBwd) {
+                const int64_t blk = static_cast<int64_t>(grow) * (p.K / kBK) + kb;
+                scb[u] = dq_constant(__ldg(p.c2_fp8 + blk), __ldg(p.c1 + (blk >> 8)), mu);
             }
         };
 #pragma unroll
-        for (int u = 0; u < kPrefetch; ++u) issue(part + kParts * u, buf[u]);
+        for (int u = 0; u < kPrefetch; ++u) issue(part + kParts * u, u);
         for (int i0 = 0; part + kParts * i0 < P.kb_total; i0 += kPrefetch) {
 #pragma unroll
             for (int u = 0; u < kPrefetch; ++u) {
                 const int kb = part + kParts * (i0 + u);
                 if (kb >= P.kb_total) break;
-                uint32_t v[32];
-                if (kb < P.kb_w) {
-                    if (kBwd)
-                        convert_cols(buf[u], mu, lut, wsm, lane, v);
-                    else
-                        convert_row(buf[u], mu, lut, v);
-                } else {
-                    const int j0 = (kb - P.kb_w) * kBK;
-                    if (kBwd) {  // A^T: lane = column k of A (r x K), in groups of 16 loads
-#pragma unroll
-                        for (int t = 0; t < 32; ++t) {
-                            const int j = j0 + 2 * t;
-                            const uint32_t a = (lane_ok && j < p.r) ? p.lora[static_cast<int64_t>(j) * p.K + grow] : 0u;
-                            const uint32_t b =
-                                (lane_ok && j + 1 < p.r) ? p.lora[static_cast<int64_t>(j + 1) * p.K + grow] : 0u;
-                            v[t] = a | (b << 16);
-                            if ((t & 7) == 7) asm volatile("" ::: "memory");  // bound loads in flight
-                        }
-                    } else {  // B: lane = row n of B (N x r)
-                        const uint16_t* brow = p.lora + static_cast<int64_t>(grow) * p.r + j0;
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            uint4 w = make_uint4(0u, 0u, 0u, 0u);
-                            if (lane_ok && j0 + 8 * c < p.r) w = *reinterpret_cast<const uint4*>(brow + 8 * c);
-                            v[4 * c + 0] = w.x;
-                            v[4 * c + 1] = w.y;
-                            v[4 * c + 2] = w.z;
-                            v[4 * c + 3] = w.w;
-                        }
-                    }
-                }
-                if (!kBwd && !lane_ok) {
-#pragma unroll
-                    for (int t = 0; t < 32; ++t) v[t] = 0u;
-                }
-                issue(kb + kParts * kPrefetch, buf[u]);
                 const uint32_t g = g0 + static_cast<uint32_t>(kb);
                 const int s = static_cast<int>(g % kStages);
                 const uint32_t ph = (g / kStages) & 1u;
-                if (!warp_wait(P.empty(s), ph ^ 1u, err, lane)) return;
+                // backward: the stage's constants come with its dY tile; once
+                // that tile has landed, the previous use of TMEM stage s is over
+                if (kBwd && !warp_wait(P.full_b(s), ph, err, lane)) return;
+                uint32_t v[32];
+                if (kb < P.kb_w) {
+                    const float* sp = P.sS + s * (kScaleStageBytes / 4) + (quarter >> 1) * kBK;
+                    convert_run<kBwd>(cb0[u], cb1[u], scb[u], sp, lut, v);
+                    if (!lane_ok) {
+#pragma unroll
+                        for (int t = 0; t < 32; ++t) v[t] = 0u;
+                    }
+                } else {  // LoRA slab: lane = row of B (forward) or of A^T (backward), r contiguous
+                    const int j0 = (kb - P.kb_w) * kBK;
+                    const uint16_t* lrow = p.lora + static_cast<int64_t>(grow) * p.r + j0;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                        if (lane_ok && j0 + 8 * c < p.r) w = *reinterpret_cast<const uint4*>(lrow + 8 * c);
+                        v[4 * c + 0] = w.x;
+                        v[4 * c + 1] = w.y;
+                        v[4 * c + 2] = w.z;
+                        v[4 * c + 3] = w.w;
+                    }
+                }
+                issue(kb + kParts * kPrefetch, u);
+                if (!kBwd && !warp_wait(P.empty(s), ph ^ 1u, err, lane)) return;
                 tmem_st_32x32b_x32(P.tmem + lane_base + kAccCols + s * kAStageCols, v);
                 tmem_wait_st();
                 tc_fence_before();
@@ -377,17 +314,17 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
 template <bool kBwd>
 __global__ void __launch_bounds__(kThreads, 1)
 k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_lora,
-              const GemmParams p) {
+              const __grid_constant__ CUtensorMap tmap_scale, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ float s_lut[16];  // static, so table reads use an immediate address
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kXStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 2);
-    uint32_t* stage_words = reinterpret_cast<uint32_t*>(smem + kStages * kXStageBytes + 1024);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     Pipe P;
     P.sA = smem;
+    P.sS = reinterpret_cast<float*>(smem + kStages * kXStageBytes + 1024);
     P.bar0 = smem_u32(bars);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -407,6 +344,7 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
     if (warp == 1 && lane == 0) {
         tma_prefetch_desc(&tmap_act);
         tma_prefetch_desc(&tmap_lora);
+        if (kBwd) tma_prefetch_desc(&tmap_scale);
     }
     tc_fence_before();
     __syncthreads();
@@ -419,19 +357,88 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
     int* err = &g_tc_error;
 
     if (warp == 0) {
-        if (lane == 0) role_tma(P, &tmap_act, &tmap_lora, err);
+        if (lane == 0) role_tma<kBwd>(P, &tmap_act, &tmap_lora, &tmap_scale, err);
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) role_mma(P, err);
         __syncwarp();
     } else {
-        role_dequant_epilogue<kBwd>(P, p, s_lut, stage_words + (warp - 2) * kStageWords, warp, lane, err);
+        role_dequant_epilogue<kBwd>(P, p, s_lut, warp, lane, err);
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(P.tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------
+// k_prep_bwd: the transposed weight the backward reads.
+//   codesT[k][j]  = (code(W[2j][k]) << 4) | code(W[2j+1][k])   (K x ldT bytes)
+//   scalesT[g][n] = c2' of the block holding W[n][64g .. 64g+63] (K/64 x ldS)
+//   AT[k][j]      = A[j][k]                                     (K x r)
+// One CTA per 64 x 64 weight tile (plus tiles for A^T); padding is zero.
+constexpr int kPrepThreads = 256;
+
+__global__ void __launch_bounds__(kPrepThreads)
+k_prep_bwd(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8, const float* __restrict__ c1,
+           const float* __restrict__ mean, const uint16_t* __restrict__ A, int N, int K, int r, int64_t ldT,
+           int64_t ldS, uint8_t* __restrict__ codesT, float* __restrict__ scalesT, uint16_t* __restrict__ AT,
+           int weight_tiles) {
+    __shared__ uint8_t tile[64][33];
+    __shared__ uint16_t at[64][65];
+    const int t = threadIdx.x;
+    const int npad_tiles = static_cast<int>(ldS / 64);
+    if (static_cast<int>(blockIdx.x) < weight_tiles) {
+        const int nt = blockIdx.x % npad_tiles, kt = blockIdx.x / npad_tiles;
+        const int n0 = nt * 64, k0 = kt * 64;
+        {   // 64 rows x 32 bytes of codes (zero beyond N)
+            const int rr = t >> 2, cc = (t & 3) * 8;
+            uint2 v = make_uint2(0u, 0u);
+            if (n0 + rr < N)
+                v = *reinterpret_cast<const uint2*>(codes + static_cast<int64_t>(n0 + rr) * (K / 2) + k0 / 2 + cc);
+            for (int b = 0; b < 4; ++b) tile[rr][cc + b] = static_cast<uint8_t>(v.x >> (8 * b));
+            for (int b = 0; b < 4; ++b) tile[rr][cc + 4 + b] = static_cast<uint8_t>(v.y >> (8 * b));
+        }
+        if (t < 64) {
+            const int n = n0 + t;
+            float c = 0.0f;
+            if (n < N) {
+                const int64_t blk = static_cast<int64_t>(n) * (K / 64) + kt;
+                c = dq_constant(c2_fp8[blk], c1[blk >> 8], *mean);
+            }
+            scalesT[static_cast<int64_t>(kt) * ldS + n] = c;
+        }
+        __syncthreads();
+        {   // row k0 + kk of W^T: bytes j0..j0+7, each two consecutive n
+            const int kk = t >> 2, j0 = (t & 3) * 8;
+            uint32_t out[2] = {0u, 0u};
+            for (int b = 0; b < 8; ++b) {
+                const int j = j0 + b;
+                const uint8_t e = tile[2 * j][kk >> 1], o = tile[2 * j + 1][kk >> 1];
+                const uint32_t ne = (kk & 1) ? (e & 15u) : (e >> 4);
+                const uint32_t no = (kk & 1) ? (o & 15u) : (o >> 4);
+                out[b >> 2] |= ((ne << 4) | no) << (8 * (b & 3));
+            }
+            *reinterpret_cast<uint2*>(codesT + static_cast<int64_t>(k0 + kk) * ldT + n0 / 2 + j0) =
+                make_uint2(out[0], out[1]);
+        }
+    } else {
+        const int kt = blockIdx.x - weight_tiles;  // 64 columns of A
+        const int k0 = kt * 64;
+        for (int j0 = 0; j0 < r; j0 += 64) {
+            for (int i = t; i < 64 * 64; i += kPrepThreads) {
+                const int jj = i >> 6, kk = i & 63;
+                at[jj][kk] = (j0 + jj < r && k0 + kk < K) ? A[static_cast<int64_t>(j0 + jj) * K + k0 + kk] : 0;
+            }
+            __syncthreads();
+            for (int i = t; i < 64 * 64; i += kPrepThreads) {
+                const int kk = i >> 6, jj = i & 63;
+                if (j0 + jj < r && k0 + kk < K) AT[static_cast<int64_t>(k0 + kk) * r + j0 + jj] = at[jj][kk];
+            }
+            __syncthreads();
+        }
     }
 }
 
@@ -464,15 +471,29 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t ou
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major fp32 matrix (outer x inner, row stride ld floats), unswizzled
+// boxes of box_inner x box_outer.
+bool make_map_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
+                  uint32_t box_inner, uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {ld * 4};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool kBwd>
-cudaError_t launch_tc(const uint16_t* act, const Nf4Weight& w, const uint16_t* lora_act,
-                      const uint16_t* lora_w, int64_t M, int r, uint16_t* out, cudaStream_t st) {
-    const int64_t ctr = kBwd ? w.N : w.K;
-    const int64_t rows = kBwd ? w.K : w.N;
-    CUtensorMap ma, ml;
-    if (!make_map_bf16(&ma, act, static_cast<uint64_t>(ctr), static_cast<uint64_t>(M), kBK, kTileT) ||
-        !make_map_bf16(&ml, lora_act, static_cast<uint64_t>(r), static_cast<uint64_t>(M), kBK, kTileT))
+cudaError_t launch_tc(const uint16_t* act, const uint16_t* lora_act, const CUtensorMap* scale_map,
+                      const GemmParams& p0, cudaStream_t st) {
+    CUtensorMap ma, ml, ms;
+    if (!make_map_bf16(&ma, act, static_cast<uint64_t>(p0.ctr), static_cast<uint64_t>(p0.M), kBK, kTileT) ||
+        !make_map_bf16(&ml, lora_act, static_cast<uint64_t>(p0.r), static_cast<uint64_t>(p0.M), kBK, kTileT))
         return cudaErrorInvalidValue;
+    ms = scale_map ? *scale_map : ma;  // unused by the forward
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
@@ -480,23 +501,11 @@ cudaError_t launch_tc(const uint16_t* act, const Nf4Weight& w, const uint16_t* l
                                         kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    GemmParams p;
-    p.codes = w.codes;
-    p.c2_fp8 = w.c2_fp8;
-    p.c1 = w.c1;
-    p.mean = w.mean;
-    p.lora = lora_w;
-    p.out = out;
-    p.M = static_cast<int>(M);
-    p.rows = static_cast<int>(rows);
-    p.ctr = static_cast<int>(ctr);
-    p.N = static_cast<int>(w.N);
-    p.K = static_cast<int>(w.K);
-    p.r = r;
+    GemmParams p = p0;
     for (int i = 0; i < 16; ++i) p.q[i] = tables().q[i];
-    const int64_t tiles = ceil_div(M, kTileT) * ceil_div(rows, kTileW);
+    const int64_t tiles = ceil_div(p.M, kTileT) * ceil_div(p.rows, kTileW);
     const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-    k_nf4_gemm_tc<kBwd><<<grid, kThreads, kSmemBytes, st>>>(ma, ml, p);
+    k_nf4_gemm_tc<kBwd><<<grid, kThreads, kSmemBytes, st>>>(ma, ml, ms, p);
     note_launches(1);
     return cudaGetLastError();
 }
@@ -506,6 +515,9 @@ bool tc_common_ok(int64_t M, const Nf4Weight& w, int r) {
            w.N < (int64_t(1) << 31) && w.K < (int64_t(1) << 31) && encode_fn() != nullptr;
 }
 
+int64_t ld_codesT(const Nf4Weight& w) { return round_up(w.N, 64) / 2; }
+int64_t ld_scalesT(const Nf4Weight& w) { return round_up(w.N, 64); }
+
 }  // namespace
 
 bool fwd_tc_supported(int64_t M, const Nf4Weight& w, int r) { return tc_common_ok(M, w, r); }
@@ -513,19 +525,62 @@ bool fwd_tc_supported(int64_t M, const Nf4Weight& w, int r) { return tc_common_o
 // The dY tensor map needs a row stride that is a multiple of 16 bytes.
 bool dx_tc_supported(int64_t M, const Nf4Weight& w, int r) { return tc_common_ok(M, w, r) && w.N % 8 == 0; }
 
+size_t dx_tc_workspace(const Nf4Weight& w, int r) {
+    const size_t a = static_cast<size_t>(w.K) * ld_codesT(w);
+    const size_t b = static_cast<size_t>(w.K / kBK) * ld_scalesT(w) * 4;
+    const size_t c = static_cast<size_t>(w.K) * r * 2;
+    return round_up(a, 256) + round_up(b, 256) + round_up(c, 256);
+}
+
 cudaError_t launch_fwd_gemm_tc(const uint16_t* X, const Nf4Weight& w, const uint16_t* T, const uint16_t* B,
                                int64_t M, int r, uint16_t* Y, cudaStream_t st) {
-    return launch_tc<false>(X, w, T, B, M, r, Y, st);
+    GemmParams p{};
+    p.codes = w.codes;
+    p.c2_fp8 = w.c2_fp8;
+    p.c1 = w.c1;
+    p.mean = w.mean;
+    p.lora = B;
+    p.out = Y;
+    p.ld_codes = w.K / 2;
+    p.M = static_cast<int>(M);
+    p.rows = static_cast<int>(w.N);
+    p.ctr = static_cast<int>(w.K);
+    p.K = static_cast<int>(w.K);
+    p.r = r;
+    return launch_tc<false>(X, T, nullptr, p, st);
 }
 
 cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U, const uint16_t* A,
-                                  int64_t M, int r, uint16_t* dX, cudaStream_t st) {
-    return launch_tc<true>(dY, w, U, A, M, r, dX, st);
+                                  int64_t M, int r, uint16_t* dX, void* ws, cudaStream_t st) {
+    const int64_t ldT = ld_codesT(w), ldS = ld_scalesT(w);
+    uint8_t* codesT = reinterpret_cast<uint8_t*>(ws);
+    float* scalesT = reinterpret_cast<float*>(codesT + round_up(static_cast<size_t>(w.K) * ldT, 256));
+    uint16_t* AT = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(scalesT) +
+                                               round_up(static_cast<size_t>(w.K / kBK) * ldS * 4, 256));
+    const int weight_tiles = static_cast<int>((ldS / 64) * (w.K / 64));
+    const int a_tiles = static_cast<int>(ceil_div(w.K, 64));
+    k_prep_bwd<<<weight_tiles + a_tiles, kPrepThreads, 0, st>>>(w.codes, w.c2_fp8, w.c1, w.mean, A,
+                                                                static_cast<int>(w.N), static_cast<int>(w.K), r,
+                                                                ldT, ldS, codesT, scalesT, AT, weight_tiles);
+    note_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    CUtensorMap msc;
+    if (!make_map_f32(&msc, scalesT, static_cast<uint64_t>(ldS), static_cast<uint64_t>(w.K / kBK),
+                      static_cast<uint64_t>(ldS), kBK, 2))
+        return cudaErrorInvalidValue;
+    GemmParams p{};
+    p.codes = codesT;
+    p.lora = AT;
+    p.out = dX;
+    p.ld_codes = ldT;
+    p.M = static_cast<int>(M);
+    p.rows = static_cast<int>(w.K);
+    p.ctr = static_cast<int>(w.N);
+    p.K = static_cast<int>(w.K);
+    p.r = r;
+    return launch_tc<true>(dY, U, &msc, p, st);
 }
-
-}  // namespace qlora
-
-namespace qlora {
 
 int gemm_device_error(int reset) {
     int v = 0;

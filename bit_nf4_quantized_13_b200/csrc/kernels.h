@@ -68,8 +68,10 @@ bool fwd_tc_supported(int64_t M, const Nf4Weight& w, int r);
 bool dx_tc_supported(int64_t M, const Nf4Weight& w, int r);
 cudaError_t launch_fwd_gemm_tc(const uint16_t* X, const Nf4Weight& w, const uint16_t* T, const uint16_t* B,
                                int64_t M, int r, uint16_t* Y, cudaStream_t stream);
+// The backward needs dx_tc_workspace bytes for the transposed weight copy.
+size_t dx_tc_workspace(const Nf4Weight& w, int r);
 cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U, const uint16_t* A,
-                                  int64_t M, int r, uint16_t* dX, cudaStream_t stream);
+                                  int64_t M, int r, uint16_t* dX, void* ws, cudaStream_t stream);
 
 // gemm_*.cu -- the frozen-weight GEMMs with the LoRA slab fused in
 //   Y  = bf16(X W'^T + T B^T)      (M x N)
@@ -77,7 +79,7 @@ cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const 
 cudaError_t launch_fwd_gemm(const uint16_t* X, const Nf4Weight& w, const uint16_t* T,
                             const uint16_t* B, int64_t M, int r, uint16_t* Y, cudaStream_t stream);
 cudaError_t launch_bwd_dx_gemm(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U,
-                               const uint16_t* A, int64_t M, int r, uint16_t* dX,
+                               const uint16_t* A, int64_t M, int r, uint16_t* dX, void* ws,
                                cudaStream_t stream);
 
 }  // namespace qlora
