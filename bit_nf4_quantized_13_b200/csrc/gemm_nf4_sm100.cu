@@ -27,8 +27,11 @@
 // 32-byte run of codes, exactly like the forward owns a row n; the
 // constants of a stage (2 x 64 floats) arrive by TMA with the dY tile.
 //
-// Tile: 128 weight rows (n forward, k backward) x 256 tokens x 64; fp32
-// accumulator in 256 TMEM columns; 6 pipeline stages.  Warp roles (576
+// Tile: 128 weight rows (n forward, k backward) x 384 tokens x 64: each
+// dequantized weight stage feeds two 128 x 192 MMAs (two fp32 accumulators,
+// 384 TMEM columns), so the conversion work per FLOP is that of a 384-token
+// tile; 4 pipeline stages (A stages in the last 128 TMEM columns).  Warp
+// roles (576
 // threads, persistent over tiles, one CTA per SM):
 //   warp 0        TMA producer for the activation tiles (and constants)
 //   warp 1        MMA issuer (one thread)
@@ -56,10 +59,13 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileW = 128;   // weight rows per tile (MMA M)
-constexpr int kTileT = 256;   // tokens per tile (MMA N)
+constexpr int kSubT = 192;    // tokens per MMA (MMA N)
+constexpr int kSubs = 2;      // MMAs per stage sharing one dequantized weight stage
+constexpr int kTileT = kSubT * kSubs;  // 384 tokens per tile
 constexpr int kBK = 64;       // contraction per stage
-constexpr int kStages = 6;
-constexpr int kXStageBytes = kTileT * kBK * 2;  // 32 KiB
+constexpr int kStages = 4;
+constexpr int kSubBytes = kSubT * kBK * 2;      // 24 KiB
+constexpr int kXStageBytes = kTileT * kBK * 2;  // 48 KiB
 constexpr int kScaleStageBytes = 2 * kBK * 4;   // backward: c2' of 2 column groups x 64 rows
 constexpr int kAccCols = kTileT;                // fp32 accumulator columns
 constexpr int kAStageCols = kBK / 2;            // bf16 pairs per TMEM column
@@ -96,10 +102,10 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
 }
 
 struct Pipe {
-    uint8_t* sA;       // kStages x 32 KiB of activation tiles
+    uint8_t* sA;       // kStages x 48 KiB of activation tiles (two 192-token halves)
     float* sS;         // backward: kStages x [2][64] block constants
     uint32_t bar0;     // full_b[S], full_a[S], empty[S], acc_full, acc_empty
-    uint32_t tmem;     // accumulator at columns [0, 256), A stages after it
+    uint32_t tmem;     // accumulators at columns [0, 384), A stages after them
     int num_t, num_tiles, kb_w, kb_total;
     __device__ uint32_t full_b(int s) const { return bar0 + 8u * s; }
     __device__ uint32_t full_a(int s) const { return bar0 + 8u * (kStages + s); }
@@ -124,21 +130,25 @@ __device__ void role_tma(const Pipe& P, const CUtensorMap* tmap_act, const CUten
             const uint32_t dst = smem_u32(P.sA + s * kXStageBytes);
             if (kb < P.kb_w) {
                 mbar_arrive_expect_tx(P.full_b(s), kXStageBytes + (kBwd ? kScaleStageBytes : 0));
-                tma_load_2d(dst, tmap_act, P.full_b(s), kb * kBK, t0);
+                for (int sub = 0; sub < kSubs; ++sub)
+                    tma_load_2d(dst + sub * kSubBytes, tmap_act, P.full_b(s), kb * kBK, t0 + sub * kSubT);
                 if (kBwd)
                     tma_load_2d(smem_u32(P.sS + s * (kScaleStageBytes / 4)), tmap_scale, P.full_b(s), kb * kBK,
                                 row0 / kBK);
             } else {
                 mbar_arrive_expect_tx(P.full_b(s), kXStageBytes);
-                tma_load_2d(dst, tmap_lora, P.full_b(s), (kb - P.kb_w) * kBK, t0);
+                for (int sub = 0; sub < kSubs; ++sub)
+                    tma_load_2d(dst + sub * kSubBytes, tmap_lora, P.full_b(s), (kb - P.kb_w) * kBK,
+                                t0 + sub * kSubT);
             }
         }
     }
 }
 
-// warp 1, one thread: four 128x256x16 MMAs per stage into the accumulator.
+// warp 1, one thread: per stage, four 128x192x16 MMAs into each of the two
+// accumulators, all reading the same weight stage in TMEM.
 __device__ void role_mma(const Pipe& P, int* err) {
-    constexpr uint32_t idesc = idesc_bf16(kTileW, kTileT);
+    constexpr uint32_t idesc = idesc_bf16(kTileW, kSubT);
     uint32_t it = 0, tcount = 0;
     for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x, ++tcount) {
         if (!mbar_wait(P.acc_empty(), (tcount & 1u) ^ 1u, err)) return;
@@ -150,10 +160,14 @@ __device__ void role_mma(const Pipe& P, int* err) {
             if (!mbar_wait(P.full_a(s), ph, err)) return;
             tc_fence_after();
             const uint32_t a_col = P.tmem + kAccCols + s * kAStageCols;
-            const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(P.sA + s * kXStageBytes));
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk)
-                mma_bf16_ts(P.tmem, a_col + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc, (kb | kk) != 0);
+            for (int sub = 0; sub < kSubs; ++sub) {
+                const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(P.sA + s * kXStageBytes + sub * kSubBytes));
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk)
+                    mma_bf16_ts(P.tmem + sub * kSubT, a_col + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                                (kb | kk) != 0);
+            }
             tc_commit(P.empty(s));
         }
         tc_commit(P.acc_full());
@@ -229,19 +243,24 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
         const uint32_t g0 = tcount * static_cast<uint32_t>(P.kb_total);  // ring index of stage 0
         const uint8_t* crow = p.codes + static_cast<int64_t>(grow) * p.ld_codes;
 
-        // codes (and, forward, the block constant) of the next kPrefetch own stages
+        // codes (and, forward, the block constant's inputs) of the next
+        // kPrefetch own stages; the constant itself is formed at use so the
+        // loads stay in flight
         uint4 cb0[kPrefetch], cb1[kPrefetch];
-        float scb[kPrefetch];
+        uint32_t sbyte[kPrefetch];
+        float sc1[kPrefetch];
         auto issue = [&](int kb, int u) {
             cb0[u] = make_uint4(0u, 0u, 0u, 0u);
             cb1[u] = cb0[u];
-            scb[u] = 0.0f;
+            sbyte[u] = 0u;
+            sc1[u] = 0.0f;
             if (kb >= P.kb_w || !lane_ok) return;
             cb0[u] = ldg_nc_v4(crow + kb * (kBK / 2));
             cb1[u] = ldg_nc_v4(crow + kb * (kBK / 2) + 16);
             if (!kBwd) {
                 const int64_t blk = static_cast<int64_t>(grow) * (p.K / kBK) + kb;
-                scb[u] = dq_constant(__ldg(p.c2_fp8 + blk), __ldg(p.c1 + (blk >> 8)), mu);
+                sbyte[u] = __ldg(p.c2_fp8 + blk);
+                sc1[u] = __ldg(p.c1 + (blk >> 8));
             }
         };
 #pragma unroll
@@ -260,7 +279,8 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
                 uint32_t v[32];
                 if (kb < P.kb_w) {
                     const float* sp = P.sS + s * (kScaleStageBytes / 4) + (quarter >> 1) * kBK;
-                    convert_run<kBwd>(cb0[u], cb1[u], scb[u], sp, lut, v);
+                    const float sc = kBwd ? 0.0f : dq_constant(static_cast<uint8_t>(sbyte[u]), sc1[u], mu);
+                    convert_run<kBwd>(cb0[u], cb1[u], sc, sp, lut, v);
                     if (!lane_ok) {
 #pragma unroll
                         for (int t = 0; t < 32; ++t) v[t] = 0u;
@@ -287,16 +307,17 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
                 if (lane == 0) mbar_arrive(P.full_a(s));
             }
         }
-        // epilogue: this warp's lane quarter, columns [64 part, 64 part + 64)
+        // epilogue: this warp's lane quarter, columns [96 part, 96 part + 96)
         if (!warp_wait(P.acc_full(), tcount & 1u, err, lane)) return;
         tc_fence_after();
+        constexpr int kChunks = kTileT / kParts / 16;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-            const int col = part * 64 + c * 16;
+        for (int c = 0; c < kChunks; ++c) {
+            const int col = part * (kTileT / kParts) + c * 16;
             uint32_t acc[16];
             tmem_ld_32x32b_x16(P.tmem + lane_base + col, acc);
             tmem_wait_ld();
-            if (c == 3) {
+            if (c == kChunks - 1) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(P.acc_empty());
@@ -490,8 +511,8 @@ template <bool kBwd>
 cudaError_t launch_tc(const uint16_t* act, const uint16_t* lora_act, const CUtensorMap* scale_map,
                       const GemmParams& p0, cudaStream_t st) {
     CUtensorMap ma, ml, ms;
-    if (!make_map_bf16(&ma, act, static_cast<uint64_t>(p0.ctr), static_cast<uint64_t>(p0.M), kBK, kTileT) ||
-        !make_map_bf16(&ml, lora_act, static_cast<uint64_t>(p0.r), static_cast<uint64_t>(p0.M), kBK, kTileT))
+    if (!make_map_bf16(&ma, act, static_cast<uint64_t>(p0.ctr), static_cast<uint64_t>(p0.M), kBK, kSubT) ||
+        !make_map_bf16(&ml, lora_act, static_cast<uint64_t>(p0.r), static_cast<uint64_t>(p0.M), kBK, kSubT))
         return cudaErrorInvalidValue;
     ms = scale_map ? *scale_map : ma;  // unused by the forward
     static std::once_flag attr_once;
