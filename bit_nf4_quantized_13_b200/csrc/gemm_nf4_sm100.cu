@@ -24,8 +24,10 @@
 // k_prep_bwd: codes of W^T (two consecutive n per byte), the block
 // constants c2' in fp32 laid out [k/64][n], and A^T.  A lane then owns one
 // weight column k and converts 64 consecutive contraction values from one
-// 32-byte run of codes, exactly like the forward owns a row n; the
-// constants of a stage (2 x 64 floats) arrive by TMA with the dY tile.
+// 32-byte run of codes, exactly like the forward owns a row n.  The 64
+// constants of a stage (one per row n, shared by the warp's 32 columns) are
+// loaded two per lane with the codes and exchanged through a small
+// warp-private shared buffer.
 //
 // Tile: 128 weight rows (n forward, k backward) x 384 tokens x 64: each
 // dequantized weight stage feeds two 128 x 192 MMAs (two fp32 accumulators,
@@ -66,7 +68,6 @@ constexpr int kBK = 64;       // contraction per stage
 constexpr int kStages = 4;
 constexpr int kSubBytes = kSubT * kBK * 2;      // 24 KiB
 constexpr int kXStageBytes = kTileT * kBK * 2;  // 48 KiB
-constexpr int kScaleStageBytes = 2 * kBK * 4;   // backward: c2' of 2 column groups x 64 rows
 constexpr int kAccCols = kTileT;                // fp32 accumulator columns
 constexpr int kAStageCols = kBK / 2;            // bf16 pairs per TMEM column
 constexpr uint32_t kTmemCols = 512;
@@ -75,7 +76,7 @@ constexpr int kParts = kDqWarps / 4;            // stage kb is converted by the 
 constexpr int kPrefetch = 2;                    // own stages of codes in flight per dequant thread
 constexpr int kThreads = 32 * (2 + kDqWarps);   // 576
 constexpr int kSmemBytes = kStages * kXStageBytes + 1024 /* align */ + 1024 /* barriers etc. */ +
-                           kStages * kScaleStageBytes;
+                           kDqWarps * kBK * 4 /* backward: per-warp constants */;
 static_assert(kAccCols + kStages * kAStageCols <= static_cast<int>(kTmemCols), "TMEM budget");
 
 struct GemmParams {
@@ -83,6 +84,8 @@ struct GemmParams {
     const uint8_t* c2_fp8; // forward only
     const float* c1;       // forward only
     const float* mean;     // forward only
+    const float* scalesT;  // backward only: c2' laid out [k/64][n], row stride ld_scales
+    int64_t ld_scales;
     const uint16_t* lora;  // forward: B (N x r); backward: A^T (K x r)
     uint16_t* out;         // forward: Y (M x N); backward: dX (M x K)
     int64_t ld_codes;      // bytes per weight row of `codes`
@@ -103,7 +106,7 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
 
 struct Pipe {
     uint8_t* sA;       // kStages x 48 KiB of activation tiles (two 192-token halves)
-    float* sS;         // backward: kStages x [2][64] block constants
+    float* sS;         // backward: per dequant warp, 64 block constants
     uint32_t bar0;     // full_b[S], full_a[S], empty[S], acc_full, acc_empty
     uint32_t tmem;     // accumulators at columns [0, 384), A stages after them
     int num_t, num_tiles, kb_w, kb_total;
@@ -114,27 +117,20 @@ struct Pipe {
     __device__ uint32_t acc_empty() const { return bar0 + 8u * (3 * kStages + 1); }
 };
 
-// warp 0, one thread: activation tiles (backward: with the stage's block
-// constants), then the LoRA slabs, into the ring.
-template <bool kBwd>
-__device__ void role_tma(const Pipe& P, const CUtensorMap* tmap_act, const CUtensorMap* tmap_lora,
-                         const CUtensorMap* tmap_scale, int* err) {
+// warp 0, one thread: activation tiles, then the LoRA slabs, into the ring.
+__device__ void role_tma(const Pipe& P, const CUtensorMap* tmap_act, const CUtensorMap* tmap_lora, int* err) {
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x) {
         const int t0 = (tile % P.num_t) * kTileT;
-        const int row0 = (tile / P.num_t) * kTileW;
         for (int kb = 0; kb < P.kb_total; ++kb, ++it) {
             const int s = static_cast<int>(it % kStages);
             const uint32_t ph = (it / kStages) & 1u;
             if (!mbar_wait(P.empty(s), ph ^ 1u, err)) return;
             const uint32_t dst = smem_u32(P.sA + s * kXStageBytes);
             if (kb < P.kb_w) {
-                mbar_arrive_expect_tx(P.full_b(s), kXStageBytes + (kBwd ? kScaleStageBytes : 0));
+                mbar_arrive_expect_tx(P.full_b(s), kXStageBytes);
                 for (int sub = 0; sub < kSubs; ++sub)
                     tma_load_2d(dst + sub * kSubBytes, tmap_act, P.full_b(s), kb * kBK, t0 + sub * kSubT);
-                if (kBwd)
-                    tma_load_2d(smem_u32(P.sS + s * (kScaleStageBytes / 4)), tmap_scale, P.full_b(s), kb * kBK,
-                                row0 / kBK);
             } else {
                 mbar_arrive_expect_tx(P.full_b(s), kXStageBytes);
                 for (int sub = 0; sub < kSubs; ++sub)
@@ -227,7 +223,7 @@ __device__ __forceinline__ void convert_run(const uint4& c0, const uint4& c1, fl
 // quarter of this tile's outputs.
 template <bool kBwd>
 __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const float* lut,
-                                                      int warp, int lane, int* err) {
+                                                      float* wsc, int warp, int lane, int* err) {
     const int dq = warp - 2;
     const int quarter = warp & 3;  // the TMEM lanes this warp may touch
     const int part = dq >> 2;      // converts the stages kb with kb % 4 == part
@@ -242,6 +238,9 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
         const bool lane_ok = grow < p.rows;
         const uint32_t g0 = tcount * static_cast<uint32_t>(P.kb_total);  // ring index of stage 0
         const uint8_t* crow = p.codes + static_cast<int64_t>(grow) * p.ld_codes;
+        // backward: this warp's 32 columns lie in one 64-wide block group
+        const float* srow = kBwd ? p.scalesT + static_cast<int64_t>((row0 + quarter * 32) / kBK) * p.ld_scales
+                                 : nullptr;
 
         // codes (and, forward, the block constant's inputs) of the next
         // kPrefetch own stages; the constant itself is formed at use so the
@@ -249,12 +248,17 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
         uint4 cb0[kPrefetch], cb1[kPrefetch];
         uint32_t sbyte[kPrefetch];
         float sc1[kPrefetch];
+        float2 s2[kPrefetch];  // backward: constants of rows 2 lane, 2 lane + 1 of the stage
         auto issue = [&](int kb, int u) {
             cb0[u] = make_uint4(0u, 0u, 0u, 0u);
             cb1[u] = cb0[u];
             sbyte[u] = 0u;
             sc1[u] = 0.0f;
-            if (kb >= P.kb_w || !lane_ok) return;
+            s2[u] = make_float2(0.0f, 0.0f);
+            if (kb >= P.kb_w) return;
+            if (kBwd && (row0 + quarter * 32) < p.rows)
+                s2[u] = __ldg(reinterpret_cast<const float2*>(srow + kb * kBK) + lane);
+            if (!lane_ok) return;
             cb0[u] = ldg_nc_v4(crow + kb * (kBK / 2));
             cb1[u] = ldg_nc_v4(crow + kb * (kBK / 2) + 16);
             if (!kBwd) {
@@ -273,14 +277,15 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
                 const uint32_t g = g0 + static_cast<uint32_t>(kb);
                 const int s = static_cast<int>(g % kStages);
                 const uint32_t ph = (g / kStages) & 1u;
-                // backward: the stage's constants come with its dY tile; once
-                // that tile has landed, the previous use of TMEM stage s is over
-                if (kBwd && !warp_wait(P.full_b(s), ph, err, lane)) return;
                 uint32_t v[32];
                 if (kb < P.kb_w) {
-                    const float* sp = P.sS + s * (kScaleStageBytes / 4) + (quarter >> 1) * kBK;
+                    if (kBwd) {
+                        reinterpret_cast<float2*>(wsc)[lane] = s2[u];
+                        __syncwarp();
+                    }
                     const float sc = kBwd ? 0.0f : dq_constant(static_cast<uint8_t>(sbyte[u]), sc1[u], mu);
-                    convert_run<kBwd>(cb0[u], cb1[u], sc, sp, lut, v);
+                    convert_run<kBwd>(cb0[u], cb1[u], sc, wsc, lut, v);
+                    if (kBwd) __syncwarp();  // wsc is rewritten by the warp's next stage
                     if (!lane_ok) {
 #pragma unroll
                         for (int t = 0; t < 32; ++t) v[t] = 0u;
@@ -299,7 +304,7 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
                     }
                 }
                 issue(kb + kParts * kPrefetch, u);
-                if (!kBwd && !warp_wait(P.empty(s), ph ^ 1u, err, lane)) return;
+                if (!warp_wait(P.empty(s), ph ^ 1u, err, lane)) return;
                 tmem_st_32x32b_x32(P.tmem + lane_base + kAccCols + s * kAStageCols, v);
                 tmem_wait_st();
                 tc_fence_before();
@@ -335,7 +340,7 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
 template <bool kBwd>
 __global__ void __launch_bounds__(kThreads, 1)
 k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_lora,
-              const __grid_constant__ CUtensorMap tmap_scale, const GemmParams p) {
+              const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ float s_lut[16];  // static, so table reads use an immediate address
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -365,7 +370,6 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
     if (warp == 1 && lane == 0) {
         tma_prefetch_desc(&tmap_act);
         tma_prefetch_desc(&tmap_lora);
-        if (kBwd) tma_prefetch_desc(&tmap_scale);
     }
     tc_fence_before();
     __syncthreads();
@@ -378,13 +382,13 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
     int* err = &g_tc_error;
 
     if (warp == 0) {
-        if (lane == 0) role_tma<kBwd>(P, &tmap_act, &tmap_lora, &tmap_scale, err);
+        if (lane == 0) role_tma(P, &tmap_act, &tmap_lora, err);
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) role_mma(P, err);
         __syncwarp();
     } else {
-        role_dequant_epilogue<kBwd>(P, p, s_lut, warp, lane, err);
+        role_dequant_epilogue<kBwd>(P, p, s_lut, P.sS + (warp - 2) * kBK, warp, lane, err);
     }
     tc_fence_before();
     __syncthreads();
@@ -492,29 +496,12 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t ou
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Row-major fp32 matrix (outer x inner, row stride ld floats), unswizzled
-// boxes of box_inner x box_outer.
-bool make_map_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
-                  uint32_t box_inner, uint32_t box_outer) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {ld * 4};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <bool kBwd>
-cudaError_t launch_tc(const uint16_t* act, const uint16_t* lora_act, const CUtensorMap* scale_map,
-                      const GemmParams& p0, cudaStream_t st) {
-    CUtensorMap ma, ml, ms;
+cudaError_t launch_tc(const uint16_t* act, const uint16_t* lora_act, const GemmParams& p0, cudaStream_t st) {
+    CUtensorMap ma, ml;
     if (!make_map_bf16(&ma, act, static_cast<uint64_t>(p0.ctr), static_cast<uint64_t>(p0.M), kBK, kSubT) ||
         !make_map_bf16(&ml, lora_act, static_cast<uint64_t>(p0.r), static_cast<uint64_t>(p0.M), kBK, kSubT))
         return cudaErrorInvalidValue;
-    ms = scale_map ? *scale_map : ma;  // unused by the forward
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
@@ -526,7 +513,7 @@ cudaError_t launch_tc(const uint16_t* act, const uint16_t* lora_act, const CUten
     for (int i = 0; i < 16; ++i) p.q[i] = tables().q[i];
     const int64_t tiles = ceil_div(p.M, kTileT) * ceil_div(p.rows, kTileW);
     const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-    k_nf4_gemm_tc<kBwd><<<grid, kThreads, kSmemBytes, st>>>(ma, ml, ms, p);
+    k_nf4_gemm_tc<kBwd><<<grid, kThreads, kSmemBytes, st>>>(ma, ml, p);
     note_launches(1);
     return cudaGetLastError();
 }
@@ -568,7 +555,7 @@ cudaError_t launch_fwd_gemm_tc(const uint16_t* X, const Nf4Weight& w, const uint
     p.ctr = static_cast<int>(w.K);
     p.K = static_cast<int>(w.K);
     p.r = r;
-    return launch_tc<false>(X, T, nullptr, p, st);
+    return launch_tc<false>(X, T, p, st);
 }
 
 cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U, const uint16_t* A,
@@ -586,12 +573,10 @@ cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const 
     note_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    CUtensorMap msc;
-    if (!make_map_f32(&msc, scalesT, static_cast<uint64_t>(ldS), static_cast<uint64_t>(w.K / kBK),
-                      static_cast<uint64_t>(ldS), kBK, 2))
-        return cudaErrorInvalidValue;
     GemmParams p{};
     p.codes = codesT;
+    p.scalesT = scalesT;
+    p.ld_scales = ldS;
     p.lora = AT;
     p.out = dX;
     p.ld_codes = ldT;
@@ -600,7 +585,7 @@ cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const 
     p.ctr = static_cast<int>(w.N);
     p.K = static_cast<int>(w.K);
     p.r = r;
-    return launch_tc<true>(dY, U, &msc, p, st);
+    return launch_tc<true>(dY, U, p, st);
 }
 
 int gemm_device_error(int reset) {
