@@ -75,7 +75,6 @@ float from_key(int64_t k) {
 // wins iff RN(n - q_j) > RN(q_{j+1} - n) (a tie keeps the lower index).
 // The predicate is monotone in n; the threshold is the smallest fp32 n in
 // [q_j, q_{j+1}] where it holds.
-volatile float g_sink;
 bool upper_wins(float n, float qj, float qj1) {
     volatile float a = n - qj;    // volatile: one fp32 rounding each, no reassociation
     volatile float b = qj1 - n;
@@ -136,6 +135,20 @@ Nf4Tables build_tables() {
             // cannot happen for the NF4 type (thresholds are >= 0.08 apart,
             // bins are 1/16 wide); keep the failure loud
             t.base[b] = -1000;
+        }
+        // rounding boundary below the threshold: the midpoint between it and
+        // its fp32 predecessor; a quotient exactly on it rounds to the even
+        // neighbour, which is the threshold when the threshold's significand
+        // is even
+        t.bnd[b] = HUGE_VAL;
+        t.tie_up[b] = 0;
+        if (inside == 1) {
+            const float th = t.thr[b];
+            const float pr = nextafterf(th, -INFINITY);
+            t.bnd[b] = 0.5 * (static_cast<double>(pr) + static_cast<double>(th));
+            uint32_t u;
+            memcpy(&u, &th, 4);
+            t.tie_up[b] = (u & 1u) == 0 ? 1 : 0;
         }
     }
     return t;

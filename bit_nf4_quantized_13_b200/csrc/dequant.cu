@@ -4,10 +4,10 @@
 // the NF4 type and scaled by its block constant.
 //
 // HBM-bound: 0.5 + 1/64 + 1/16384 bytes read and 4 (fp32) or 2 (bf16) bytes
-// written per weight.  A warp owns 1024 consecutive weights (16 blocks):
-// lanes 0-15 first expand the 16 block constants, then in store step i
-// lane l writes the i-th 16-byte row slot of the warp's output, so every
-// store instruction is one contiguous run across the warp.
+// written per weight.  Each lane expands 32 consecutive weights per step
+// from one 16-byte load of codes and one block constant; code nibbles become
+// table byte offsets with shift/mask and byte_perm, and pairs of weights are
+// scaled with one f32x2 multiply.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -15,89 +15,101 @@ namespace qlora {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kWarpElems = 1024;
+constexpr int kRun = 32;  // weights per lane per step: 16 code bytes, one block constant
 
-__device__ __forceinline__ uint32_t ld_nc_u32(const uint8_t* p) {
-    uint32_t v;
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
-}
-__device__ __forceinline__ uint32_t ld_nc_u16(const uint8_t* p) {
-    unsigned short v;
-    asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+__device__ __forceinline__ uint4 ld_nc_v4(const uint8_t* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
     return v;
 }
 
-// OUT_BF16 = false: fp32 output, 4 weights (2 code bytes) per lane per step.
-// OUT_BF16 = true : bf16 output, 8 weights (4 code bytes) per lane per step.
+// q[code] from the 16-entry table by byte offset (code * 4)
+__device__ __forceinline__ float lut_at(const float* lut, uint32_t byte_off) {
+    return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(lut) + byte_off);
+}
+
+// 32 weights of one block from 16 code bytes: element 2t is the high nibble
+// of byte t.  out[i] = RN32(q[code_i] * c2').
+__device__ __forceinline__ void expand32(const uint4& cw, float cp, const float* lut, float (&w)[kRun]) {
+    const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const uint32_t hi4 = (w4[h] >> 2) & 0x3C3C3C3Cu;
+        const uint32_t lo4 = (w4[h] << 2) & 0x3C3C3C3Cu;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 x = __fmul2_rn(make_float2(lut_at(lut, __byte_perm(hi4, 0u, 0x4440u | j)),
+                                                    lut_at(lut, __byte_perm(lo4, 0u, 0x4440u | j))),
+                                        make_float2(cp, cp));
+            w[8 * h + 2 * j] = x.x;
+            w[8 * h + 2 * j + 1] = x.y;
+        }
+    }
+}
+
+// Each lane owns 32 consecutive weights per step (one 16-byte load of
+// codes, one block constant), grid-stride with the next step's loads in
+// flight.  OUT_BF16 selects bf16 (64-byte) or fp32 (128-byte) output runs.
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(kThreads)
 k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
           const float* __restrict__ c1, const float* __restrict__ mean, int64_t numel,
           void* __restrict__ out, Nf4Tables tabs) {
-    __shared__ float sq[16];
-    if (threadIdx.x < 16) sq[threadIdx.x] = tabs.q[threadIdx.x];
+    __shared__ float s_lut[16];
+    if (threadIdx.x < 16) s_lut[threadIdx.x] = tabs.q[threadIdx.x];
     __syncthreads();
     const float mu = *mean;
-    const int lane = threadIdx.x & 31;
-    const int64_t nb = ceil_div(numel, kBlock);
-    const int64_t nwc = ceil_div(numel, kWarpElems);
-    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    constexpr int kPer = OUT_BF16 ? 8 : 4;           // weights per lane per step
-    constexpr int kSteps = kWarpElems / (32 * kPer);  // 8 (fp32) or 4 (bf16)
+    const int64_t nfull = numel / kRun;  // whole 32-weight runs
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
 
-    for (int64_t c = warp0; c < nwc; c += nwarps) {
-        const int64_t base = c * kWarpElems;
-        // block constants of the warp's 16 blocks, one per lane 0..15
-        float cp = 0.0f;
-        {
-            const int64_t blk = (base >> 6) + (lane & 15);
-            if (blk < nb) cp = dq_constant(c2_fp8[blk], c1[blk >> 8], mu);
+    uint4 cw = make_uint4(0u, 0u, 0u, 0u);
+    uint32_t sb = 0u;
+    float sc1 = 0.0f;
+    auto load = [&](int64_t run, uint4& c, uint32_t& b, float& s1) {
+        const int64_t e = run * kRun;
+        c = ld_nc_v4(codes + (e >> 1));
+        b = __ldg(c2_fp8 + (e >> 6));
+        s1 = __ldg(c1 + (e >> 14));
+    };
+    if (t < nfull) load(t, cw, sb, sc1);
+    for (; t < nfull; t += stride) {
+        uint4 ncw = cw;
+        uint32_t nsb = sb;
+        float ns1 = sc1;
+        if (t + stride < nfull) load(t + stride, ncw, nsb, ns1);
+        float w[kRun];
+        expand32(cw, dq_constant(static_cast<uint8_t>(sb), sc1, mu), s_lut, w);
+        const int64_t e = t * kRun;
+        if (OUT_BF16) {
+            uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + e);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                __stcs(o + c, make_uint4(pack_bf16x2(w[8 * c + 0], w[8 * c + 1]), pack_bf16x2(w[8 * c + 2], w[8 * c + 3]),
+                                         pack_bf16x2(w[8 * c + 4], w[8 * c + 5]), pack_bf16x2(w[8 * c + 6], w[8 * c + 7])));
+        } else {
+            float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + e);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                __stcs(o + c, make_float4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]));
         }
-        const bool full = base + kWarpElems <= numel;
-#pragma unroll
-        for (int i = 0; i < kSteps; ++i) {
-            const int64_t e = base + static_cast<int64_t>(kPer) * (32 * i + lane);
-            // weights e .. e+kPer-1 share one block: kPer divides 64
-            const float scale = __shfl_sync(0xffffffffu, cp, static_cast<int>(((e - base) >> 6) & 15));
-            uint32_t cw;
-            if (full) {
-                cw = OUT_BF16 ? ld_nc_u32(codes + (e >> 1)) : ld_nc_u16(codes + (e >> 1));
-            } else {
-                cw = 0;
-                for (int b = 0; b < kPer / 2; ++b)
-                    if (e + 2 * b < numel) cw |= static_cast<uint32_t>(codes[(e >> 1) + b]) << (8 * b);
-            }
-            float w[kPer];
-#pragma unroll
-            for (int b = 0; b < kPer / 2; ++b) {
-                const uint32_t byte = (cw >> (8 * b)) & 0xffu;
-                w[2 * b] = __fmul_rn(sq[byte >> 4], scale);
-                w[2 * b + 1] = __fmul_rn(sq[byte & 15u], scale);
-            }
-            if (OUT_BF16) {
-                uint16_t* o = reinterpret_cast<uint16_t*>(out) + e;
-                if (full) {
-                    uint4 v;
-                    v.x = pack_bf16x2(w[0], w[1]);
-                    v.y = pack_bf16x2(w[2], w[3]);
-                    v.z = pack_bf16x2(w[4], w[5]);
-                    v.w = pack_bf16x2(w[6], w[7]);
-                    __stcs(reinterpret_cast<uint4*>(o), v);
-                } else {
-                    for (int t = 0; t < kPer; ++t)
-                        if (e + t < numel) o[t] = f32_to_bf16_bits(w[t]);
-                }
-            } else {
-                float* o = reinterpret_cast<float*>(out) + e;
-                if (full) {
-                    __stcs(reinterpret_cast<float4*>(o), make_float4(w[0], w[1], w[2], w[3]));
-                } else {
-                    for (int t = 0; t < kPer; ++t)
-                        if (e + t < numel) o[t] = w[t];
-                }
-            }
+        cw = ncw;
+        sb = nsb;
+        sc1 = ns1;
+    }
+    // ragged tail (< 32 weights), one thread
+    if (blockIdx.x == 0 && threadIdx.x == 0 && nfull * kRun < numel) {
+        for (int64_t e = nfull * kRun; e < numel; ++e) {
+            const uint8_t byte = codes[e >> 1];
+            const int code = (e & 1) ? (byte & 15) : (byte >> 4);
+            const float cp = dq_constant(c2_fp8[e >> 6], c1[e >> 14], mu);
+            const float v = __fmul_rn(s_lut[code], cp);
+            if (OUT_BF16)
+                reinterpret_cast<uint16_t*>(out)[e] = f32_to_bf16_bits(v);
+            else
+                reinterpret_cast<float*>(out)[e] = v;
         }
     }
 }
@@ -107,9 +119,9 @@ k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,
                               const float* mean, int64_t numel, void* out, int out_dtype,
                               cudaStream_t stream) {
-    const int64_t nwc = ceil_div(numel, kWarpElems);
-    const int64_t want = ceil_div(nwc, kThreads / 32);
-    const int grid = static_cast<int>(want < num_sms() * 8LL ? want : num_sms() * 8LL);
+    const int64_t runs = ceil_div(numel, kRun);
+    const int64_t want = ceil_div(runs, kThreads);
+    const int grid = static_cast<int>(want < num_sms() * 8LL ? (want > 0 ? want : 1) : num_sms() * 8LL);
     if (out_dtype == 1)
         k_dequant<true><<<grid, kThreads, 0, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables());
     else

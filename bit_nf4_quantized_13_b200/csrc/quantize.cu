@@ -29,6 +29,13 @@ struct EncTab {
     int base;
 };
 
+// Exact encoder entry per bin (see Nf4Tables::bnd): 16 bytes, one LDS.128.
+struct __align__(16) ExactTab {
+    int base;
+    int tie_up;
+    double bnd;
+};
+
 // Nearest NF4 code of n in [-1, 1] (exact fp32 nearest-value rule, ties to
 // the lower code): a 33-bin table built on the host gives the code at the
 // bin's lower end and the one threshold that may lie inside the bin.
@@ -40,6 +47,24 @@ __device__ __forceinline__ int nf4_code(float n, const EncTab* tab) {
     return e.base + (n >= e.thr ? 1 : 0);
 }
 
+__device__ __forceinline__ unsigned bin_of(float n) {
+    const unsigned b = (__float_as_uint(__fadd_rn(n, 3.0f)) >> 18) - 0x1000u;
+    return b > 32u ? 32u : b;
+}
+
+// The same code without the division: the bin is chosen from the
+// approximate quotient w * RN(1/a) (within 2^-23 of w/a, while every
+// threshold lies at least 1.6e-3 from a bin edge, so a neighbouring bin
+// gives the same code), and the one comparison that decides between two
+// codes, RN(w / a) >= thr, is made exactly as w against a * bnd in fp64.
+__device__ __forceinline__ int nf4_code_exact(float w, float y, double a64, const ExactTab* tab) {
+    const ExactTab e = tab[bin_of(__fmul_rn(w, y))];
+    const double p = a64 * e.bnd;  // exact: 24-bit a times a 25-bit boundary
+    const double wd = static_cast<double>(w);
+    const bool up = (wd > p) || (e.tie_up && wd == p);
+    return e.base + (up ? 1 : 0);
+}
+
 __device__ __forceinline__ float4 ld_stream(const float* p) {
     float4 v;
     asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
@@ -48,84 +73,126 @@ __device__ __forceinline__ float4 ld_stream(const float* p) {
     return v;
 }
 
-__device__ __forceinline__ bool finite4(const float4& v) {
-    return isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
+// max that propagates NaN, so one test per block catches NaN and Inf
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float d;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
 }
 
 constexpr int kQuantThreads = 256;
 constexpr int kChunk = 512;  // weights per warp step
+
+// One 64-block per 16 lanes: v holds this lane's 4 weights of the block.
+// Returns the lane's 4 codes packed as two bytes, and the block absmax.
+__device__ __forceinline__ uint32_t encode4(const float4& v, float& m_out, bool& bad, const ExactTab* xtab,
+                                            const EncTab* tab) {
+    float m = max_nan(max_nan(fabsf(v.x), fabsf(v.y)), max_nan(fabsf(v.z), fabsf(v.w)));
+    m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 8));
+    m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m_out = m;
+    int q0 = 7, q1 = 7, q2 = 7, q3 = 7;
+    if (!(m <= 3.402823466e38f)) {  // NaN or Inf in the block: flagged, codes unspecified
+        bad = true;
+    } else if (m > 0.0f) {
+        if (m >= 0x1p-120f && m <= 0x1p120f) {
+            const float y = __frcp_rn(m);
+            const double a64 = static_cast<double>(m);
+            q0 = nf4_code_exact(v.x, y, a64, xtab);
+            q1 = nf4_code_exact(v.y, y, a64, xtab);
+            q2 = nf4_code_exact(v.z, y, a64, xtab);
+            q3 = nf4_code_exact(v.w, y, a64, xtab);
+        } else {  // extreme block scales: divide exactly
+            q0 = nf4_code(__fdiv_rn(v.x, m), tab);
+            q1 = nf4_code(__fdiv_rn(v.y, m), tab);
+            q2 = nf4_code(__fdiv_rn(v.z, m), tab);
+            q3 = nf4_code(__fdiv_rn(v.w, m), tab);
+        }
+    }
+    // byte e/2 = (code e << 4) | code e+1, little-endian in the returned pair
+    return static_cast<uint32_t>((q0 << 4) | q1) | (static_cast<uint32_t>((q2 << 4) | q3) << 8);
+}
 
 __global__ void __launch_bounds__(kQuantThreads)
 k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__ codes,
                float* __restrict__ c2, unsigned long long* __restrict__ bins,
                int* __restrict__ flag, Nf4Tables tabs) {
     __shared__ EncTab tab[33];
+    __shared__ ExactTab xtab[33];
     __shared__ unsigned long long sbins[256];
     __shared__ int sbad;
     for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
-    if (threadIdx.x < 33) tab[threadIdx.x] = EncTab{tabs.thr[threadIdx.x], tabs.base[threadIdx.x]};
+    if (threadIdx.x < 33) {
+        tab[threadIdx.x] = EncTab{tabs.thr[threadIdx.x], tabs.base[threadIdx.x]};
+        xtab[threadIdx.x] = ExactTab{tabs.base[threadIdx.x], tabs.tie_up[threadIdx.x], tabs.bnd[threadIdx.x]};
+    }
     if (threadIdx.x == 0) sbad = 0;
     __syncthreads();
 
     const int lane = threadIdx.x & 31;
     const int64_t nb = ceil_div(numel, kBlock);
+    const int64_t nfull = numel / kChunk;  // whole 512-weight chunks
     const int64_t nchunks = ceil_div(numel, kChunk);
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     bool bad = false;
 
-    for (int64_t c = warp0; c < nchunks; c += nwarps) {
-        const int64_t base = c * kChunk;
-        const bool full = base + kChunk <= numel;
-        float4 v[4];
-        if (full) {
+    auto load_full = [&](int64_t c, float4 (&v)[4]) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[i] = ld_stream(W + base + 4 * (32 * i + lane));
-        } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int64_t e = base + 4 * (32 * i + lane);
-                v[i].x = e + 0 < numel ? W[e + 0] : 0.0f;
-                v[i].y = e + 1 < numel ? W[e + 1] : 0.0f;
-                v[i].z = e + 2 < numel ? W[e + 2] : 0.0f;
-                v[i].w = e + 3 < numel ? W[e + 3] : 0.0f;
+        for (int i = 0; i < 4; ++i) v[i] = ld_stream(W + c * kChunk + 4 * (32 * i + lane));
+    };
+    auto finish_block = [&](int64_t base, int i, float m) {
+        if ((lane & 15) == 0) {
+            const int64_t blk = (base >> 6) + 2 * i + (lane >> 4);
+            if (blk < nb) {
+                c2[blk] = m;
+                const uint32_t u = __float_as_uint(m);
+                const uint32_t ex = u >> 23;
+                const unsigned long long mant = ex ? ((u & 0x7fffffu) | 0x800000u) : (u & 0x7fffffu);
+                if (mant) atomicAdd(&sbins[ex & 255u], mant);
             }
         }
+    };
+
+    // whole chunks, loads for the next chunk in flight while this one encodes
+    int64_t c = warp0;
+    float4 cur[4], nxt[4];
+    if (c < nfull) load_full(c, cur);
+    for (; c < nfull; c += nwarps) {
+        const bool more = c + nwarps < nfull;
+        if (more) load_full(c + nwarps, nxt);
+        const int64_t base = c * kChunk;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            bad |= !finite4(v[i]);
-            float m = fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w)));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            int q0 = 7, q1 = 7, q2 = 7, q3 = 7;
-            if (m > 0.0f) {
-                q0 = nf4_code(__fdiv_rn(v[i].x, m), tab);
-                q1 = nf4_code(__fdiv_rn(v[i].y, m), tab);
-                q2 = nf4_code(__fdiv_rn(v[i].z, m), tab);
-                q3 = nf4_code(__fdiv_rn(v[i].w, m), tab);
-            }
-            const int64_t e = base + 4 * (32 * i + lane);  // first weight of this lane
-            // byte e/2 = (code e << 4) | code e+1; byte e/2+1 likewise
-            const uint32_t b01 = static_cast<uint32_t>((q0 << 4) | q1) |
-                                 (static_cast<uint32_t>((q2 << 4) | q3) << 8);
-            if (full) {
-                *reinterpret_cast<uint16_t*>(codes + (e >> 1)) = static_cast<uint16_t>(b01);
-            } else {
-                if (e < numel) codes[e >> 1] = static_cast<uint8_t>(e + 1 < numel ? (b01 & 0xff) : (b01 & 0xf0));
-                if (e + 2 < numel) codes[(e >> 1) + 1] = static_cast<uint8_t>(e + 3 < numel ? (b01 >> 8) : ((b01 >> 8) & 0xf0));
-            }
-            if ((lane & 15) == 0) {
-                const int64_t blk = (base >> 6) + 2 * i + (lane >> 4);
-                if (blk < nb) {
-                    c2[blk] = m;
-                    const uint32_t u = __float_as_uint(m);
-                    const uint32_t ex = u >> 23;
-                    const unsigned long long mant = ex ? ((u & 0x7fffffu) | 0x800000u) : (u & 0x7fffffu);
-                    if (mant) atomicAdd(&sbins[ex & 255u], mant);
-                }
-            }
+            float m;
+            const uint32_t b01 = encode4(cur[i], m, bad, xtab, tab);
+            const int64_t e = base + 4 * (32 * i + lane);
+            *reinterpret_cast<uint16_t*>(codes + (e >> 1)) = static_cast<uint16_t>(b01);
+            finish_block(base, i, m);
+        }
+        if (more) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
+        }
+    }
+    // the ragged last chunk (at most one), by the warp whose turn it is
+    if (nfull < nchunks && (nfull % nwarps) == warp0) {
+        const int64_t base = nfull * kChunk;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t e = base + 4 * (32 * i + lane);
+            float4 v;
+            v.x = e + 0 < numel ? W[e + 0] : 0.0f;
+            v.y = e + 1 < numel ? W[e + 1] : 0.0f;
+            v.z = e + 2 < numel ? W[e + 2] : 0.0f;
+            v.w = e + 3 < numel ? W[e + 3] : 0.0f;
+            float m;
+            const uint32_t b01 = encode4(v, m, bad, xtab, tab);
+            if (e < numel) codes[e >> 1] = static_cast<uint8_t>(e + 1 < numel ? (b01 & 0xff) : (b01 & 0xf0));
+            if (e + 2 < numel) codes[(e >> 1) + 1] = static_cast<uint8_t>(e + 3 < numel ? (b01 >> 8) : ((b01 >> 8) & 0xf0));
+            finish_block(base, i, m);
         }
     }
     if (bad) sbad = 1;
@@ -203,7 +270,7 @@ __device__ float mean_from_bins(const unsigned long long* __restrict__ bins, int
     return __shfl_sync(0xffffffffu, mu, 0);
 }
 
-constexpr int kDqThreads = 256;  // one thread per constant of a 256-group
+constexpr int kDqThreads = 256;  // 8 warps, one 256-group per warp at a time
 
 __global__ void __launch_bounds__(kDqThreads)
 k_double_quant(const float* __restrict__ c2, int64_t nb, const unsigned long long* __restrict__ bins,
@@ -211,10 +278,10 @@ k_double_quant(const float* __restrict__ c2, int64_t nb, const unsigned long lon
                float* __restrict__ mean_out, int32_t* __restrict__ status) {
     __shared__ unsigned long long sdig[kDigits];
     __shared__ float smu;
-    __shared__ float sred[kDqThreads / 32];
-    if (threadIdx.x < 32) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp == 0) {
         const float mu = mean_from_bins(bins, nb, sdig);
-        if (threadIdx.x == 0) smu = mu;
+        if (lane == 0) smu = mu;
     }
     __syncthreads();
     const float mu = smu;
@@ -223,22 +290,25 @@ k_double_quant(const float* __restrict__ c2, int64_t nb, const unsigned long lon
         if (status) *status = (*flag) ? QLORA_ERR_NONFINITE : QLORA_OK;
     }
     const int64_t ng = ceil_div(nb, kBlock2);
-    for (int64_t g = blockIdx.x; g < ng; g += gridDim.x) {
-        const int64_t j = g * kBlock2 + threadIdx.x;
-        const bool valid = j < nb;
-        const float y = valid ? __fsub_rn(c2[j], mu) : 0.0f;
-        float a = fabsf(y);
+    const int64_t wpb = kDqThreads / 32;
+    for (int64_t g = static_cast<int64_t>(blockIdx.x) * wpb + warp; g < ng; g += static_cast<int64_t>(gridDim.x) * wpb) {
+        float y[kBlock2 / 32];
+        float a = 0.0f;
+#pragma unroll
+        for (int i = 0; i < kBlock2 / 32; ++i) {
+            const int64_t j = g * kBlock2 + 32 * i + lane;
+            y[i] = j < nb ? __fsub_rn(c2[j], mu) : 0.0f;
+            a = fmaxf(a, fabsf(y[i]));
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-        if ((threadIdx.x & 31) == 0) sred[threadIdx.x >> 5] = a;
-        __syncthreads();
-        float amax = sred[0];
+        const float c = __fdiv_rn(a, 448.0f);
+        if (lane == 0) c1[g] = c;
 #pragma unroll
-        for (int w = 1; w < kDqThreads / 32; ++w) amax = fmaxf(amax, sred[w]);
-        __syncthreads();  // sred is reused by the next group
-        const float c = __fdiv_rn(amax, 448.0f);
-        if (threadIdx.x == 0) c1[g] = c;
-        if (valid) c2_fp8[j] = (c == 0.0f) ? static_cast<uint8_t>(0) : f32_to_e4m3(__fdiv_rn(y, c));
+        for (int i = 0; i < kBlock2 / 32; ++i) {
+            const int64_t j = g * kBlock2 + 32 * i + lane;
+            if (j < nb) c2_fp8[j] = (c == 0.0f) ? static_cast<uint8_t>(0) : f32_to_e4m3(__fdiv_rn(y[i], c));
+        }
     }
 }
 
@@ -261,13 +331,21 @@ cudaError_t launch_quantize_nf4_dq(const float* W, int64_t numel, uint8_t* codes
     if (err != cudaSuccess) return err;
     const int64_t nchunks = ceil_div(numel, kChunk);
     const int64_t want = ceil_div(nchunks, kQuantThreads / 32);
-    const int grid1 = static_cast<int>(want < num_sms() * 8LL ? want : num_sms() * 8LL);
+    static int resident = 0;  // CTAs of k_nf4_quantize per SM
+    if (!resident) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, k_nf4_quantize, kQuantThreads, 0) != cudaSuccess ||
+            resident < 1)
+            resident = 2;
+    }
+    const int64_t cap = static_cast<int64_t>(num_sms()) * resident;
+    const int grid1 = static_cast<int>(want < cap ? want : cap);
     k_nf4_quantize<<<grid1, kQuantThreads, 0, stream>>>(W, numel, codes, c2, bins, flag, tables());
     note_launches(1);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     const int64_t ng = ceil_div(nb, kBlock2);
-    const int grid2 = static_cast<int>(ng < num_sms() * 4LL ? ng : num_sms() * 4LL);
+    const int64_t want2 = ceil_div(ng, kDqThreads / 32);
+    const int grid2 = static_cast<int>(want2 < num_sms() * 4LL ? want2 : num_sms() * 4LL);
     k_double_quant<<<grid2, kDqThreads, 0, stream>>>(c2, nb, bins, flag, c2_fp8, c1, mean, status);
     note_launches(1);
     return cudaGetLastError();

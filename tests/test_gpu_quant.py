@@ -89,7 +89,10 @@ def test_encode_near_every_decision_boundary():
     qv = oracle.nf4_codebook().astype(np.float64)
     mids = (qv[1:] + qv[:-1]) / 2
     rows = []
-    for a in (1.0, 0.0731, 3.3e-5, 1.7e3, 2.0 ** -100, 1.0e30, 2.0 ** 126 * 1.5):
+    scales = [1.0, 0.0731, 3.3e-5, 1.7e3, 2.0 ** -100, 1.0e30, 2.0 ** 126 * 1.5, 2.0 ** -125, 2.0 ** -119.5,
+              2.0 ** 119.5, 2.0 ** 121]
+    scales += list(np.exp2(synth.rng(0, 4242).uniform(-118, 118, 24)))
+    for a in scales:
         for m in mids:
             c = np.float32(m * a)
             near = (c.view(np.uint32).astype(np.int64) + np.arange(-3, 4)).astype(np.uint32).view(np.float32)
