@@ -136,20 +136,6 @@ Nf4Tables build_tables() {
             // bins are 1/16 wide); keep the failure loud
             t.base[b] = -1000;
         }
-        // rounding boundary below the threshold: the midpoint between it and
-        // its fp32 predecessor; a quotient exactly on it rounds to the even
-        // neighbour, which is the threshold when the threshold's significand
-        // is even
-        t.bnd[b] = HUGE_VAL;
-        t.tie_up[b] = 0;
-        if (inside == 1) {
-            const float th = t.thr[b];
-            const float pr = nextafterf(th, -INFINITY);
-            t.bnd[b] = 0.5 * (static_cast<double>(pr) + static_cast<double>(th));
-            uint32_t u;
-            memcpy(&u, &th, 4);
-            t.tie_up[b] = (u & 1u) == 0 ? 1 : 0;
-        }
     }
     return t;
 }

@@ -24,13 +24,6 @@ struct Nf4Tables {
     // 0x1000 (33 bins).  code(n) = base[b] + (n >= thr[b]).
     float thr[33];
     int base[33];
-    // The same decision made on w and the block absmax a without forming
-    // n = RN(w / a): RN(w / a) >= thr[b] exactly when w > a * bnd[b], or
-    // w == a * bnd[b] and tie_up[b], where bnd[b] is the rounding boundary
-    // just below thr[b] (a 25-bit number, so a * bnd[b] is exact in fp64).
-    // bnd[b] = +inf where the bin holds no threshold.
-    double bnd[33];
-    int tie_up[33];
 };
 
 const Nf4Tables& tables();  // host: lazily built, immutable

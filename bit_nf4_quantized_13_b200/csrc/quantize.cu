@@ -29,13 +29,6 @@ struct EncTab {
     int base;
 };
 
-// Exact encoder entry per bin (see Nf4Tables::bnd): 16 bytes, one LDS.128.
-struct __align__(16) ExactTab {
-    int base;
-    int tie_up;
-    double bnd;
-};
-
 // Nearest NF4 code of n in [-1, 1] (exact fp32 nearest-value rule, ties to
 // the lower code): a 33-bin table built on the host gives the code at the
 // bin's lower end and the one threshold that may lie inside the bin.
@@ -47,22 +40,20 @@ __device__ __forceinline__ int nf4_code(float n, const EncTab* tab) {
     return e.base + (n >= e.thr ? 1 : 0);
 }
 
-__device__ __forceinline__ unsigned bin_of(float n) {
-    const unsigned b = (__float_as_uint(__fadd_rn(n, 3.0f)) >> 18) - 0x1000u;
-    return b > 32u ? 32u : b;
-}
-
-// The same code without the division: the bin is chosen from the
-// approximate quotient w * RN(1/a) (within 2^-23 of w/a, while every
-// threshold lies at least 1.6e-3 from a bin edge, so a neighbouring bin
-// gives the same code), and the one comparison that decides between two
-// codes, RN(w / a) >= thr, is made exactly as w against a * bnd in fp64.
-__device__ __forceinline__ int nf4_code_exact(float w, float y, double a64, const ExactTab* tab) {
-    const ExactTab e = tab[bin_of(__fmul_rn(w, y))];
-    const double p = a64 * e.bnd;  // exact: 24-bit a times a 25-bit boundary
-    const double wd = static_cast<double>(w);
-    const bool up = (wd > p) || (e.tie_up && wd == p);
-    return e.base + (up ? 1 : 0);
+// The same code without dividing in the common case.  With y = RN(1/a),
+// n~ = RN(w y) lies within 3 * 2^-24 of n = RN(w / a) (|n| <= 1).  The code
+// is a step function of n whose steps (thresholds) lie at least 1.6e-3
+// from the table's bin edges, so the bin of n~ serves n as well, and the one
+// threshold comparison agrees for n~ and n whenever n~ is more than 2^-21
+// from the threshold; only closer quotients (rare) take the exact division.
+__device__ __forceinline__ int nf4_code_fast(float w, float a, float y, const EncTab* tab) {
+    const float na = __fmul_rn(w, y);
+    const float v = __fadd_rn(na, 3.0f);
+    unsigned b = (__float_as_uint(v) >> 18) - 0x1000u;
+    b = b > 32u ? 32u : b;
+    const EncTab e = tab[b];
+    if (fabsf(__fsub_rn(na, e.thr)) > 0x1p-21f) return e.base + (na >= e.thr ? 1 : 0);
+    return e.base + (__fdiv_rn(w, a) >= e.thr ? 1 : 0);
 }
 
 __device__ __forceinline__ float4 ld_stream(const float* p) {
@@ -85,8 +76,7 @@ constexpr int kChunk = 512;  // weights per warp step
 
 // One 64-block per 16 lanes: v holds this lane's 4 weights of the block.
 // Returns the lane's 4 codes packed as two bytes, and the block absmax.
-__device__ __forceinline__ uint32_t encode4(const float4& v, float& m_out, bool& bad, const ExactTab* xtab,
-                                            const EncTab* tab) {
+__device__ __forceinline__ uint32_t encode4(const float4& v, float& m_out, bool& bad, const EncTab* tab) {
     float m = max_nan(max_nan(fabsf(v.x), fabsf(v.y)), max_nan(fabsf(v.z), fabsf(v.w)));
     m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 8));
     m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 4));
@@ -99,11 +89,10 @@ __device__ __forceinline__ uint32_t encode4(const float4& v, float& m_out, bool&
     } else if (m > 0.0f) {
         if (m >= 0x1p-120f && m <= 0x1p120f) {
             const float y = __frcp_rn(m);
-            const double a64 = static_cast<double>(m);
-            q0 = nf4_code_exact(v.x, y, a64, xtab);
-            q1 = nf4_code_exact(v.y, y, a64, xtab);
-            q2 = nf4_code_exact(v.z, y, a64, xtab);
-            q3 = nf4_code_exact(v.w, y, a64, xtab);
+            q0 = nf4_code_fast(v.x, m, y, tab);
+            q1 = nf4_code_fast(v.y, m, y, tab);
+            q2 = nf4_code_fast(v.z, m, y, tab);
+            q3 = nf4_code_fast(v.w, m, y, tab);
         } else {  // extreme block scales: divide exactly
             q0 = nf4_code(__fdiv_rn(v.x, m), tab);
             q1 = nf4_code(__fdiv_rn(v.y, m), tab);
@@ -120,13 +109,11 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
                float* __restrict__ c2, unsigned long long* __restrict__ bins,
                int* __restrict__ flag, Nf4Tables tabs) {
     __shared__ EncTab tab[33];
-    __shared__ ExactTab xtab[33];
     __shared__ unsigned long long sbins[256];
     __shared__ int sbad;
     for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
     if (threadIdx.x < 33) {
         tab[threadIdx.x] = EncTab{tabs.thr[threadIdx.x], tabs.base[threadIdx.x]};
-        xtab[threadIdx.x] = ExactTab{tabs.base[threadIdx.x], tabs.tie_up[threadIdx.x], tabs.bnd[threadIdx.x]};
     }
     if (threadIdx.x == 0) sbad = 0;
     __syncthreads();
@@ -167,7 +154,7 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             float m;
-            const uint32_t b01 = encode4(cur[i], m, bad, xtab, tab);
+            const uint32_t b01 = encode4(cur[i], m, bad, tab);
             const int64_t e = base + 4 * (32 * i + lane);
             *reinterpret_cast<uint16_t*>(codes + (e >> 1)) = static_cast<uint16_t>(b01);
             finish_block(base, i, m);
@@ -189,7 +176,7 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
             v.z = e + 2 < numel ? W[e + 2] : 0.0f;
             v.w = e + 3 < numel ? W[e + 3] : 0.0f;
             float m;
-            const uint32_t b01 = encode4(v, m, bad, xtab, tab);
+            const uint32_t b01 = encode4(v, m, bad, tab);
             if (e < numel) codes[e >> 1] = static_cast<uint8_t>(e + 1 < numel ? (b01 & 0xff) : (b01 & 0xf0));
             if (e + 2 < numel) codes[(e >> 1) + 1] = static_cast<uint8_t>(e + 3 < numel ? (b01 >> 8) : ((b01 >> 8) & 0xf0));
             finish_block(base, i, m);
