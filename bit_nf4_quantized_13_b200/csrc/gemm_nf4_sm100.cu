@@ -208,12 +208,9 @@ __device__ __forceinline__ void convert_run(const uint4& c0, const uint4& c1, fl
         for (int j = 0; j < 4; ++j) {
             const float a = lut_at(lut, __byte_perm(hi4, 0u, 0x4440u | j));
             const float b = lut_at(lut, __byte_perm(lo4, 0u, 0x4440u | j));
-            const float2 s2 = j == 0 ? make_float2(s01.x, s01.y)
-                            : j == 1 ? make_float2(s01.z, s01.w)
-                            : j == 2 ? make_float2(s23.x, s23.y)
-                                     : make_float2(s23.z, s23.w);
-            const float2 x = __fmul2_rn(make_float2(a, b), s2);
-            v[4 * h + j] = pack_bf16x2(x.x, x.y);
+            const float sa = j == 0 ? s01.x : j == 1 ? s01.z : j == 2 ? s23.x : s23.z;
+            const float sb = j == 0 ? s01.y : j == 1 ? s01.w : j == 2 ? s23.y : s23.w;
+            v[4 * h + j] = pack_bf16x2(__fmul_rn(a, sa), __fmul_rn(b, sb));
         }
     }
 }
@@ -284,12 +281,11 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
                         __syncwarp();
                     }
                     const float sc = kBwd ? 0.0f : dq_constant(static_cast<uint8_t>(sbyte[u]), sc1[u], mu);
+                    // rows beyond the weight hold finite garbage (zero codes times
+                    // the constant of empty inputs): their outputs are never
+                    // stored and rows do not mix in this product
                     convert_run<kBwd>(cb0[u], cb1[u], sc, wsc, lut, v);
                     if (kBwd) __syncwarp();  // wsc is rewritten by the warp's next stage
-                    if (!lane_ok) {
-#pragma unroll
-                        for (int t = 0; t < 32; ++t) v[t] = 0u;
-                    }
                 } else {  // LoRA slab: lane = row of B (forward) or of A^T (backward), r contiguous
                     const int j0 = (kb - P.kb_w) * kBK;
                     const uint16_t* lrow = p.lora + static_cast<int64_t>(grow) * p.r + j0;

@@ -29,31 +29,12 @@ struct EncTab {
     int base;
 };
 
-// Nearest NF4 code of n in [-1, 1] (exact fp32 nearest-value rule, ties to
-// the lower code): a 33-bin table built on the host gives the code at the
-// bin's lower end and the one threshold that may lie inside the bin.
-__device__ __forceinline__ int nf4_code(float n, const EncTab* tab) {
-    const float v = __fadd_rn(n, 3.0f);
-    unsigned b = (__float_as_uint(v) >> 18) - 0x1000u;
-    b = b > 32u ? 32u : b;  // NaN / out-of-range guard (status is flagged)
-    const EncTab e = tab[b];
-    return e.base + (n >= e.thr ? 1 : 0);
-}
-
-// The same code without dividing in the common case.  With y = RN(1/a),
-// n~ = RN(w y) lies within 3 * 2^-24 of n = RN(w / a) (|n| <= 1).  The code
-// is a step function of n whose steps (thresholds) lie at least 1.6e-3
-// from the table's bin edges, so the bin of n~ serves n as well, and the one
-// threshold comparison agrees for n~ and n whenever n~ is more than 2^-21
-// from the threshold; only closer quotients (rare) take the exact division.
-__device__ __forceinline__ int nf4_code_fast(float w, float a, float y, const EncTab* tab) {
-    const float na = __fmul_rn(w, y);
-    const float v = __fadd_rn(na, 3.0f);
-    unsigned b = (__float_as_uint(v) >> 18) - 0x1000u;
-    b = b > 32u ? 32u : b;
-    const EncTab e = tab[b];
-    if (fabsf(__fsub_rn(na, e.thr)) > 0x1p-21f) return e.base + (na >= e.thr ? 1 : 0);
-    return e.base + (__fdiv_rn(w, a) >= e.thr ? 1 : 0);
+// rcp.approx: within 2^-22 relative of 1/a for normal a (the PTX ISA
+// bounds its error by 1 ulp)
+__device__ __forceinline__ float rcp_approx(float a) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(a));
+    return y;
 }
 
 __device__ __forceinline__ float4 ld_stream(const float* p) {
@@ -76,6 +57,16 @@ constexpr int kChunk = 512;  // weights per warp step
 
 // One 64-block per 16 lanes: v holds this lane's 4 weights of the block.
 // Returns the lane's 4 codes packed as two bytes, and the block absmax.
+//
+// Codes without dividing in the common case: with y ~ 1/a (relative error
+// <= 2^-22), n~ = RN(w y) lies within 2^-21 of n = RN(w / a) for |n| <= 1.
+// The code is a step function of n whose steps (thresholds) lie at least
+// 1.6e-3 from the table's bin edges, so the bin of n~ serves n as well, and
+// the one threshold comparison agrees for n~ and n whenever n~ is more than
+// 2^-20 from the threshold.  A lane whose four quotients are all clear of
+// their thresholds is done; otherwise (rarely) it divides exactly.  The
+// table has one extra entry below -1 (index 0) because n~ may undershoot
+// -1 by a rounding, so finite inputs never need clamping.
 __device__ __forceinline__ uint32_t encode4(const float4& v, float& m_out, bool& bad, const EncTab* tab) {
     float m = max_nan(max_nan(fabsf(v.x), fabsf(v.y)), max_nan(fabsf(v.z), fabsf(v.w)));
     m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 8));
@@ -83,38 +74,50 @@ __device__ __forceinline__ uint32_t encode4(const float4& v, float& m_out, bool&
     m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
     m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
     m_out = m;
-    int q0 = 7, q1 = 7, q2 = 7, q3 = 7;
     if (!(m <= 3.402823466e38f)) {  // NaN or Inf in the block: flagged, codes unspecified
         bad = true;
-    } else if (m > 0.0f) {
-        if (m >= 0x1p-120f && m <= 0x1p120f) {
-            const float y = __frcp_rn(m);
-            q0 = nf4_code_fast(v.x, m, y, tab);
-            q1 = nf4_code_fast(v.y, m, y, tab);
-            q2 = nf4_code_fast(v.z, m, y, tab);
-            q3 = nf4_code_fast(v.w, m, y, tab);
-        } else {  // extreme block scales: divide exactly
-            q0 = nf4_code(__fdiv_rn(v.x, m), tab);
-            q1 = nf4_code(__fdiv_rn(v.y, m), tab);
-            q2 = nf4_code(__fdiv_rn(v.z, m), tab);
-            q3 = nf4_code(__fdiv_rn(v.w, m), tab);
+        return 0x7777u;
+    }
+    if (m == 0.0f) return 0x7777u;  // all-zero block: the zero code
+    const float w[4] = {v.x, v.y, v.z, v.w};
+    int q[4];
+    bool exact = !(m >= 0x1p-120f && m <= 0x1p120f);  // extreme scales: always divide
+    if (!exact) {
+        const float y = rcp_approx(m);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float na = __fmul_rn(w[i], y);
+            const unsigned b = (__float_as_uint(__fadd_rn(na, 3.0f)) >> 18) - 0xFFFu;
+            const EncTab e = tab[b];
+            q[i] = e.base + (na >= e.thr ? 1 : 0);
+            exact |= fabsf(__fsub_rn(na, e.thr)) <= 0x1p-20f;
+        }
+    }
+    if (exact) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float n = __fdiv_rn(w[i], m);
+            const unsigned b = (__float_as_uint(__fadd_rn(n, 3.0f)) >> 18) - 0xFFFu;
+            const EncTab e = tab[b > 33u ? 33u : b];
+            q[i] = e.base + (n >= e.thr ? 1 : 0);
         }
     }
     // byte e/2 = (code e << 4) | code e+1, little-endian in the returned pair
-    return static_cast<uint32_t>((q0 << 4) | q1) | (static_cast<uint32_t>((q2 << 4) | q3) << 8);
+    const uint32_t b0 = (static_cast<uint32_t>(q[0]) << 4) + static_cast<uint32_t>(q[1]);
+    const uint32_t b1 = (static_cast<uint32_t>(q[2]) << 4) + static_cast<uint32_t>(q[3]);
+    return (b1 << 8) + b0;
 }
 
 __global__ void __launch_bounds__(kQuantThreads)
 k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__ codes,
                float* __restrict__ c2, unsigned long long* __restrict__ bins,
                int* __restrict__ flag, Nf4Tables tabs) {
-    __shared__ EncTab tab[33];
+    __shared__ EncTab tab[34];  // [0]: below -1; [1 + b]: bin b of the host table
     __shared__ unsigned long long sbins[256];
     __shared__ int sbad;
     for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
-    if (threadIdx.x < 33) {
-        tab[threadIdx.x] = EncTab{tabs.thr[threadIdx.x], tabs.base[threadIdx.x]};
-    }
+    if (threadIdx.x < 33) tab[1 + threadIdx.x] = EncTab{tabs.thr[threadIdx.x], tabs.base[threadIdx.x]};
+    if (threadIdx.x == 33) tab[0] = EncTab{2.0f, 0};
     if (threadIdx.x == 0) sbad = 0;
     __syncthreads();
 
