@@ -332,10 +332,36 @@ def run_native(args, world, rank, local):
             dq_ms += e0.elapsed_time(e1)
             dq_bytes += dequant_bytes(b["case"].W.size, 2)
 
+    # unfused comparator: dequantize to a bf16 W in HBM, then library GEMMs
+    # (torch.matmul / cuBLAS) for the base product and the LoRA path
+    k9_ms = 0.0
+    k9_reps = max(3, args.steps // 4)
+    for rep in range(k9_reps + 2):
+        for b in bufs:
+            c = b["case"]
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            q.qlora_dequantize(b["wq"], torch.bfloat16, out=b["Wdq"])
+            yk = torch.matmul(b["X"], b["Wdq"].t())
+            tk = torch.matmul(b["X"], b["A"].t()).mul_(c.s)
+            yk.addmm_(tk, b["B"].t())
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 2:
+                k9_ms += e0.elapsed_time(e1)
+    k9_tflops = sum(fwd_flops(c.M, c.N, c.K, c.r) for c in cases) * k9_reps / (k9_ms * 1e-3) / 1e12
+
+    decode = run_decode(q, torch, dev, stream, flush, args) if rank == 0 and not args.no_decode else None
+
     peaks, peak_src = load_peaks()
     # the GEMM is timed in short bursts between L2 flushes: the burst peak
     tc_peak = peaks["bf16_tflops"]
     fwd_tflops = fflops / (ft * 1e-3) / 1e12
+    if decode:
+        for v in decode.values():
+            v["frac_hbm"] = v["gbs"] / peaks["hbm_gbs"]
+            v["graph_frac_hbm"] = v["graph_gbs"] / peaks["hbm_gbs"]
     roofline = {"kernel": "qlora_linear_fwd (T = X A^T, then the NF4-dequant GEMM with the LoRA slab)",
                 "bound": "tensor", "achieved": fwd_tflops, "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": fwd_tflops / tc_peak, "traffic": None, "peak_source": peak_src,
@@ -401,6 +427,8 @@ def run_native(args, world, rank, local):
                 "dequant_bf16_gbs": dq_bytes / (dq_ms * 1e-3) / 1e9 if dq_ms else None,
                 "dequant_bf16_frac_hbm": (dq_bytes / (dq_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]) if dq_ms else None,
                 "fwd_tflops": fwd_tflops, "bwd_tflops": bflops / (bt * 1e-3) / 1e12,
+                "unfused_fwd_tflops": k9_tflops,
+                "decode": decode,
                 "ms": {"quantize": qt / args.steps, "fwd": ft / args.steps, "bwd": bt / args.steps},
                 "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": tc_peak, "source": peak_src}},
             "clocks": clocks.summary(t_wall0, t_wall1),
@@ -414,6 +442,74 @@ def run_native(args, world, rank, local):
     return 0
 
 
+def decode_bytes(M, N, K, r):
+    """Algorithmic bytes of one small-batch forward: the quantized weight
+    (0.5 + 1/64 + 1/4096 B/param) plus X, A, B read and Y, T written."""
+    return N * K // 2 + N * K // 64 + -(-(N * K // 64) // 256) * 4 + 2 * (M * K + r * K + N * r + M * N + M * r)
+
+
+def run_decode(q, torch, dev, stream, flush, args):
+    """LLaMA-13B-shaped decode forward (W 5120x5120 and 13824x5120, M = 1,
+    4, 16 tokens, r = 16): per call device time with L2 flushed before
+    each call, launched directly and replayed from a CUDA graph."""
+    out = {}
+    reps = max(10, args.steps)
+    for which in range(2):
+        if args.decode_case and not args.decode_case.startswith(f"{synth.DECODE13B[which][1]}x"):
+            continue
+        base = synth.decode13b_linear(which, 16, seed=0)
+        W = torch.from_numpy(base.W).to(dev)
+        wq = q.qlora_quantize_nf4_dq(W)
+        del W
+        for M in (1, 4, 16):
+            if args.decode_case and not args.decode_case.endswith(f"_m{M}"):
+                continue
+            c = synth.decode13b_linear(which, M, seed=0) if M != 16 else base
+            X = torch.from_numpy(c.X.view(np.int16)).to(dev).view(torch.bfloat16)
+            A = torch.from_numpy(c.A.view(np.int16)).to(dev).view(torch.bfloat16)
+            B = torch.from_numpy(c.B.view(np.int16)).to(dev).view(torch.bfloat16)
+            Y = torch.empty((M, c.N), dtype=torch.bfloat16, device=dev)
+            T = torch.empty((M, c.r), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(q.qlora_linear_fwd_workspace_size(M, c.N, c.K, c.r), dtype=torch.uint8, device=dev)
+
+            def call():
+                q.qlora_linear_fwd(X, wq, A, B, c.s, Y=Y, T_save=T, ws=ws)
+
+            for _ in range(3):
+                call()
+            torch.cuda.synchronize()
+            direct = []
+            for _ in range(reps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                call()
+                e1.record(stream)
+                direct.append((e0, e1))
+            torch.cuda.synchronize()
+            ms = statistics.median(a.elapsed_time(b) for a, b in direct)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                call()
+            g.replay()
+            torch.cuda.synchronize()
+            graphed = []
+            for _ in range(reps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                graphed.append((e0, e1))
+            torch.cuda.synchronize()
+            gms = statistics.median(a.elapsed_time(b) for a, b in graphed)
+            del g
+            nbytes = decode_bytes(M, c.N, c.K, c.r)
+            out[f"{c.N}x{c.K}_m{M}"] = {"bytes": nbytes, "ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                                        "graph_ms": gms, "graph_gbs": nbytes / (gms * 1e-3) / 1e9}
+    return out
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -422,8 +518,26 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the small-batch forward (LLaMA-13B decode shapes) and print it")
+    ap.add_argument("--decode-case", default="", help="e.g. 13824x5120_m16: one decode configuration")
     args = ap.parse_args(argv)
     world, rank, local = dist_setup()
+    if args.decode_only:
+        import torch
+
+        import bit_nf4_quantized_13_b200 as q
+        dev = torch.device("cuda", local)
+        torch.cuda.set_device(dev)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        res = run_decode(q, torch, dev, torch.cuda.current_stream(), flush, args)
+        peaks, src = load_peaks()
+        for v in res.values():
+            v["frac_hbm"] = v["gbs"] / peaks["hbm_gbs"]
+            v["graph_frac_hbm"] = v["graph_gbs"] / peaks["hbm_gbs"]
+        print(json.dumps({"decode": res, "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": src}), flush=True)
+        return 0
     if args.impl == "reference":
         return run_reference(args, world, rank)
     return run_native(args, world, rank, local)

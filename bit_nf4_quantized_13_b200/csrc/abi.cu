@@ -154,6 +154,10 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + align256(static_cast<size_t>(M) * r * 2));
     cudaStream_t cs = as_stream(stream);
     Nf4Weight w{codes, c2_fp8, c1, mean, N, K};
+    if (gemv_supported(M, N, K, r)) {  // a few tokens: one stream over the weight
+        const cudaError_t g = launch_fwd_gemv(X, w, A, B, M, r, s, Y, T_save, cs);
+        if (g != cudaErrorNotSupported) return cuda_status(g);  // else: no cluster shape fits
+    }
     cudaError_t e = lora_xat(X, A, M, N, K, r, s, T, part, cs);
     if (e == cudaSuccess) e = launch_fwd_gemm(X, w, T, B, M, r, Y, cs);
     return cuda_status(e);
@@ -198,7 +202,8 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N
 int qlora_device_error(int reset) {
     const int a = gemm_device_error(reset);
     const int b = lora_device_error(reset);
-    return a != QLORA_OK ? a : b;
+    const int c = gemv_device_error(reset);
+    return a != QLORA_OK ? a : b != QLORA_OK ? b : c;
 }
 
 uint64_t qlora_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -1,0 +1,686 @@
+// gemv_sm100.cu -- the small-batch QLoRA forward (1 <= M <= 16 tokens):
+//
+//   T = bf16(s * X A^T)          (M x r)
+//   Y = bf16(X W'^T + T B^T)     (M x N)
+//
+// QLoRA study notes (gitcode.csdn.net), section 3.5, eq. (5) with the LoRA
+// scalar of section 4, eq. (3).  With a handful of tokens the product is a
+// stream over the NF4 weight (0.516 bytes per parameter), so the design
+// targets HBM bandwidth, not tensor throughput:
+//
+//  * Work unit: 16 consecutive weight rows over all of K.  Each CTA of a
+//    cluster of C CTAs copies its K-slice of the 16 rows (one tensor-map
+//    box) plus the rows' FP8 constants (one bulk copy) into a stage of a
+//    shared-memory ring (3 to 6 deep).  Few, large copies matter: issuing
+//    a copy costs the producer thread on the order of a hundred cycles.
+//  * Decode: a 256-entry table maps one code byte (two 4-bit codes) to the
+//    two bf16 codebook values as one 32-bit MMA operand register.  Each
+//    table entry is replicated across the 32 banks (lane l reads word l of
+//    a 256-byte row), so the lookups of a warp never conflict; the byte and
+//    the lane offset form the address in one byte permute.
+//  * Math: mma.m16n8k16 with the 16 weight rows as the A operand and up to
+//    8 tokens per B tile.  K inside each 64-block is permuted consistently
+//    in both operands so a lane's codes are 8 contiguous bytes per row.  The
+//    block constant c2' multiplies each block's 64-term partial product
+//    (the weight enters as bf16(q[code]) * c2' instead of
+//    bf16(RN(q[code] * c2')); both are one bf16 rounding from w').
+//  * X fragments stay in registers for the whole kernel: a warp always owns
+//    the same K-blocks of its CTA's slice.
+//  * Split-K across the cluster: each CTA reduces its warps' partials in
+//    shared memory, then CTA rank 0 sums the C partials in rank order
+//    (deterministic), adds T B^T with one more MMA per 16 ranks and stores
+//    Y.
+//  * T = bf16(s X A^T) is formed in the same kernel from the register
+//    resident X fragments (the rows of A take the MMA's A operand in the
+//    permuted k order), reduced over the cluster like the unit partials.
+//  * 15 decode warps per CTA run free of one another; a 16th warp issues
+//    the copies and sums their partials (named-barrier hand-off).  It pushes
+//    the CTA's partial into rank 0's shared memory with st.async (completing
+//    on an mbarrier); rank 0's producer warp finishes each unit one unit
+//    behind and hands the slot buffers (up to 4) back with remote arrives.
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+#include "tma_host.h"
+
+namespace qlora {
+namespace {
+
+using namespace sm100;
+
+__device__ int g_gemv_error;
+
+constexpr int kRows = 16;                    // weight rows per unit
+constexpr int kWarps = 15;                   // decode + MMA warps
+constexpr int kCompute = kWarps * 32;
+constexpr int kThreads = kCompute + 32;      // + the producer warp (16 warps: 128 registers a thread)
+constexpr int kMaxBw = 3;                    // 64-blocks per warp per unit
+constexpr int kMaxCtaBlocks = kWarps * kMaxBw;
+constexpr int kMaxCl = 8;                    // CTAs per cluster
+constexpr int kStages = 6;                   // most stages a launch uses
+constexpr int kSlotBufs = 4;                 // most units a CTA may run ahead of rank 0's epilogue
+constexpr int kLutBytes = 256 * 256;         // 256 entries x 64 words (32 used)
+constexpr int kMaxRankTiles = 4;             // r <= 64
+constexpr int kBRingMax = 8;                 // LoRA B tiles in flight ahead of the epilogue
+constexpr int kBRingBytes = 8192;            // ring size: kBRingMax tiles of 32 r bytes, at most
+constexpr int kTStride = 16 * kMaxRankTiles; // T staging row (ranks), bf16
+constexpr int kBarRedFull = 1;               // named barrier: partials written (compute warps arrive)
+constexpr int kBarRedFree = 2;               // named barrier: partials read (producer arrives)
+
+struct GemvParams {
+    const uint8_t* codes;
+    const uint8_t* c2_fp8;
+    const float* c1;
+    const float* mean;
+    const uint16_t* X;      // M x K
+    const uint16_t* A;      // r x K
+    const uint16_t* B;      // N x r
+    uint16_t* Y;            // M x N
+    uint16_t* T_save;       // M x r or null
+    int M, N, K, r;
+    float s;
+    int KB;                 // K / 64
+    int units;              // N / 16
+    int cl;                 // CTAs per cluster
+    int row_stride;         // bytes between rows of a stage
+    int stage_bytes;
+    int nstages;            // ring depth, <= kStages
+    int nslot;              // slot buffers: 2 or kSlotBufs
+    float q[16];
+};
+
+struct GemvSmem {
+    size_t red_off, slot_off, tslot_off, tbuf_off, bring_off, bar_off, total;
+};
+
+__host__ __device__ constexpr GemvSmem gemv_smem(int NT, int stage_bytes, int nstages, int cl, int rt, int nslot) {
+    GemvSmem m{};
+    m.red_off = kLutBytes + static_cast<size_t>(nstages) * stage_bytes;
+    m.slot_off = m.red_off + kWarps * NT * 32 * 16;
+    m.tslot_off = m.slot_off + static_cast<size_t>(nslot) * cl * NT * 32 * 16;
+    m.tbuf_off = m.tslot_off + static_cast<size_t>(cl) * rt * NT * 32 * 16;
+    m.bring_off = m.tbuf_off + 16 * kTStride * 2;
+    m.bar_off = m.bring_off + kBRingBytes;
+    m.total = m.bar_off + (kStages + 2 * kSlotBufs + 1 + kBRingMax) * 8;
+    return m;
+}
+
+// Two bf16 codebook values for one code byte: the lower half holds the even
+// element (high nibble), the upper half the odd one.
+__device__ __forceinline__ uint32_t lut_pair(const uint8_t* lut, uint32_t word, uint32_t lane_off, int byte) {
+    const uint32_t addr = __byte_perm(word, lane_off, 0x5504u | (static_cast<uint32_t>(byte) << 4));
+    return *reinterpret_cast<const uint32_t*>(lut + addr);
+}
+
+// Named-barrier hand-off between the compute warps and the producer warp;
+// the warp is reconverged first (the barriers are warp-aligned).
+__device__ __forceinline__ void bar_arrive(int id) {
+    __syncwarp();
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
+}
+__device__ __forceinline__ void bar_wait(int id) {
+    __syncwarp();
+    named_bar_sync(id, kThreads);
+}
+
+// Issues the copies of unit `u` into `stage`, completing on `bar`: one
+// tensor-map box of the codes (16 rows x row_stride bytes from block b0 on;
+// this CTA's blocks plus a few of the next slice, or zeros past the row,
+// which also pads the rows to a bank-friendly pitch) and one bulk copy of
+// the rows' FP8 constants.
+__device__ __forceinline__ void issue_unit(const CUtensorMap* map, const GemvParams& p, int u, uint8_t* stage,
+                                           uint64_t* bar, int b0) {
+    const uint32_t b = smem_u32(bar);
+    const uint32_t strip_bytes = static_cast<uint32_t>(kRows * p.KB);
+    mbar_arrive_expect_tx(b, kRows * p.row_stride + strip_bytes);
+    tma_load_2d(smem_u32(stage), map, b, b0 * 4, u * kRows);
+    bulk_load(smem_u32(stage + kRows * p.row_stride), p.c2_fp8 + static_cast<int64_t>(u) * kRows * p.KB,
+              strip_bytes, b);
+}
+
+// The 16 rows of B that unit `u` needs (rows 16u .. 16u+15, contiguous
+// 32 r bytes) into ring tile `tile`, completing on `bar`.
+__device__ __forceinline__ void issue_b_tile(const GemvParams& p, int u, uint8_t* tile, uint64_t* bar) {
+    const uint32_t bytes = static_cast<uint32_t>(kRows * p.r * 2);
+    mbar_arrive_expect_tx(smem_u32(bar), bytes);
+    bulk_load(smem_u32(tile), p.B + static_cast<int64_t>(u) * kRows * p.r, bytes, smem_u32(bar));
+}
+
+// Sum of the 15 compute warps' partials (fragment layout), warp order.
+template <int NT>
+__device__ __forceinline__ void sum_partials(const float4* red, int lane, float4 (&v)[NT]) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        float4 sum = red[nt * 32 + lane];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) {
+            const float4 x = red[(w * NT + nt) * 32 + lane];
+            sum.x += x.x; sum.y += x.y; sum.z += x.z; sum.w += x.w;
+        }
+        v[nt] = sum;
+    }
+}
+
+// The producer warp of every CTA: issues the stage copies, reduces the
+// compute warps' partials and pushes the CTA's partial of T and of every
+// unit into rank 0's shared memory (st.async).  In rank 0 it also runs the
+// epilogue, one unit behind: T = bf16(s * sum of the T partials in rank
+// order) once, then per unit the C partials summed in rank order, the slot
+// buffer handed back to every CTA, T B^T added with one MMA per 16 ranks
+// and Y stored.
+template <int NT>
+__device__ __forceinline__ void producer_warp(const CUtensorMap* map, const GemvParams& p, uint8_t* smem, const GemvSmem& L, uint64_t* full,
+                                              uint64_t* slot_full, uint64_t* slot_empty, uint64_t* t_full,
+                                              uint64_t* bfull, uint32_t crank, int cid, int ncl, int n_local,
+                                              int b0, int nblk, int lane) {
+    const int g = lane >> 2, qd = lane & 3;
+    const int RT = (p.r + 15) >> 4;
+    const int nst = p.nstages;
+    uint8_t* stages = smem + kLutBytes;
+    const float4* red = reinterpret_cast<const float4*>(smem + L.red_off);
+    const float4* slot = reinterpret_cast<const float4*>(smem + L.slot_off);
+    const float4* tslot = reinterpret_cast<const float4*>(smem + L.tslot_off);
+    uint16_t* tbuf = reinterpret_cast<uint16_t*>(smem + L.tbuf_off);  // [16 tokens][kTStride]
+    uint8_t* bring = smem + L.bring_off;
+    const uint32_t slot_bytes = static_cast<uint32_t>(p.cl) * NT * 32 * 16;
+    const int tile_bytes = kRows * p.r * 2;
+    int nring = kBRingBytes / tile_bytes;
+    nring = nring < kBRingMax ? nring : kBRingMax;
+    const bool rank0 = crank == 0;
+
+    if (lane == 0) {
+        const int pre = n_local < nst ? n_local : nst;
+        for (int i = 0; i < pre; ++i) issue_unit(map, p, cid + i * ncl, stages + i * p.stage_bytes, &full[i], b0);
+        if (rank0) {
+            mbar_arrive_expect_tx(smem_u32(t_full), static_cast<uint32_t>(p.cl) * RT * NT * 32 * 16);
+            for (int b = 0; b < p.nslot; ++b) mbar_arrive_expect_tx(smem_u32(&slot_full[b]), slot_bytes);
+            for (int u = 0; u < nring && u < n_local; ++u)
+                issue_b_tile(p, cid + u * ncl, bring + u * tile_bytes, &bfull[u]);
+        }
+    }
+    const uint32_t tslot_r0 = cluster_map(smem_u32(smem + L.tslot_off), 0);
+    const uint32_t t_full_r0 = cluster_map(smem_u32(t_full), 0);
+    const uint32_t slot_r0 = cluster_map(smem_u32(smem + L.slot_off), 0);
+    const uint32_t slot_full_r0 = cluster_map(smem_u32(slot_full), 0);
+
+    // this CTA's part of X A^T, one 16-rank tile per round
+    for (int rt = 0; rt < RT; ++rt) {
+        bar_wait(kBarRedFull);
+        float4 v[NT];
+        sum_partials<NT>(red, lane, v);
+        bar_arrive(kBarRedFree);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+            st_async_f4(tslot_r0 + static_cast<uint32_t>((((crank * RT + rt) * NT + nt) * 32 + lane) * 16), v[nt],
+                        t_full_r0);
+    }
+
+    uint32_t tf[NT][kMaxRankTiles][2];
+    bool t_ready = false;
+    auto finish = [&](int i) {
+        if (!t_ready) {  // T: lane holds (rank 16 rt + g (+8), token 8 nt + 2 qd (+1)) of every tile
+            mbar_wait(smem_u32(t_full), 0, &g_gemv_error);
+            for (int rt = 0; rt < RT; ++rt) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    float4 v = tslot[((0 * RT + rt) * NT + nt) * 32 + lane];
+                    for (int rk = 1; rk < p.cl; ++rk) {
+                        const float4 w = tslot[((rk * RT + rt) * NT + nt) * 32 + lane];
+                        v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+                    }
+                    const float e4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 16 * rt + g + 8 * (e >> 1);
+                        const int tok = 8 * nt + 2 * qd + (e & 1);
+                        const uint16_t tb = f32_to_bf16_bits(e4[e] * p.s);
+                        tbuf[tok * kTStride + j] = tb;
+                        if (p.T_save && cid == 0 && tok < p.M && j < p.r)
+                            p.T_save[static_cast<int64_t>(tok) * p.r + j] = tb;
+                    }
+                }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int st = 0; st < kMaxRankTiles; ++st)
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf)  // T as the B operand of the LoRA MMA: (k = rank, n = token)
+                        tf[nt][st][hf] = (16 * st < p.r) ? *reinterpret_cast<const uint32_t*>(
+                                                               &tbuf[(8 * nt + g) * kTStride + 16 * st + 2 * qd + 8 * hf])
+                                                         : 0u;
+            t_ready = true;
+        }
+        const int b = i % p.nslot, k = i / p.nslot, rb = i % nring;
+        const int n0 = (cid + i * ncl) * kRows;
+        mbar_wait(smem_u32(&slot_full[b]), k & 1, &g_gemv_error);
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float4 sum = slot[((b * p.cl + 0) * NT + nt) * 32 + lane];
+            for (int rk = 1; rk < p.cl; ++rk) {
+                const float4 v = slot[((b * p.cl + rk) * NT + nt) * 32 + lane];
+                sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+            }
+            acc[nt][0] = sum.x; acc[nt][1] = sum.y; acc[nt][2] = sum.z; acc[nt][3] = sum.w;
+        }
+        __syncwarp();
+        if (i + p.nslot < n_local) {  // the buffer's next use: arm it, then release it to every CTA
+            if (lane == 0) mbar_arrive_expect_tx(smem_u32(&slot_full[b]), slot_bytes);
+            __syncwarp();
+            if (lane < p.cl) mbar_arrive_cluster(cluster_map(smem_u32(&slot_empty[b]), lane));
+        }
+        mbar_wait(smem_u32(&bfull[rb]), (i / nring) & 1, &g_gemv_error);
+        const uint16_t* bt = reinterpret_cast<const uint16_t*>(bring + rb * tile_bytes);
+#pragma unroll
+        for (int st = 0; st < kMaxRankTiles; ++st) {
+            if (16 * st >= p.r) break;
+            uint32_t a[4];  // a0a1: row g, a2a3: row g+8, a4..a7: the same 8 ranks further
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const int j = 16 * st + 2 * qd + 8 * (h >> 1);
+                a[h] = j < p.r ? *reinterpret_cast<const uint32_t*>(bt + (g + 8 * (h & 1)) * p.r + j) : 0u;
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                mma_16816(acc[nt], a[0], a[1], a[2], a[3], tf[nt][st][0], tf[nt][st][1]);
+        }
+        __syncwarp();
+        if (lane == 0 && i + nring < n_local) {  // refill the tile just read
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue_b_tile(p, cid + (i + nring) * ncl, bring + rb * tile_bytes, &bfull[rb]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int tok = nt * 8 + 2 * qd + (e & 1);
+                const int row = n0 + g + 8 * (e >> 1);
+                if (tok < p.M) p.Y[static_cast<int64_t>(tok) * p.N + row] = f32_to_bf16_bits(acc[nt][e]);
+            }
+        }
+    };
+
+#pragma unroll 1
+    for (int i = 0; i < n_local; ++i) {
+        bar_wait(kBarRedFull);  // unit i's partials are written: its stage is free too
+        if (lane == 0 && i + nst < n_local)
+            issue_unit(map, p, cid + (i + nst) * ncl, stages + (i % nst) * p.stage_bytes, &full[i % nst], b0);
+        float4 v[NT];
+        sum_partials<NT>(red, lane, v);
+        bar_arrive(kBarRedFree);
+        const int b = i % p.nslot, k = i / p.nslot;
+        if (k >= 1) mbar_wait(smem_u32(&slot_empty[b]), (k - 1) & 1, &g_gemv_error);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+            st_async_f4(slot_r0 + static_cast<uint32_t>((((b * p.cl + crank) * NT + nt) * 32 + lane) * 16), v[nt],
+                        slot_full_r0 + static_cast<uint32_t>(b * 8));
+        if (rank0 && i >= 1) finish(i - 1);
+    }
+    if (rank0 && n_local > 0) finish(n_local - 1);
+}
+
+template <int NT>
+__device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem, const GemvSmem& L, uint64_t* full,
+                                             int cid, int ncl, int n_local, int b0, int nblk, int warp, int lane) {
+    const int g = lane >> 2, qd = lane & 3;
+    const int RT = (p.r + 15) >> 4;
+    const int nst = p.nstages;
+    const uint8_t* lut = smem;
+    const uint8_t* stages = smem + kLutBytes;
+    float4* red = reinterpret_cast<float4*>(smem + L.red_off) + warp * NT * 32;  // this warp's [NT][32]
+
+    // X fragments of this warp's blocks: block jloc = warp + kWarps * jj.
+    // Lane (g, qd) of token tile nt holds X[nt*8 + g][64*kb + 16*qd .. +16);
+    // inside a block, k is permuted alike in both MMA operands so that
+    // MMA t of the block takes the elements 4t .. 4t+3 of every lane's run.
+    uint32_t xf[kMaxBw][NT][8];
+#pragma unroll
+    for (int jj = 0; jj < kMaxBw; ++jj) {
+        const int jloc = warp + kWarps * jj;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int tok = nt * 8 + g;
+            uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+            if (jloc < nblk && tok < p.M) {
+                const uint4* src = reinterpret_cast<const uint4*>(
+                    p.X + static_cast<int64_t>(tok) * p.K + static_cast<int64_t>(b0 + jloc) * 64 + 16 * qd);
+                lo = __ldg(src);
+                hi = __ldg(src + 1);
+            }
+            xf[jj][nt][0] = lo.x; xf[jj][nt][1] = lo.y; xf[jj][nt][2] = lo.z; xf[jj][nt][3] = lo.w;
+            xf[jj][nt][4] = hi.x; xf[jj][nt][5] = hi.y; xf[jj][nt][6] = hi.z; xf[jj][nt][7] = hi.w;
+        }
+    }
+
+    // This CTA's part of X A^T, one 16-rank tile at a time: the rows of A
+    // are the MMA's A operand in the same permuted k order as the codes.
+    for (int rt = 0; rt < RT; ++rt) {
+        float ta[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) ta[nt][0] = ta[nt][1] = ta[nt][2] = ta[nt][3] = 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < kMaxBw; ++jj) {
+            const int jloc = warp + kWarps * jj;
+            if (jloc < nblk) {
+                uint4 ra[2][2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int j = 16 * rt + g + 8 * h;
+                    ra[h][0] = ra[h][1] = make_uint4(0, 0, 0, 0);
+                    if (j < p.r) {
+                        const uint4* src = reinterpret_cast<const uint4*>(
+                            p.A + static_cast<int64_t>(j) * p.K + static_cast<int64_t>(b0 + jloc) * 64 + 16 * qd);
+                        ra[h][0] = __ldg(src);
+                        ra[h][1] = __ldg(src + 1);
+                    }
+                }
+                const uint32_t wg[8] = {ra[0][0].x, ra[0][0].y, ra[0][0].z, ra[0][0].w,
+                                        ra[0][1].x, ra[0][1].y, ra[0][1].z, ra[0][1].w};
+                const uint32_t wh[8] = {ra[1][0].x, ra[1][0].y, ra[1][0].z, ra[1][0].w,
+                                        ra[1][1].x, ra[1][1].y, ra[1][1].z, ra[1][1].w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_16816(ta[nt], wg[2 * t], wh[2 * t], wg[2 * t + 1], wh[2 * t + 1], xf[jj][nt][2 * t],
+                                  xf[jj][nt][2 * t + 1]);
+            }
+        }
+        if (rt > 0) bar_wait(kBarRedFree);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) red[nt * 32 + lane] = make_float4(ta[nt][0], ta[nt][1], ta[nt][2], ta[nt][3]);
+        bar_arrive(kBarRedFull);
+    }
+
+    const float mean = __ldg(p.mean);
+    const uint32_t lane_off = static_cast<uint32_t>(lane) * 4;
+    // c1 of (row = lane, block jloc) of unit i, for lanes < 16
+    auto load_c1 = [&](int i, float (&c1v)[kMaxBw]) {
+#pragma unroll
+        for (int jj = 0; jj < kMaxBw; ++jj) {
+            const int jloc = warp + kWarps * jj;
+            c1v[jj] = 0.0f;
+            if (lane < kRows && jloc < nblk && i < n_local) {
+                const int64_t blk = (static_cast<int64_t>(cid + i * ncl) * kRows + lane) * p.KB + b0 + jloc;
+                c1v[jj] = __ldg(p.c1 + (blk >> 8));
+            }
+        }
+    };
+    float c1c[kMaxBw], c1n[kMaxBw];
+    load_c1(0, c1c);
+
+#pragma unroll 1
+    for (int i = 0; i < n_local; ++i) {
+        const int s = i % nst;
+        load_c1(i + 1, c1n);  // the next unit's: the loads overlap this unit
+        mbar_wait(smem_u32(&full[s]), (i / nst) & 1, &g_gemv_error);
+        const uint8_t* stg = stages + s * p.stage_bytes;
+        const uint8_t* strip = stg + kRows * p.row_stride;
+
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < kMaxBw; ++jj) {
+            const int jloc = warp + kWarps * jj;
+            if (jloc < nblk) {
+                const uint2 cg = *reinterpret_cast<const uint2*>(stg + g * p.row_stride + jloc * 32 + qd * 8);
+                const uint2 ch = *reinterpret_cast<const uint2*>(stg + (g + 8) * p.row_stride + jloc * 32 + qd * 8);
+                // block constants c2' of the 16 rows: lane r < 16 forms row r's, then shuffles
+                float c2v = 0.0f;
+                if (lane < kRows) c2v = dq_constant(strip[lane * p.KB + b0 + jloc], c1c[jj], mean);
+                const float sg = __shfl_sync(0xffffffffu, c2v, g);
+                const float sh = __shfl_sync(0xffffffffu, c2v, g + 8);
+                float bacc[NT][4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const uint32_t wg = t < 2 ? cg.x : cg.y, wh = t < 2 ? ch.x : ch.y;
+                    const int by = (t & 1) * 2;
+                    const uint32_t a0 = lut_pair(lut, wg, lane_off, by);
+                    const uint32_t a1 = lut_pair(lut, wh, lane_off, by);
+                    const uint32_t a2 = lut_pair(lut, wg, lane_off, by + 1);
+                    const uint32_t a3 = lut_pair(lut, wh, lane_off, by + 1);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        if (t == 0)
+                            mma_16816_zc(bacc[nt], a0, a1, a2, a3, xf[jj][nt][0], xf[jj][nt][1]);
+                        else
+                            mma_16816(bacc[nt], a0, a1, a2, a3, xf[jj][nt][2 * t], xf[jj][nt][2 * t + 1]);
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    acc[nt][0] = fmaf(bacc[nt][0], sg, acc[nt][0]);
+                    acc[nt][1] = fmaf(bacc[nt][1], sg, acc[nt][1]);
+                    acc[nt][2] = fmaf(bacc[nt][2], sh, acc[nt][2]);
+                    acc[nt][3] = fmaf(bacc[nt][3], sh, acc[nt][3]);
+                }
+            }
+        }
+#pragma unroll
+        for (int jj = 0; jj < kMaxBw; ++jj) c1c[jj] = c1n[jj];
+        bar_wait(kBarRedFree);  // the producer has read the previous partials
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) red[nt * 32 + lane] = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
+        bar_arrive(kBarRedFull);
+    }
+    bar_wait(kBarRedFree);  // pairs with the producer's last release
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1) k_gemv_nf4(const __grid_constant__ CUtensorMap map_codes,
+                                                           const __grid_constant__ GemvParams p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int RT = (p.r + 15) >> 4;
+    const GemvSmem L = gemv_smem(NT, p.stage_bytes, p.nstages, p.cl, RT, p.nslot);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+    uint64_t* slot_full = full + kStages;          // rank 0: a unit's partials have all landed
+    uint64_t* slot_empty = slot_full + kSlotBufs;  // every rank: rank 0 has read the buffer
+    uint64_t* t_full = slot_empty + kSlotBufs;     // rank 0: the T partials have all landed
+    uint64_t* bfull = t_full + 1;                  // rank 0: LoRA B tiles
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t crank = cluster_ctarank();
+    const int cid = static_cast<int>(cluster_id_x());
+    const int ncl = static_cast<int>(num_clusters_x());
+    const int b0 = static_cast<int>(static_cast<int64_t>(crank) * p.KB / p.cl);
+    const int nblk = static_cast<int>(static_cast<int64_t>(crank + 1) * p.KB / p.cl) - b0;
+    const int n_local = cid < p.units ? (p.units - 1 - cid) / ncl + 1 : 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < kStages + 2 * kSlotBufs + 1 + kBRingMax; ++i) mbar_init(smem_u32(&full[i]), 1);
+        fence_barrier_init();
+    }
+    if (tid < 256) {  // the decode table: entry v replicated into words 0..31 of row v
+        const uint32_t e = pack_bf16x2(p.q[tid >> 4], p.q[tid & 15]);
+        uint4* row = reinterpret_cast<uint4*>(smem + tid * 256);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) row[i] = make_uint4(e, e, e, e);
+    }
+    __syncthreads();
+    cluster_arrive();  // every CTA's barriers are initialised before any remote traffic
+    cluster_wait();
+
+    if (warp == kWarps)
+        producer_warp<NT>(&map_codes, p, smem, L, full, slot_full, slot_empty, t_full, bfull, crank, cid, ncl, n_local, b0, nblk,
+                          lane);
+    else
+        compute_warp<NT>(p, smem, L, full, cid, ncl, n_local, b0, nblk, warp, lane);
+    cluster_arrive();  // no CTA leaves while cluster peers may still address its shared memory
+    cluster_wait();
+}
+
+struct Plan {
+    int cl, clusters, row_stride, stage_bytes, nstages, nslot;
+    size_t smem;
+};
+
+// Largest number of co-resident clusters of `cl` CTAs with `smem` bytes of
+// shared memory each, cached per (device, tile count, cluster size, smem).
+template <int NT>
+int max_clusters(int cl, size_t smem) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, size_t>, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const auto key = std::make_tuple(dev, cl, smem);
+    std::lock_guard<std::mutex> lk(mu);
+    const auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    if (cudaFuncSetAttribute(k_gemv_nf4<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(cl * num_sms());
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_gemv_nf4<NT>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    cache[key] = n;
+    return n;
+}
+
+template <int NT>
+bool make_plan(int64_t N, int64_t K, int r, Plan& best) {
+    const int KB = static_cast<int>(K / 64);
+    const int units = static_cast<int>(N / kRows);
+    const int RT = (r + 15) / 16;
+    double best_eff = -1.0;
+    const int sms = num_sms();
+    for (int cl : {1, 2, 4, 8}) {
+        const int maxblk = static_cast<int>(ceil_div(KB, cl));
+        if (maxblk > kMaxCtaBlocks || KB < cl) continue;
+        Plan pl{};
+        pl.cl = cl;
+        pl.row_stride = static_cast<int>(round_up(maxblk * 32, 128) + 32);  // = 32 mod 128: no bank conflicts
+        if (pl.row_stride / 8 > 256) continue;                                 // tensor-map box width
+        pl.stage_bytes = static_cast<int>(round_up(kRows * pl.row_stride + round_up(kRows * KB, 128), 128));
+        pl.nstages = 0;
+        for (int nslot = kSlotBufs; nslot >= 2 && !pl.nstages; nslot /= 2) {
+            for (int ns = kStages; ns >= 3 && !pl.nstages; --ns)
+                if (gemv_smem(NT, pl.stage_bytes, ns, cl, RT, nslot).total <= 227 * 1024) pl.nstages = ns;
+            pl.nslot = nslot;
+        }
+        if (!pl.nstages) continue;
+        pl.smem = gemv_smem(NT, pl.stage_bytes, pl.nstages, cl, RT, pl.nslot).total;
+        const int maxc = max_clusters<NT>(cl, pl.smem);
+        if (maxc <= 0) continue;
+        pl.clusters = units < maxc ? units : maxc;
+        const int per = static_cast<int>(ceil_div(units, pl.clusters));
+        const double eff = static_cast<double>(units) / (static_cast<double>(pl.clusters) * per) *
+                           (static_cast<double>(pl.clusters) * cl / sms);
+        if (eff > best_eff + 0.01) {
+            best_eff = eff;
+            best = pl;
+        }
+    }
+    return best_eff > 0.0;
+}
+
+// The codes as a row-major [N][K/16] array of 64-bit words; boxes of
+// row_stride / 8 words x 16 rows, zero fill past the end of a row.
+bool make_codes_map(CUtensorMap* m, const GemvParams& p) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.K / 16), static_cast<cuuint64_t>(p.N)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.K / 2)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(p.row_stride / 8), static_cast<cuuint32_t>(kRows)};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t*>(p.codes), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NT>
+cudaError_t launch_gemv(const GemvParams& p, const Plan& pl, cudaStream_t st) {
+    CUtensorMap map;
+    if (!make_codes_map(&map, p)) return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(k_gemv_nf4<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(pl.smem));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(pl.cl * pl.clusters);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_gemv_nf4<NT>, map, p);
+    note_launches(1);
+    return e;
+}
+
+}  // namespace
+
+bool gemv_supported(int64_t M, int64_t N, int64_t K, int r) {
+    return M >= 1 && M <= 16 && N >= kRows && N % kRows == 0 && K >= 64 && K % 64 == 0 &&
+           K / 64 <= kMaxCl * kMaxCtaBlocks && N / kRows < (int64_t(1) << 30) && r >= 8 && r % 8 == 0 &&
+           r <= 16 * kMaxRankTiles;
+}
+
+cudaError_t launch_fwd_gemv(const uint16_t* X, const Nf4Weight& w, const uint16_t* A, const uint16_t* B, int64_t M,
+                            int r, float s, uint16_t* Y, uint16_t* T_save, cudaStream_t st) {
+    const bool two = M > 8;
+    Plan pl{};
+    if (!(two ? make_plan<2>(w.N, w.K, r, pl) : make_plan<1>(w.N, w.K, r, pl))) return cudaErrorNotSupported;
+    GemvParams p{};
+    p.codes = w.codes;
+    p.c2_fp8 = w.c2_fp8;
+    p.c1 = w.c1;
+    p.mean = w.mean;
+    p.X = X;
+    p.A = A;
+    p.B = B;
+    p.Y = Y;
+    p.T_save = T_save;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(w.N);
+    p.K = static_cast<int>(w.K);
+    p.r = r;
+    p.s = s;
+    p.KB = static_cast<int>(w.K / 64);
+    p.units = static_cast<int>(w.N / kRows);
+    p.cl = pl.cl;
+    p.row_stride = pl.row_stride;
+    p.stage_bytes = pl.stage_bytes;
+    p.nstages = pl.nstages;
+    p.nslot = pl.nslot;
+    const float* q = tables().q;
+    for (int i = 0; i < 16; ++i) p.q[i] = q[i];
+    return two ? launch_gemv<2>(p, pl, st) : launch_gemv<1>(p, pl, st);
+}
+
+int gemv_device_error(int reset) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_gemv_error, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (reset && v) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_gemv_error, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    }
+    return v;
+}
+
+}  // namespace qlora

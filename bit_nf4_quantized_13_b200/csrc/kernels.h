@@ -73,6 +73,15 @@ size_t dx_tc_workspace(const Nf4Weight& w, int r);
 cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U, const uint16_t* A,
                                   int64_t M, int r, uint16_t* dX, void* ws, cudaStream_t stream);
 
+// gemv_sm100.cu -- the small-batch forward (1 <= M <= 16): T and Y in one
+// kernel that streams the weight once; T is written to T_save when it is not
+// null.  Returns cudaErrorNotSupported (nothing launched) when no cluster
+// shape fits the device.
+bool gemv_supported(int64_t M, int64_t N, int64_t K, int r);
+cudaError_t launch_fwd_gemv(const uint16_t* X, const Nf4Weight& w, const uint16_t* A, const uint16_t* B, int64_t M,
+                            int r, float s, uint16_t* Y, uint16_t* T_save, cudaStream_t stream);
+int gemv_device_error(int reset);
+
 // gemm_*.cu -- the frozen-weight GEMMs with the LoRA slab fused in
 //   Y  = bf16(X W'^T + T B^T)      (M x N)
 //   dX = bf16(dY W' + U A)         (M x K)

@@ -154,6 +154,12 @@ size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r);
  * where W' = bf16 of the double-dequantized weight (eq. 6).  W is given by
  * the four buffers of qlora_quantize_nf4_dq for an N x K row-major weight.
  * Requires K % 64 == 0, 1 <= r <= 256, M >= 0, N >= 1.
+ * Small batches (1 <= M <= 16 with N % 16 == 0, 8 <= r <= 64, r % 8 == 0,
+ * K <= 23040) take a single weight-streaming kernel that applies each
+ * 64-block's constant c2' to the block's partial dot product, i.e. the
+ * weight enters as bf16(q[code]) * c2' rather than bf16(q[code] * c2'):
+ * the same value up to one bf16 rounding, within the forward's tolerance.
+ * That path uses no workspace and computes T itself.
  */
 int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                      const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,

@@ -134,3 +134,12 @@ LLAMA65B_LAYER = [("q", 8192, 8192), ("k", 8192, 8192), ("v", 8192, 8192), ("o",
                   ("gate", 22016, 8192), ("up", 22016, 8192), ("down", 8192, 22016)]
 
 DECODE13B = [("w5120x5120", 5120, 5120), ("w13824x5120", 13824, 5120)]
+
+
+def decode13b_linear(which: int, M: int, seed: int = 0) -> LinearCase:
+    """LLaMA-13B-shaped decode linear: W 5120x5120 or 13824x5120 ~N(0,0.02)
+    without outliers; X M x 5120 (M in 1, 4, 16) ~N(0,1) bf16; r=16,
+    alpha=16 (s=1); forward only."""
+    name, N, K = DECODE13B[which]
+    return linear_case(f"decode13b_{name}_m{M}_r16", M, N, K, 16, 16.0, seed, wid=2 + which,
+                       with_dy=False)

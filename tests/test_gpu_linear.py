@@ -122,3 +122,22 @@ def test_llama7b_shapes_sampled_rows(which):
     case = synth.llama7b_linear(which, seed=0)
     rows = np.sort(synth.rng(0, 99 + which).choice(case.M, 64, replace=False)).astype(np.int64)
     _run_case(case, rows=rows)
+
+
+def test_unfused_library_path_agrees():
+    """Second opinion: dequantize to bf16 with the library, then torch.matmul
+    (cuBLAS) for X W'^T + (s X A^T) B^T and dY W' + (s dY B) A; the fused
+    kernels agree within the same tolerance."""
+    case = synth.linear_case("k9", 512, 1536, 2048, 64, 16.0, seed=11, outlier_frac=0.001)
+    wq = q.qlora_quantize_nf4_dq(dev_f32(case.W))
+    X, A, B, dY = dev_bf16(case.X), dev_bf16(case.A), dev_bf16(case.B), dev_bf16(case.dY)
+    Y, T = q.qlora_linear_fwd(X, wq, A, B, case.s)
+    dX, _, _ = q.qlora_linear_bwd(dY, X, wq, A, B, case.s, T=T)
+    Wd = q.qlora_dequantize(wq, torch.bfloat16).view(case.N, case.K)
+    Tk = (X.float() @ A.float().t() * case.s).bfloat16()
+    Yk = X.float() @ Wd.float().t() + Tk.float() @ B.float().t()
+    Uk = (dY.float() @ B.float() * case.s).bfloat16()
+    dXk = dY.float() @ Wd.float() + Uk.float() @ A.float()
+    torch.cuda.synchronize()
+    check_close(host_f64(Y), Yk.double().cpu().numpy(), "Y vs unfused")
+    check_close(host_f64(dX), dXk.double().cpu().numpy(), "dX vs unfused")
