@@ -39,6 +39,10 @@ WORKLOAD = "llama7b_linears_w4096x4096_w11008x4096_m4096_r64_alpha16_quantize_fw
 M_TOKENS, RANK, ALPHA = 4096, 64, 16.0
 L2_FLUSH_BYTES = 256 << 20
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) per call of the dX path (k_prep_bwd + k_nf4_gemm_tc<1>), mean over
+# the two linears, from one ncu capture of the kernels as they are now (profiles/); None when
+# the kernels have changed since that capture.
+DX_TRAFFIC_BYTES = None
 
 
 def linear_flops(M, N, K, r):
@@ -74,7 +78,7 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int, interval_ms: int = 50):
+    def __init__(self, device_index: int, interval_ms: int = 10):
         self.lines = []
         self.proc = None
         try:
@@ -332,6 +336,28 @@ def run_native(args, world, rank, local):
             dq_ms += e0.elapsed_time(e1)
             dq_bytes += dequant_bytes(b["case"].W.size, 2)
 
+    # the dominant kernel: the backward's dX path (the transposed-weight prep
+    # and the NF4 GEMM dX = dY W' + U A), timed live as the backward with dX
+    # minus the backward without it, per call, L2 flushed before each
+    dx_ms, dx_flops, dx_reps = 0.0, 0.0, max(5, args.steps // 4)
+    for rep in range(dx_reps + 2):
+        for b in bufs:
+            c = b["case"]
+            tt = []
+            for want in (True, False):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                q.qlora_linear_bwd(b["dY"], b["X"], b["wq"], b["A"], b["B"], c.s, T=b["T"],
+                                   dX=b["dX"] if want else None, dA=b["dA"], dB=b["dB"], ws=b["bws"],
+                                   want_dx=want)
+                e1.record(stream)
+                tt.append((e0, e1))
+            torch.cuda.synchronize()
+            if rep >= 2:
+                dx_ms += tt[0][0].elapsed_time(tt[0][1]) - tt[1][0].elapsed_time(tt[1][1])
+                dx_flops += 2.0 * c.M * c.N * c.K + 2.0 * c.M * c.r * c.K
+
     # unfused comparator: dequantize to a bf16 W in HBM, then library GEMMs
     # (torch.matmul / cuBLAS) for the base product and the LoRA path
     k9_ms = 0.0
@@ -362,10 +388,14 @@ def run_native(args, world, rank, local):
         for v in decode.values():
             v["frac_hbm"] = v["gbs"] / peaks["hbm_gbs"]
             v["graph_frac_hbm"] = v["graph_gbs"] / peaks["hbm_gbs"]
-    roofline = {"kernel": "qlora_linear_fwd (T = X A^T, then the NF4-dequant GEMM with the LoRA slab)",
-                "bound": "tensor", "achieved": fwd_tflops, "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": fwd_tflops / tc_peak, "traffic": None, "peak_source": peak_src,
-                "algorithmic": "2MNK + 2Mr(N+K) per launch"}
+    dx_tflops = dx_flops / (dx_ms * 1e-3) / 1e12
+    roofline = {"kernel": "k_nf4_gemm_tc<1> with k_prep_bwd: dX = dY W'^T' + U A of qlora_linear_bwd "
+                          "(largest share of the step in the ncu launch list)",
+                "bound": "tensor", "achieved": dx_tflops, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": dx_tflops / tc_peak, "traffic": DX_TRAFFIC_BYTES, "peak_source": peak_src,
+                "algorithmic": "2MNK + 2MrK per call (both linears, M=4096, r=64)",
+                "timing": "per call: backward with dX minus backward without dX, CUDA events, L2 flushed",
+                "peak_kind": "burst (clocks stay at max in the timed region)"}
 
     # end to end through the C ABI with host buffers: H2D of the step's
     # inputs from pinned memory, the step, D2H of its outputs
@@ -426,7 +456,8 @@ def run_native(args, world, rank, local):
                 "quantize_frac_hbm": qbytes / (qt * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "dequant_bf16_gbs": dq_bytes / (dq_ms * 1e-3) / 1e9 if dq_ms else None,
                 "dequant_bf16_frac_hbm": (dq_bytes / (dq_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]) if dq_ms else None,
-                "fwd_tflops": fwd_tflops, "bwd_tflops": bflops / (bt * 1e-3) / 1e12,
+                "fwd_tflops": fwd_tflops, "fwd_frac_tensor": fwd_tflops / tc_peak,
+                "bwd_tflops": bflops / (bt * 1e-3) / 1e12, "dx_path_tflops": dx_tflops,
                 "unfused_fwd_tflops": k9_tflops,
                 "decode": decode,
                 "ms": {"quantize": qt / args.steps, "fwd": ft / args.steps, "bwd": bt / args.steps},
@@ -513,7 +544,7 @@ def run_decode(q, torch, dev, stream, flush, args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-e2e", action="store_true")
