@@ -43,23 +43,23 @@ cudaError_t launch_bwd_dx_gemm(const uint16_t* dY, const Nf4Weight& w, const uin
 // The rank-r products: tensor cores where the shapes allow TMA (r % 8 == 0,
 // N % 8 == 0), CUDA cores otherwise.
 cudaError_t lora_xat(const uint16_t* X, const uint16_t* A, int64_t M, int64_t N, int64_t K, int r, float s,
-                     uint16_t* T, float* part, cudaStream_t st) {
-    if (lora_tc_supported(M, N, K, r)) return launch_lora_xat_tc(X, A, M, K, r, s, T, part, st);
+                     uint16_t* T, cudaStream_t st) {
+    if (lora_tc_supported(M, N, K, r)) return launch_lora_xat_tc(X, A, M, K, r, s, T, st);
     return launch_lora_xat_simt(X, A, M, K, r, s, T, st);
 }
 
 cudaError_t lora_dyb(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t N, int64_t K, int r, float s,
-                     uint16_t* U, float* part, cudaStream_t st) {
-    if (lora_tc_supported(M, N, K, r)) return launch_lora_dyb_tc(dY, B, M, N, r, s, U, part, st);
+                     uint16_t* U, cudaStream_t st) {
+    if (lora_tc_supported(M, N, K, r)) return launch_lora_dyb_tc(dY, B, M, N, r, s, U, st);
     return launch_lora_dyb_simt(dY, B, M, N, r, s, U, st);
 }
 
 cudaError_t lora_grads(const uint16_t* dY, const uint16_t* X, const uint16_t* T, const uint16_t* U, int64_t M,
-                       int64_t N, int64_t K, int r, uint16_t* dA, uint16_t* dB, float* part, cudaStream_t st) {
+                       int64_t N, int64_t K, int r, uint16_t* dA, uint16_t* dB, cudaStream_t st) {
     if (!lora_tc_supported(M, N, K, r)) return launch_lora_grads_simt(dY, X, T, U, M, N, K, r, dA, dB, st);
-    cudaError_t e = launch_lora_da_tc(X, U, M, K, r, dA, part, st);
+    cudaError_t e = launch_lora_da_tc(X, U, M, K, r, dA, st);
     if (e != cudaSuccess) return e;
-    return launch_lora_db_tc(dY, T, M, N, r, dB, part, st);
+    return launch_lora_db_tc(dY, T, M, N, r, dB, st);
 }
 
 }  // namespace qlora
@@ -126,16 +126,16 @@ int qlora_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c
 
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
     if (check_linear(M, N, K, r) != QLORA_OK) return 0;
-    // T (used when T_save is NULL), then the split-K partials of the rank-r products
-    return align256(static_cast<size_t>(M) * r * 2) + align256(lora_tc_workspace(M, N, K, r));
+    // T (used when T_save is NULL)
+    return align256(static_cast<size_t>(M) * r * 2);
 }
 
 size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
     if (check_linear(M, N, K, r) != QLORA_OK) return 0;
     const size_t mr = align256(static_cast<size_t>(M) * r * 2);
-    // U, T (when T is NULL), the rank-r partials, the transposed weight of the dX GEMM
+    // U, T (when T is NULL), the transposed weight of the dX GEMM
     Nf4Weight w{nullptr, nullptr, nullptr, nullptr, N, K};
-    return 2 * mr + align256(lora_tc_workspace(M, N, K, r)) + align256(dx_tc_workspace(w, r));
+    return 2 * mr + align256(dx_tc_workspace(w, r));
 }
 
 int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
@@ -151,14 +151,13 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     if (!ws || !aligned16(ws) || ws_bytes < qlora_linear_fwd_workspace_size(M, N, K, r))
         return QLORA_ERR_WORKSPACE;
     uint16_t* T = T_save ? T_save : reinterpret_cast<uint16_t*>(ws);
-    float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + align256(static_cast<size_t>(M) * r * 2));
     cudaStream_t cs = as_stream(stream);
     Nf4Weight w{codes, c2_fp8, c1, mean, N, K};
     if (gemv_supported(M, N, K, r)) {  // a few tokens: one stream over the weight
         const cudaError_t g = launch_fwd_gemv(X, w, A, B, M, r, s, Y, T_save, cs);
         if (g != cudaErrorNotSupported) return cuda_status(g);  // else: no cluster shape fits
     }
-    cudaError_t e = lora_xat(X, A, M, N, K, r, s, T, part, cs);
+    cudaError_t e = lora_xat(X, A, M, N, K, r, s, T, cs);
     if (e == cudaSuccess) e = launch_fwd_gemm(X, w, T, B, M, r, Y, cs);
     return cuda_status(e);
 }
@@ -185,17 +184,16 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N
     const size_t mr = align256(static_cast<size_t>(M) * r * 2);
     uint16_t* U = reinterpret_cast<uint16_t*>(ws);
     uint16_t* Tw = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + mr);
-    float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 2 * mr);
     Nf4Weight w{codes, c2_fp8, c1, mean, N, K};
-    void* dxws = reinterpret_cast<char*>(ws) + 2 * mr + align256(lora_tc_workspace(M, N, K, r));
+    void* dxws = reinterpret_cast<char*>(ws) + 2 * mr;
     cudaError_t e = cudaSuccess;
     if (!T) {
-        e = lora_xat(X, A, M, N, K, r, s, Tw, part, cs);
+        e = lora_xat(X, A, M, N, K, r, s, Tw, cs);
         T = Tw;
     }
-    if (e == cudaSuccess) e = lora_dyb(dY, B, M, N, K, r, s, U, part, cs);
+    if (e == cudaSuccess) e = lora_dyb(dY, B, M, N, K, r, s, U, cs);
     if (e == cudaSuccess && dX) e = launch_bwd_dx_gemm(dY, w, U, A, M, r, dX, dxws, cs);
-    if (e == cudaSuccess) e = lora_grads(dY, X, T, U, M, N, K, r, dA, dB, part, cs);
+    if (e == cudaSuccess) e = lora_grads(dY, X, T, U, M, N, K, r, dA, dB, cs);
     return cuda_status(e);
 }
 

@@ -33,17 +33,17 @@ struct Nf4Weight {
 //   U  = bf16(s * dY B)    (M x r)
 //   dA = bf16(U^T X)       (r x K)
 //   dB = bf16(dY^T T)      (N x r)
-// lora_sm100.cu: tensor-core versions (fp32 split-K partials in `part`)
+// lora_sm100.cu: tensor-core versions (split-K over a thread-block cluster,
+// reduced in distributed shared memory: no workspace)
 bool lora_tc_supported(int64_t M, int64_t N, int64_t K, int r);
-size_t lora_tc_workspace(int64_t M, int64_t N, int64_t K, int r);
 cudaError_t launch_lora_xat_tc(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, float s,
-                               uint16_t* T, float* part, cudaStream_t stream);
+                               uint16_t* T, cudaStream_t stream);
 cudaError_t launch_lora_dyb_tc(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t N, int r, float s,
-                               uint16_t* U, float* part, cudaStream_t stream);
+                               uint16_t* U, cudaStream_t stream);
 cudaError_t launch_lora_da_tc(const uint16_t* X, const uint16_t* U, int64_t M, int64_t K, int r, uint16_t* dA,
-                              float* part, cudaStream_t stream);
+                              cudaStream_t stream);
 cudaError_t launch_lora_db_tc(const uint16_t* dY, const uint16_t* T, int64_t M, int64_t N, int r, uint16_t* dB,
-                              float* part, cudaStream_t stream);
+                              cudaStream_t stream);
 int lora_device_error(int reset);
 int gemm_device_error(int reset);  // gemm_nf4_sm100.cu
 // gemm_simt.cu: CUDA-core versions (any shape)

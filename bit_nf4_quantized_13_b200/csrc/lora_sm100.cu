@@ -11,13 +11,16 @@
 // operands are row-major bf16 matrices read either along their contiguous
 // dimension (K-major) or across it (MN-major); TMA loads both in the
 // 128-byte swizzled layout and tcgen05.mma takes either major-ness.  The
-// outputs have only r columns, so the contraction is split across CTAs
-// (split-K) to fill the GPU; each split writes fp32 partials that a second
-// kernel sums in a fixed order (deterministic), scales and rounds to bf16.
+// outputs have only r columns, so the contraction is split across the S
+// CTAs (S = 1..8, a power of two) of a thread-block cluster to fill the GPU.
 //
 // One CTA = one 128-row tile x one contraction split: warp 0 issues TMA,
 // warp 1 the MMAs (M = 128, N = r rounded up to 16), then all four warps
-// read the accumulator from tensor memory and store the partials.
+// copy the fp32 accumulator from tensor memory into the CTA's shared
+// memory.  After a cluster barrier, rank c sums rows [c 128/S, (c+1) 128/S)
+// of the tile over the S CTAs in rank order (distributed shared memory;
+// deterministic), scales, rounds to bf16 and stores them: no partials in
+// HBM and no second kernel.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -43,11 +46,14 @@ constexpr int kABytes = kRows * kBK * 2;  // 16 KiB
 constexpr int kMaxSmem = 200 * 1024;
 
 struct SkinnyParams {
-    float* part;   // [splits][rows][nt] fp32
+    uint16_t* out;  // rows x r bf16, or r x rows when transposed
+    float scale;
+    int transposed;
     int rows;      // output rows
+    int r;
     int nt;        // r rounded up to 16 (MMA N)
     int kb_total;  // 64-wide contraction blocks
-    int kb_per_split;
+    int splits;    // CTAs per cluster, a power of two
     int stages;
     int b_bytes;   // bytes of one B stage
     uint32_t tmem_cols;
@@ -68,9 +74,9 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
     const uint32_t done = bar0 + 8u * (2 * p.stages);
 
     const int row0 = blockIdx.x * kRows;
-    const int split = blockIdx.y;
-    const int kb_begin = split * p.kb_per_split;
-    const int kb_end = min(p.kb_total, kb_begin + p.kb_per_split);
+    const int split = static_cast<int>(cluster_ctarank());  // == blockIdx.y: the cluster spans the splits
+    const int kb_begin = static_cast<int>(static_cast<int64_t>(split) * p.kb_total / p.splits);
+    const int kb_end = static_cast<int>(static_cast<int64_t>(split + 1) * p.kb_total / p.splits);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
@@ -136,55 +142,64 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
         if (ok) tc_commit(done);
     }
     __syncwarp();
-    // epilogue: lane quarter of each warp = 32 output rows, 16 columns at a time
+    // the split's accumulator -> this CTA's shared memory [128][nt + 4] fp32
+    // (the pipeline stages are free once `done` has fired)
+    const int ld = p.nt + 4;
+    float* acc = reinterpret_cast<float*>(smem);
     const bool fin = __all_sync(0xffffffffu, mbar_wait(done, 0, err));
     if (fin) {
         tc_fence_after();
-        const int row = row0 + warp * 32 + lane;
-        float* dst = p.part + (static_cast<int64_t>(split) * p.rows + row) * p.nt;
+        const int lr = warp * 32 + lane;
         for (int c0 = 0; c0 < p.nt; c0 += 16) {
             uint32_t v[16];
             tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
             tmem_wait_ld();
-            if (row < p.rows) {
 #pragma unroll
-                for (int t = 0; t < 16; t += 4)
-                    *reinterpret_cast<float4*>(dst + c0 + t) = make_float4(
-                        __uint_as_float(v[t]), __uint_as_float(v[t + 1]), __uint_as_float(v[t + 2]),
-                        __uint_as_float(v[t + 3]));
+            for (int t = 0; t < 16; t += 4)
+                *reinterpret_cast<float4*>(acc + lr * ld + c0 + t) = make_float4(
+                    __uint_as_float(v[t]), __uint_as_float(v[t + 1]), __uint_as_float(v[t + 2]),
+                    __uint_as_float(v[t + 3]));
+        }
+    } else {
+        for (int i = threadIdx.x; i < kRows * ld; i += kThreads) acc[i] = 0.0f;
+    }
+    tc_fence_before();
+    cluster_arrive();  // every split's accumulator is in its CTA's shared memory
+    cluster_wait();
+    {
+        const int rows_per = kRows / p.splits;
+        const int q4 = p.nt / 4;
+        const uint32_t acc_s = smem_u32(acc);
+        for (int idx = threadIdx.x; idx < rows_per * q4; idx += kThreads) {
+            const int lr = split * rows_per + idx / q4;
+            const int c = (idx % q4) * 4;
+            const uint32_t off = static_cast<uint32_t>((lr * ld + c) * 4);
+            float4 sum = ld_cluster_f4(cluster_map(acc_s + off, 0));
+            for (int q = 1; q < p.splits; ++q) {
+                const float4 v = ld_cluster_f4(cluster_map(acc_s + off, static_cast<uint32_t>(q)));
+                sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+            }
+            const int row = row0 + lr;
+            if (row < p.rows && c < p.r) {
+                const uint32_t lo = pack_bf16x2(sum.x * p.scale, sum.y * p.scale);
+                const uint32_t hi = pack_bf16x2(sum.z * p.scale, sum.w * p.scale);
+                if (p.transposed) {
+                    uint16_t* o = p.out + static_cast<int64_t>(c) * p.rows + row;
+                    o[0] = static_cast<uint16_t>(lo & 0xffffu);
+                    o[p.rows] = static_cast<uint16_t>(lo >> 16);
+                    o[2 * static_cast<int64_t>(p.rows)] = static_cast<uint16_t>(hi & 0xffffu);
+                    o[3 * static_cast<int64_t>(p.rows)] = static_cast<uint16_t>(hi >> 16);
+                } else {
+                    *reinterpret_cast<uint2*>(p.out + static_cast<int64_t>(row) * p.r + c) = make_uint2(lo, hi);
+                }
             }
         }
     }
-    tc_fence_before();
-    __syncthreads();
+    cluster_arrive();  // no CTA leaves while its shared memory may still be read
+    cluster_wait();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, p.tmem_cols);
-    }
-}
-
-// out = bf16(scale * sum_s part[s]) in a fixed order; `transposed` writes
-// out[j][i] (dA) instead of out[i][j].
-__global__ void k_lora_reduce(const float* __restrict__ part, int splits, int rows, int nt, int r, float scale,
-                              uint16_t* __restrict__ out, int transposed) {
-    const int64_t total = static_cast<int64_t>(rows) * r;
-    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        int64_t i, j;
-        if (transposed) {  // consecutive threads walk i so the stores are contiguous
-            j = idx / rows;
-            i = idx % rows;
-        } else {
-            i = idx / r;
-            j = idx % r;
-        }
-        float acc = 0.0f;
-        for (int s = 0; s < splits; ++s) acc += part[(static_cast<int64_t>(s) * rows + i) * nt + j];
-        const uint16_t b = f32_to_bf16_bits(scale * acc);
-        if (transposed)
-            out[j * rows + i] = b;
-        else
-            out[i * r + j] = b;
     }
 }
 
@@ -205,39 +220,37 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
 }
 
 struct Plan {
-    int nt, kb_total, kb_per_split, splits, stages, b_bytes, smem;
+    int nt, kb_total, splits, stages, b_bytes, smem;
     uint32_t tmem_cols;
     int64_t tiles;
 };
 
+// Splits: the smallest power of two (<= 8, <= the contraction blocks) that
+// gives about two CTAs per SM.
 Plan plan(int64_t rows, int64_t ctr, int r, bool b_mn) {
     Plan pl;
     pl.nt = static_cast<int>(round_up(r, 16));
     pl.kb_total = static_cast<int>(ceil_div(ctr > 0 ? ctr : 1, kBK));
     pl.tiles = ceil_div(rows > 0 ? rows : 1, kRows);
-    const int64_t target = 2LL * num_sms();
-    int64_t splits = ceil_div(target, pl.tiles);
-    splits = splits < 1 ? 1 : (splits > pl.kb_total ? pl.kb_total : splits);
-    pl.kb_per_split = static_cast<int>(ceil_div(pl.kb_total, splits));
-    pl.splits = static_cast<int>(ceil_div(pl.kb_total, pl.kb_per_split));  // no empty split
+    const int64_t want = ceil_div(2LL * num_sms(), pl.tiles);
+    int splits = 1;
+    while (splits < want && splits * 2 <= 8 && splits * 2 <= pl.kb_total) splits *= 2;
+    pl.splits = splits;
     pl.b_bytes = b_mn ? static_cast<int>(ceil_div(pl.nt, 64)) * 8192 : pl.nt * kBK * 2;
     const int stage = kABytes + pl.b_bytes;
     pl.stages = (kMaxSmem - 2048) / stage;
     pl.stages = pl.stages > 4 ? 4 : pl.stages;  // keeps two CTAs per SM for r <= 64
-    pl.smem = pl.stages * stage + 1024 + 1024;
+    const int staging = kRows * (pl.nt + 4) * 4;  // the accumulator, reusing the stages
+    pl.smem = (pl.stages * stage > staging ? pl.stages * stage : staging) + 1024 + 1024;
     uint32_t c = 32;
     while (c < static_cast<uint32_t>(pl.nt)) c <<= 1;
     pl.tmem_cols = c;
     return pl;
 }
 
-size_t partial_bytes(const Plan& pl, int64_t rows) {
-    return static_cast<size_t>(pl.splits) * static_cast<size_t>(rows) * pl.nt * 4;
-}
-
 template <bool A_MN, bool B_MN>
 cudaError_t run(const Plan& pl, const CUtensorMap& ma, const CUtensorMap& mb, int64_t rows, int r, float scale,
-                float* part, uint16_t* out, bool transposed, cudaStream_t st) {
+                uint16_t* out, bool transposed, cudaStream_t st) {
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [] {
@@ -245,25 +258,32 @@ cudaError_t run(const Plan& pl, const CUtensorMap& ma, const CUtensorMap& mb, in
     });
     if (attr != cudaSuccess) return attr;
     SkinnyParams p;
-    p.part = part;
+    p.out = out;
+    p.scale = scale;
+    p.transposed = transposed ? 1 : 0;
     p.rows = static_cast<int>(rows);
+    p.r = r;
     p.nt = pl.nt;
     p.kb_total = pl.kb_total;
-    p.kb_per_split = pl.kb_per_split;
+    p.splits = pl.splits;
     p.stages = pl.stages;
     p.b_bytes = pl.b_bytes;
     p.tmem_cols = pl.tmem_cols;
-    dim3 grid(static_cast<unsigned>(pl.tiles), static_cast<unsigned>(pl.splits));
-    k_lora_tc<A_MN, B_MN><<<grid, kThreads, pl.smem, st>>>(ma, mb, p);
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr_c[1];
+    attr_c[0].id = cudaLaunchAttributeClusterDimension;
+    attr_c[0].val.clusterDim.x = 1;
+    attr_c[0].val.clusterDim.y = static_cast<unsigned>(pl.splits);
+    attr_c[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.tiles), static_cast<unsigned>(pl.splits));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(pl.smem);
+    cfg.stream = st;
+    cfg.attrs = attr_c;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_lora_tc<A_MN, B_MN>, ma, mb, p);
     note_launches(1);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    const int64_t total = rows * r;
-    const int64_t want = ceil_div(total, 256);
-    const int g2 = static_cast<int>(want < num_sms() * 8LL ? want : num_sms() * 8LL);
-    k_lora_reduce<<<g2, 256, 0, st>>>(part, pl.splits, static_cast<int>(rows), pl.nt, r, scale, out, transposed ? 1 : 0);
-    note_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace
@@ -273,49 +293,40 @@ bool lora_tc_supported(int64_t M, int64_t N, int64_t K, int r) {
            N < (int64_t(1) << 31) && encode_fn() != nullptr;
 }
 
-size_t lora_tc_workspace(int64_t M, int64_t N, int64_t K, int r) {
-    if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return 0;
-    size_t b = partial_bytes(plan(M, K, r, false), M);                    // T
-    b = std::max(b, partial_bytes(plan(M, N, r, true), M));               // U
-    b = std::max(b, partial_bytes(plan(K, M, r, true), K));               // dA^T
-    b = std::max(b, partial_bytes(plan(N, M, r, true), N));               // dB
-    return b;
-}
-
 // T = bf16(s X A^T): A operand X (K-major), B operand A (K-major).
 cudaError_t launch_lora_xat_tc(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, float s,
-                               uint16_t* T, float* part, cudaStream_t st) {
+                               uint16_t* T, cudaStream_t st) {
     const Plan pl = plan(M, K, r, false);
     CUtensorMap ma, mb;
     if (!make_map(&ma, X, K, M, kBK, kRows) || !make_map(&mb, A, K, r, kBK, pl.nt)) return cudaErrorInvalidValue;
-    return run<false, false>(pl, ma, mb, M, r, s, part, T, false, st);
+    return run<false, false>(pl, ma, mb, M, r, s, T, false, st);
 }
 
 // U = bf16(s dY B): A operand dY (K-major over n), B operand B^T (MN-major).
 cudaError_t launch_lora_dyb_tc(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t N, int r, float s,
-                               uint16_t* U, float* part, cudaStream_t st) {
+                               uint16_t* U, cudaStream_t st) {
     const Plan pl = plan(M, N, r, true);
     CUtensorMap ma, mb;
     if (!make_map(&ma, dY, N, M, kBK, kRows) || !make_map(&mb, B, r, N, 64, kBK)) return cudaErrorInvalidValue;
-    return run<false, true>(pl, ma, mb, M, r, s, part, U, false, st);
+    return run<false, true>(pl, ma, mb, M, r, s, U, false, st);
 }
 
 // dA = bf16(U^T X) computed as dA^T[k][j] = sum_m X[m][k] U[m][j]: both MN-major.
 cudaError_t launch_lora_da_tc(const uint16_t* X, const uint16_t* U, int64_t M, int64_t K, int r, uint16_t* dA,
-                              float* part, cudaStream_t st) {
+                              cudaStream_t st) {
     const Plan pl = plan(K, M, r, true);
     CUtensorMap ma, mb;
     if (!make_map(&ma, X, K, M, 64, kBK) || !make_map(&mb, U, r, M, 64, kBK)) return cudaErrorInvalidValue;
-    return run<true, true>(pl, ma, mb, K, r, 1.0f, part, dA, true, st);
+    return run<true, true>(pl, ma, mb, K, r, 1.0f, dA, true, st);
 }
 
 // dB = bf16(dY^T T), dB[n][j] = sum_m dY[m][n] T[m][j]: both MN-major.
 cudaError_t launch_lora_db_tc(const uint16_t* dY, const uint16_t* T, int64_t M, int64_t N, int r, uint16_t* dB,
-                              float* part, cudaStream_t st) {
+                              cudaStream_t st) {
     const Plan pl = plan(N, M, r, true);
     CUtensorMap ma, mb;
     if (!make_map(&ma, dY, N, M, 64, kBK) || !make_map(&mb, T, r, M, 64, kBK)) return cudaErrorInvalidValue;
-    return run<true, true>(pl, ma, mb, N, r, 1.0f, part, dB, false, st);
+    return run<true, true>(pl, ma, mb, N, r, 1.0f, dB, false, st);
 }
 
 int lora_device_error(int reset) {

@@ -137,11 +137,11 @@ int qlora_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c
                      void* out, int out_dtype, void* stream);
 
 /*
- * Workspace bytes for qlora_linear_fwd / qlora_linear_bwd (depends on the
- * current device's SM count: query with the device current).  The forward
- * needs M*r*2 bytes for T (used when T_save is NULL) plus the fp32 split-K
- * partials of the rank-r products; the backward needs U and T plus the same
- * partials.  A workspace of the larger size serves both.
+ * Workspace bytes for qlora_linear_fwd / qlora_linear_bwd.  The forward
+ * needs M*r*2 bytes for T (used when T_save is NULL); the backward needs U
+ * and T (M*r*2 bytes each, 256-byte aligned) plus, for dX, the transposed
+ * copy of the weight its GEMM reads (about 1.1 bytes per weight).  A
+ * workspace of the larger size serves both.
  */
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int r);
 size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r);
