@@ -32,13 +32,18 @@
 // Tile: 128 weight rows (n forward, k backward) x 384 tokens x 64: each
 // dequantized weight stage feeds two 128 x 192 MMAs (two fp32 accumulators,
 // 384 TMEM columns), so the conversion work per FLOP is that of a 384-token
-// tile; 4 pipeline stages (A stages in the last 128 TMEM columns).  Warp
-// roles (576
+// tile; 3 pipeline stages (A stages in TMEM after the accumulators).  The
+// codes are expanded through a 64 KiB table that maps a code byte to both
+// of its fp32 codebook values (one 8-byte copy per lane: no bank
+// conflicts), so a pair of weights costs one byte permute, one shared load,
+// two multiplies and one pack.  Warp
+// roles (448
 // threads, persistent over tiles, one CTA per SM):
 //   warp 0        TMA producer for the activation tiles (and constants)
 //   warp 1        MMA issuer (one thread)
-//   warps 2..17   dequant producers: warp w converts the stages kb with
-//                 kb % 4 == (w - 2) / 4 for the TMEM lane quarter w % 4, then
+//   warps 2..13   dequant producers: warp w converts the stages kb with
+//                 kb % 3 == (w - 2) / 4 (always ring slot kb % 3) for the
+//                 TMEM lane quarter w % 4, then
 //                 the epilogue of the tile: tcgen05.ld, bf16, stores
 //                 coalesced along the weight-row index
 // Every wait is bounded; a timeout records QLORA_ERR_TIMEOUT in a sticky
@@ -66,18 +71,21 @@ constexpr int kSubT = 192;    // tokens per MMA (MMA N)
 constexpr int kSubs = 2;      // MMAs per stage sharing one dequantized weight stage
 constexpr int kTileT = kSubT * kSubs;  // 384 tokens per tile
 constexpr int kBK = 64;       // contraction per stage
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kSubBytes = kSubT * kBK * 2;      // 24 KiB
 constexpr int kXStageBytes = kTileT * kBK * 2;  // 48 KiB
 constexpr int kAccCols = kTileT;                // fp32 accumulator columns
 constexpr int kAStageCols = kBK / 2;            // bf16 pairs per TMEM column
 constexpr uint32_t kTmemCols = 512;
-constexpr int kDqWarps = 16;                    // four per TMEM lane quarter
-constexpr int kParts = kDqWarps / 4;            // stage kb is converted by the warps with part == kb % 4
-constexpr int kPrefetch = 2;                    // own stages of codes in flight per dequant thread
-constexpr int kThreads = 32 * (2 + kDqWarps);   // 576
-constexpr int kSmemBytes = kStages * kXStageBytes + 1024 /* align */ + 1024 /* barriers etc. */ +
-                           kDqWarps * kBK * 4 /* backward: per-warp constants */;
+constexpr int kDqWarps = 12;                    // three per TMEM lane quarter
+constexpr int kParts = kDqWarps / 4;            // stage kb is converted by the warps with part == kb % 3
+static_assert(kParts == kStages, "a part's stages must always use the same ring slot");
+constexpr int kPrefetchFwd = 2;                 // own stages of codes in flight per dequant thread
+constexpr int kPrefetchBwd = 2;                 // (the backward also holds its constants)
+constexpr int kThreads = 32 * (2 + kDqWarps);   // 448: 128 registers a thread
+constexpr int kLutBytes = 256 * 256;             // code byte -> fp32 pair, one 8-byte copy per lane
+constexpr int kLutOff = kStages * kXStageBytes + 1024 + kDqWarps * kBK * 4;
+constexpr int kSmemBytes = 1024 /* align */ + kLutOff + kLutBytes;
 static_assert(kAccCols + kStages * kAStageCols <= static_cast<int>(kTmemCols), "TMEM budget");
 
 struct GemmParams {
@@ -118,14 +126,25 @@ struct Pipe {
     __device__ uint32_t acc_empty() const { return bar0 + 8u * (3 * kStages + 1); }
 };
 
+// Ring slot of contraction stage kb: slot kb % kStages, always, so the
+// dequant warps of part p (the stages kb % kStages == p) own slot p for the
+// whole kernel and no two parts ever wait on the same slot's barriers.
+// Returns the slot's use count before this stage (tile tcount): its parity
+// is the phase every role waits on.
+__device__ __forceinline__ uint32_t slot_use(int kb, uint32_t tcount, int kb_total) {
+    const int s = kb % kStages;
+    const uint32_t uses_per_tile = static_cast<uint32_t>((kb_total - s + kStages - 1) / kStages);
+    return tcount * uses_per_tile + static_cast<uint32_t>(kb / kStages);
+}
+
 // warp 0, one thread: activation tiles, then the LoRA slabs, into the ring.
 __device__ void role_tma(const Pipe& P, const CUtensorMap* tmap_act, const CUtensorMap* tmap_lora, int* err) {
-    uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x) {
+    uint32_t tcount = 0;
+    for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x, ++tcount) {
         const int t0 = (tile % P.num_t) * kTileT;
-        for (int kb = 0; kb < P.kb_total; ++kb, ++it) {
-            const int s = static_cast<int>(it % kStages);
-            const uint32_t ph = (it / kStages) & 1u;
+        for (int kb = 0; kb < P.kb_total; ++kb) {
+            const int s = kb % kStages;
+            const uint32_t ph = slot_use(kb, tcount, P.kb_total) & 1u;
             if (!mbar_wait(P.empty(s), ph ^ 1u, err)) return;
             const uint32_t dst = smem_u32(P.sA + s * kXStageBytes);
             if (kb < P.kb_w) {
@@ -146,13 +165,13 @@ __device__ void role_tma(const Pipe& P, const CUtensorMap* tmap_act, const CUten
 // accumulators, all reading the same weight stage in TMEM.
 __device__ void role_mma(const Pipe& P, int* err) {
     constexpr uint32_t idesc = idesc_bf16(kTileW, kSubT);
-    uint32_t it = 0, tcount = 0;
+    uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x, ++tcount) {
         if (!mbar_wait(P.acc_empty(), (tcount & 1u) ^ 1u, err)) return;
         tc_fence_after();
-        for (int kb = 0; kb < P.kb_total; ++kb, ++it) {
-            const int s = static_cast<int>(it % kStages);
-            const uint32_t ph = (it / kStages) & 1u;
+        for (int kb = 0; kb < P.kb_total; ++kb) {
+            const int s = kb % kStages;
+            const uint32_t ph = slot_use(kb, tcount, P.kb_total) & 1u;
             if (!mbar_wait(P.full_b(s), ph, err)) return;
             if (!mbar_wait(P.full_a(s), ph, err)) return;
             tc_fence_after();
@@ -182,9 +201,13 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* er
     return ok != 0;
 }
 
-// q[code] read from the 16-entry table by a byte offset (code * 4).
-__device__ __forceinline__ float lut_at(const float* lut, uint32_t byte_off) {
-    return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(lut) + byte_off);
+// The two codebook values of one code byte, (q[high nibble], q[low nibble]),
+// from the lane's own copy of the 256-entry table: entry b, lane l at byte
+// 256 b + 8 l, so a warp's reads never share a bank; the byte and the lane
+// offset form the address in one byte permute.
+__device__ __forceinline__ float2 lut_pair(const uint8_t* lut, uint32_t word, uint32_t lane_off, int byte) {
+    const uint32_t addr = __byte_perm(word, lane_off, 0x5504u | (static_cast<uint32_t>(byte) << 4));
+    return *reinterpret_cast<const float2*>(lut + addr);
 }
 
 // 64 contraction values of one weight row (forward) or column (backward):
@@ -194,37 +217,30 @@ __device__ __forceinline__ float lut_at(const float* lut, uint32_t byte_off) {
 // shared memory).
 template <bool kPerElem>
 __device__ __forceinline__ void convert_run(const uint4& c0, const uint4& c1, float sc, const float* sp,
-                                            const float* lut, uint32_t (&v)[32]) {
+                                            const uint8_t* lut, uint32_t lane_off, uint32_t (&v)[32]) {
     const uint32_t w8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
-        const uint32_t hi4 = (w8[h] >> 2) & 0x3C3C3C3Cu;  // even-element code * 4, per byte
-        const uint32_t lo4 = (w8[h] << 2) & 0x3C3C3C3Cu;  // odd-element code * 4, per byte
-        float4 s01 = make_float4(sc, sc, sc, sc), s23 = s01;
-        if (kPerElem) {
-            s01 = *reinterpret_cast<const float4*>(sp + 8 * h);
-            s23 = *reinterpret_cast<const float4*>(sp + 8 * h + 4);
-        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const float a = lut_at(lut, __byte_perm(hi4, 0u, 0x4440u | j));
-            const float b = lut_at(lut, __byte_perm(lo4, 0u, 0x4440u | j));
-            const float sa = j == 0 ? s01.x : j == 1 ? s01.z : j == 2 ? s23.x : s23.z;
-            const float sb = j == 0 ? s01.y : j == 1 ? s01.w : j == 2 ? s23.y : s23.w;
-            v[4 * h + j] = pack_bf16x2(__fmul_rn(a, sa), __fmul_rn(b, sb));
+            const float2 q2 = lut_pair(lut, w8[h], lane_off, j);
+            // backward: the constants of contraction values 8h + 2j, 8h + 2j + 1
+            const float2 s2 = kPerElem ? *reinterpret_cast<const float2*>(sp + 8 * h + 2 * j) : make_float2(sc, sc);
+            v[4 * h + j] = pack_bf16x2(__fmul_rn(q2.x, s2.x), __fmul_rn(q2.y, s2.y));
         }
     }
 }
 
-// warps 2..17: each converts every fourth stage of the weight tile into
+// warps 2..13: each converts every third stage of the weight tile into
 // TMEM (quarter = its TMEM lanes, part = which stages), then writes a
 // quarter of this tile's outputs.
 template <bool kBwd>
-__device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const float* lut,
+__device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const uint8_t* lut,
                                                       float* wsc, int warp, int lane, int* err) {
+    const uint32_t lane_off = static_cast<uint32_t>(lane) * 8;
     const int dq = warp - 2;
     const int quarter = warp & 3;  // the TMEM lanes this warp may touch
-    const int part = dq >> 2;      // converts the stages kb with kb % 4 == part
+    const int part = dq >> 2;      // converts the stages kb with kb % 3 == part
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float mu = kBwd ? 0.0f : *p.mean;
@@ -234,7 +250,6 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
         const int row0 = (tile / P.num_t) * kTileW;
         const int grow = row0 + row;             // this lane's weight row of the product
         const bool lane_ok = grow < p.rows;
-        const uint32_t g0 = tcount * static_cast<uint32_t>(P.kb_total);  // ring index of stage 0
         const uint8_t* crow = p.codes + static_cast<int64_t>(grow) * p.ld_codes;
         // backward: this warp's 32 columns lie in one 64-wide block group
         const float* srow = kBwd ? p.scalesT + static_cast<int64_t>((row0 + quarter * 32) / kBK) * p.ld_scales
@@ -243,6 +258,7 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
         // codes (and, forward, the block constant's inputs) of the next
         // kPrefetch own stages; the constant itself is formed at use so the
         // loads stay in flight
+        constexpr int kPrefetch = kBwd ? kPrefetchBwd : kPrefetchFwd;
         uint4 cb0[kPrefetch], cb1[kPrefetch];
         uint32_t sbyte[kPrefetch];
         float sc1[kPrefetch];
@@ -272,9 +288,8 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
             for (int u = 0; u < kPrefetch; ++u) {
                 const int kb = part + kParts * (i0 + u);
                 if (kb >= P.kb_total) break;
-                const uint32_t g = g0 + static_cast<uint32_t>(kb);
-                const int s = static_cast<int>(g % kStages);
-                const uint32_t ph = (g / kStages) & 1u;
+                const int s = part;  // == kb % kStages
+                const uint32_t ph = slot_use(kb, tcount, P.kb_total) & 1u;
                 uint32_t v[32];
                 if (kb < P.kb_w) {
                     if (kBwd) {
@@ -285,7 +300,7 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
                     // rows beyond the weight hold finite garbage (zero codes times
                     // the constant of empty inputs): their outputs are never
                     // stored and rows do not mix in this product
-                    convert_run<kBwd>(cb0[u], cb1[u], sc, wsc, lut, v);
+                    convert_run<kBwd>(cb0[u], cb1[u], sc, wsc, lut, lane_off, v);
                     if (kBwd) __syncwarp();  // wsc is rewritten by the warp's next stage
                 } else {  // LoRA slab: lane = row of B (forward) or of A^T (backward), r contiguous
                     const int j0 = (kb - P.kb_w) * kBK;
@@ -337,10 +352,11 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
 template <bool kBwd>
 __global__ void __launch_bounds__(kThreads, 1)
 k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_lora,
-              const GemmParams p) {
+              const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ float s_lut[16];  // static, so table reads use an immediate address
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base, derived by pointer arithmetic so that every
+    // access below stays a (32-bit) shared-memory access
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kXStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 2);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -359,7 +375,9 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
         mbar_init(P.acc_empty(), kDqWarps);
         fence_barrier_init();
     }
-    if (threadIdx.x < 16) s_lut[threadIdx.x] = p.q[threadIdx.x];
+    uint8_t* lut = smem + kLutOff;
+    for (int i = threadIdx.x; i < 256 * 32; i += kThreads)
+        reinterpret_cast<float2*>(lut)[i] = make_float2(p.q[i >> 9], p.q[(i >> 5) & 15]);
     if (warp == 0) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
@@ -385,7 +403,7 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
         if (lane == 0) role_mma(P, err);
         __syncwarp();
     } else {
-        role_dequant_epilogue<kBwd>(P, p, s_lut, P.sS + (warp - 2) * kBK, warp, lane, err);
+        role_dequant_epilogue<kBwd>(P, p, lut, P.sS + (warp - 2) * kBK, warp, lane, err);
     }
     tc_fence_before();
     __syncthreads();
