@@ -55,42 +55,45 @@ __device__ __forceinline__ float max_nan(float a, float b) {
 constexpr int kQuantThreads = 256;
 constexpr int kChunk = 512;  // weights per warp step
 
-// One 64-block per 16 lanes: v holds this lane's 4 weights of the block.
-// Returns the lane's 4 codes packed as two bytes, and the block absmax.
+// Absmax of the two 64-blocks a warp holds in one load (lanes 0-15: the
+// first, lanes 16-31: the second), as fp32 bit patterns with the sign
+// cleared: two whole-warp integer max reductions.  |NaN| (max.NaN gives the
+// canonical NaN) and Inf compare above every finite value.
+__device__ __forceinline__ void block_absmax_bits(const float4& v, int lane, uint32_t& lo, uint32_t& hi) {
+    const float a = max_nan(max_nan(fabsf(v.x), fabsf(v.y)), max_nan(fabsf(v.z), fabsf(v.w)));
+    const uint32_t u = __float_as_uint(a);
+    const bool upper = lane >= 16;
+    lo = __reduce_max_sync(0xffffffffu, upper ? 0u : u);
+    hi = __reduce_max_sync(0xffffffffu, upper ? u : 0u);
+}
+
+// The lane's 4 codes (two bytes, little-endian) for block absmax m (finite,
+// non-zero).
 //
-// Codes without dividing in the common case: with y ~ 1/a (relative error
-// <= 2^-22), n~ = RN(w y) lies within 2^-21 of n = RN(w / a) for |n| <= 1.
+// Codes without dividing in the common case: with y ~ 1/m (relative error
+// <= 2^-22), n~ = RN(w y) lies within 2^-21 of n = RN(w / m) for |n| <= 1.
 // The code is a step function of n whose steps (thresholds) lie at least
 // 1.6e-3 from the table's bin edges, so the bin of n~ serves n as well, and
 // the one threshold comparison agrees for n~ and n whenever n~ is more than
-// 2^-20 from the threshold.  A lane whose four quotients are all clear of
-// their thresholds is done; otherwise (rarely) it divides exactly.  The
-// table has one extra entry below -1 (index 0) because n~ may undershoot
-// -1 by a rounding, so finite inputs never need clamping.
-__device__ __forceinline__ uint32_t encode4(const float4& v, float& m_out, bool& bad, const EncTab* tab) {
-    float m = max_nan(max_nan(fabsf(v.x), fabsf(v.y)), max_nan(fabsf(v.z), fabsf(v.w)));
-    m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 8));
-    m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 4));
-    m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m_out = m;
-    if (!(m <= 3.402823466e38f)) {  // NaN or Inf in the block: flagged, codes unspecified
-        bad = true;
-        return 0x7777u;
-    }
-    if (m == 0.0f) return 0x7777u;  // all-zero block: the zero code
+// 2^-20 from the threshold (d = RN(n~ - thr) gives both: d >= 0 iff
+// n~ >= thr).  A lane whose four quotients are all clear of their
+// thresholds is done; otherwise (rarely) it divides exactly.  The table has
+// one extra entry below -1 (index 0) because n~ may undershoot -1 by a
+// rounding, so finite inputs never need clamping.  `tabx` is the table
+// shifted by the 0xFFF bin-index bias, indexed by bits(n + 3) >> 18.
+__device__ __forceinline__ uint32_t encode4(const float4& v, float m, const EncTab* tab, const EncTab* tabx) {
     const float w[4] = {v.x, v.y, v.z, v.w};
-    int q[4];
+    uint32_t q[4];
     bool exact = !(m >= 0x1p-120f && m <= 0x1p120f);  // extreme scales: always divide
     if (!exact) {
         const float y = rcp_approx(m);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const float na = __fmul_rn(w[i], y);
-            const unsigned b = (__float_as_uint(__fadd_rn(na, 3.0f)) >> 18) - 0xFFFu;
-            const EncTab e = tab[b];
-            q[i] = e.base + (na >= e.thr ? 1 : 0);
-            exact |= fabsf(__fsub_rn(na, e.thr)) <= 0x1p-20f;
+            const EncTab e = tabx[__float_as_uint(__fadd_rn(na, 3.0f)) >> 18];
+            const float d = __fsub_rn(na, e.thr);
+            q[i] = static_cast<uint32_t>(e.base) + (d >= 0.0f ? 1u : 0u);
+            exact |= fabsf(d) <= 0x1p-20f;
         }
     }
     if (exact) {
@@ -99,13 +102,11 @@ __device__ __forceinline__ uint32_t encode4(const float4& v, float& m_out, bool&
             const float n = __fdiv_rn(w[i], m);
             const unsigned b = (__float_as_uint(__fadd_rn(n, 3.0f)) >> 18) - 0xFFFu;
             const EncTab e = tab[b > 33u ? 33u : b];
-            q[i] = e.base + (n >= e.thr ? 1 : 0);
+            q[i] = static_cast<uint32_t>(e.base) + (n >= e.thr ? 1u : 0u);
         }
     }
     // byte e/2 = (code e << 4) | code e+1, little-endian in the returned pair
-    const uint32_t b0 = (static_cast<uint32_t>(q[0]) << 4) + static_cast<uint32_t>(q[1]);
-    const uint32_t b1 = (static_cast<uint32_t>(q[2]) << 4) + static_cast<uint32_t>(q[3]);
-    return (b1 << 8) + b0;
+    return (q[0] << 4) | q[1] | (q[2] << 12) | (q[3] << 8);
 }
 
 __global__ void __launch_bounds__(kQuantThreads)
@@ -120,6 +121,7 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
     if (threadIdx.x == 33) tab[0] = EncTab{2.0f, 0};
     if (threadIdx.x == 0) sbad = 0;
     __syncthreads();
+    const EncTab* tabx = tab - 0xFFF;  // tabx[bits(n + 3) >> 18] == tab[bin + 1]
 
     const int lane = threadIdx.x & 31;
     const int64_t nb = ceil_div(numel, kBlock);
@@ -130,46 +132,62 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
     bool bad = false;
 
     auto load_full = [&](int64_t c, float4 (&v)[4]) {
+        const float* src = W + c * kChunk + 4 * lane;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = ld_stream(W + c * kChunk + 4 * (32 * i + lane));
+        for (int i = 0; i < 4; ++i) v[i] = ld_stream(src + 128 * i);
     };
-    auto finish_block = [&](int64_t base, int i, float m) {
-        if ((lane & 15) == 0) {
-            const int64_t blk = (base >> 6) + 2 * i + (lane >> 4);
+    // Lanes 0-7 finish the chunk's 8 blocks: the constant c2 (coalesced) and
+    // its exact addition into the exponent bins.
+    auto finish_chunk = [&](int64_t base, float mb) {
+        if (lane < 8) {
+            const int64_t blk = (base >> 6) + lane;
             if (blk < nb) {
-                c2[blk] = m;
-                const uint32_t u = __float_as_uint(m);
+                c2[blk] = mb;
+                const uint32_t u = __float_as_uint(mb);
                 const uint32_t ex = u >> 23;
                 const unsigned long long mant = ex ? ((u & 0x7fffffu) | 0x800000u) : (u & 0x7fffffu);
                 if (mant) atomicAdd(&sbins[ex & 255u], mant);
             }
         }
     };
-
-    // whole chunks, loads for the next chunk in flight while this one encodes
-    int64_t c = warp0;
-    float4 cur[4], nxt[4];
-    if (c < nfull) load_full(c, cur);
-    for (; c < nfull; c += nwarps) {
-        const bool more = c + nwarps < nfull;
-        if (more) load_full(c + nwarps, nxt);
+    // One chunk: 4 loads of 512 bytes, each holding two 64-blocks.
+    auto encode_chunk = [&](int64_t c, const float4 (&v)[4]) {
         const int64_t base = c * kChunk;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(codes + (base >> 1)) + lane;
+        float mb = 0.0f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            float m;
-            const uint32_t b01 = encode4(cur[i], m, bad, tab);
-            const int64_t e = base + 4 * (32 * i + lane);
-            *reinterpret_cast<uint16_t*>(codes + (e >> 1)) = static_cast<uint16_t>(b01);
-            finish_block(base, i, m);
+            uint32_t lo, hi;
+            block_absmax_bits(v[i], lane, lo, hi);
+            const uint32_t mine = lane >= 16 ? hi : lo;
+            if ((lane >> 1) == i) mb = __uint_as_float((lane & 1) ? hi : lo);
+            uint32_t b01 = 0x7777u;  // all-zero block: the zero code
+            if (mine >= 0x7f800000u)
+                bad = true;  // NaN or Inf in the block: flagged, codes unspecified
+            else if (mine != 0u)
+                b01 = encode4(v[i], __uint_as_float(mine), tab, tabx);
+            dst[32 * i] = static_cast<uint16_t>(b01);  // bytes (base + 128 i + 4 lane) / 2
         }
-        if (more) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
-        }
+        finish_chunk(base, mb);
+    };
+
+    // whole chunks, the next chunk's loads in flight while one encodes
+    int64_t c = warp0;
+    float4 va[4], vb[4];
+    if (c < nfull) load_full(c, va);
+    while (c < nfull) {
+        if (c + nwarps < nfull) load_full(c + nwarps, vb);
+        encode_chunk(c, va);
+        c += nwarps;
+        if (c >= nfull) break;
+        if (c + nwarps < nfull) load_full(c + nwarps, va);
+        encode_chunk(c, vb);
+        c += nwarps;
     }
     // the ragged last chunk (at most one), by the warp whose turn it is
     if (nfull < nchunks && (nfull % nwarps) == warp0) {
         const int64_t base = nfull * kChunk;
+        float mb = 0.0f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int64_t e = base + 4 * (32 * i + lane);
@@ -178,12 +196,19 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
             v.y = e + 1 < numel ? W[e + 1] : 0.0f;
             v.z = e + 2 < numel ? W[e + 2] : 0.0f;
             v.w = e + 3 < numel ? W[e + 3] : 0.0f;
-            float m;
-            const uint32_t b01 = encode4(v, m, bad, tab);
+            uint32_t lo, hi;
+            block_absmax_bits(v, lane, lo, hi);
+            const uint32_t mine = lane >= 16 ? hi : lo;
+            if ((lane >> 1) == i) mb = __uint_as_float((lane & 1) ? hi : lo);
+            uint32_t b01 = 0x7777u;
+            if (mine >= 0x7f800000u)
+                bad = true;
+            else if (mine != 0u)
+                b01 = encode4(v, __uint_as_float(mine), tab, tabx);
             if (e < numel) codes[e >> 1] = static_cast<uint8_t>(e + 1 < numel ? (b01 & 0xff) : (b01 & 0xf0));
             if (e + 2 < numel) codes[(e >> 1) + 1] = static_cast<uint8_t>(e + 3 < numel ? (b01 >> 8) : ((b01 >> 8) & 0xf0));
-            finish_block(base, i, m);
         }
+        finish_chunk(base, mb);
     }
     if (bad) sbad = 1;
     __syncthreads();
