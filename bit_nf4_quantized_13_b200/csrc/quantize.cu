@@ -79,9 +79,15 @@ __device__ __forceinline__ void block_absmax_bits(const float4& v, int lane, uin
 // n~ >= thr).  A lane whose four quotients are all clear of their
 // thresholds is done; otherwise (rarely) it divides exactly.  The table has
 // one extra entry below -1 (index 0) because n~ may undershoot -1 by a
-// rounding, so finite inputs never need clamping.  `tabx` is the table
-// shifted by the 0xFFF bin-index bias, indexed by bits(n + 3) >> 18.
-__device__ __forceinline__ uint32_t encode4(const float4& v, float m, const EncTab* tab, const EncTab* tabx) {
+// rounding, so finite inputs never need clamping.  Every lane reads its own
+// copy of the table (entry i of lane l at 8 (32 i + l) bytes, so a warp's
+// lookups never share a bank): `tabl` is the lane's copy shifted by the
+// 0xFFF bin-index bias, addressed by (bits(n + 3) >> 18) * 256 bytes.
+__device__ __forceinline__ const EncTab& lane_entry(const uint8_t* tabl, float n) {
+    return *reinterpret_cast<const EncTab*>(tabl + ((__float_as_uint(n) >> 10) & ~0xFFu));
+}
+
+__device__ __forceinline__ uint32_t encode4(const float4& v, float m, const EncTab* tab, const uint8_t* tabl) {
     const float w[4] = {v.x, v.y, v.z, v.w};
     uint32_t q[4];
     bool exact = !(m >= 0x1p-120f && m <= 0x1p120f);  // extreme scales: always divide
@@ -90,7 +96,7 @@ __device__ __forceinline__ uint32_t encode4(const float4& v, float m, const EncT
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const float na = __fmul_rn(w[i], y);
-            const EncTab e = tabx[__float_as_uint(__fadd_rn(na, 3.0f)) >> 18];
+            const EncTab e = lane_entry(tabl, __fadd_rn(na, 3.0f));
             const float d = __fsub_rn(na, e.thr);
             q[i] = static_cast<uint32_t>(e.base) + (d >= 0.0f ? 1u : 0u);
             exact |= fabsf(d) <= 0x1p-20f;
@@ -109,21 +115,27 @@ __device__ __forceinline__ uint32_t encode4(const float4& v, float m, const EncT
     return (q[0] << 4) | q[1] | (q[2] << 12) | (q[3] << 8);
 }
 
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, 4)
 k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__ codes,
                float* __restrict__ c2, unsigned long long* __restrict__ bins,
                int* __restrict__ flag, Nf4Tables tabs) {
-    __shared__ EncTab tab[34];  // [0]: below -1; [1 + b]: bin b of the host table
+    __shared__ EncTab tab[34];       // [0]: below -1; [1 + b]: bin b of the host table
+    __shared__ EncTab tabr[34 * 32];  // the same, one copy per lane: [i][lane]
     __shared__ unsigned long long sbins[256];
     __shared__ int sbad;
     for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
+    for (int i = threadIdx.x; i < 34 * 32; i += blockDim.x) {
+        const int e = i >> 5;
+        tabr[i] = e == 0 ? EncTab{2.0f, 0} : EncTab{tabs.thr[e - 1], tabs.base[e - 1]};
+    }
     if (threadIdx.x < 33) tab[1 + threadIdx.x] = EncTab{tabs.thr[threadIdx.x], tabs.base[threadIdx.x]};
     if (threadIdx.x == 33) tab[0] = EncTab{2.0f, 0};
     if (threadIdx.x == 0) sbad = 0;
     __syncthreads();
-    const EncTab* tabx = tab - 0xFFF;  // tabx[bits(n + 3) >> 18] == tab[bin + 1]
 
     const int lane = threadIdx.x & 31;
+    // this lane's copy, biased so that byte offset (bits >> 18) * 256 finds entry (bits >> 18) - 0xFFF
+    const uint8_t* tabl = reinterpret_cast<const uint8_t*>(tabr) + 8 * lane - 0xFFF * 256;
     const int64_t nb = ceil_div(numel, kBlock);
     const int64_t nfull = numel / kChunk;  // whole 512-weight chunks
     const int64_t nchunks = ceil_div(numel, kChunk);
@@ -165,7 +177,7 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
             if (mine >= 0x7f800000u)
                 bad = true;  // NaN or Inf in the block: flagged, codes unspecified
             else if (mine != 0u)
-                b01 = encode4(v[i], __uint_as_float(mine), tab, tabx);
+                b01 = encode4(v[i], __uint_as_float(mine), tab, tabl);
             dst[32 * i] = static_cast<uint16_t>(b01);  // bytes (base + 128 i + 4 lane) / 2
         }
         finish_chunk(base, mb);
@@ -204,7 +216,7 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
             if (mine >= 0x7f800000u)
                 bad = true;
             else if (mine != 0u)
-                b01 = encode4(v, __uint_as_float(mine), tab, tabx);
+                b01 = encode4(v, __uint_as_float(mine), tab, tabl);
             if (e < numel) codes[e >> 1] = static_cast<uint8_t>(e + 1 < numel ? (b01 & 0xff) : (b01 & 0xf0));
             if (e + 2 < numel) codes[(e >> 1) + 1] = static_cast<uint8_t>(e + 3 < numel ? (b01 >> 8) : ((b01 >> 8) & 0xf0));
         }
