@@ -115,15 +115,17 @@ __device__ __forceinline__ uint32_t encode4(const float4& v, float m, const EncT
     return (q[0] << 4) | q[1] | (q[2] << 12) | (q[3] << 8);
 }
 
-__global__ void __launch_bounds__(kQuantThreads, 4)
+__global__ void __launch_bounds__(kQuantThreads, 3)
 k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__ codes,
                float* __restrict__ c2, unsigned long long* __restrict__ bins,
                int* __restrict__ flag, Nf4Tables tabs) {
     __shared__ EncTab tab[34];       // [0]: below -1; [1 + b]: bin b of the host table
     __shared__ EncTab tabr[34 * 32];  // the same, one copy per lane: [i][lane]
-    __shared__ unsigned long long sbins[256];
+    // exact-sum bins of this CTA, as 32-bit words plus carry counts (native
+    // 32-bit shared atomics; a carry out of the low word is counted apart)
+    __shared__ uint32_t sbin_lo[256], sbin_hi[256];
     __shared__ int sbad;
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) sbin_lo[i] = sbin_hi[i] = 0u;
     for (int i = threadIdx.x; i < 34 * 32; i += blockDim.x) {
         const int e = i >> 5;
         tabr[i] = e == 0 ? EncTab{2.0f, 0} : EncTab{tabs.thr[e - 1], tabs.base[e - 1]};
@@ -157,8 +159,11 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
                 c2[blk] = mb;
                 const uint32_t u = __float_as_uint(mb);
                 const uint32_t ex = u >> 23;
-                const unsigned long long mant = ex ? ((u & 0x7fffffu) | 0x800000u) : (u & 0x7fffffu);
-                if (mant) atomicAdd(&sbins[ex & 255u], mant);
+                const uint32_t mant = ex ? ((u & 0x7fffffu) | 0x800000u) : (u & 0x7fffffu);
+                if (mant) {
+                    const uint32_t old = atomicAdd(&sbin_lo[ex & 255u], mant);
+                    if (old + mant < old) atomicAdd(&sbin_hi[ex & 255u], 1u);
+                }
             }
         }
     };
@@ -173,12 +178,14 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
             block_absmax_bits(v[i], lane, lo, hi);
             const uint32_t mine = lane >= 16 ? hi : lo;
             if ((lane >> 1) == i) mb = __uint_as_float((lane & 1) ? hi : lo);
-            uint32_t b01 = 0x7777u;  // all-zero block: the zero code
-            if (mine >= 0x7f800000u)
-                bad = true;  // NaN or Inf in the block: flagged, codes unspecified
-            else if (mine != 0u)
-                b01 = encode4(v[i], __uint_as_float(mine), tab, tabl);
-            dst[32 * i] = static_cast<uint16_t>(b01);  // bytes (base + 128 i + 4 lane) / 2
+            // NaN or Inf in the block: flagged, codes unspecified; an all-zero
+            // block gets the zero code
+            bad |= mine >= 0x7f800000u;
+            const bool ok = mine - 1u < 0x7f7fffffu;  // finite and non-zero
+            // otherwise encode zeros: the table index stays in range only for |w| <= m
+            const float4 vi = ok ? v[i] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            const uint32_t b01 = encode4(vi, ok ? __uint_as_float(mine) : 1.0f, tab, tabl);
+            dst[32 * i] = static_cast<uint16_t>(ok ? b01 : 0x7777u);  // bytes (base + 128 i + 4 lane) / 2
         }
         finish_chunk(base, mb);
     };
@@ -224,8 +231,10 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
     }
     if (bad) sbad = 1;
     __syncthreads();
-    for (int i = threadIdx.x; i < 256; i += blockDim.x)
-        if (sbins[i]) atomicAdd(&bins[i], sbins[i]);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+        const unsigned long long t = (static_cast<unsigned long long>(sbin_hi[i]) << 32) | sbin_lo[i];
+        if (t) atomicAdd(&bins[i], t);
+    }
     if (threadIdx.x == 0 && sbad) atomicOr(flag, 1);
 }
 
