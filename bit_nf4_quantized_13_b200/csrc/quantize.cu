@@ -241,65 +241,79 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
 // ------------------------------------------------------------------------
 // Exact mean from the exponent bins.  Bin E holds the integer sum of the
 // 24-bit significands of all c2 with exponent field E; its value is
-// bins[E] * 2^(max(E,1) - 150).  The total, as an integer multiple of
-// 2^-149, is accumulated in 32-bit digits (carries deferred), rounded once
-// to the nearest double, divided by nb and rounded to fp32.
+// bins[E] * 2^(max(E,1) - 150).  As an integer multiple of 2^-149 the total
+// is sum_E bins[E] << (max(E,1) - 1).  Lane l folds its eight bins
+// E = 8l .. 8l+7 into one 128-bit value relative to 2^(max(8l,1) - 1)
+// (each term < 2^64 shifted by at most 7: the sum stays below 2^75); lane 0
+// adds the non-zero lane values into 32-bit digits, rounds the total once to
+// the nearest double (round bit and sticky bit), divides by nb in double
+// and rounds to fp32.
 constexpr int kDigits = 12;
 
 __device__ float mean_from_bins(const unsigned long long* __restrict__ bins, int64_t nb,
-                                unsigned long long* sdig /* shared, kDigits */) {
+                                unsigned long long* sv /* shared, 64: lane values lo, hi */) {
     const int lane = threadIdx.x & 31;
-    if (lane < kDigits) sdig[lane] = 0ull;
-    __syncwarp();
-    for (int e = lane; e < 256; e += 32) {
+    unsigned long long lo = 0, hi = 0;
+    const int e0 = 8 * lane, base = e0 ? e0 : 1;  // exponent field whose bin shift is the lane's origin
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int e = e0 + k;
         const unsigned long long v = bins[e];
-        if (!v) continue;
-        const int sh = (e ? e : 1) - 1;
-        const int d0 = sh >> 5, off = sh & 31;
-        const unsigned long long lo = (v << off) & 0xffffffffull;
-        const unsigned long long mid = (off ? (v >> (32 - off)) : (v >> 32)) & 0xffffffffull;
-        const unsigned long long hi = off ? (v >> (64 - off)) : 0ull;
-        atomicAdd(&sdig[d0], lo);
-        atomicAdd(&sdig[d0 + 1], mid);
-        if (hi) atomicAdd(&sdig[d0 + 2], hi);
+        const int sh = (e ? e : 1) - base;  // 0..7
+        const unsigned long long vlo = v << sh, vhi = sh ? (v >> (64 - sh)) : 0ull;
+        lo += vlo;
+        hi += vhi + (lo < vlo ? 1ull : 0ull);
     }
+    sv[2 * lane] = lo;
+    sv[2 * lane + 1] = hi;
     __syncwarp();
     float mu = 0.0f;
     if (lane == 0) {
-        unsigned long long d[kDigits + 1];
-        unsigned long long carry = 0;
-        for (int i = 0; i < kDigits; ++i) {
-            const unsigned long long t = sdig[i] + carry;
-            d[i] = t & 0xffffffffull;
-            carry = t >> 32;
+        uint32_t d[kDigits + 1];
+#pragma unroll
+        for (int i = 0; i <= kDigits; ++i) d[i] = 0u;
+        for (int l = 0; l < 32; ++l) {
+            const unsigned long long vlo = sv[2 * l], vhi = sv[2 * l + 1];
+            if ((vlo | vhi) == 0ull) continue;
+            const int sh = (l ? 8 * l : 1) - 1;  // bit position of the lane value's origin
+            const int d0 = sh >> 5, off = sh & 31;
+            // the value (< 2^75) as 32-bit words, shifted by off into 4 words
+            const uint32_t w[3] = {static_cast<uint32_t>(vlo), static_cast<uint32_t>(vlo >> 32),
+                                   static_cast<uint32_t>(vhi)};
+            uint32_t p[4];
+            p[0] = w[0] << off;
+            p[1] = off ? (w[1] << off) | (w[0] >> (32 - off)) : w[1];
+            p[2] = off ? (w[2] << off) | (w[1] >> (32 - off)) : w[2];
+            p[3] = off ? (w[2] >> (32 - off)) : 0u;
+            unsigned long long carry = 0;
+            for (int i = 0; d0 + i <= kDigits; ++i) {
+                const unsigned long long t = static_cast<unsigned long long>(d[d0 + i]) + (i < 4 ? p[i] : 0u) + carry;
+                d[d0 + i] = static_cast<uint32_t>(t);
+                carry = t >> 32;
+                if (i >= 3 && carry == 0) break;
+            }
         }
-        d[kDigits] = carry;
         int top = -1;
         for (int i = kDigits; i >= 0; --i)
             if (d[i]) { top = i; break; }
         double sum = 0.0;
         if (top >= 0) {
-            const int msb = 32 * top + 63 - __clzll(d[top]);  // bit index of the leading 1 (digits are < 2^32)
-            auto bit = [&](int k) -> unsigned long long {
-                return k < 0 ? 0ull : (d[k >> 5] >> (k & 31)) & 1ull;
-            };
-            // the 53 bits [msb-52, msb], the round bit below them, and a
-            // sticky bit for everything further down
-            const int lsb = msb - 52;
-            unsigned long long m = 0;
-            for (int k = msb; k >= (lsb > 0 ? lsb : 0); --k) m = (m << 1) | bit(k);
-            if (lsb > 0) {
-                const unsigned long long rnd = bit(lsb - 1);
-                const int below = lsb - 1;  // bits [0, below) feed the sticky bit
-                bool sticky = false;
-                for (int i = 0; i < (below >> 5) && !sticky; ++i) sticky = d[i] != 0;
-                if (!sticky && (below & 31))
-                    sticky = (d[below >> 5] & ((1ull << (below & 31)) - 1ull)) != 0;
-                if (rnd && (sticky || (m & 1ull))) m += 1ull;  // 2^53 stays exact
-                sum = ldexp(static_cast<double>(m), lsb - 149);
-            } else {
-                sum = ldexp(static_cast<double>(m), -149);
-            }
+            // the leading 64 bits of the total (digits top, top-1, top-2), left aligned
+            const unsigned long long t0 = (static_cast<unsigned long long>(d[top]) << 32) | (top >= 1 ? d[top - 1] : 0u);
+            const uint32_t t1 = top >= 2 ? d[top - 2] : 0u;
+            const int lz = __clzll(t0);  // < 32: d[top] != 0
+            const unsigned long long lead = lz ? (t0 << lz) | (static_cast<unsigned long long>(t1) >> (32 - lz)) : t0;
+            // bit position (over the whole total) of the lead's lowest bit
+            const int lead_lsb = 32 * top + 32 - lz - 64;  // = msb - 63, may be negative
+            unsigned long long m = lead >> 11;              // 53 bits
+            const bool rnd = (lead >> 10) & 1ull;
+            bool sticky = (lead & 0x3ffull) != 0;
+            // bits below the lead: the low lz bits of t1 and the digits under it
+            const uint32_t t1_below = lz ? (t1 & ((1u << (32 - lz)) - 1u)) : t1;  // t1's bits under the lead
+            sticky |= t1_below != 0u;
+            for (int i = 0; i < top - 2 && !sticky; ++i) sticky = d[i] != 0u;
+            if (rnd && (sticky || (m & 1ull))) m += 1ull;  // 2^53 stays exact
+            sum = ldexp(static_cast<double>(m), lead_lsb + 11 - 149);
         }
         mu = __double2float_rn(__ddiv_rn(sum, static_cast<double>(nb)));
     }
@@ -312,11 +326,11 @@ __global__ void __launch_bounds__(kDqThreads)
 k_double_quant(const float* __restrict__ c2, int64_t nb, const unsigned long long* __restrict__ bins,
                const int* __restrict__ flag, uint8_t* __restrict__ c2_fp8, float* __restrict__ c1,
                float* __restrict__ mean_out, int32_t* __restrict__ status) {
-    __shared__ unsigned long long sdig[kDigits];
+    __shared__ unsigned long long sv[64];
     __shared__ float smu;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == 0) {
-        const float mu = mean_from_bins(bins, nb, sdig);
+        const float mu = mean_from_bins(bins, nb, sv);
         if (lane == 0) smu = mu;
     }
     __syncthreads();
