@@ -137,11 +137,31 @@ __device__ __forceinline__ uint32_t slot_use(int kb, uint32_t tcount, int kb_tot
     return tcount * uses_per_tile + static_cast<uint32_t>(kb / kStages);
 }
 
+// Token tile and weight-row tile of persistent tile index `tile`.  The
+// forward walks the token tiles fastest (its activation X is shared by all
+// weight tiles and stays in L2); the backward walks the weight tiles
+// fastest, so the CTAs working at the same time share a few token tiles of
+// dY (whose full size can exceed L2) while the small transposed weight is
+// reused from L2.
+template <bool kBwd>
+__device__ __forceinline__ void tile_coords(const Pipe& P, int tile, int& t0, int& row0) {
+    if (kBwd) {
+        const int num_w = P.num_tiles / P.num_t;
+        t0 = (tile / num_w) * kTileT;
+        row0 = (tile % num_w) * kTileW;
+    } else {
+        t0 = (tile % P.num_t) * kTileT;
+        row0 = (tile / P.num_t) * kTileW;
+    }
+}
+
 // warp 0, one thread: activation tiles, then the LoRA slabs, into the ring.
+template <bool kBwd>
 __device__ void role_tma(const Pipe& P, const CUtensorMap* tmap_act, const CUtensorMap* tmap_lora, int* err) {
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x, ++tcount) {
-        const int t0 = (tile % P.num_t) * kTileT;
+        int t0, row0;
+        tile_coords<kBwd>(P, tile, t0, row0);
         for (int kb = 0; kb < P.kb_total; ++kb) {
             const int s = kb % kStages;
             const uint32_t ph = slot_use(kb, tcount, P.kb_total) & 1u;
@@ -246,8 +266,8 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
     const float mu = kBwd ? 0.0f : *p.mean;
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x, ++tcount) {
-        const int t0 = (tile % P.num_t) * kTileT;
-        const int row0 = (tile / P.num_t) * kTileW;
+        int t0, row0;
+        tile_coords<kBwd>(P, tile, t0, row0);
         const int grow = row0 + row;             // this lane's weight row of the product
         const bool lane_ok = grow < p.rows;
         const uint8_t* crow = p.codes + static_cast<int64_t>(grow) * p.ld_codes;
@@ -397,7 +417,7 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
     int* err = &g_tc_error;
 
     if (warp == 0) {
-        if (lane == 0) role_tma(P, &tmap_act, &tmap_lora, err);
+        if (lane == 0) role_tma<kBwd>(P, &tmap_act, &tmap_lora, err);
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) role_mma(P, err);
