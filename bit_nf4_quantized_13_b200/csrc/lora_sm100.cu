@@ -174,10 +174,17 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
             const int lr = split * rows_per + idx / q4;
             const int c = (idx % q4) * 4;
             const uint32_t off = static_cast<uint32_t>((lr * ld + c) * 4);
-            float4 sum = ld_cluster_f4(cluster_map(acc_s + off, 0));
-            for (int q = 1; q < p.splits; ++q) {
-                const float4 v = ld_cluster_f4(cluster_map(acc_s + off, static_cast<uint32_t>(q)));
-                sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+            // all ranks' values in flight together, then summed in rank order
+            float4 v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (q < p.splits) v[q] = ld_cluster_f4(cluster_map(acc_s + off, static_cast<uint32_t>(q)));
+            float4 sum = v[0];
+#pragma unroll
+            for (int q = 1; q < 8; ++q) {
+                if (q < p.splits) {
+                    sum.x += v[q].x; sum.y += v[q].y; sum.z += v[q].z; sum.w += v[q].w;
+                }
             }
             const int row = row0 + lr;
             if (row < p.rows && c < p.r) {
