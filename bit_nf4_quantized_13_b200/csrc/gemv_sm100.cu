@@ -9,10 +9,11 @@
 // targets HBM bandwidth, not tensor throughput:
 //
 //  * Work unit: 16 consecutive weight rows over all of K.  Each CTA of a
-//    cluster of C CTAs copies its K-slice of the 16 rows (one tensor-map
-//    box) plus the rows' FP8 constants (one bulk copy) into a stage of a
-//    shared-memory ring (3 to 6 deep).  Few, large copies matter: issuing
-//    a copy costs the producer thread on the order of a hundred cycles.
+//    cluster of C CTAs copies its K-slice of the 16 rows' codes (one
+//    tensor-map box) into a stage of a shared-memory ring (3 to 6 deep);
+//    the rows' FP8 block constants and c1 are plain loads, a unit ahead, by
+//    the lanes that form c2'.  Few, large copies matter: issuing a copy
+//    costs the producer thread hundreds of cycles under load.
 //  * Decode: a 256-entry table maps one code byte (two 4-bit codes) to the
 //    two bf16 codebook values as one 32-bit MMA operand register.  Each
 //    table entry is replicated across the 32 banks (lane l reads word l of
@@ -65,8 +66,6 @@ constexpr int kStages = 6;                   // most stages a launch uses
 constexpr int kSlotBufs = 4;                 // most units a CTA may run ahead of rank 0's epilogue
 constexpr int kLutBytes = 256 * 256;         // 256 entries x 64 words (32 used)
 constexpr int kMaxRankTiles = 4;             // r <= 64
-constexpr int kBRingMax = 8;                 // LoRA B tiles in flight ahead of the epilogue
-constexpr int kBRingBytes = 8192;            // ring size: kBRingMax tiles of 32 r bytes, at most
 constexpr int kTStride = 16 * kMaxRankTiles; // T staging row (ranks), bf16
 constexpr int kBarRedFull = 1;               // named barrier: partials written (compute warps arrive)
 constexpr int kBarRedFree = 2;               // named barrier: partials read (producer arrives)
@@ -94,7 +93,7 @@ struct GemvParams {
 };
 
 struct GemvSmem {
-    size_t red_off, slot_off, tslot_off, tbuf_off, bring_off, bar_off, total;
+    size_t red_off, slot_off, tslot_off, tbuf_off, bar_off, total;
 };
 
 __host__ __device__ constexpr GemvSmem gemv_smem(int NT, int stage_bytes, int nstages, int cl, int rt, int nslot) {
@@ -103,9 +102,8 @@ __host__ __device__ constexpr GemvSmem gemv_smem(int NT, int stage_bytes, int ns
     m.slot_off = m.red_off + kWarps * NT * 32 * 16;
     m.tslot_off = m.slot_off + static_cast<size_t>(nslot) * cl * NT * 32 * 16;
     m.tbuf_off = m.tslot_off + static_cast<size_t>(cl) * rt * NT * 32 * 16;
-    m.bring_off = m.tbuf_off + 16 * kTStride * 2;
-    m.bar_off = m.bring_off + kBRingBytes;
-    m.total = m.bar_off + (kStages + 2 * kSlotBufs + 1 + kBRingMax) * 8;
+    m.bar_off = m.tbuf_off + 16 * kTStride * 2;
+    m.total = m.bar_off + (kStages + 2 * kSlotBufs + 1) * 8;
     return m;
 }
 
@@ -127,27 +125,30 @@ __device__ __forceinline__ void bar_wait(int id) {
     named_bar_sync(id, kThreads);
 }
 
-// Issues the copies of unit `u` into `stage`, completing on `bar`: one
+// Issues the copy of unit `u` into `stage`, completing on `bar`: one
 // tensor-map box of the codes (16 rows x row_stride bytes from block b0 on;
 // this CTA's blocks plus a few of the next slice, or zeros past the row,
-// which also pads the rows to a bank-friendly pitch) and one bulk copy of
-// the rows' FP8 constants.
+// which also pads the rows to a bank-friendly pitch).
 __device__ __forceinline__ void issue_unit(const CUtensorMap* map, const GemvParams& p, int u, uint8_t* stage,
                                            uint64_t* bar, int b0) {
     const uint32_t b = smem_u32(bar);
-    const uint32_t strip_bytes = static_cast<uint32_t>(kRows * p.KB);
-    mbar_arrive_expect_tx(b, kRows * p.row_stride + strip_bytes);
+    mbar_arrive_expect_tx(b, kRows * p.row_stride);
     tma_load_2d(smem_u32(stage), map, b, b0 * 4, u * kRows);
-    bulk_load(smem_u32(stage + kRows * p.row_stride), p.c2_fp8 + static_cast<int64_t>(u) * kRows * p.KB,
-              strip_bytes, b);
 }
 
-// The 16 rows of B that unit `u` needs (rows 16u .. 16u+15, contiguous
-// 32 r bytes) into ring tile `tile`, completing on `bar`.
-__device__ __forceinline__ void issue_b_tile(const GemvParams& p, int u, uint8_t* tile, uint64_t* bar) {
-    const uint32_t bytes = static_cast<uint32_t>(kRows * p.r * 2);
-    mbar_arrive_expect_tx(smem_u32(bar), bytes);
-    bulk_load(smem_u32(tile), p.B + static_cast<int64_t>(u) * kRows * p.r, bytes, smem_u32(bar));
+// Rows 16u + g and 16u + g + 8 of B as the A operand of the LoRA MMA
+// (ranks 16 st ..), plain loads issued a unit ahead of their use.
+__device__ __forceinline__ void load_b_rows(const GemvParams& p, int u, int g, int qd,
+                                            uint32_t (&a)[kMaxRankTiles][4]) {
+#pragma unroll
+    for (int st = 0; st < kMaxRankTiles; ++st) {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const int64_t row = static_cast<int64_t>(u) * kRows + g + 8 * (h & 1);
+            const int j = 16 * st + 2 * qd + 8 * (h >> 1);
+            a[st][h] = j < p.r ? __ldg(reinterpret_cast<const uint32_t*>(p.B + row * p.r + j)) : 0u;
+        }
+    }
 }
 
 // Sum of the 15 compute warps' partials (fragment layout), warp order.
@@ -175,7 +176,7 @@ __device__ __forceinline__ void sum_partials(const float4* red, int lane, float4
 template <int NT>
 __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const GemvParams& p, uint8_t* smem, const GemvSmem& L, uint64_t* full,
                                               uint64_t* slot_full, uint64_t* slot_empty, uint64_t* t_full,
-                                              uint64_t* bfull, uint32_t crank, int cid, int ncl, int n_local,
+                                              uint32_t crank, int cid, int ncl, int n_local,
                                               int b0, int nblk, int lane) {
     const int g = lane >> 2, qd = lane & 3;
     const int RT = (p.r + 15) >> 4;
@@ -185,12 +186,10 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const Gemv
     const float4* slot = reinterpret_cast<const float4*>(smem + L.slot_off);
     const float4* tslot = reinterpret_cast<const float4*>(smem + L.tslot_off);
     uint16_t* tbuf = reinterpret_cast<uint16_t*>(smem + L.tbuf_off);  // [16 tokens][kTStride]
-    uint8_t* bring = smem + L.bring_off;
     const uint32_t slot_bytes = static_cast<uint32_t>(p.cl) * NT * 32 * 16;
-    const int tile_bytes = kRows * p.r * 2;
-    int nring = kBRingBytes / tile_bytes;
-    nring = nring < kBRingMax ? nring : kBRingMax;
     const bool rank0 = crank == 0;
+    uint32_t ba[kMaxRankTiles][4];  // rank 0: B rows of the next unit to finish
+    if (rank0 && n_local > 0) load_b_rows(p, cid, g, qd, ba);
 
     if (lane == 0) {
         const int pre = n_local < nst ? n_local : nst;
@@ -198,8 +197,6 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const Gemv
         if (rank0) {
             mbar_arrive_expect_tx(smem_u32(t_full), static_cast<uint32_t>(p.cl) * RT * NT * 32 * 16);
             for (int b = 0; b < p.nslot; ++b) mbar_arrive_expect_tx(smem_u32(&slot_full[b]), slot_bytes);
-            for (int u = 0; u < nring && u < n_local; ++u)
-                issue_b_tile(p, cid + u * ncl, bring + u * tile_bytes, &bfull[u]);
         }
     }
     const uint32_t tslot_r0 = cluster_map(smem_u32(smem + L.tslot_off), 0);
@@ -256,7 +253,7 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const Gemv
                                                          : 0u;
             t_ready = true;
         }
-        const int b = i % p.nslot, k = i / p.nslot, rb = i % nring;
+        const int b = i % p.nslot, k = i / p.nslot;
         const int n0 = (cid + i * ncl) * kRows;
         mbar_wait(smem_u32(&slot_full[b]), k & 1, &g_gemv_error);
         float acc[NT][4];
@@ -275,26 +272,14 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const Gemv
             __syncwarp();
             if (lane < p.cl) mbar_arrive_cluster(cluster_map(smem_u32(&slot_empty[b]), lane));
         }
-        mbar_wait(smem_u32(&bfull[rb]), (i / nring) & 1, &g_gemv_error);
-        const uint16_t* bt = reinterpret_cast<const uint16_t*>(bring + rb * tile_bytes);
 #pragma unroll
         for (int st = 0; st < kMaxRankTiles; ++st) {
             if (16 * st >= p.r) break;
-            uint32_t a[4];  // a0a1: row g, a2a3: row g+8, a4..a7: the same 8 ranks further
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const int j = 16 * st + 2 * qd + 8 * (h >> 1);
-                a[h] = j < p.r ? *reinterpret_cast<const uint32_t*>(bt + (g + 8 * (h & 1)) * p.r + j) : 0u;
-            }
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-                mma_16816(acc[nt], a[0], a[1], a[2], a[3], tf[nt][st][0], tf[nt][st][1]);
+            for (int nt = 0; nt < NT; ++nt)  // A: a0a1 row g, a2a3 row g+8, a4..a7 the same 8 ranks further
+                mma_16816(acc[nt], ba[st][0], ba[st][1], ba[st][2], ba[st][3], tf[nt][st][0], tf[nt][st][1]);
         }
-        __syncwarp();
-        if (lane == 0 && i + nring < n_local) {  // refill the tile just read
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            issue_b_tile(p, cid + (i + nring) * ncl, bring + rb * tile_bytes, &bfull[rb]);
-        }
+        if (i + 1 < n_local) load_b_rows(p, cid + (i + 1) * ncl, g, qd, ba);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -325,21 +310,14 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const Gemv
     if (rank0 && n_local > 0) finish(n_local - 1);
 }
 
+// X fragments of warp `warp`'s blocks: block jloc = warp + kWarps * jj.
+// Lane (g, qd) of token tile nt holds X[nt*8 + g][64*kb + 16*qd .. +16);
+// inside a block, k is permuted alike in both MMA operands so that MMA t of
+// the block takes the elements 4t .. 4t+3 of every lane's run.
 template <int NT>
-__device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem, const GemvSmem& L, uint64_t* full,
-                                             int cid, int ncl, int n_local, int b0, int nblk, int warp, int lane) {
+__device__ __forceinline__ void load_x_frags(const GemvParams& p, int b0, int nblk, int warp, int lane,
+                                             uint32_t (&xf)[kMaxBw][NT][8]) {
     const int g = lane >> 2, qd = lane & 3;
-    const int RT = (p.r + 15) >> 4;
-    const int nst = p.nstages;
-    const uint8_t* lut = smem;
-    const uint8_t* stages = smem + kLutBytes;
-    float4* red = reinterpret_cast<float4*>(smem + L.red_off) + warp * NT * 32;  // this warp's [NT][32]
-
-    // X fragments of this warp's blocks: block jloc = warp + kWarps * jj.
-    // Lane (g, qd) of token tile nt holds X[nt*8 + g][64*kb + 16*qd .. +16);
-    // inside a block, k is permuted alike in both MMA operands so that
-    // MMA t of the block takes the elements 4t .. 4t+3 of every lane's run.
-    uint32_t xf[kMaxBw][NT][8];
 #pragma unroll
     for (int jj = 0; jj < kMaxBw; ++jj) {
         const int jloc = warp + kWarps * jj;
@@ -357,6 +335,18 @@ __device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem,
             xf[jj][nt][4] = hi.x; xf[jj][nt][5] = hi.y; xf[jj][nt][6] = hi.z; xf[jj][nt][7] = hi.w;
         }
     }
+}
+
+template <int NT>
+__device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem, const GemvSmem& L, uint64_t* full,
+                                             int cid, int ncl, int n_local, int b0, int nblk, int warp, int lane,
+                                             const uint32_t (&xf)[kMaxBw][NT][8]) {
+    const int g = lane >> 2, qd = lane & 3;
+    const int RT = (p.r + 15) >> 4;
+    const int nst = p.nstages;
+    const uint8_t* lut = smem;
+    const uint8_t* stages = smem + kLutBytes;
+    float4* red = reinterpret_cast<float4*>(smem + L.red_off) + warp * NT * 32;  // this warp's [NT][32]
 
     // This CTA's part of X A^T, one 16-rank tile at a time: the rows of A
     // are the MMA's A operand in the same permuted k order as the codes.
@@ -400,28 +390,31 @@ __device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem,
 
     const float mean = __ldg(p.mean);
     const uint32_t lane_off = static_cast<uint32_t>(lane) * 4;
-    // c1 of (row = lane, block jloc) of unit i, for lanes < 16
-    auto load_c1 = [&](int i, float (&c1v)[kMaxBw]) {
+    // inputs of the block constant of (row = lane, block jloc) of unit i, for
+    // lanes < 16: the FP8 byte and c1, loaded a unit ahead of their use
+    auto load_consts = [&](int i, float (&c1v)[kMaxBw], uint32_t (&fb)[kMaxBw]) {
 #pragma unroll
         for (int jj = 0; jj < kMaxBw; ++jj) {
             const int jloc = warp + kWarps * jj;
             c1v[jj] = 0.0f;
+            fb[jj] = 0u;
             if (lane < kRows && jloc < nblk && i < n_local) {
                 const int64_t blk = (static_cast<int64_t>(cid + i * ncl) * kRows + lane) * p.KB + b0 + jloc;
                 c1v[jj] = __ldg(p.c1 + (blk >> 8));
+                fb[jj] = __ldg(p.c2_fp8 + blk);
             }
         }
     };
     float c1c[kMaxBw], c1n[kMaxBw];
-    load_c1(0, c1c);
+    uint32_t fbc[kMaxBw], fbn[kMaxBw];
+    load_consts(0, c1c, fbc);
 
 #pragma unroll 1
     for (int i = 0; i < n_local; ++i) {
         const int s = i % nst;
-        load_c1(i + 1, c1n);  // the next unit's: the loads overlap this unit
+        load_consts(i + 1, c1n, fbn);  // the next unit's: the loads overlap this unit
         mbar_wait(smem_u32(&full[s]), (i / nst) & 1, &g_gemv_error);
         const uint8_t* stg = stages + s * p.stage_bytes;
-        const uint8_t* strip = stg + kRows * p.row_stride;
 
         float acc[NT][4];
 #pragma unroll
@@ -434,7 +427,7 @@ __device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem,
                 const uint2 ch = *reinterpret_cast<const uint2*>(stg + (g + 8) * p.row_stride + jloc * 32 + qd * 8);
                 // block constants c2' of the 16 rows: lane r < 16 forms row r's, then shuffles
                 float c2v = 0.0f;
-                if (lane < kRows) c2v = dq_constant(strip[lane * p.KB + b0 + jloc], c1c[jj], mean);
+                if (lane < kRows) c2v = dq_constant(static_cast<uint8_t>(fbc[jj]), c1c[jj], mean);
                 const float sg = __shfl_sync(0xffffffffu, c2v, g);
                 const float sh = __shfl_sync(0xffffffffu, c2v, g + 8);
                 float bacc[NT][4];
@@ -464,7 +457,10 @@ __device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem,
             }
         }
 #pragma unroll
-        for (int jj = 0; jj < kMaxBw; ++jj) c1c[jj] = c1n[jj];
+        for (int jj = 0; jj < kMaxBw; ++jj) {
+            c1c[jj] = c1n[jj];
+            fbc[jj] = fbn[jj];
+        }
         bar_wait(kBarRedFree);  // the producer has read the previous partials
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) red[nt * 32 + lane] = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
@@ -483,7 +479,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemv_nf4(const __grid_constant_
     uint64_t* slot_full = full + kStages;          // rank 0: a unit's partials have all landed
     uint64_t* slot_empty = slot_full + kSlotBufs;  // every rank: rank 0 has read the buffer
     uint64_t* t_full = slot_empty + kSlotBufs;     // rank 0: the T partials have all landed
-    uint64_t* bfull = t_full + 1;                  // rank 0: LoRA B tiles
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t crank = cluster_ctarank();
@@ -493,8 +488,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemv_nf4(const __grid_constant_
     const int nblk = static_cast<int>(static_cast<int64_t>(crank + 1) * p.KB / p.cl) - b0;
     const int n_local = cid < p.units ? (p.units - 1 - cid) / ncl + 1 : 0;
 
+    // the compute warps' X fragments first: their loads fly during the set-up
+    uint32_t xf[kMaxBw][NT][8];
+    if (warp < kWarps) load_x_frags<NT>(p, b0, nblk, warp, lane, xf);
     if (tid == 0) {
-        for (int i = 0; i < kStages + 2 * kSlotBufs + 1 + kBRingMax; ++i) mbar_init(smem_u32(&full[i]), 1);
+        for (int i = 0; i < kStages + 2 * kSlotBufs + 1; ++i) mbar_init(smem_u32(&full[i]), 1);
         fence_barrier_init();
     }
     if (tid < 256) {  // the decode table: entry v replicated into words 0..31 of row v
@@ -508,10 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemv_nf4(const __grid_constant_
     cluster_wait();
 
     if (warp == kWarps)
-        producer_warp<NT>(&map_codes, p, smem, L, full, slot_full, slot_empty, t_full, bfull, crank, cid, ncl, n_local, b0, nblk,
-                          lane);
+        producer_warp<NT>(&map_codes, p, smem, L, full, slot_full, slot_empty, t_full, crank, cid, ncl, n_local, b0,
+                          nblk, lane);
     else
-        compute_warp<NT>(p, smem, L, full, cid, ncl, n_local, b0, nblk, warp, lane);
+        compute_warp<NT>(p, smem, L, full, cid, ncl, n_local, b0, nblk, warp, lane, xf);
     cluster_arrive();  // no CTA leaves while cluster peers may still address its shared memory
     cluster_wait();
 }
@@ -572,7 +570,7 @@ bool make_plan(int64_t N, int64_t K, int r, Plan& best) {
         pl.cl = cl;
         pl.row_stride = static_cast<int>(round_up(maxblk * 32, 128) + 32);  // = 32 mod 128: no bank conflicts
         if (pl.row_stride / 8 > 256) continue;                                 // tensor-map box width
-        pl.stage_bytes = static_cast<int>(round_up(kRows * pl.row_stride + round_up(kRows * KB, 128), 128));
+        pl.stage_bytes = static_cast<int>(round_up(kRows * pl.row_stride, 128));
         pl.nstages = 0;
         for (int nslot = kSlotBufs; nslot >= 2 && !pl.nstages; nslot /= 2) {
             for (int ns = kStages; ns >= 3 && !pl.nstages; --ns)
