@@ -34,11 +34,12 @@
 //  * T = bf16(s X A^T) is formed in the same kernel from the register
 //    resident X fragments (the rows of A take the MMA's A operand in the
 //    permuted k order), reduced over the cluster like the unit partials.
-//  * 15 decode warps per CTA run free of one another; a 16th warp issues
-//    the copies and sums their partials (named-barrier hand-off).  It pushes
+//  * 14 decode warps per CTA run free of one another; a 15th warp issues
+//    the copies and sums their partials (named-barrier hand-off) and pushes
 //    the CTA's partial into rank 0's shared memory with st.async (completing
-//    on an mbarrier); rank 0's producer warp finishes each unit one unit
-//    behind and hands the slot buffers (up to 4) back with remote arrives.
+//    on an mbarrier); in rank 0 a 16th warp finishes the units as their
+//    partials land and hands the slot buffers (up to 4) back with remote
+//    arrives, so no warp's per-unit work serialises behind another's.
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -56,9 +57,10 @@ using namespace sm100;
 __device__ int g_gemv_error;
 
 constexpr int kRows = 16;                    // weight rows per unit
-constexpr int kWarps = 15;                   // decode + MMA warps
+constexpr int kWarps = 14;                   // decode + MMA warps
 constexpr int kCompute = kWarps * 32;
-constexpr int kThreads = kCompute + 32;      // + the producer warp (16 warps: 128 registers a thread)
+constexpr int kBarThreads = kCompute + 32;   // named-barrier hand-off: compute warps + producer warp
+constexpr int kThreads = kBarThreads + 32;   // + the epilogue warp (16 warps: 128 registers a thread)
 constexpr int kMaxBw = 3;                    // 64-blocks per warp per unit
 constexpr int kMaxCtaBlocks = kWarps * kMaxBw;
 constexpr int kMaxCl = 8;                    // CTAs per cluster
@@ -118,11 +120,11 @@ __device__ __forceinline__ uint32_t lut_pair(const uint8_t* lut, uint32_t word, 
 // the warp is reconverged first (the barriers are warp-aligned).
 __device__ __forceinline__ void bar_arrive(int id) {
     __syncwarp();
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(kBarThreads) : "memory");
 }
 __device__ __forceinline__ void bar_wait(int id) {
     __syncwarp();
-    named_bar_sync(id, kThreads);
+    named_bar_sync(id, kBarThreads);
 }
 
 // Issues the copy of unit `u` into `stage`, completing on `bar`: one
@@ -168,11 +170,7 @@ __device__ __forceinline__ void sum_partials(const float4* red, int lane, float4
 
 // The producer warp of every CTA: issues the stage copies, reduces the
 // compute warps' partials and pushes the CTA's partial of T and of every
-// unit into rank 0's shared memory (st.async).  In rank 0 it also runs the
-// epilogue, one unit behind: T = bf16(s * sum of the T partials in rank
-// order) once, then per unit the C partials summed in rank order, the slot
-// buffer handed back to every CTA, T B^T added with one MMA per 16 ranks
-// and Y stored.
+// unit into rank 0's shared memory (st.async).
 template <int NT>
 __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const GemvParams& p, uint8_t* smem, const GemvSmem& L, uint64_t* full,
                                               uint64_t* slot_full, uint64_t* slot_empty, uint64_t* t_full,
@@ -185,19 +183,10 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const Gemv
     const float4* red = reinterpret_cast<const float4*>(smem + L.red_off);
     const float4* slot = reinterpret_cast<const float4*>(smem + L.slot_off);
     const float4* tslot = reinterpret_cast<const float4*>(smem + L.tslot_off);
-    uint16_t* tbuf = reinterpret_cast<uint16_t*>(smem + L.tbuf_off);  // [16 tokens][kTStride]
-    const uint32_t slot_bytes = static_cast<uint32_t>(p.cl) * NT * 32 * 16;
-    const bool rank0 = crank == 0;
-    uint32_t ba[kMaxRankTiles][4];  // rank 0: B rows of the next unit to finish
-    if (rank0 && n_local > 0) load_b_rows(p, cid, g, qd, ba);
 
     if (lane == 0) {
         const int pre = n_local < nst ? n_local : nst;
         for (int i = 0; i < pre; ++i) issue_unit(map, p, cid + i * ncl, stages + i * p.stage_bytes, &full[i], b0);
-        if (rank0) {
-            mbar_arrive_expect_tx(smem_u32(t_full), static_cast<uint32_t>(p.cl) * RT * NT * 32 * 16);
-            for (int b = 0; b < p.nslot; ++b) mbar_arrive_expect_tx(smem_u32(&slot_full[b]), slot_bytes);
-        }
     }
     const uint32_t tslot_r0 = cluster_map(smem_u32(smem + L.tslot_off), 0);
     const uint32_t t_full_r0 = cluster_map(smem_u32(t_full), 0);
@@ -216,9 +205,47 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const Gemv
                         t_full_r0);
     }
 
+#pragma unroll 1
+    for (int i = 0; i < n_local; ++i) {
+        bar_wait(kBarRedFull);  // unit i's partials are written: its stage is free too
+        if (lane == 0 && i + nst < n_local)
+            issue_unit(map, p, cid + (i + nst) * ncl, stages + (i % nst) * p.stage_bytes, &full[i % nst], b0);
+        float4 v[NT];
+        sum_partials<NT>(red, lane, v);
+        bar_arrive(kBarRedFree);
+        const int b = i % p.nslot, k = i / p.nslot;
+        if (k >= 1) mbar_wait(smem_u32(&slot_empty[b]), (k - 1) & 1, &g_gemv_error);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+            st_async_f4(slot_r0 + static_cast<uint32_t>((((b * p.cl + crank) * NT + nt) * 32 + lane) * 16), v[nt],
+                        slot_full_r0 + static_cast<uint32_t>(b * 8));
+    }
+}
+
+// Rank 0's epilogue warp, one unit behind the partials: T = bf16(s * sum of
+// the T partials in rank order) once, then per unit the C partials summed in
+// rank order, the slot buffer handed back to every CTA, T B^T added with one
+// MMA per 16 ranks and Y stored.
+template <int NT>
+__device__ __forceinline__ void epilogue_warp(const GemvParams& p, uint8_t* smem, const GemvSmem& L,
+                                              uint64_t* slot_full, uint64_t* slot_empty, uint64_t* t_full, int cid,
+                                              int ncl, int n_local, int lane) {
+    const int g = lane >> 2, qd = lane & 3;
+    const int RT = (p.r + 15) >> 4;
+    const float4* slot = reinterpret_cast<const float4*>(smem + L.slot_off);
+    const float4* tslot = reinterpret_cast<const float4*>(smem + L.tslot_off);
+    uint16_t* tbuf = reinterpret_cast<uint16_t*>(smem + L.tbuf_off);  // [16 tokens][kTStride]
+    const uint32_t slot_bytes = static_cast<uint32_t>(p.cl) * NT * 32 * 16;
+    if (lane == 0) {
+        mbar_arrive_expect_tx(smem_u32(t_full), static_cast<uint32_t>(p.cl) * RT * NT * 32 * 16);
+        for (int b = 0; b < p.nslot; ++b) mbar_arrive_expect_tx(smem_u32(&slot_full[b]), slot_bytes);
+    }
+    uint32_t ba[kMaxRankTiles][4];  // B rows of the next unit to finish
+    if (n_local > 0) load_b_rows(p, cid, g, qd, ba);
     uint32_t tf[NT][kMaxRankTiles][2];
     bool t_ready = false;
-    auto finish = [&](int i) {
+#pragma unroll 1
+    for (int i = 0; i < n_local; ++i) {
         if (!t_ready) {  // T: lane holds (rank 16 rt + g (+8), token 8 nt + 2 qd (+1)) of every tile
             mbar_wait(smem_u32(t_full), 0, &g_gemv_error);
             for (int rt = 0; rt < RT; ++rt) {
@@ -289,25 +316,8 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const Gemv
                 if (tok < p.M) p.Y[static_cast<int64_t>(tok) * p.N + row] = f32_to_bf16_bits(acc[nt][e]);
             }
         }
-    };
-
-#pragma unroll 1
-    for (int i = 0; i < n_local; ++i) {
-        bar_wait(kBarRedFull);  // unit i's partials are written: its stage is free too
-        if (lane == 0 && i + nst < n_local)
-            issue_unit(map, p, cid + (i + nst) * ncl, stages + (i % nst) * p.stage_bytes, &full[i % nst], b0);
-        float4 v[NT];
-        sum_partials<NT>(red, lane, v);
-        bar_arrive(kBarRedFree);
-        const int b = i % p.nslot, k = i / p.nslot;
-        if (k >= 1) mbar_wait(smem_u32(&slot_empty[b]), (k - 1) & 1, &g_gemv_error);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-            st_async_f4(slot_r0 + static_cast<uint32_t>((((b * p.cl + crank) * NT + nt) * 32 + lane) * 16), v[nt],
-                        slot_full_r0 + static_cast<uint32_t>(b * 8));
-        if (rank0 && i >= 1) finish(i - 1);
     }
-    if (rank0 && n_local > 0) finish(n_local - 1);
+
 }
 
 // X fragments of warp `warp`'s blocks: block jloc = warp + kWarps * jj.
@@ -508,7 +518,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemv_nf4(const __grid_constant_
     if (warp == kWarps)
         producer_warp<NT>(&map_codes, p, smem, L, full, slot_full, slot_empty, t_full, crank, cid, ncl, n_local, b0,
                           nblk, lane);
-    else
+    else if (warp == kWarps + 1) {
+        if (crank == 0) epilogue_warp<NT>(p, smem, L, slot_full, slot_empty, t_full, cid, ncl, n_local, lane);
+    } else
         compute_warp<NT>(p, smem, L, full, cid, ncl, n_local, b0, nblk, warp, lane, xf);
     cluster_arrive();  // no CTA leaves while cluster peers may still address its shared memory
     cluster_wait();
