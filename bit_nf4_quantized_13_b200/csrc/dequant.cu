@@ -4,10 +4,13 @@
 // the NF4 type and scaled by its block constant.
 //
 // HBM-bound: 0.5 + 1/64 + 1/16384 bytes read and 4 (fp32) or 2 (bf16) bytes
-// written per weight.  Each lane expands 32 consecutive weights per step
-// from one 16-byte load of codes and one block constant; code nibbles become
-// table byte offsets with shift/mask and byte_perm, and pairs of weights are
-// scaled with one f32x2 multiply.
+// written per weight, the writes dominating.  A warp expands 1024 weights
+// per step; lane l takes the four 8-weight groups at 8 l + 256 i, so each
+// load instruction reads one contiguous 128-byte run of codes and each
+// bf16 store instruction writes one contiguous 512-byte run (whole sectors).
+// A code byte becomes both of its fp32 codebook values through a 256-entry
+// table with one copy per lane (no bank conflicts): one byte permute and
+// one shared load per two weights.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -15,101 +18,118 @@ namespace qlora {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kRun = 32;  // weights per lane per step: 16 code bytes, one block constant
+constexpr int kChunk = 1024;  // weights per warp per step
+constexpr int kLutBytes = 256 * 256;
 
-__device__ __forceinline__ uint4 ld_nc_v4(const uint8_t* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
+// (q[high nibble], q[low nibble]) of one code byte from the lane's copy
+__device__ __forceinline__ float2 lut_pair(const uint8_t* lut, uint32_t word, uint32_t lane_off, int byte) {
+    const uint32_t addr = __byte_perm(word, lane_off, 0x5504u | (static_cast<uint32_t>(byte) << 4));
+    return *reinterpret_cast<const float2*>(lut + addr);
+}
+
+__device__ __forceinline__ uint32_t ld_nc_u32(const uint8_t* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
     return v;
 }
 
-// q[code] from the 16-entry table by byte offset (code * 4)
-__device__ __forceinline__ float lut_at(const float* lut, uint32_t byte_off) {
-    return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(lut) + byte_off);
-}
-
-// 32 weights of one block from 16 code bytes: element 2t is the high nibble
-// of byte t.  out[i] = RN32(q[code_i] * c2').
-__device__ __forceinline__ void expand32(const uint4& cw, float cp, const float* lut, float (&w)[kRun]) {
-    const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+// 8 weights of one group (4 code bytes, element 2t the high nibble of byte
+// t) scaled by the block constant: w[i] = RN32(q[code_i] * c2').
+__device__ __forceinline__ void expand8(uint32_t cw, float cp, const uint8_t* lut, uint32_t lane_off, float (&w)[8]) {
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        const uint32_t hi4 = (w4[h] >> 2) & 0x3C3C3C3Cu;
-        const uint32_t lo4 = (w4[h] << 2) & 0x3C3C3C3Cu;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float2 x = __fmul2_rn(make_float2(lut_at(lut, __byte_perm(hi4, 0u, 0x4440u | j)),
-                                                    lut_at(lut, __byte_perm(lo4, 0u, 0x4440u | j))),
-                                        make_float2(cp, cp));
-            w[8 * h + 2 * j] = x.x;
-            w[8 * h + 2 * j + 1] = x.y;
-        }
+    for (int j = 0; j < 4; ++j) {
+        const float2 q2 = lut_pair(lut, cw, lane_off, j);
+        w[2 * j] = __fmul_rn(q2.x, cp);
+        w[2 * j + 1] = __fmul_rn(q2.y, cp);
     }
 }
 
-// Each lane owns 32 consecutive weights per step (one 16-byte load of
-// codes, one block constant), grid-stride with the next step's loads in
-// flight.  OUT_BF16 selects bf16 (64-byte) or fp32 (128-byte) output runs.
+template <bool OUT_BF16>
+__device__ __forceinline__ void store8(void* out, int64_t e, const float (&w)[8]) {
+    if (OUT_BF16) {
+        __stcs(reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + e),
+               make_uint4(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]), pack_bf16x2(w[4], w[5]),
+                          pack_bf16x2(w[6], w[7])));
+    } else {
+        float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + e);
+        __stcs(o, make_float4(w[0], w[1], w[2], w[3]));
+        __stcs(o + 1, make_float4(w[4], w[5], w[6], w[7]));
+    }
+}
+
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(kThreads)
 k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
           const float* __restrict__ c1, const float* __restrict__ mean, int64_t numel,
           void* __restrict__ out, Nf4Tables tabs) {
-    __shared__ float s_lut[16];
-    if (threadIdx.x < 16) s_lut[threadIdx.x] = tabs.q[threadIdx.x];
+    extern __shared__ __align__(16) uint8_t lut[];  // entry b, lane l at 256 b + 8 l
+    for (int i = threadIdx.x; i < 256 * 32; i += kThreads)
+        reinterpret_cast<float2*>(lut)[i] = make_float2(tabs.q[i >> 9], tabs.q[(i >> 5) & 15]);
     __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const uint32_t lane_off = static_cast<uint32_t>(lane) * 8;
     const float mu = *mean;
-    const int64_t nfull = numel / kRun;  // whole 32-weight runs
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t nfull = numel / kChunk;  // whole 1024-weight chunks
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+    int64_t c = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
 
-    uint4 cw = make_uint4(0u, 0u, 0u, 0u);
-    uint32_t sb = 0u;
-    float sc1 = 0.0f;
-    auto load = [&](int64_t run, uint4& c, uint32_t& b, float& s1) {
-        const int64_t e = run * kRun;
-        c = ld_nc_v4(codes + (e >> 1));
-        b = __ldg(c2_fp8 + (e >> 6));
-        s1 = __ldg(c1 + (e >> 14));
-    };
-    if (t < nfull) load(t, cw, sb, sc1);
-    for (; t < nfull; t += stride) {
-        uint4 ncw = cw;
-        uint32_t nsb = sb;
-        float ns1 = sc1;
-        if (t + stride < nfull) load(t + stride, ncw, nsb, ns1);
-        float w[kRun];
-        expand32(cw, dq_constant(static_cast<uint8_t>(sb), sc1, mu), s_lut, w);
-        const int64_t e = t * kRun;
-        if (OUT_BF16) {
-            uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + e);
+    // the lane's four groups of chunk c: codes and the constants' inputs
+    uint32_t cw[4], fb[4];
+    float s1[4];
+    auto load = [&](int64_t ch, uint32_t (&w)[4], uint32_t (&b)[4], float (&x)[4]) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                __stcs(o + c, make_uint4(pack_bf16x2(w[8 * c + 0], w[8 * c + 1]), pack_bf16x2(w[8 * c + 2], w[8 * c + 3]),
-                                         pack_bf16x2(w[8 * c + 4], w[8 * c + 5]), pack_bf16x2(w[8 * c + 6], w[8 * c + 7])));
-        } else {
-            float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + e);
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                __stcs(o + c, make_float4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]));
+        for (int i = 0; i < 4; ++i) {
+            const int64_t e = ch * kChunk + 8 * lane + 256 * i;
+            w[i] = ld_nc_u32(codes + (e >> 1));
+            b[i] = __ldg(c2_fp8 + (e >> 6));
+            x[i] = __ldg(c1 + (e >> 14));
         }
-        cw = ncw;
-        sb = nsb;
-        sc1 = ns1;
+    };
+    if (c < nfull) load(c, cw, fb, s1);
+    for (; c < nfull; c += nwarps) {
+        uint32_t ncw[4] = {cw[0], cw[1], cw[2], cw[3]}, nfb[4] = {fb[0], fb[1], fb[2], fb[3]};
+        float ns1[4] = {s1[0], s1[1], s1[2], s1[3]};
+        if (c + nwarps < nfull) load(c + nwarps, ncw, nfb, ns1);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float w[8];
+            expand8(cw[i], dq_constant(static_cast<uint8_t>(fb[i]), s1[i], mu), lut, lane_off, w);
+            store8<OUT_BF16>(out, c * kChunk + 8 * lane + 256 * i, w);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            cw[i] = ncw[i];
+            fb[i] = nfb[i];
+            s1[i] = ns1[i];
+        }
     }
-    // ragged tail (< 32 weights), one thread
-    if (blockIdx.x == 0 && threadIdx.x == 0 && nfull * kRun < numel) {
-        for (int64_t e = nfull * kRun; e < numel; ++e) {
-            const uint8_t byte = codes[e >> 1];
-            const int code = (e & 1) ? (byte & 15) : (byte >> 4);
+    // the ragged last chunk (< 1024 weights), by one warp: whole 8-weight
+    // groups vectorized, the last partial group element by element
+    const int64_t wid = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    if (nfull * kChunk < numel && wid == nfull % nwarps) {
+#pragma unroll 1
+        for (int i = 0; i < 4; ++i) {
+            const int64_t e = nfull * kChunk + 8 * lane + 256 * i;
+            if (e >= numel) continue;
             const float cp = dq_constant(c2_fp8[e >> 6], c1[e >> 14], mu);
-            const float v = __fmul_rn(s_lut[code], cp);
-            if (OUT_BF16)
-                reinterpret_cast<uint16_t*>(out)[e] = f32_to_bf16_bits(v);
-            else
-                reinterpret_cast<float*>(out)[e] = v;
+            if (e + 8 <= numel) {
+                const uint32_t w4 = static_cast<uint32_t>(codes[e >> 1]) | (static_cast<uint32_t>(codes[(e >> 1) + 1]) << 8) |
+                                    (static_cast<uint32_t>(codes[(e >> 1) + 2]) << 16) |
+                                    (static_cast<uint32_t>(codes[(e >> 1) + 3]) << 24);
+                float w[8];
+                expand8(w4, cp, lut, lane_off, w);
+                store8<OUT_BF16>(out, e, w);
+            } else {
+                for (int64_t k = e; k < numel; ++k) {
+                    const uint8_t byte = codes[k >> 1];
+                    const int code = (k & 1) ? (byte & 15) : (byte >> 4);
+                    const float v = __fmul_rn(tabs.q[code], cp);
+                    if (OUT_BF16)
+                        reinterpret_cast<uint16_t*>(out)[k] = f32_to_bf16_bits(v);
+                    else
+                        reinterpret_cast<float*>(out)[k] = v;
+                }
+            }
         }
     }
 }
@@ -119,13 +139,19 @@ k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,
                               const float* mean, int64_t numel, void* out, int out_dtype,
                               cudaStream_t stream) {
-    const int64_t runs = ceil_div(numel, kRun);
-    const int64_t want = ceil_div(runs, kThreads);
-    const int grid = static_cast<int>(want < num_sms() * 8LL ? (want > 0 ? want : 1) : num_sms() * 8LL);
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(k_dequant<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutBytes);
+        cudaFuncSetAttribute(k_dequant<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutBytes);
+        attr = true;
+    }
+    const int64_t chunks = ceil_div(numel, kChunk);
+    const int64_t want = ceil_div(chunks, kThreads / 32);
+    const int grid = static_cast<int>(want < num_sms() * 3LL ? (want > 0 ? want : 1) : num_sms() * 3LL);
     if (out_dtype == 1)
-        k_dequant<true><<<grid, kThreads, 0, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables());
+        k_dequant<true><<<grid, kThreads, kLutBytes, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables());
     else
-        k_dequant<false><<<grid, kThreads, 0, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables());
+        k_dequant<false><<<grid, kThreads, kLutBytes, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables());
     note_launches(1);
     return cudaGetLastError();
 }
