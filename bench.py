@@ -40,9 +40,9 @@ M_TOKENS, RANK, ALPHA = 4096, 64, 16.0
 L2_FLUSH_BYTES = 256 << 20
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) per call of the dX path (k_prep_bwd + k_nf4_gemm_tc<1>), mean over
-# the two linears (59.1 MB and 217.0 MB), from one ncu capture of the kernels as they are now
-# (profiles/k_nf4_gemm_tc_llama7b_m4096.md); None when the kernels have changed since then.
-DX_TRAFFIC_BYTES = 138.05e6
+# the two linears, from one ncu capture of the kernels as they are now (profiles/); None when
+# the kernels have changed since the last capture.
+DX_TRAFFIC_BYTES = None
 
 
 def linear_flops(M, N, K, r):
@@ -535,9 +535,34 @@ def run_decode(q, torch, dev, stream, flush, args):
             torch.cuda.synchronize()
             gms = statistics.median(a.elapsed_time(b) for a, b in graphed)
             del g
+            # unfused comparator: the library's dequantize to a bf16 W in HBM,
+            # then torch.matmul (cuBLAS) for the base and LoRA products
+            Wdq = torch.empty((c.N, c.K), dtype=torch.bfloat16, device=dev)
+
+            def unfused():
+                q.qlora_dequantize(wq, torch.bfloat16, out=Wdq)
+                yk = torch.matmul(X, Wdq.t())
+                tk = torch.matmul(X, A.t()).mul_(c.s)
+                yk.addmm_(tk, B.t())
+
+            for _ in range(3):
+                unfused()
+            torch.cuda.synchronize()
+            uf = []
+            for _ in range(reps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                unfused()
+                e1.record(stream)
+                uf.append((e0, e1))
+            torch.cuda.synchronize()
+            ums = statistics.median(a.elapsed_time(b) for a, b in uf)
+            del Wdq
             nbytes = decode_bytes(M, c.N, c.K, c.r)
             out[f"{c.N}x{c.K}_m{M}"] = {"bytes": nbytes, "ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
-                                        "graph_ms": gms, "graph_gbs": nbytes / (gms * 1e-3) / 1e9}
+                                        "graph_ms": gms, "graph_gbs": nbytes / (gms * 1e-3) / 1e9,
+                                        "unfused_ms": ums}
     return out
 
 

@@ -29,10 +29,12 @@
 // loaded two per lane with the codes and exchanged through a small
 // warp-private shared buffer.
 //
-// Tile: 128 weight rows (n forward, k backward) x 384 tokens x 64: each
-// dequantized weight stage feeds two 128 x 192 MMAs (two fp32 accumulators,
-// 384 TMEM columns), so the conversion work per FLOP is that of a 384-token
-// tile; 3 pipeline stages (A stages in TMEM after the accumulators).  The
+// Tile: 128 weight rows (n forward, k backward) x 2w tokens x 64, w = 128,
+// 160, 176 or 192 chosen per problem so the tiles fill the CTAs' rounds
+// evenly: each dequantized weight stage feeds two 128 x w MMAs (two fp32
+// accumulators, 2w TMEM columns), so the conversion work per FLOP is that
+// of a 2w-token tile; 3 pipeline stages (A stages in TMEM after the
+// accumulators).  The
 // codes are expanded through a 64 KiB table that maps a code byte to both
 // of its fp32 codebook values (one 8-byte copy per lane: no bank
 // conflicts), so a pair of weights costs one byte permute, one shared load,
@@ -67,14 +69,9 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileW = 128;   // weight rows per tile (MMA M)
-constexpr int kSubT = 192;    // tokens per MMA (MMA N)
 constexpr int kSubs = 2;      // MMAs per stage sharing one dequantized weight stage
-constexpr int kTileT = kSubT * kSubs;  // 384 tokens per tile
 constexpr int kBK = 64;       // contraction per stage
 constexpr int kStages = 3;
-constexpr int kSubBytes = kSubT * kBK * 2;      // 24 KiB
-constexpr int kXStageBytes = kTileT * kBK * 2;  // 48 KiB
-constexpr int kAccCols = kTileT;                // fp32 accumulator columns
 constexpr int kAStageCols = kBK / 2;            // bf16 pairs per TMEM column
 constexpr uint32_t kTmemCols = 512;
 constexpr int kDqWarps = 12;                    // three per TMEM lane quarter
@@ -84,9 +81,26 @@ constexpr int kPrefetchFwd = 2;                 // own stages of codes in flight
 constexpr int kPrefetchBwd = 2;                 // (the backward also holds its constants)
 constexpr int kThreads = 32 * (2 + kDqWarps);   // 448: 128 registers a thread
 constexpr int kLutBytes = 256 * 256;             // code byte -> fp32 pair, one 8-byte copy per lane
-constexpr int kLutOff = kStages * kXStageBytes + 1024 + kDqWarps * kBK * 4;
-constexpr int kSmemBytes = 1024 /* align */ + kLutOff + kLutBytes;
-static_assert(kAccCols + kStages * kAStageCols <= static_cast<int>(kTmemCols), "TMEM budget");
+
+// Token-tile geometry: a tile is kSubs MMAs of kSubT tokens that share every
+// dequantized weight stage.  The launcher picks kSubT per problem so that
+// the tiles fill the persistent CTAs' rounds evenly (a 384-token tile leaves
+// a 4096-token, 4096-row product at 77% of its last round's slots).
+template <int kSubT>
+struct Geo {
+    static constexpr int kTileT = kSubT * kSubs;          // tokens per tile
+    static constexpr int kSubBytes = kSubT * kBK * 2;     // one MMA's activation tile
+    static constexpr int kXStageBytes = kTileT * kBK * 2;
+    static constexpr int kAccCols = kTileT;               // fp32 accumulator columns
+    static constexpr int kChunks = kTileT / 16;           // epilogue chunks of 16 columns
+    static constexpr int kLutOff = kStages * kXStageBytes + 1024 + kDqWarps * kBK * 4;
+    static constexpr int kSmemBytes = 1024 /* align */ + kLutOff + kLutBytes;
+    static_assert(kSubT % 16 == 0 && kSubT >= 64 && kSubT <= 256, "MMA N for M = 128");
+    static_assert(kSubBytes % 1024 == 0, "128-byte swizzle atoms stay aligned");
+    static_assert(kAccCols + kStages * kAStageCols <= static_cast<int>(kTmemCols), "TMEM budget");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+    static_assert(kChunks >= kDqWarps / 4, "every part stores at least one chunk");
+};
 
 struct GemmParams {
     const uint8_t* codes;  // forward: W codes (N x K/2); backward: W^T codes (K x ldT)
@@ -117,7 +131,7 @@ struct Pipe {
     uint8_t* sA;       // kStages x 48 KiB of activation tiles (two 192-token halves)
     float* sS;         // backward: per dequant warp, 64 block constants
     uint32_t bar0;     // full_b[S], full_a[S], empty[S], acc_full, acc_empty
-    uint32_t tmem;     // accumulators at columns [0, 384), A stages after them
+    uint32_t tmem;     // accumulators at columns [0, 2w), A stages after them
     int num_t, num_tiles, kb_w, kb_total;
     __device__ uint32_t full_b(int s) const { return bar0 + 8u * s; }
     __device__ uint32_t full_a(int s) const { return bar0 + 8u * (kStages + s); }
@@ -143,8 +157,9 @@ __device__ __forceinline__ uint32_t slot_use(int kb, uint32_t tcount, int kb_tot
 // fastest, so the CTAs working at the same time share a few token tiles of
 // dY (whose full size can exceed L2) while the small transposed weight is
 // reused from L2.
-template <bool kBwd>
+template <bool kBwd, int kSubT>
 __device__ __forceinline__ void tile_coords(const Pipe& P, int tile, int& t0, int& row0) {
+    constexpr int kTileT = Geo<kSubT>::kTileT;
     if (kBwd) {
         const int num_w = P.num_tiles / P.num_t;
         t0 = (tile / num_w) * kTileT;
@@ -156,34 +171,37 @@ __device__ __forceinline__ void tile_coords(const Pipe& P, int tile, int& t0, in
 }
 
 // warp 0, one thread: activation tiles, then the LoRA slabs, into the ring.
-template <bool kBwd>
+template <bool kBwd, int kSubT>
 __device__ void role_tma(const Pipe& P, const CUtensorMap* tmap_act, const CUtensorMap* tmap_lora, int* err) {
+    using G = Geo<kSubT>;
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x, ++tcount) {
         int t0, row0;
-        tile_coords<kBwd>(P, tile, t0, row0);
+        tile_coords<kBwd, kSubT>(P, tile, t0, row0);
         for (int kb = 0; kb < P.kb_total; ++kb) {
             const int s = kb % kStages;
             const uint32_t ph = slot_use(kb, tcount, P.kb_total) & 1u;
             if (!mbar_wait(P.empty(s), ph ^ 1u, err)) return;
-            const uint32_t dst = smem_u32(P.sA + s * kXStageBytes);
+            const uint32_t dst = smem_u32(P.sA + s * G::kXStageBytes);
             if (kb < P.kb_w) {
-                mbar_arrive_expect_tx(P.full_b(s), kXStageBytes);
+                mbar_arrive_expect_tx(P.full_b(s), G::kXStageBytes);
                 for (int sub = 0; sub < kSubs; ++sub)
-                    tma_load_2d(dst + sub * kSubBytes, tmap_act, P.full_b(s), kb * kBK, t0 + sub * kSubT);
+                    tma_load_2d(dst + sub * G::kSubBytes, tmap_act, P.full_b(s), kb * kBK, t0 + sub * kSubT);
             } else {
-                mbar_arrive_expect_tx(P.full_b(s), kXStageBytes);
+                mbar_arrive_expect_tx(P.full_b(s), G::kXStageBytes);
                 for (int sub = 0; sub < kSubs; ++sub)
-                    tma_load_2d(dst + sub * kSubBytes, tmap_lora, P.full_b(s), (kb - P.kb_w) * kBK,
+                    tma_load_2d(dst + sub * G::kSubBytes, tmap_lora, P.full_b(s), (kb - P.kb_w) * kBK,
                                 t0 + sub * kSubT);
             }
         }
     }
 }
 
-// warp 1, one thread: per stage, four 128x192x16 MMAs into each of the two
+// warp 1, one thread: per stage, four 128 x w x 16 MMAs into each of the two
 // accumulators, all reading the same weight stage in TMEM.
+template <int kSubT>
 __device__ void role_mma(const Pipe& P, int* err) {
+    using G = Geo<kSubT>;
     constexpr uint32_t idesc = idesc_bf16(kTileW, kSubT);
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x, ++tcount) {
@@ -195,10 +213,10 @@ __device__ void role_mma(const Pipe& P, int* err) {
             if (!mbar_wait(P.full_b(s), ph, err)) return;
             if (!mbar_wait(P.full_a(s), ph, err)) return;
             tc_fence_after();
-            const uint32_t a_col = P.tmem + kAccCols + s * kAStageCols;
+            const uint32_t a_col = P.tmem + G::kAccCols + s * kAStageCols;
 #pragma unroll
             for (int sub = 0; sub < kSubs; ++sub) {
-                const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(P.sA + s * kXStageBytes + sub * kSubBytes));
+                const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(P.sA + s * G::kXStageBytes + sub * G::kSubBytes));
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk)
                     mma_bf16_ts(P.tmem + sub * kSubT, a_col + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
@@ -254,7 +272,7 @@ __device__ __forceinline__ void convert_run(const uint4& c0, const uint4& c1, fl
 // warps 2..13: each converts every third stage of the weight tile into
 // TMEM (quarter = its TMEM lanes, part = which stages), then writes a
 // quarter of this tile's outputs.
-template <bool kBwd>
+template <bool kBwd, int kSubT>
 __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const uint8_t* lut,
                                                       float* wsc, int warp, int lane, int* err) {
     const uint32_t lane_off = static_cast<uint32_t>(lane) * 8;
@@ -263,11 +281,12 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
     const int part = dq >> 2;      // converts the stages kb with kb % 3 == part
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    using G = Geo<kSubT>;
     const float mu = kBwd ? 0.0f : *p.mean;
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x, ++tcount) {
         int t0, row0;
-        tile_coords<kBwd>(P, tile, t0, row0);
+        tile_coords<kBwd, kSubT>(P, tile, t0, row0);
         const int grow = row0 + row;             // this lane's weight row of the product
         const bool lane_ok = grow < p.rows;
         const uint8_t* crow = p.codes + static_cast<int64_t>(grow) * p.ld_codes;
@@ -337,24 +356,24 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
                 }
                 issue(kb + kParts * kPrefetch, u);
                 if (!warp_wait(P.empty(s), ph ^ 1u, err, lane)) return;
-                tmem_st_32x32b_x32(P.tmem + lane_base + kAccCols + s * kAStageCols, v);
+                tmem_st_32x32b_x32(P.tmem + lane_base + G::kAccCols + s * kAStageCols, v);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(P.full_a(s));
             }
         }
-        // epilogue: this warp's lane quarter, columns [96 part, 96 part + 96)
+        // epilogue: this warp's lane quarter, the 16-column chunks
+        // part, part + 3, part + 6, ...
         if (!warp_wait(P.acc_full(), tcount & 1u, err, lane)) return;
         tc_fence_after();
-        constexpr int kChunks = kTileT / kParts / 16;
 #pragma unroll 1
-        for (int c = 0; c < kChunks; ++c) {
-            const int col = part * (kTileT / kParts) + c * 16;
+        for (int c = part; c < G::kChunks; c += kParts) {
+            const int col = c * 16;
             uint32_t acc[16];
             tmem_ld_32x32b_x16(P.tmem + lane_base + col, acc);
             tmem_wait_ld();
-            if (c == kChunks - 1) {
+            if (c + kParts >= G::kChunks) {  // this warp's last chunk
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(P.acc_empty());
@@ -369,21 +388,22 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
     }
 }
 
-template <bool kBwd>
+template <bool kBwd, int kSubT>
 __global__ void __launch_bounds__(kThreads, 1)
 k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_lora,
               const __grid_constant__ GemmParams p) {
+    using G = Geo<kSubT>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base, derived by pointer arithmetic so that every
     // access below stays a (32-bit) shared-memory access
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kXStageBytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * G::kXStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 2);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     Pipe P;
     P.sA = smem;
-    P.sS = reinterpret_cast<float*>(smem + kStages * kXStageBytes + 1024);
+    P.sS = reinterpret_cast<float*>(smem + kStages * G::kXStageBytes + 1024);
     P.bar0 = smem_u32(bars);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -395,7 +415,7 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
         mbar_init(P.acc_empty(), kDqWarps);
         fence_barrier_init();
     }
-    uint8_t* lut = smem + kLutOff;
+    uint8_t* lut = smem + G::kLutOff;
     for (int i = threadIdx.x; i < 256 * 32; i += kThreads)
         reinterpret_cast<float2*>(lut)[i] = make_float2(p.q[i >> 9], p.q[(i >> 5) & 15]);
     if (warp == 0) {
@@ -410,20 +430,20 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
     __syncthreads();
     tc_fence_after();
     P.tmem = *tmem_slot;
-    P.num_t = (p.M + kTileT - 1) / kTileT;
+    P.num_t = (p.M + G::kTileT - 1) / G::kTileT;
     P.num_tiles = P.num_t * ((p.rows + kTileW - 1) / kTileW);
     P.kb_w = (p.ctr + kBK - 1) / kBK;
     P.kb_total = P.kb_w + (p.r + kBK - 1) / kBK;
     int* err = &g_tc_error;
 
     if (warp == 0) {
-        if (lane == 0) role_tma<kBwd>(P, &tmap_act, &tmap_lora, err);
+        if (lane == 0) role_tma<kBwd, kSubT>(P, &tmap_act, &tmap_lora, err);
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) role_mma(P, err);
+        if (lane == 0) role_mma<kSubT>(P, err);
         __syncwarp();
     } else {
-        role_dequant_epilogue<kBwd>(P, p, lut, P.sS + (warp - 2) * kBK, warp, lane, err);
+        role_dequant_epilogue<kBwd, kSubT>(P, p, lut, P.sS + (warp - 2) * kBK, warp, lane, err);
     }
     tc_fence_before();
     __syncthreads();
@@ -438,51 +458,69 @@ k_nf4_gemm_tc(const __grid_constant__ CUtensorMap tmap_act, const __grid_constan
 //   codesT[k][j]  = (code(W[2j][k]) << 4) | code(W[2j+1][k])   (K x ldT bytes)
 //   scalesT[g][n] = c2' of the block holding W[n][64g .. 64g+63] (K/64 x ldS)
 //   AT[k][j]      = A[j][k]                                     (K x r)
-// One CTA per 64 x 64 weight tile (plus tiles for A^T); padding is zero.
+// One CTA per 64 x 256 weight tile (64 rows n, up to 256 columns k; plus
+// CTAs for A^T); padding is zero.  A thread loads 32 bytes of one row n
+// (two 16-byte loads), then builds the 32 bytes of one row k of W^T from
+// shared memory and stores them as two 16-byte stores.
 constexpr int kPrepThreads = 256;
+constexpr int kPrepK = 256;  // weight columns per CTA
 
 __global__ void __launch_bounds__(kPrepThreads)
 k_prep_bwd(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8, const float* __restrict__ c1,
            const float* __restrict__ mean, const uint16_t* __restrict__ A, int N, int K, int r, int64_t ldT,
            int64_t ldS, uint8_t* __restrict__ codesT, float* __restrict__ scalesT, uint16_t* __restrict__ AT,
            int weight_tiles) {
-    __shared__ uint8_t tile[64][33];
+    __shared__ __align__(16) uint8_t tile[64][kPrepK / 2];
     __shared__ uint16_t at[64][65];
     const int t = threadIdx.x;
     const int npad_tiles = static_cast<int>(ldS / 64);
     if (static_cast<int>(blockIdx.x) < weight_tiles) {
-        const int nt = blockIdx.x % npad_tiles, kt = blockIdx.x / npad_tiles;
-        const int n0 = nt * 64, k0 = kt * 64;
-        {   // 64 rows x 32 bytes of codes (zero beyond N)
-            const int rr = t >> 2, cc = (t & 3) * 8;
-            uint2 v = make_uint2(0u, 0u);
-            if (n0 + rr < N)
-                v = *reinterpret_cast<const uint2*>(codes + static_cast<int64_t>(n0 + rr) * (K / 2) + k0 / 2 + cc);
-            for (int b = 0; b < 4; ++b) tile[rr][cc + b] = static_cast<uint8_t>(v.x >> (8 * b));
-            for (int b = 0; b < 4; ++b) tile[rr][cc + 4 + b] = static_cast<uint8_t>(v.y >> (8 * b));
-        }
-        if (t < 64) {
-            const int n = n0 + t;
-            float c = 0.0f;
-            if (n < N) {
-                const int64_t blk = static_cast<int64_t>(n) * (K / 64) + kt;
-                c = dq_constant(c2_fp8[blk], c1[blk >> 8], *mean);
+        const int nt = blockIdx.x % npad_tiles, kq = blockIdx.x / npad_tiles;
+        const int n0 = nt * 64, k0 = kq * kPrepK;
+        const int kspan = min(kPrepK, K - k0);  // a multiple of 64
+        {   // rows n0 .. n0 + 63, bytes k0/2 .. (k0 + kspan)/2 of the codes (zero beyond N)
+            const int rr = t >> 2, cc = (t & 3) * 32;
+            uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+            if (n0 + rr < N && 2 * cc < kspan) {
+                const uint8_t* src = codes + static_cast<int64_t>(n0 + rr) * (K / 2) + k0 / 2 + cc;
+                v0 = *reinterpret_cast<const uint4*>(src);
+                v1 = *reinterpret_cast<const uint4*>(src + 16);
             }
-            scalesT[static_cast<int64_t>(kt) * ldS + n] = c;
+            *reinterpret_cast<uint4*>(&tile[rr][cc]) = v0;
+            *reinterpret_cast<uint4*>(&tile[rr][cc + 16]) = v1;
+        }
+        {   // the constants of the (up to) four 64-blocks of each row
+            const int n = n0 + (t & 63), g = t >> 6;
+            if (64 * g < kspan) {
+                const int kt = k0 / 64 + g;
+                float c = 0.0f;
+                if (n < N) {
+                    const int64_t blk = static_cast<int64_t>(n) * (K / 64) + kt;
+                    c = dq_constant(c2_fp8[blk], c1[blk >> 8], *mean);
+                }
+                scalesT[static_cast<int64_t>(kt) * ldS + n] = c;
+            }
         }
         __syncthreads();
-        {   // row k0 + kk of W^T: bytes j0..j0+7, each two consecutive n
-            const int kk = t >> 2, j0 = (t & 3) * 8;
-            uint32_t out[2] = {0u, 0u};
-            for (int b = 0; b < 8; ++b) {
-                const int j = j0 + b;
-                const uint8_t e = tile[2 * j][kk >> 1], o = tile[2 * j + 1][kk >> 1];
-                const uint32_t ne = (kk & 1) ? (e & 15u) : (e >> 4);
-                const uint32_t no = (kk & 1) ? (o & 15u) : (o >> 4);
-                out[b >> 2] |= ((ne << 4) | no) << (8 * (b & 3));
+        if (t < kspan) {  // row k0 + t of W^T: 32 bytes, each two consecutive n
+            const int col = t >> 1;
+            const int shift = (t & 1) ? 0 : 4;  // even k: the high nibble
+            uint32_t out[8];
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                uint32_t acc = 0u;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int j = 4 * w + b;
+                    const uint32_t ne = (tile[2 * j][col] >> shift) & 15u;
+                    const uint32_t no = (tile[2 * j + 1][col] >> shift) & 15u;
+                    acc |= ((ne << 4) | no) << (8 * b);
+                }
+                out[w] = acc;
             }
-            *reinterpret_cast<uint2*>(codesT + static_cast<int64_t>(k0 + kk) * ldT + n0 / 2 + j0) =
-                make_uint2(out[0], out[1]);
+            uint8_t* dst = codesT + static_cast<int64_t>(k0 + t) * ldT + n0 / 2;
+            *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+            *reinterpret_cast<uint4*>(dst + 16) = make_uint4(out[4], out[5], out[6], out[7]);
         }
     } else {
         const int kt = blockIdx.x - weight_tiles;  // 64 columns of A
@@ -520,8 +558,10 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t ou
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kBwd>
-cudaError_t launch_tc(const uint16_t* act, const uint16_t* lora_act, const GemmParams& p0, cudaStream_t st) {
+template <bool kBwd, int kSubT>
+cudaError_t launch_tc_geo(const uint16_t* act, const uint16_t* lora_act, const GemmParams& p0, int grid,
+                          cudaStream_t st) {
+    using G = Geo<kSubT>;
     CUtensorMap ma, ml;
     if (!make_map_bf16(&ma, act, static_cast<uint64_t>(p0.ctr), static_cast<uint64_t>(p0.M), kBK, kSubT) ||
         !make_map_bf16(&ml, lora_act, static_cast<uint64_t>(p0.r), static_cast<uint64_t>(p0.M), kBK, kSubT))
@@ -529,17 +569,51 @@ cudaError_t launch_tc(const uint16_t* act, const uint16_t* lora_act, const GemmP
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(k_nf4_gemm_tc<kBwd>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kSmemBytes);
+        attr_err = cudaFuncSetAttribute(k_nf4_gemm_tc<kBwd, kSubT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        G::kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
     GemmParams p = p0;
     for (int i = 0; i < 16; ++i) p.q[i] = tables().q[i];
-    const int64_t tiles = ceil_div(p.M, kTileT) * ceil_div(p.rows, kTileW);
-    const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-    k_nf4_gemm_tc<kBwd><<<grid, kThreads, kSmemBytes, st>>>(ma, ml, p);
+    k_nf4_gemm_tc<kBwd, kSubT><<<grid, kThreads, G::kSmemBytes, st>>>(ma, ml, p);
     note_launches(1);
     return cudaGetLastError();
+}
+
+// MMA widths the launcher chooses from (tokens per tile = 2 x width).
+constexpr int kSubChoices[] = {128, 160, 176, 192};
+
+// The width whose tiles finish soonest on `sms` persistent CTAs: rounds
+// (tiles per CTA, rounded up) times the tile's token count plus a fixed
+// per-tile cost (the stage conversions, the epilogue) of about 48 tokens'
+// worth of MMA time.  Ties go to the wider tile.
+int pick_sub(int64_t M, int64_t rows, int64_t sms) {
+    int best = kSubChoices[0];
+    int64_t best_cost = -1;
+    for (int sub : kSubChoices) {
+        const int64_t tiles = ceil_div(M, 2 * sub) * ceil_div(rows, kTileW);
+        const int64_t rounds = ceil_div(tiles, sms);
+        const int64_t cost = rounds * (2 * sub + 48);
+        if (best_cost < 0 || cost <= best_cost) {
+            best = sub;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+template <bool kBwd>
+cudaError_t launch_tc(const uint16_t* act, const uint16_t* lora_act, const GemmParams& p0, cudaStream_t st) {
+    const int64_t sms = num_sms();
+    const int sub = pick_sub(p0.M, p0.rows, sms);
+    const int64_t tiles = ceil_div(static_cast<int64_t>(p0.M), 2 * sub) * ceil_div(static_cast<int64_t>(p0.rows), kTileW);
+    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+    switch (sub) {
+        case 128: return launch_tc_geo<kBwd, 128>(act, lora_act, p0, grid, st);
+        case 160: return launch_tc_geo<kBwd, 160>(act, lora_act, p0, grid, st);
+        case 176: return launch_tc_geo<kBwd, 176>(act, lora_act, p0, grid, st);
+        default: return launch_tc_geo<kBwd, 192>(act, lora_act, p0, grid, st);
+    }
 }
 
 bool tc_common_ok(int64_t M, const Nf4Weight& w, int r) {
@@ -589,7 +663,7 @@ cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const 
     float* scalesT = reinterpret_cast<float*>(codesT + round_up(static_cast<size_t>(w.K) * ldT, 256));
     uint16_t* AT = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(scalesT) +
                                                round_up(static_cast<size_t>(w.K / kBK) * ldS * 4, 256));
-    const int weight_tiles = static_cast<int>((ldS / 64) * (w.K / 64));
+    const int weight_tiles = static_cast<int>((ldS / 64) * ceil_div(w.K, kPrepK));
     const int a_tiles = static_cast<int>(ceil_div(w.K, 64));
     k_prep_bwd<<<weight_tiles + a_tiles, kPrepThreads, 0, st>>>(w.codes, w.c2_fp8, w.c1, w.mean, A,
                                                                 static_cast<int>(w.N), static_cast<int>(w.K), r,

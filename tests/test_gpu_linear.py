@@ -73,6 +73,18 @@ def test_tile_spanning_shape():
     _run_case(case)
 
 
+@pytest.mark.parametrize("M,N,K", [(830, 4864, 128), (1001, 4864, 128), (1090, 4864, 128),
+                                   (830, 128, 4864), (1001, 128, 4864), (1090, 128, 4864)])
+def test_every_token_tile_width(M, N, K):
+    """The GEMMs pick a token-tile width of 256, 320, 352 or 384 per problem
+    from the tile count per CTA round (148 CTAs): these shapes select 320,
+    352 and 384 in the forward (weight rows N = 4864) and in the dX product
+    (rows K = 4864), each with a ragged token tail; 64 sampled rows."""
+    case = synth.linear_case(f"w{M}n{N}k{K}", M, N, K, 16, 16.0, seed=21, outlier_frac=0.001)
+    rows = np.sort(synth.rng(0, 121).choice(M, 64, replace=False)).astype(np.int64)
+    _run_case(case, rows=rows)
+
+
 def test_T_recompute_matches_saved_T():
     case = synth.linear_case("m96n256k256r16", 96, 256, 256, 16, 16.0, seed=3)
     wq = q.qlora_quantize_nf4_dq(dev_f32(case.W))
