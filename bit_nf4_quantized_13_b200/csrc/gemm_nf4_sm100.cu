@@ -269,9 +269,76 @@ __device__ __forceinline__ void convert_run(const uint4& c0, const uint4& c1, fl
     }
 }
 
-// warps 2..13: each converts every third stage of the weight tile into
-// TMEM (quarter = its TMEM lanes, part = which stages), then writes a
-// quarter of this tile's outputs.
+// A position in one part's sequence of stages over all of this CTA's
+// tiles: the stages kb == part (mod 3) of tile 0, then of tile 1, ...
+struct Cursor {
+    int tile;         // persistent tile index (>= num_tiles: past the end)
+    uint32_t tcount;  // tiles of this CTA before it
+    int kb;           // contraction stage
+    int t0, row0;     // the tile's first token and first weight row
+};
+
+template <bool kBwd, int kSubT>
+__device__ __forceinline__ void cursor_start(Cursor& c, const Pipe& P, int part) {
+    c.tile = blockIdx.x;
+    c.tcount = 0;
+    c.kb = part;
+    tile_coords<kBwd, kSubT>(P, c.tile, c.t0, c.row0);
+}
+
+template <bool kBwd, int kSubT>
+__device__ __forceinline__ void cursor_next(Cursor& c, const Pipe& P, int part) {
+    c.kb += kParts;
+    if (c.kb >= P.kb_total) {
+        c.kb = part;
+        c.tile += gridDim.x;
+        ++c.tcount;
+        if (c.tile < P.num_tiles) tile_coords<kBwd, kSubT>(P, c.tile, c.t0, c.row0);
+    }
+}
+
+// Epilogue of this CTA's tile number tcount (first token t0, first weight
+// row row0): this warp's lane quarter, the 16-column chunks part, part + 3,
+// part + 6, ...; the accumulator is released after the warp's last load.
+template <int kSubT>
+__device__ __forceinline__ void tile_epilogue(const Pipe& P, const GemmParams& p, uint32_t tcount, int t0,
+                                              int row0, int part, int row, uint32_t lane_base, int lane,
+                                              int* err, bool& ok) {
+    using G = Geo<kSubT>;
+    if (!warp_wait(P.acc_full(), tcount & 1u, err, lane)) {
+        ok = false;
+        return;
+    }
+    tc_fence_after();
+    const int grow = row0 + row;
+    const bool lane_ok = grow < p.rows;
+#pragma unroll 1
+    for (int c = part; c < G::kChunks; c += kParts) {
+        const int col = c * 16;
+        uint32_t acc[16];
+        tmem_ld_32x32b_x16(P.tmem + lane_base + col, acc);
+        tmem_wait_ld();
+        if (c + kParts >= G::kChunks) {  // this warp's last chunk
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(P.acc_empty());
+        }
+        if (lane_ok) {
+            uint16_t* o = p.out + static_cast<int64_t>(t0 + col) * p.rows + grow;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (t0 + col + j < p.M) o[static_cast<int64_t>(j) * p.rows] = f32_to_bf16_bits(__uint_as_float(acc[j]));
+        }
+    }
+}
+
+// warps 2..13: each converts every third stage of the weight tiles into
+// TMEM (quarter = its TMEM lanes, part = which stages) and writes a third
+// of each tile's outputs for its lane quarter.  The stages form one stream
+// over all of the CTA's tiles (the codes of the next tile are loaded while
+// the current one ends), and a tile's epilogue runs after the warp has
+// stored its first stage of the next tile, so the MMAs of the next tile
+// find their first stages ready once the accumulator is free.
 template <bool kBwd, int kSubT>
 __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmParams& p, const uint8_t* lut,
                                                       float* wsc, int warp, int lane, int* err) {
@@ -281,111 +348,112 @@ __device__ __forceinline__ void role_dequant_epilogue(const Pipe& P, const GemmP
     const int part = dq >> 2;      // converts the stages kb with kb % 3 == part
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    using G = Geo<kSubT>;
     const float mu = kBwd ? 0.0f : *p.mean;
-    uint32_t tcount = 0;
-    for (int tile = blockIdx.x; tile < P.num_tiles; tile += gridDim.x, ++tcount) {
-        int t0, row0;
-        tile_coords<kBwd, kSubT>(P, tile, t0, row0);
-        const int grow = row0 + row;             // this lane's weight row of the product
-        const bool lane_ok = grow < p.rows;
-        const uint8_t* crow = p.codes + static_cast<int64_t>(grow) * p.ld_codes;
-        // backward: this warp's 32 columns lie in one 64-wide block group
-        const float* srow = kBwd ? p.scalesT + static_cast<int64_t>((row0 + quarter * 32) / kBK) * p.ld_scales
-                                 : nullptr;
+    bool ok = true;
 
-        // codes (and, forward, the block constant's inputs) of the next
-        // kPrefetch own stages; the constant itself is formed at use so the
-        // loads stay in flight
-        constexpr int kPrefetch = kBwd ? kPrefetchBwd : kPrefetchFwd;
-        uint4 cb0[kPrefetch], cb1[kPrefetch];
-        uint32_t sbyte[kPrefetch];
-        float sc1[kPrefetch];
-        float2 s2[kPrefetch];  // backward: constants of rows 2 lane, 2 lane + 1 of the stage
-        auto issue = [&](int kb, int u) {
-            cb0[u] = make_uint4(0u, 0u, 0u, 0u);
-            cb1[u] = cb0[u];
-            sbyte[u] = 0u;
-            sc1[u] = 0.0f;
-            s2[u] = make_float2(0.0f, 0.0f);
-            if (kb >= P.kb_w) return;
-            if (kBwd && (row0 + quarter * 32) < p.rows)
-                s2[u] = __ldg(reinterpret_cast<const float2*>(srow + kb * kBK) + lane);
-            if (!lane_ok) return;
-            cb0[u] = ldg_nc_v4(crow + kb * (kBK / 2));
-            cb1[u] = ldg_nc_v4(crow + kb * (kBK / 2) + 16);
-            if (!kBwd) {
-                const int64_t blk = static_cast<int64_t>(grow) * (p.K / kBK) + kb;
-                sbyte[u] = __ldg(p.c2_fp8 + blk);
-                sc1[u] = __ldg(p.c1 + (blk >> 8));
-            }
-        };
-#pragma unroll
-        for (int u = 0; u < kPrefetch; ++u) issue(part + kParts * u, u);
-        for (int i0 = 0; part + kParts * i0 < P.kb_total; i0 += kPrefetch) {
-#pragma unroll
-            for (int u = 0; u < kPrefetch; ++u) {
-                const int kb = part + kParts * (i0 + u);
-                if (kb >= P.kb_total) break;
-                const int s = part;  // == kb % kStages
-                const uint32_t ph = slot_use(kb, tcount, P.kb_total) & 1u;
-                uint32_t v[32];
-                if (kb < P.kb_w) {
-                    if (kBwd) {
-                        reinterpret_cast<float2*>(wsc)[lane] = s2[u];
-                        __syncwarp();
-                    }
-                    const float sc = kBwd ? 0.0f : dq_constant(static_cast<uint8_t>(sbyte[u]), sc1[u], mu);
-                    // rows beyond the weight hold finite garbage (zero codes times
-                    // the constant of empty inputs): their outputs are never
-                    // stored and rows do not mix in this product
-                    convert_run<kBwd>(cb0[u], cb1[u], sc, wsc, lut, lane_off, v);
-                    if (kBwd) __syncwarp();  // wsc is rewritten by the warp's next stage
-                } else {  // LoRA slab: lane = row of B (forward) or of A^T (backward), r contiguous
-                    const int j0 = (kb - P.kb_w) * kBK;
-                    const uint16_t* lrow = p.lora + static_cast<int64_t>(grow) * p.r + j0;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-                        if (lane_ok && j0 + 8 * c < p.r) w = *reinterpret_cast<const uint4*>(lrow + 8 * c);
-                        v[4 * c + 0] = w.x;
-                        v[4 * c + 1] = w.y;
-                        v[4 * c + 2] = w.z;
-                        v[4 * c + 3] = w.w;
-                    }
-                }
-                issue(kb + kParts * kPrefetch, u);
-                if (!warp_wait(P.empty(s), ph ^ 1u, err, lane)) return;
-                tmem_st_32x32b_x32(P.tmem + lane_base + G::kAccCols + s * kAStageCols, v);
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(P.full_a(s));
-            }
+    if (part >= P.kb_total) {  // no stages for this part: epilogues only
+        uint32_t tcount = 0;
+        for (int tile = blockIdx.x; tile < P.num_tiles && ok; tile += gridDim.x, ++tcount) {
+            int t0, row0;
+            tile_coords<kBwd, kSubT>(P, tile, t0, row0);
+            tile_epilogue<kSubT>(P, p, tcount, t0, row0, part, row, lane_base, lane, err, ok);
         }
-        // epilogue: this warp's lane quarter, the 16-column chunks
-        // part, part + 3, part + 6, ...
-        if (!warp_wait(P.acc_full(), tcount & 1u, err, lane)) return;
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = part; c < G::kChunks; c += kParts) {
-            const int col = c * 16;
-            uint32_t acc[16];
-            tmem_ld_32x32b_x16(P.tmem + lane_base + col, acc);
-            tmem_wait_ld();
-            if (c + kParts >= G::kChunks) {  // this warp's last chunk
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(P.acc_empty());
-            }
-            if (lane_ok) {
-                uint16_t* o = p.out + static_cast<int64_t>(t0 + col) * p.rows + grow;
+        return;
+    }
+
+    // codes (and, forward, the block constant's inputs) of the next
+    // kPrefetch own stages; the constant itself is formed at use so the
+    // loads stay in flight
+    constexpr int kPrefetch = kBwd ? kPrefetchBwd : kPrefetchFwd;
+    uint4 cb0[kPrefetch], cb1[kPrefetch];
+    uint32_t sbyte[kPrefetch];
+    float sc1[kPrefetch];
+    float2 s2[kPrefetch];  // backward: constants of rows 2 lane, 2 lane + 1 of the stage
+    auto issue = [&](const Cursor& c, int u) {
+        cb0[u] = make_uint4(0u, 0u, 0u, 0u);
+        cb1[u] = cb0[u];
+        sbyte[u] = 0u;
+        sc1[u] = 0.0f;
+        s2[u] = make_float2(0.0f, 0.0f);
+        if (c.tile >= P.num_tiles || c.kb >= P.kb_w) return;
+        const int grow = c.row0 + row;
+        if (kBwd && (c.row0 + quarter * 32) < p.rows) {
+            // this warp's 32 columns lie in one 64-wide block group
+            const float* srow = p.scalesT + static_cast<int64_t>((c.row0 + quarter * 32) / kBK) * p.ld_scales;
+            s2[u] = __ldg(reinterpret_cast<const float2*>(srow + c.kb * kBK) + lane);
+        }
+        if (grow >= p.rows) return;
+        const uint8_t* crow = p.codes + static_cast<int64_t>(grow) * p.ld_codes;
+        cb0[u] = ldg_nc_v4(crow + c.kb * (kBK / 2));
+        cb1[u] = ldg_nc_v4(crow + c.kb * (kBK / 2) + 16);
+        if (!kBwd) {
+            const int64_t blk = static_cast<int64_t>(grow) * (p.K / kBK) + c.kb;
+            sbyte[u] = __ldg(p.c2_fp8 + blk);
+            sc1[u] = __ldg(p.c1 + (blk >> 8));
+        }
+    };
+
+    Cursor ci, cc;  // the next stage to load, the next stage to convert
+    cursor_start<kBwd, kSubT>(ci, P, part);
+    cursor_start<kBwd, kSubT>(cc, P, part);
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    if (t0 + col + j < p.M) o[static_cast<int64_t>(j) * p.rows] = f32_to_bf16_bits(__uint_as_float(acc[j]));
+    for (int u = 0; u < kPrefetch; ++u) {
+        issue(ci, u);
+        cursor_next<kBwd, kSubT>(ci, P, part);
+    }
+    int prev_t0 = 0, prev_row0 = 0;  // the tile whose epilogue is pending
+    while (cc.tile < P.num_tiles) {
+#pragma unroll
+        for (int u = 0; u < kPrefetch; ++u) {
+            if (cc.tile >= P.num_tiles) break;
+            const int kb = cc.kb;
+            const int s = part;  // == kb % kStages
+            const uint32_t ph = slot_use(kb, cc.tcount, P.kb_total) & 1u;
+            const int grow = cc.row0 + row;  // this lane's weight row of the product
+            uint32_t v[32];
+            if (kb < P.kb_w) {
+                if (kBwd) {
+                    reinterpret_cast<float2*>(wsc)[lane] = s2[u];
+                    __syncwarp();
+                }
+                const float sc = kBwd ? 0.0f : dq_constant(static_cast<uint8_t>(sbyte[u]), sc1[u], mu);
+                // rows beyond the weight hold finite garbage (zero codes times
+                // the constant of empty inputs): their outputs are never
+                // stored and rows do not mix in this product
+                convert_run<kBwd>(cb0[u], cb1[u], sc, wsc, lut, lane_off, v);
+                if (kBwd) __syncwarp();  // wsc is rewritten by the warp's next stage
+            } else {  // LoRA slab: lane = row of B (forward) or of A^T (backward), r contiguous
+                const int j0 = (kb - P.kb_w) * kBK;
+                const uint16_t* lrow = p.lora + static_cast<int64_t>(grow) * p.r + j0;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                    if (grow < p.rows && j0 + 8 * c < p.r) w = *reinterpret_cast<const uint4*>(lrow + 8 * c);
+                    v[4 * c + 0] = w.x;
+                    v[4 * c + 1] = w.y;
+                    v[4 * c + 2] = w.z;
+                    v[4 * c + 3] = w.w;
+                }
             }
+            issue(ci, u);
+            cursor_next<kBwd, kSubT>(ci, P, part);
+            if (!warp_wait(P.empty(s), ph ^ 1u, err, lane)) return;
+            tmem_st_32x32b_x32(P.tmem + lane_base + Geo<kSubT>::kAccCols + s * kAStageCols, v);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(P.full_a(s));
+            if (kb == part && cc.tcount > 0) {  // first own stage of a tile: end the previous one
+                tile_epilogue<kSubT>(P, p, cc.tcount - 1, prev_t0, prev_row0, part, row, lane_base, lane, err, ok);
+                if (!ok) return;
+            }
+            prev_t0 = cc.t0;
+            prev_row0 = cc.row0;
+            cursor_next<kBwd, kSubT>(cc, P, part);
         }
     }
+    // the CTA's last tile
+    tile_epilogue<kSubT>(P, p, cc.tcount - 1, prev_t0, prev_row0, part, row, lane_base, lane, err, ok);
 }
 
 template <bool kBwd, int kSubT>
