@@ -40,9 +40,9 @@ M_TOKENS, RANK, ALPHA = 4096, 64, 16.0
 L2_FLUSH_BYTES = 256 << 20
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) per call of the dX path (k_prep_bwd + k_nf4_gemm_tc<1>), mean over
-# the two linears, from one ncu capture of the kernels as they are now (profiles/); None when
-# the kernels have changed since the last capture.
-DX_TRAFFIC_BYTES = None
+# the two linears (57.5 MB and 217.4 MB), from one ncu capture of the kernels as they are now
+# (profiles/k_nf4_gemm_tc_llama7b_m4096.md); None when the kernels have changed since then.
+DX_TRAFFIC_BYTES = 137.45e6
 
 
 def linear_flops(M, N, K, r):
