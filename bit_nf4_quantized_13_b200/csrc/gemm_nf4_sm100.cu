@@ -30,7 +30,7 @@
 // warp-private shared buffer.
 //
 // Tile: 128 weight rows (n forward, k backward) x 2w tokens x 64, w = 128,
-// 160, 176 or 192 chosen per problem so the tiles fill the CTAs' rounds
+// 160, 176, 192 or 208 chosen per problem so the tiles fill the CTAs' rounds
 // evenly: each dequantized weight stage feeds two 128 x w MMAs (two fp32
 // accumulators, 2w TMEM columns), so the conversion work per FLOP is that
 // of a 2w-token tile; 3 pipeline stages (A stages in TMEM after the
@@ -649,19 +649,22 @@ cudaError_t launch_tc_geo(const uint16_t* act, const uint16_t* lora_act, const G
 }
 
 // MMA widths the launcher chooses from (tokens per tile = 2 x width).
-constexpr int kSubChoices[] = {128, 160, 176, 192};
+constexpr int kSubChoices[] = {128, 160, 176, 192, 208};
 
 // The width whose tiles finish soonest on `sms` persistent CTAs: rounds
-// (tiles per CTA, rounded up) times the tile's token count plus a fixed
-// per-tile cost (the stage conversions, the epilogue) of about 48 tokens'
-// worth of MMA time.  Ties go to the wider tile.
+// (tiles per CTA, rounded up) times the time of one tile.  A 128-row MMA
+// instruction costs about the same issue time whatever its width up to 256
+// (measured on B200: 187 cycles per instruction with two accumulators in
+// turn, for widths 64 to 256), so a tile's time is mostly a fixed cost per
+// 64-wide stage: measured, about 790 tokens' worth of width-proportional
+// time.  Ties go to the wider tile.
 int pick_sub(int64_t M, int64_t rows, int64_t sms) {
     int best = kSubChoices[0];
     int64_t best_cost = -1;
     for (int sub : kSubChoices) {
         const int64_t tiles = ceil_div(M, 2 * sub) * ceil_div(rows, kTileW);
         const int64_t rounds = ceil_div(tiles, sms);
-        const int64_t cost = rounds * (2 * sub + 48);
+        const int64_t cost = rounds * (2 * sub + 790);
         if (best_cost < 0 || cost <= best_cost) {
             best = sub;
             best_cost = cost;
@@ -680,7 +683,8 @@ cudaError_t launch_tc(const uint16_t* act, const uint16_t* lora_act, const GemmP
         case 128: return launch_tc_geo<kBwd, 128>(act, lora_act, p0, grid, st);
         case 160: return launch_tc_geo<kBwd, 160>(act, lora_act, p0, grid, st);
         case 176: return launch_tc_geo<kBwd, 176>(act, lora_act, p0, grid, st);
-        default: return launch_tc_geo<kBwd, 192>(act, lora_act, p0, grid, st);
+        case 192: return launch_tc_geo<kBwd, 192>(act, lora_act, p0, grid, st);
+        default: return launch_tc_geo<kBwd, 208>(act, lora_act, p0, grid, st);
     }
 }
 

@@ -73,13 +73,14 @@ def test_tile_spanning_shape():
     _run_case(case)
 
 
-@pytest.mark.parametrize("M,N,K", [(830, 4864, 128), (1001, 4864, 128), (1090, 4864, 128),
-                                   (830, 128, 4864), (1001, 128, 4864), (1090, 128, 4864)])
+@pytest.mark.parametrize("M,N,K", [(830, 4864, 128), (1001, 4864, 128), (1090, 4864, 128), (1200, 4864, 128),
+                                   (830, 128, 4864), (1001, 128, 4864), (1090, 128, 4864), (1200, 128, 4864)])
 def test_every_token_tile_width(M, N, K):
-    """The GEMMs pick a token-tile width of 256, 320, 352 or 384 per problem
-    from the tile count per CTA round (148 CTAs): these shapes select 320,
-    352 and 384 in the forward (weight rows N = 4864) and in the dX product
-    (rows K = 4864), each with a ragged token tail; 64 sampled rows."""
+    """The GEMMs pick a token-tile width of 256, 320, 352, 384 or 416 per
+    problem from the tile count per CTA round (148 CTAs): these shapes
+    select 320, 352, 384 and 416 in the forward (weight rows N = 4864) and
+    in the dX product (rows K = 4864), each with a ragged token tail; 64
+    sampled rows."""
     case = synth.linear_case(f"w{M}n{N}k{K}", M, N, K, 16, 16.0, seed=21, outlier_frac=0.001)
     rows = np.sort(synth.rng(0, 121).choice(M, 64, replace=False)).astype(np.int64)
     _run_case(case, rows=rows)
