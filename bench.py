@@ -72,6 +72,67 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
+class NvmlClockSampler:
+    """SM clock and clock-event reasons read through NVML (read-only
+    queries) every millisecond from a thread, so that even a timed region of
+    a few milliseconds holds many samples.  Raises if NVML is unavailable."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, torch_device_index: int, interval_s: float = 0.001):
+        import pynvml
+        import torch
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        handle = None
+        try:  # the CUDA device's own GPU, whatever the visible-device mapping
+            pr = torch.cuda.get_device_properties(torch_device_index)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            handle = pynvml.nvmlDeviceGetHandleByIndex(torch_device_index)
+        self.h = handle
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM))
+        self.masks = [(nm, getattr(pynvml, attr)) for nm, attr in self.REASONS]
+        self.lines = []
+        self.stop_flag = False
+        self.interval = interval_s
+        self.t = threading.Thread(target=self._poll, daemon=True)
+        self.t.start()
+
+    def _poll(self):
+        nv = self.nv
+        while not self.stop_flag:
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+                self.lines.append((time.time(), sm, rs))
+            except Exception:
+                pass
+            time.sleep(self.interval)
+
+    def stop(self):
+        self.stop_flag = True
+        self.t.join(timeout=5)
+
+    def summary(self, t0, t1):
+        rows = [x for x in self.lines if t0 <= x[0] <= t1] or list(self.lines)
+        if not rows:
+            return None
+        reasons = sorted({nm for (_, _, rs) in rows for nm, m in self.masks if rs & m})
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(rows), "source": "nvml, 1 ms polling"}
+
+
+def clock_sampler(device_index: int):
+    try:
+        return NvmlClockSampler(device_index)
+    except Exception:
+        return ClockSampler(device_index)
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during a window."""
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -280,7 +341,7 @@ def run_native(args, world, rank, local):
         dist.barrier()
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(local)
+    clocks = clock_sampler(local)
     time.sleep(0.3)
     launches0 = q.qlora_kernel_launch_count()
     steps_ev, phase_ev = [], []
