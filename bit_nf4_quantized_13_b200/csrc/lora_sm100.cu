@@ -15,9 +15,9 @@
 // CTAs (S = 1..8, a power of two) of a thread-block cluster to fill the GPU.
 //
 // One CTA = one 128-row tile x one contraction split: warp 0 issues TMA,
-// warp 1 the MMAs (M = 128, N = r rounded up to 16), then all four warps
-// copy the fp32 accumulator from tensor memory into the CTA's shared
-// memory.  After a cluster barrier, rank c sums rows [c 128/S, (c+1) 128/S)
+// warp 1 the MMAs (M = 128, N = r rounded up to 16) into two accumulators
+// in turn (even and odd 16-wide k steps), then all four warps add the two
+// and copy the fp32 sum from tensor memory into the CTA's shared memory.  After a cluster barrier, rank c sums rows [c 128/S, (c+1) 128/S)
 // of the tile over the S CTAs in rank order (distributed shared memory;
 // deterministic), scales, rounds to bf16 and stores them: no partials in
 // HBM and no second kernel.
@@ -135,7 +135,9 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                                          : sdesc_kmajor_sw128(sa) + static_cast<uint64_t>(kk * 2);
                 const uint64_t bd = B_MN ? sdesc_mnmajor_sw128(sb + kk * 2048, 8192)
                                          : sdesc_kmajor_sw128(sb) + static_cast<uint64_t>(kk * 2);
-                mma_bf16_ss(tmem, ad, bd, idesc, (kb > kb_begin || kk > 0) ? 1u : 0u);
+                // two accumulators in turn (even and odd k steps): consecutive
+                // MMAs are independent, which nearly halves their issue time
+                mma_bf16_ss(tmem + (kk & 1) * (p.tmem_cols / 2), ad, bd, idesc, (kb > kb_begin || kk >= 2) ? 1u : 0u);
             }
             tc_commit(empty(s));
         }
@@ -151,14 +153,16 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
         tc_fence_after();
         const int lr = warp * 32 + lane;
         for (int c0 = 0; c0 < p.nt; c0 += 16) {
-            uint32_t v[16];
+            uint32_t v[16], w[16];
             tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
+            tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + p.tmem_cols / 2 + c0, w);
             tmem_wait_ld();
 #pragma unroll
-            for (int t = 0; t < 16; t += 4)
+            for (int t = 0; t < 16; t += 4)  // even k steps + odd k steps
                 *reinterpret_cast<float4*>(acc + lr * ld + c0 + t) = make_float4(
-                    __uint_as_float(v[t]), __uint_as_float(v[t + 1]), __uint_as_float(v[t + 2]),
-                    __uint_as_float(v[t + 3]));
+                    __uint_as_float(v[t]) + __uint_as_float(w[t]), __uint_as_float(v[t + 1]) + __uint_as_float(w[t + 1]),
+                    __uint_as_float(v[t + 2]) + __uint_as_float(w[t + 2]),
+                    __uint_as_float(v[t + 3]) + __uint_as_float(w[t + 3]));
         }
     } else {
         for (int i = threadIdx.x; i < kRows * ld; i += kThreads) acc[i] = 0.0f;
@@ -251,7 +255,8 @@ Plan plan(int64_t rows, int64_t ctr, int r, bool b_mn) {
     pl.smem = (pl.stages * stage > staging ? pl.stages * stage : staging) + 1024 + 1024;
     uint32_t c = 32;
     while (c < static_cast<uint32_t>(pl.nt)) c <<= 1;
-    pl.tmem_cols = c;
+    pl.tmem_cols = 2 * c;  // two accumulators of c columns; at most 512 per SM for every r <= 256
+                           // (r > 64 leaves room for one CTA per SM, r <= 64 for two)
     return pl;
 }
 
