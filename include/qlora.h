@@ -44,7 +44,7 @@ typedef enum qlora_status {
     QLORA_ERR_WORKSPACE = 3,   /* ws NULL or ws_bytes below the documented size       */
     QLORA_ERR_CUDA = 4,        /* a kernel launch or CUDA runtime call failed          */
     QLORA_ERR_NONFINITE = 5,   /* written to the device status word: NaN/Inf in W      */
-    QLORA_ERR_TIMEOUT = 6      /* reserved: a bounded device wait gave up              */
+    QLORA_ERR_TIMEOUT = 6      /* from qlora_device_error: a device-side wait gave up  */
 } qlora_status;
 
 #define QLORA_BLOCK 64       /* first-level block: elements per absmax constant  */
@@ -59,7 +59,7 @@ typedef enum qlora_status {
  * probabilities from 1/2 out to delta = ((1 - 1/30) + (1 - 1/32)) / 2.
  * out_host: HOST array of 16 floats, sorted ascending (out[7] == 0,
  * out[0] == -1, out[15] == +1).  Pure host function; never touches the GPU.
- * Returns QLORA_INVALID_ARG for a NULL pointer.
+ * Returns QLORA_ERR_INVALID_ARG for a NULL pointer.
  */
 int qlora_nf4_codebook(float out_host[16]);
 
