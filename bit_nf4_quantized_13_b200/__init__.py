@@ -110,9 +110,63 @@ def _check(fn: str, st: int) -> None:
 
 
 def _need_cuda(*ts):
+    """Contiguous CUDA tensors, all on one device (the current one while the
+    call runs: the library launches on the current device's stream)."""
+    dev = None
     for t in ts:
-        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+        if t is None:
+            continue
+        if not t.is_cuda or not t.is_contiguous():
             raise ValueError("tensors must be contiguous CUDA tensors")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors on different devices: {dev} and {t.device}")
+    if dev is not None and dev.index is not None and dev.index != _torch().cuda.current_device():
+        raise ValueError(f"tensors are on {dev} but the current device is cuda:"
+                         f"{_torch().cuda.current_device()}")
+
+
+def _need_dtype(dtype, **ts):
+    for name, t in ts.items():
+        if t is not None and t.dtype != dtype:
+            raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _need_shape(name, t, shape):
+    if t is not None and tuple(t.shape) != tuple(int(d) for d in shape):
+        raise ValueError(f"{name} must have shape {tuple(int(d) for d in shape)}, got {tuple(t.shape)}")
+
+
+def _need_weight(w, numel):
+    """The four buffers of an Nf4Weight hold at least what `numel` weights need
+    (the kernels read exactly that much)."""
+    nb = -(-numel // BLOCK)
+    need = {"codes": (numel + 1) // 2, "c2_fp8": nb, "c1": -(-nb // BLOCK2), "mean": 1}
+    for name, n in need.items():
+        t = getattr(w, name)
+        if t.numel() < n:
+            raise ValueError(f"Nf4Weight.{name} holds {t.numel()} elements, {n} needed")
+    torch = _torch()
+    _need_dtype(torch.uint8, codes=w.codes, c2_fp8=w.c2_fp8)
+    _need_dtype(torch.float32, c1=w.c1, mean=w.mean)
+
+
+def _linear_dims(X, w, A, B):
+    """(M, N, K, r) of a linear call, checking that the operands agree."""
+    if X.dim() != 2 or len(w.shape) != 2 or A.dim() != 2 or B.dim() != 2:
+        raise ValueError("X, the weight, A and B must be 2-D")
+    M, K = (int(d) for d in X.shape)
+    N, Kw = (int(d) for d in w.shape)
+    if Kw != K:
+        raise ValueError(f"X has K = {K} columns but the weight is {N} x {Kw}")
+    r = int(A.shape[0])
+    _need_shape("A", A, (r, K))
+    _need_shape("B", B, (N, r))
+    _need_weight(w, N * K)
+    torch = _torch()
+    _need_dtype(torch.bfloat16, X=X, A=A, B=B)
+    return M, N, K, r
 
 
 def _workspace(nbytes: int, device):
@@ -175,6 +229,10 @@ def qlora_quantize_nf4_dq(W, out: Nf4Weight | None = None, ws=None, status=None,
         raise ValueError("W must be float32")
     n = W.numel()
     w = out if out is not None else alloc_nf4_weight(tuple(W.shape), W.device)
+    _need_weight(w, n)
+    _need_cuda(W, w.codes, w.c2_fp8, w.c1, w.mean, ws, status)
+    if status is not None:
+        _need_dtype(torch.int32, status=status)
     if ws is None:
         ws = _workspace(qlora_quantize_workspace_size(n), W.device)
     st = _get_lib().qlora_quantize_nf4_dq(_ptr(W), n, BLOCK, BLOCK2, _ptr(w.codes), _ptr(w.c2_fp8),
@@ -188,8 +246,13 @@ def qlora_dequantize(w: Nf4Weight, out_dtype=None, out=None, stream=None):
     torch = _torch()
     out_dtype = out_dtype or torch.float32
     code = {torch.float32: 0, torch.bfloat16: 1}[out_dtype]
+    _need_weight(w, w.numel)
     if out is None:
         out = torch.empty(w.shape, dtype=out_dtype, device=w.codes.device)
+    _need_dtype(out_dtype, out=out)
+    if out.numel() < w.numel:
+        raise ValueError(f"out holds {out.numel()} elements, {w.numel} needed")
+    _need_cuda(w.codes, w.c2_fp8, w.c1, w.mean, out)
     st = _get_lib().qlora_dequantize(_ptr(w.codes), _ptr(w.c2_fp8), _ptr(w.c1), _ptr(w.mean), w.numel,
                               BLOCK, BLOCK2, _ptr(out), code, _stream(stream))
     _check("qlora_dequantize", st)
@@ -209,10 +272,11 @@ def qlora_linear_bwd_workspace_size(M, N, K, r) -> int:
 def qlora_linear_fwd(X, w: Nf4Weight, A, B, s: float, Y=None, T_save=None, ws=None, stream=None):
     """Y = X W'^T + s (X A^T) B^T; returns (Y, T) with T = bf16(s X A^T)."""
     torch = _torch()
-    _need_cuda(X, A, B)
-    M, K = X.shape
-    N = w.shape[0]
-    r = A.shape[0]
+    M, N, K, r = _linear_dims(X, w, A, B)
+    _need_shape("Y", Y, (M, N))
+    _need_shape("T_save", T_save, (M, r))
+    _need_dtype(torch.bfloat16, Y=Y, T_save=T_save)
+    _need_cuda(X, A, B, Y, T_save, ws, w.codes, w.c2_fp8, w.c1, w.mean)
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
     if T_save is None:
@@ -230,10 +294,14 @@ def qlora_linear_bwd(dY, X, w: Nf4Weight, A, B, s: float, T=None, dX=None, dA=No
                      ws=None, want_dx: bool = True, stream=None):
     """Adapter gradients and the input gradient; no gradient for W."""
     torch = _torch()
-    _need_cuda(dY, X, A, B, T)
-    M, K = X.shape
-    N = w.shape[0]
-    r = A.shape[0]
+    M, N, K, r = _linear_dims(X, w, A, B)
+    _need_shape("dY", dY, (M, N))
+    _need_shape("T", T, (M, r))
+    _need_shape("dX", dX, (M, K))
+    _need_shape("dA", dA, (r, K))
+    _need_shape("dB", dB, (N, r))
+    _need_dtype(torch.bfloat16, dY=dY, T=T, dX=dX, dA=dA, dB=dB)
+    _need_cuda(dY, X, A, B, T, dX, dA, dB, ws, w.codes, w.c2_fp8, w.c1, w.mean)
     if want_dx and dX is None:
         dX = torch.empty((M, K), dtype=torch.bfloat16, device=X.device)
     if dA is None:
@@ -252,7 +320,12 @@ def qlora_linear_bwd(dY, X, w: Nf4Weight, A, B, s: float, T=None, dX=None, dA=No
 
 def qlora_fp8_e4m3_encode(x, out=None, stream=None):
     torch = _torch()
-    _need_cuda(x)
+    _need_dtype(torch.float32, x=x)
+    if out is not None:
+        _need_dtype(torch.uint8, out=out)
+        if out.numel() < x.numel():
+            raise ValueError(f"out holds {out.numel()} elements, {x.numel()} needed")
+    _need_cuda(x, out)
     if out is None:
         out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     _check("qlora_fp8_e4m3_encode",
@@ -283,6 +356,10 @@ def qlora_quantize_nf4_dq_noalloc(W, out: Nf4Weight | None = None, status=None,
     if W.dtype != torch.float32:
         raise ValueError("W must be float32")
     w = out if out is not None else alloc_nf4_weight(tuple(W.shape), W.device)
+    _need_weight(w, W.numel())
+    _need_cuda(W, w.codes, w.c2_fp8, w.c1, w.mean, status)
+    if status is not None:
+        _need_dtype(torch.int32, status=status)
     st = _get_lib().qlora_quantize_nf4_dq_noalloc(_ptr(W), W.numel(), BLOCK, BLOCK2, _ptr(w.codes),
                                            _ptr(w.c2_fp8), _ptr(w.c1), _ptr(w.mean), _ptr(status),
                                            _stream(stream))

@@ -119,10 +119,13 @@ def test_unsupported_shapes_raise():
     case = synth.linear_case("bad", 4, 64, 128, 8, 16.0, seed=5)
     wq = q.qlora_quantize_nf4_dq(dev_f32(case.W))
     X, A, B = dev_bf16(case.X), dev_bf16(case.A), dev_bf16(case.B)
-    with pytest.raises(q.QloraError) as e:
+    with pytest.raises(q.QloraError) as e:  # K % 64 != 0, operands consistent: refused by the library
         Xbad = torch.zeros((4, 100), dtype=torch.bfloat16, device="cuda")
-        q.qlora_linear_fwd(Xbad, q.Nf4Weight(wq.codes, wq.c2_fp8, wq.c1, wq.mean, (64, 100)), A, B, 1.0)
+        Abad = torch.zeros((8, 100), dtype=torch.bfloat16, device="cuda")
+        q.qlora_linear_fwd(Xbad, q.Nf4Weight(wq.codes, wq.c2_fp8, wq.c1, wq.mean, (64, 100)), Abad, B, 1.0)
     assert e.value.status == 2
+    with pytest.raises(ValueError):  # operands that disagree: refused by the binding
+        q.qlora_linear_fwd(X, wq, torch.zeros((8, 64), dtype=torch.bfloat16, device="cuda"), B, 1.0)
     Abig = torch.zeros((257, 128), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(q.QloraError):
         q.qlora_linear_fwd(X, wq, Abig, torch.zeros((64, 257), dtype=torch.bfloat16, device="cuda"), 1.0)
