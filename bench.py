@@ -396,6 +396,23 @@ def run_native(args, world, rank, local):
             torch.cuda.synchronize()
             dq_ms += e0.elapsed_time(e1)
             dq_bytes += dequant_bytes(b["case"].W.size, 2)
+    # the same to fp32 (the other output type of row a7), into one buffer sized
+    # for the larger weight
+    dq32_ms, dq32_bytes = 0.0, 0
+    w32buf = torch.empty(max(b["case"].W.size for b in bufs), dtype=torch.float32, device=dev)
+    for rep in range(max(3, args.steps // 4) + 2):
+        for b in bufs:
+            n = b["case"].W.size
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            q.qlora_dequantize(b["wq"], torch.float32, out=w32buf[:n])
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 2:
+                dq32_ms += e0.elapsed_time(e1)
+                dq32_bytes += dequant_bytes(n, 4)
+    del w32buf
 
     # the dominant kernel: the backward's dX path (the transposed-weight prep
     # and the NF4 GEMM dX = dY W' + U A), timed live as the backward with dX
@@ -517,6 +534,8 @@ def run_native(args, world, rank, local):
                 "quantize_frac_hbm": qbytes / (qt * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "dequant_bf16_gbs": dq_bytes / (dq_ms * 1e-3) / 1e9 if dq_ms else None,
                 "dequant_bf16_frac_hbm": (dq_bytes / (dq_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]) if dq_ms else None,
+                "dequant_fp32_gbs": dq32_bytes / (dq32_ms * 1e-3) / 1e9 if dq32_ms else None,
+                "dequant_fp32_frac_hbm": (dq32_bytes / (dq32_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]) if dq32_ms else None,
                 "fwd_tflops": fwd_tflops, "fwd_frac_tensor": fwd_tflops / tc_peak,
                 "bwd_tflops": bflops / (bt * 1e-3) / 1e12, "dx_path_tflops": dx_tflops,
                 "unfused_fwd_tflops": k9_tflops,
