@@ -128,7 +128,7 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
 }
 
 struct Pipe {
-    uint8_t* sA;       // kStages x 48 KiB of activation tiles (two 192-token halves)
+    uint8_t* sA;       // kStages activation stages of 2w tokens x 64 (two w-token halves)
     float* sS;         // backward: per dequant warp, 64 block constants
     uint32_t bar0;     // full_b[S], full_a[S], empty[S], acc_full, acc_empty
     uint32_t tmem;     // accumulators at columns [0, 2w), A stages after them
