@@ -188,6 +188,23 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+class L2Flush:
+    """Leaves the L2 cache holding only clean lines of a buffer no kernel
+    uses: a write of one buffer larger than L2, then a read of another one.
+    The read evicts the write's dirty lines (their write-back happens here,
+    outside any timed region), so the next timed kernel neither finds its
+    inputs in L2 nor pays for writing back someone else's dirty lines."""
+
+    def __init__(self, torch, dev, nbytes: int = L2_FLUSH_BYTES):
+        self.w = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(nbytes // 4, dtype=torch.int32, device=dev)
+        self.sink = torch.empty((), dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.sink.copy_(self.r.max())
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -238,6 +255,25 @@ def oracle_baseline(cases, wbs, rows_m=4, quant_elems=1 << 22):
             "sample": (f"fwd+bwd of {rows_m} tokens per linear (full N, K, r=64) and quantization of "
                        f"the first {quant_elems} weights per linear, both linears"),
             "quant_gbs": qb_tot / tq_tot / 1e9, "seconds": tl_tot + tq_tot}
+
+
+def oracle_decode_baseline():
+    """The oracle's small-batch forward at the LLaMA-13B decode shapes, in
+    full: W 5120x5120 and 13824x5120, one token, r = 16 (the forward over
+    the oracle's own bf16 dequantized weight; its NF4 round trip is done
+    beforehand, untimed).  GB/s counts the same algorithmic bytes as the
+    GPU's decode entries."""
+    import oracle
+    out = {}
+    for which in range(2):
+        c = synth.decode13b_linear(which, 1, seed=0)
+        wb = oracle_weight_bf16(c)
+        t0 = time.perf_counter()
+        oracle.linear_fwd(c.X, wb, c.A, c.B, c.s)
+        dt = time.perf_counter() - t0
+        nbytes = decode_bytes(1, c.N, c.K, c.r)
+        out[f"{c.N}x{c.K}_m1"] = {"ms": dt * 1e3, "gbs": nbytes / dt / 1e9}
+    return out
 
 
 def run_reference(args, world, rank):
@@ -310,7 +346,7 @@ def run_native(args, world, rank, local):
                                device=dev)
         b["Wdq"] = torch.empty((c.N, c.K), dtype=torch.bfloat16, device=dev)
         bufs.append(b)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(torch, dev)
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
@@ -347,7 +383,7 @@ def run_native(args, world, rank, local):
     steps_ev, phase_ev = [], []
     t_wall0 = time.time()
     for _ in range(args.steps):
-        flush.zero_()  # L2 flush between timed steps (outside the step's events)
+        flush()  # L2 flush between timed steps (outside the step's events)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         pe = new_events()
         s0.record(stream)
@@ -388,7 +424,7 @@ def run_native(args, world, rank, local):
             q.qlora_dequantize(b["wq"], torch.bfloat16, out=b["Wdq"])
     for _ in range(max(3, args.steps // 4)):
         for b in bufs:
-            flush.zero_()
+            flush()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             q.qlora_dequantize(b["wq"], torch.bfloat16, out=b["Wdq"])
@@ -403,7 +439,7 @@ def run_native(args, world, rank, local):
     for rep in range(max(3, args.steps // 4) + 2):
         for b in bufs:
             n = b["case"].W.size
-            flush.zero_()
+            flush()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             q.qlora_dequantize(b["wq"], torch.float32, out=w32buf[:n])
@@ -423,7 +459,7 @@ def run_native(args, world, rank, local):
             c = b["case"]
             tt = []
             for want in (True, False):
-                flush.zero_()
+                flush()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 q.qlora_linear_bwd(b["dY"], b["X"], b["wq"], b["A"], b["B"], c.s, T=b["T"],
@@ -443,7 +479,7 @@ def run_native(args, world, rank, local):
     for rep in range(k9_reps + 2):
         for b in bufs:
             c = b["case"]
-            flush.zero_()
+            flush()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             q.qlora_dequantize(b["wq"], torch.bfloat16, out=b["Wdq"])
@@ -457,8 +493,10 @@ def run_native(args, world, rank, local):
     k9_tflops = sum(fwd_flops(c.M, c.N, c.K, c.r) for c in cases) * k9_reps / (k9_ms * 1e-3) / 1e12
 
     decode = run_decode(q, torch, dev, stream, flush, args) if rank == 0 and not args.no_decode else None
-
     peaks, peak_src = load_peaks()
+    full7b = run_full_7b_set(q, torch, dev, stream, peaks) if rank == 0 and not args.no_c3 else None
+    l65b = run_llama65b_layer(q, torch, dev, stream, flush, peaks, args) if rank == 0 and not args.no_c4 else None
+
     # the GEMM is timed in short bursts between L2 flushes: the burst peak
     tc_peak = peaks["bf16_tflops"]
     fwd_tflops = fflops / (ft * 1e-3) / 1e12
@@ -517,6 +555,8 @@ def run_native(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_baseline(cases, [oracle_weight_bf16(c) for c in cases], rows_m=256, quant_elems=1 << 24)
+        cpu["decode_13b"] = oracle_decode_baseline()
+        cpu["sample"] += "; plus the 13B decode forward (M = 1, both shapes) in full"
 
     if rank == 0:
         line = {
@@ -525,7 +565,8 @@ def run_native(args, world, rank, local):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": WORKLOAD, "linears": ["4096x4096", "11008x4096"], "tokens_per_gpu": M_TOKENS,
                        "rank": RANK, "alpha": ALPHA, "block": 64, "block2": 256,
-                       "l2": "flushed between timed steps (256 MiB write); inputs also exceed L2",
+                       "l2": ("flushed between timed steps (256 MiB write, then a 256 MiB read of another buffer, "
+                              "so L2 holds only clean lines); inputs also exceed L2"),
                        "parallelism": f"dp{world}"},
             "gpu_launches": int(launches),
             "roofline": roofline,
@@ -540,6 +581,8 @@ def run_native(args, world, rank, local):
                 "bwd_tflops": bflops / (bt * 1e-3) / 1e12, "dx_path_tflops": dx_tflops,
                 "unfused_fwd_tflops": k9_tflops,
                 "decode": decode,
+                "full_llama7b_weight_set": full7b,
+                "llama65b_layer": l65b,
                 "ms": {"quantize": qt / args.steps, "fwd": ft / args.steps, "bwd": bt / args.steps},
                 "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": tc_peak, "source": peak_src}},
             "clocks": clocks.summary(t_wall0, t_wall1),
@@ -551,6 +594,145 @@ def run_native(args, world, rank, local):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def run_full_7b_set(q, torch, dev, stream, peaks):
+    """The full LLaMA-7B-shaped weight set (224 tensors: 32 layers x q, k, v,
+    o 4096^2, gate, up 11008x4096, down 4096x11008; 6 476 005 376 weights,
+    Student-t df=5 rescaled to std 0.02), all resident in HBM: quantized
+    tensor by tensor, back to back, then dequantized to fp32 and to bf16 the
+    same way.  Every pass reads data written long before (26 GB of inputs
+    against a 126 MB L2), so no flush is needed.  bits/param counts the four
+    stored buffers of every tensor."""
+    shapes = synth.llama7b_weight_shapes()
+    Ws, wqs = [], []
+    for i, (_, n, k) in enumerate(shapes):
+        Ws.append(synth.student_t_device(0, 1000 + i, n * k, dev).view(n, k))
+        wqs.append(q.alloc_nf4_weight((n, k), dev))
+    params = sum(n * k for _, n, k in shapes)
+    qws = torch.empty(q.qlora_quantize_workspace_size(max(n * k for _, n, k in shapes)), dtype=torch.uint8,
+                      device=dev)
+    stored = sum(w.nbytes() for w in wqs)
+
+    def timed(fn, reps=2):
+        best = None
+        for _ in range(reps):
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        return best
+
+    def quant_all():
+        for W, wq in zip(Ws, wqs):
+            q.qlora_quantize_nf4_dq(W, out=wq, ws=qws)
+
+    quant_all()  # warm-up (first launches)
+    tq = timed(quant_all)
+    qbytes = sum(quant_bytes(n * k) for _, n, k in shapes)
+    del Ws
+    out32 = torch.empty(params, dtype=torch.float32, device=dev)
+    offs = np.cumsum([0] + [n * k for _, n, k in shapes])
+
+    def dq_all(dtype, out):
+        for j, wq in enumerate(wqs):
+            q.qlora_dequantize(wq, dtype, out=out[offs[j]:offs[j + 1]])
+
+    dq_all(torch.float32, out32)
+    t32 = timed(lambda: dq_all(torch.float32, out32))
+    out16 = out32.view(torch.bfloat16)[:params]
+    dq_all(torch.bfloat16, out16)
+    t16 = timed(lambda: dq_all(torch.bfloat16, out16))
+    b32 = sum(dequant_bytes(n * k, 4) for _, n, k in shapes)
+    b16 = sum(dequant_bytes(n * k, 2) for _, n, k in shapes)
+    del out32, out16, wqs
+    hbm = peaks["hbm_gbs"]
+    return {"tensors": len(shapes), "params": params, "bits_per_param": 8.0 * stored / params,
+            "stored_bytes": stored,
+            "quantize_ms": tq, "quantize_gbs": qbytes / (tq * 1e-3) / 1e9,
+            "quantize_frac_hbm": qbytes / (tq * 1e-3) / 1e9 / hbm,
+            "dequant_fp32_ms": t32, "dequant_fp32_gbs": b32 / (t32 * 1e-3) / 1e9,
+            "dequant_fp32_frac_hbm": b32 / (t32 * 1e-3) / 1e9 / hbm,
+            "dequant_bf16_ms": t16, "dequant_bf16_gbs": b16 / (t16 * 1e-3) / 1e9,
+            "dequant_bf16_frac_hbm": b16 / (t16 * 1e-3) / 1e9 / hbm,
+            "inputs": "Student-t df=5 x 0.02/sqrt(5/3), generated on the GPU (synth.student_t_device, seed 0)"}
+
+
+def run_llama65b_layer(q, torch, dev, stream, flush, peaks, args):
+    """A LLaMA-65B-shaped decoder layer's seven linears (q, k, v, o 8192^2,
+    gate, up 22016x8192, down 8192x22016; r=64, alpha=16, LoRA on every
+    linear): per token count M in 512/2048/8192, the forward and backward
+    (dX, dA, dB) of all seven, timed per linear with CUDA events; one layer
+    pass per timed iteration, L2 flushed between iterations."""
+    layer = synth.LLAMA65B_LAYER
+    wqs = []
+    for i, (_, n, k) in enumerate(layer):
+        W = synth.normal_device(0, 2000 + i, (n, k), dev, std=0.02)
+        wqs.append(q.qlora_quantize_nf4_dq(W))
+        del W
+    reps = max(3, min(10, args.steps // 5))
+    out = {}
+    tc_b, tc_s = peaks["bf16_tflops"], peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    for M in synth.LLAMA65B_TOKENS:
+        lin = []
+        for i, (nm, n, k) in enumerate(layer):
+            d = {"name": nm, "N": n, "K": k}
+            d["X"] = synth.normal_device(1, 3000 + 10 * i, (M, k), dev, dtype=torch.bfloat16)
+            d["dY"] = synth.normal_device(1, 3001 + 10 * i, (M, n), dev, dtype=torch.bfloat16)
+            d["A"] = synth.normal_device(1, 3002 + 10 * i, (RANK, k), dev, std=0.01, dtype=torch.bfloat16)
+            d["B"] = synth.normal_device(1, 3003 + 10 * i, (n, RANK), dev, std=0.01, dtype=torch.bfloat16)
+            d["Y"] = torch.empty((M, n), dtype=torch.bfloat16, device=dev)
+            d["T"] = torch.empty((M, RANK), dtype=torch.bfloat16, device=dev)
+            d["dX"] = torch.empty((M, k), dtype=torch.bfloat16, device=dev)
+            d["dA"] = torch.empty((RANK, k), dtype=torch.bfloat16, device=dev)
+            d["dB"] = torch.empty((n, RANK), dtype=torch.bfloat16, device=dev)
+            d["ws"] = torch.empty(q.qlora_linear_bwd_workspace_size(M, n, k, RANK), dtype=torch.uint8, device=dev)
+            lin.append(d)
+        s_lora = ALPHA / RANK
+
+        def layer_pass(ev=None):
+            for i, (d, wq) in enumerate(zip(lin, wqs)):
+                if ev is not None:
+                    ev[i][0].record(stream)
+                q.qlora_linear_fwd(d["X"], wq, d["A"], d["B"], s_lora, Y=d["Y"], T_save=d["T"], ws=d["ws"])
+                if ev is not None:
+                    ev[i][1].record(stream)
+                q.qlora_linear_bwd(d["dY"], d["X"], wq, d["A"], d["B"], s_lora, T=d["T"], dX=d["dX"],
+                                   dA=d["dA"], dB=d["dB"], ws=d["ws"])
+                if ev is not None:
+                    ev[i][2].record(stream)
+
+        layer_pass()
+        torch.cuda.synchronize()
+        fwd_ms = [0.0] * len(layer)
+        bwd_ms = [0.0] * len(layer)
+        tot_ms = 0.0
+        for _ in range(reps):
+            flush()
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in layer]
+            layer_pass(ev)
+            torch.cuda.synchronize()
+            for i in range(len(layer)):
+                fwd_ms[i] += ev[i][0].elapsed_time(ev[i][1]) / reps
+                bwd_ms[i] += ev[i][1].elapsed_time(ev[i][2]) / reps
+            tot_ms += ev[0][0].elapsed_time(ev[-1][2]) / reps
+        per = []
+        fl_tot = 0.0
+        for i, (nm, n, k) in enumerate(layer):
+            ff, fb = fwd_flops(M, n, k, RANK), linear_flops(M, n, k, RANK) - fwd_flops(M, n, k, RANK)
+            fl_tot += ff + fb
+            per.append({"linear": f"{nm} {n}x{k}", "fwd_ms": fwd_ms[i], "bwd_ms": bwd_ms[i],
+                        "fwd_tflops": ff / (fwd_ms[i] * 1e-3) / 1e12, "bwd_tflops": fb / (bwd_ms[i] * 1e-3) / 1e12,
+                        "fwd_bwd_tflops": (ff + fb) / ((fwd_ms[i] + bwd_ms[i]) * 1e-3) / 1e12})
+        tf = fl_tot / (tot_ms * 1e-3) / 1e12
+        out[f"m{M}"] = {"layer_ms": tot_ms, "layer_flops": fl_tot, "layer_tflops": tf,
+                        "frac_burst": tf / tc_b, "frac_sustained": tf / tc_s, "linears": per}
+        del lin
+    return out
 
 
 def decode_bytes(M, N, K, r):
@@ -591,7 +773,7 @@ def run_decode(q, torch, dev, stream, flush, args):
             torch.cuda.synchronize()
             direct = []
             for _ in range(reps):
-                flush.zero_()
+                flush()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 call()
@@ -606,7 +788,7 @@ def run_decode(q, torch, dev, stream, flush, args):
             torch.cuda.synchronize()
             graphed = []
             for _ in range(reps):
-                flush.zero_()
+                flush()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 g.replay()
@@ -630,7 +812,7 @@ def run_decode(q, torch, dev, stream, flush, args):
             torch.cuda.synchronize()
             uf = []
             for _ in range(reps):
-                flush.zero_()
+                flush()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 unfused()
@@ -655,6 +837,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-c3", action="store_true", help="skip the full LLaMA-7B-shaped weight set")
+    ap.add_argument("--no-c4", action="store_true", help="skip the LLaMA-65B-shaped layer")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the small-batch forward (LLaMA-13B decode shapes) and print it")
     ap.add_argument("--decode-case", default="", help="e.g. 13824x5120_m16: one decode configuration")
@@ -666,7 +850,7 @@ def main(argv=None):
         import bit_nf4_quantized_13_b200 as q
         dev = torch.device("cuda", local)
         torch.cuda.set_device(dev)
-        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        flush = L2Flush(torch, dev)
         res = run_decode(q, torch, dev, torch.cuda.current_stream(), flush, args)
         peaks, src = load_peaks()
         for v in res.values():

@@ -63,6 +63,7 @@ def _load() -> ctypes.CDLL:
         "qlora_kernel_launch_count": (ctypes.c_uint64, []),
         "qlora_device_error": (i32, [i32]),
         "qlora_quantize_nf4_dq_noalloc": (i32, [vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]),
+        "qlora_debug_wait_timeout": (i32, [ctypes.c_uint64, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -337,6 +338,13 @@ def qlora_device_error(reset: bool = False) -> int:
     """Sticky error word of the tensor-core kernels (0 = none, 6 = a bounded
     in-kernel wait timed out)."""
     return int(_get_lib().qlora_device_error(1 if reset else 0))
+
+
+def qlora_debug_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Failure-detection self-test: one kernel whose bounded wait is never
+    satisfied gives up after limit_ns (<= 1e9) and records QLORA_ERR_TIMEOUT
+    for qlora_device_error."""
+    _check("qlora_debug_wait_timeout", _get_lib().qlora_debug_wait_timeout(int(limit_ns), _stream(stream)))
 
 
 def qlora_kernel_launch_count() -> int:

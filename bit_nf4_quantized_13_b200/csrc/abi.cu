@@ -75,6 +75,7 @@ inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLO
 inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 
 constexpr int64_t kMaxNumel = int64_t(1) << 46;
+constexpr uint64_t kMaxSelftestWaitNs = 1000000000ull;  // the self-test waits at most 1 s
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -202,6 +203,11 @@ int qlora_device_error(int reset) {
     const int b = lora_device_error(reset);
     const int c = gemv_device_error(reset);
     return a != QLORA_OK ? a : b != QLORA_OK ? b : c;
+}
+
+int qlora_debug_wait_timeout(uint64_t limit_ns, void* stream) {
+    if (limit_ns == 0 || limit_ns > kMaxSelftestWaitNs) return QLORA_ERR_INVALID_ARG;
+    return cuda_status(launch_wait_selftest(limit_ns, as_stream(stream)));
 }
 
 uint64_t qlora_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include "../../include/qlora.h"
+#include "ctx_memo.h"
 
 namespace qlora {
 
@@ -69,6 +70,28 @@ __host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return ceil_
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int num_sms();  // cached SM count of the current device
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` once per CUDA
+// context (function attributes belong to the loaded module, which a device
+// reset unloads); `memo` is the launcher's own, one per kernel instance.
+template <typename Kernel>
+cudaError_t ensure_smem_limit(ContextMemo<int>& memo, Kernel kernel, int bytes) {
+    uint64_t ctx = 0;
+    if (!current_context_id(&ctx)) return cudaErrorDeviceUninitialized;
+    cudaError_t err = cudaSuccess;
+    int have = 0;
+    const bool ok = memo.get(ctx, &have, [&](int* v) {
+        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        *v = bytes;
+        return err == cudaSuccess;
+    });
+    if (!ok) return err != cudaSuccess ? err : cudaErrorUnknown;
+    if (have < bytes) {  // a larger request than the one made in this context
+        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (err != cudaSuccess) return err;
+    }
+    return cudaSuccess;
+}
 
 // Counts kernel launches for qlora_kernel_launch_count (host side).
 void note_launches(int n);

@@ -139,12 +139,10 @@ k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,
                               const float* mean, int64_t numel, void* out, int out_dtype,
                               cudaStream_t stream) {
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(k_dequant<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutBytes);
-        cudaFuncSetAttribute(k_dequant<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutBytes);
-        attr = true;
-    }
+    static ContextMemo<int> memo_bf16, memo_f32;
+    const cudaError_t attr = out_dtype == 1 ? ensure_smem_limit(memo_bf16, k_dequant<true>, kLutBytes)
+                                            : ensure_smem_limit(memo_f32, k_dequant<false>, kLutBytes);
+    if (attr != cudaSuccess) return attr;
     const int64_t chunks = ceil_div(numel, kChunk);
     const int64_t want = ceil_div(chunks, kThreads / 32);
     const int grid = static_cast<int>(want < num_sms() * 3LL ? (want > 0 ? want : 1) : num_sms() * 3LL);

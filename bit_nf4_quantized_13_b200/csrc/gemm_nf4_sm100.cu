@@ -634,12 +634,8 @@ cudaError_t launch_tc_geo(const uint16_t* act, const uint16_t* lora_act, const G
     if (!make_map_bf16(&ma, act, static_cast<uint64_t>(p0.ctr), static_cast<uint64_t>(p0.M), kBK, kSubT) ||
         !make_map_bf16(&ml, lora_act, static_cast<uint64_t>(p0.r), static_cast<uint64_t>(p0.M), kBK, kSubT))
         return cudaErrorInvalidValue;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(k_nf4_gemm_tc<kBwd, kSubT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        G::kSmemBytes);
-    });
+    static ContextMemo<int> attr_memo;
+    const cudaError_t attr_err = ensure_smem_limit(attr_memo, k_nf4_gemm_tc<kBwd, kSubT>, G::kSmemBytes);
     if (attr_err != cudaSuccess) return attr_err;
     GemmParams p = p0;
     for (int i = 0; i < 16; ++i) p.q[i] = tables().q[i];
@@ -756,6 +752,27 @@ cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const 
     p.K = static_cast<int>(w.K);
     p.r = r;
     return launch_tc<true>(dY, U, p, st);
+}
+
+// The failure-detection self-test: one thread waits, with the given limit,
+// for a phase of an mbarrier that nothing ever arrives on.  No copy or MMA
+// is in flight, so when the limit passes the wait records QLORA_ERR_TIMEOUT
+// in the sticky word and the kernel simply returns.
+__global__ void k_wait_selftest(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(sm100::smem_u32(&bar), 1);
+        sm100::fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) sm100::mbar_wait(sm100::smem_u32(&bar), 0u, &g_tc_error, limit_ns);
+    __syncthreads();
+}
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st) {
+    k_wait_selftest<<<1, 32, 0, st>>>(limit_ns);
+    note_launches(1);
+    return cudaGetLastError();
 }
 
 int gemm_device_error(int reset) {

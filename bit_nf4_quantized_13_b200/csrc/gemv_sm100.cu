@@ -532,14 +532,14 @@ struct Plan {
 };
 
 // Largest number of co-resident clusters of `cl` CTAs with `smem` bytes of
-// shared memory each, cached per (device, tile count, cluster size, smem).
+// shared memory each, cached per (CUDA context, cluster size, smem).
 template <int NT>
 int max_clusters(int cl, size_t smem) {
     static std::mutex mu;
-    static std::map<std::tuple<int, int, size_t>, int> cache;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    const auto key = std::make_tuple(dev, cl, smem);
+    static std::map<std::tuple<uint64_t, int, size_t>, int> cache;
+    uint64_t ctx = 0;
+    if (!current_context_id(&ctx)) return 0;
+    const auto key = std::make_tuple(ctx, cl, smem);
     std::lock_guard<std::mutex> lk(mu);
     const auto it = cache.find(key);
     if (it != cache.end()) return it->second;

@@ -46,6 +46,9 @@ cudaError_t launch_lora_db_tc(const uint16_t* dY, const uint16_t* T, int64_t M, 
                               cudaStream_t stream);
 int lora_device_error(int reset);
 int gemm_device_error(int reset);  // gemm_nf4_sm100.cu
+// gemm_nf4_sm100.cu: a kernel whose one bounded wait is never satisfied
+// (records QLORA_ERR_TIMEOUT after limit_ns)
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
 // gemm_simt.cu: CUDA-core versions (any shape)
 cudaError_t launch_lora_xat_simt(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, float s,
                                  uint16_t* T, cudaStream_t stream);

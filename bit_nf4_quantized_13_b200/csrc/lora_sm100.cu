@@ -263,11 +263,8 @@ Plan plan(int64_t rows, int64_t ctr, int r, bool b_mn) {
 template <bool A_MN, bool B_MN>
 cudaError_t run(const Plan& pl, const CUtensorMap& ma, const CUtensorMap& mb, int64_t rows, int r, float scale,
                 uint16_t* out, bool transposed, cudaStream_t st) {
-    static std::once_flag once;
-    static cudaError_t attr = cudaSuccess;
-    std::call_once(once, [] {
-        attr = cudaFuncSetAttribute(k_lora_tc<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem + 2048);
-    });
+    static ContextMemo<int> attr_memo;
+    const cudaError_t attr = ensure_smem_limit(attr_memo, k_lora_tc<A_MN, B_MN>, kMaxSmem + 2048);
     if (attr != cudaSuccess) return attr;
     SkinnyParams p;
     p.out = out;

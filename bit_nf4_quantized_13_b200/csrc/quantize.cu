@@ -381,12 +381,19 @@ cudaError_t launch_quantize_nf4_dq(const float* W, int64_t numel, uint8_t* codes
     if (err != cudaSuccess) return err;
     const int64_t nchunks = ceil_div(numel, kChunk);
     const int64_t want = ceil_div(nchunks, kQuantThreads / 32);
-    static int resident = 0;  // CTAs of k_nf4_quantize per SM
-    if (!resident) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, k_nf4_quantize, kQuantThreads, 0) != cudaSuccess ||
-            resident < 1)
-            resident = 2;
-    }
+    // CTAs of k_nf4_quantize per SM, asked once per context
+    static ContextMemo<int> resident_memo;
+    int resident = 2;
+    uint64_t ctx = 0;
+    if (current_context_id(&ctx))
+        resident_memo.get(ctx, &resident, [](int* v) {
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, k_nf4_quantize, kQuantThreads, 0) != cudaSuccess ||
+                *v < 1) {
+                cudaGetLastError();
+                *v = 2;
+            }
+            return true;
+        });
     const int64_t cap = static_cast<int64_t>(num_sms()) * resident;
     const int grid1 = static_cast<int>(want < cap ? want : cap);
     k_nf4_quantize<<<grid1, kQuantThreads, 0, stream>>>(W, numel, codes, c2, bins, flag, tables());

@@ -12,12 +12,14 @@
 // the process exits.
 //
 // Host code must not hand the array's symbol to a kernel: on the host that
-// name is only a stand-in, not a device address.  The first call on each
-// device (with that device current) looks up the real address once with
-// cudaGetSymbolAddress and caches it; later calls reuse it.
-#include <mutex>
-
+// name is only a stand-in, not a device address.  The first call in each
+// CUDA context (with that context's device current) looks up the real
+// address with cudaGetSymbolAddress and memoizes it under the context's
+// process-unique id; later calls in the same context reuse it.  A context
+// made again after a device reset has a new id, so its first call looks the
+// address up afresh (the reloaded module's array may sit elsewhere).
 #include "common.cuh"
+#include "ctx_memo.h"
 #include "kernels.h"
 
 namespace qlora {
@@ -29,24 +31,19 @@ constexpr size_t kNoAllocScratchBytes =
 
 static __device__ __align__(256) unsigned char g_quant_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_addr_mu;
-void* g_addr[kMaxDevices] = {};
+ContextMemo<void*> g_addr;
 
-// Device address of g_quant_scratch on the current device (looked up once).
+// Device address of g_quant_scratch in the current context (looked up once
+// per context).
 cudaError_t scratch_address(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_addr_mu);
-    if (!g_addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_quant_scratch);
-        if (e != cudaSuccess) return e;
-        g_addr[dev] = p;
-    }
-    *out = g_addr[dev];
+    uint64_t ctx = 0;
+    if (!current_context_id(&ctx)) return cudaErrorDeviceUninitialized;
+    cudaError_t err = cudaSuccess;
+    const bool ok = g_addr.get(ctx, out, [&](void** p) {
+        err = cudaGetSymbolAddress(p, g_quant_scratch);
+        return err == cudaSuccess && *p != nullptr;
+    });
+    if (!ok) return err != cudaSuccess ? err : cudaErrorInvalidSymbol;
     return cudaSuccess;
 }
 

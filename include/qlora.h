@@ -112,9 +112,13 @@ int qlora_quantize_nf4_dq(const float* W, int64_t numel, int block, int block2,
  * per 64-block, sized for numel <= QLORA_NOALLOC_MAX_NUMEL (2^28 weights,
  * about 16 MiB).  Larger numel returns QLORA_ERR_WORKSPACE without
  * launching anything.  The call allocates nothing (no cudaMalloc/cudaFree).
- * The first call on each device, made with that device current, looks up
- * the array's device address once (cudaGetSymbolAddress); make that first
- * call before any stream capture.  All calls share the one array: calls
+ * The first call in each CUDA context (i.e. per device, with that device
+ * current) looks up the array's device address (cudaGetSymbolAddress) and
+ * remembers it for that context; make that first call before any stream
+ * capture.  After a device reset the next call runs in a new context and
+ * looks the address up again, so it never uses an address from before the
+ * reset (the array's contents do not survive a reset; nothing relies on
+ * them between calls).  All calls share the one array: calls
  * whose kernels overlap on the GPU (different streams without ordering,
  * or several host threads) race on it and must be serialised by the
  * caller.  Each call clears the parts that must start at zero.
@@ -200,6 +204,18 @@ int qlora_fp8_e4m3_encode(const float* x, uint8_t* out, int64_t n, void* stream)
  * Returns QLORA_ERR_CUDA if the word cannot be read.
  */
 int qlora_device_error(int reset);
+
+/*
+ * qlora_debug_wait_timeout -- failure-detection self-test (no counterpart
+ * in the paper).  Launches one single-thread kernel on `stream` whose
+ * bounded wait (the same wait every pipeline stage of the tensor-core
+ * kernels uses) is never satisfied: after limit_ns nanoseconds of GPU time
+ * it gives up, records QLORA_ERR_TIMEOUT in the sticky word that
+ * qlora_device_error reads, and returns.  Nothing else is in flight in that
+ * kernel, so the context stays usable and later calls work as usual.
+ * 0 < limit_ns <= 1e9, else QLORA_ERR_INVALID_ARG (nothing launched).
+ */
+int qlora_debug_wait_timeout(uint64_t limit_ns, void* stream);
 
 /*
  * qlora_kernel_launch_count -- number of kernels this library has launched

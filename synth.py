@@ -65,6 +65,37 @@ def weight_student_t(seed: int, tid: int, shape, df: float = 5.0, std: float = 0
     return (t * (std / math.sqrt(df / (df - 2.0)))).astype(np.float32)
 
 
+def student_t_device(seed: int, tid: int, numel: int, device, df: int = 5, std: float = 0.02):
+    """fp32 torch tensor of `numel` Student-t(df) draws, rescaled to the given
+    standard deviation, generated on `device` by torch's counter-based
+    generator seeded with (seed, tid).  For integer df the variate is built
+    from its definition: Z / sqrt(V / df) with Z ~ N(0,1) and V the sum of
+    df squared N(0,1) draws.  Used where a workload is too large to draw on
+    the host (the full LLaMA-7B-shaped weight set)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed((int(seed) << 24) ^ int(tid))
+    z = torch.randn(numel, generator=g, device=device, dtype=torch.float32)
+    v = torch.zeros(numel, device=device, dtype=torch.float32)
+    for _ in range(int(df)):
+        v.add_(torch.randn(numel, generator=g, device=device, dtype=torch.float32).square_())
+    z.div_(v.div_(float(df)).sqrt_())
+    return z.mul_(std / math.sqrt(df / (df - 2.0)))
+
+
+def normal_device(seed: int, tid: int, shape, device, std: float = 1.0, dtype=None):
+    """N(0, std^2) draws generated on `device` by torch's counter-based
+    generator seeded with (seed, tid), optionally cast (round to nearest
+    even) to `dtype`.  Used for the activations of the largest workloads."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed((int(seed) << 24) ^ int(tid))
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x if dtype is None else x.to(dtype)
+
+
 @dataclass
 class LinearCase:
     """One QLoRA linear: W (N x K) fp32, X (M x K), A (r x K), B (N x r) and dY
@@ -132,6 +163,19 @@ def llama7b_weight_shapes():
 
 LLAMA65B_LAYER = [("q", 8192, 8192), ("k", 8192, 8192), ("v", 8192, 8192), ("o", 8192, 8192),
                   ("gate", 22016, 8192), ("up", 22016, 8192), ("down", 8192, 22016)]
+
+LLAMA65B_TOKENS = (512, 2048, 8192)
+
+
+def llama65b_linear(which: int, M: int, seed: int = 0, r: int = 64, with_dy: bool = True) -> LinearCase:
+    """One linear of a LLaMA-65B-shaped decoder layer (LLAMA65B_LAYER[which]):
+    W ~N(0,0.02) with 0.1% entries x8 (the 7B-shaped recipe; the 65B case
+    states no distribution), X M x K ~N(0,1) bf16 with M in 512/2048/8192,
+    r=64, alpha=16."""
+    name, N, K = LLAMA65B_LAYER[which]
+    return linear_case(f"llama65b_{name}_{N}x{K}_m{M}_r{r}", M, N, K, r, 16.0, seed,
+                       outlier_frac=0.001, wid=20 + which, with_dy=with_dy)
+
 
 DECODE13B = [("w5120x5120", 5120, 5120), ("w13824x5120", 13824, 5120)]
 

@@ -88,3 +88,6 @@ def test_argument_validation_on_host(q):
                               1 << 20, None) == 1
     assert L.qlora_fp8_e4m3_encode(P, P, -1, None) == 1
     assert L.qlora_fp8_e4m3_encode(None, None, 0, None) == 0
+    # the failure-detection self-test refuses limits outside (0, 1 s]
+    assert L.qlora_debug_wait_timeout(0, None) == 1
+    assert L.qlora_debug_wait_timeout(2_000_000_000, None) == 1

@@ -140,6 +140,23 @@ def test_llama7b_shapes_sampled_rows(which):
     _run_case(case, rows=rows)
 
 
+# q/o (8192 x 8192), gate/up (22016 x 8192) and down (8192 x 22016: the
+# 344-block contraction) of a LLaMA-65B-shaped layer
+LLAMA65B_DISTINCT = [0, 4, 6]
+
+
+@pytest.mark.parametrize("M", [512, 8192])
+@pytest.mark.parametrize("which", LLAMA65B_DISTINCT)
+def test_llama65b_shapes(which, M):
+    """LLaMA-65B-shaped linears, r=64, alpha=16: Y, T and dX on 512 seeded
+    token rows (all rows at M = 512), dA and dB in full."""
+    case = synth.llama65b_linear(which, M, seed=0)
+    rows = None
+    if M > 512:
+        rows = np.sort(synth.rng(0, 650 + which).choice(M, 512, replace=False)).astype(np.int64)
+    _run_case(case, rows=rows)
+
+
 def test_unfused_library_path_agrees():
     """Second opinion: dequantize to bf16 with the library, then torch.matmul
     (cuBLAS) for X W'^T + (s X A^T) B^T and dY W' + (s dY B) A; the fused

@@ -66,6 +66,44 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row():
     _same(again, first)
 
 
+@pytest.mark.parametrize("numel", [1, 17, 63, 64, 65, 64 * 257 + 3])
+def test_noalloc_small_and_ragged_sizes(numel):
+    W = torch.from_numpy(synth.weight_normal(0, 503, (numel,), 0.02, 0.01)).cuda()
+    got, st = _via_abi_noalloc(W)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    _same(got, _via_abi_workspace(W))
+
+
+def test_noalloc_empty_input_launches_nothing():
+    n0 = q.qlora_kernel_launch_count()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert q.lib.qlora_quantize_nf4_dq_noalloc(None, 0, 64, 256, None, None, None, None, None, stream) == 0
+    assert q.qlora_kernel_launch_count() == n0
+
+
+def test_noalloc_call_takes_no_device_memory():
+    """With torch's caching allocator holding everything the call needs, a
+    warmed-up call leaves the device's free memory exactly where it was."""
+    W = torch.from_numpy(synth.weight_normal(0, 504, (4096, 1024), 0.02, 0.001)).cuda()
+    out = q.alloc_nf4_weight(tuple(W.shape), W.device)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def call():
+        st = q.lib.qlora_quantize_nf4_dq_noalloc(_p(W), W.numel(), 64, 256, _p(out.codes), _p(out.c2_fp8),
+                                                 _p(out.c1), _p(out.mean), None, stream)
+        assert st == 0
+
+    call()  # first call in this context: the scratch address is looked up here
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     P = 1 << 20  # never dereferenced: the size check comes first
     st = q.lib.qlora_quantize_nf4_dq_noalloc(P, q.NOALLOC_MAX_NUMEL + 1, 64, 256, P, P, P, P, None, None)
