@@ -30,12 +30,20 @@ int num_sms() {
 
 cudaError_t launch_fwd_gemm(const uint16_t* X, const Nf4Weight& w, const uint16_t* T,
                             const uint16_t* B, int64_t M, int r, uint16_t* Y, cudaStream_t st) {
+    if (pair_gemm_supported(M, w, r, false)) {
+        const cudaError_t e = launch_fwd_gemm_pair(X, w, T, B, M, r, Y, st);
+        if (e != cudaErrorNotSupported) return e;
+    }
     if (fwd_tc_supported(M, w, r)) return launch_fwd_gemm_tc(X, w, T, B, M, r, Y, st);
     return launch_fwd_gemm_simt(X, w, T, B, M, r, Y, st);
 }
 
 cudaError_t launch_bwd_dx_gemm(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U,
                                const uint16_t* A, int64_t M, int r, uint16_t* dX, void* ws, cudaStream_t st) {
+    if (pair_gemm_supported(M, w, r, true)) {
+        const cudaError_t e = launch_bwd_dx_gemm_pair(dY, w, U, A, M, r, dX, st);
+        if (e != cudaErrorNotSupported) return e;
+    }
     if (dx_tc_supported(M, w, r)) return launch_bwd_dx_gemm_tc(dY, w, U, A, M, r, dX, ws, st);
     return launch_bwd_dx_gemm_simt(dY, w, U, A, M, r, dX, st);
 }
@@ -202,7 +210,8 @@ int qlora_device_error(int reset) {
     const int a = gemm_device_error(reset);
     const int b = lora_device_error(reset);
     const int c = gemv_device_error(reset);
-    return a != QLORA_OK ? a : b != QLORA_OK ? b : c;
+    const int d = pair_device_error(reset);
+    return a != QLORA_OK ? a : b != QLORA_OK ? b : c != QLORA_OK ? c : d;
 }
 
 int qlora_debug_wait_timeout(uint64_t limit_ns, void* stream) {

@@ -1,0 +1,663 @@
+// gemm_pair_sm100.cu -- the two frozen-weight GEMMs of the QLoRA linear on
+// pairs of SMs (QLoRA study notes, gitcode.csdn.net, section 3.5 eq. 5 and
+// 6, section 4 eq. 3, and the gradient through the bf16 weight of 3.5):
+//
+//   forward:  Y  = X  W'^T + T B^T     T = bf16(s X A^T)      (M x N)
+//   backward: dX = dY W'   + U A       U = bf16(s dY B)       (M x K)
+//   W' = bf16(q[code] * c2'), double-dequantized on the fly, never stored.
+//
+// Both compute the transposed product tile by tile with the weight as the
+// MMA's A operand:
+//
+//   forward:  D[n][m] += W'[n][k]   * X[m][k]     (contract over k)
+//   backward: D[k][m] += W'^T[k][n] * dY[m][n]    (contract over n)
+//
+// A tile is 256 weight rows x 512 tokens, computed by a pair of CTAs on two
+// SMs with tcgen05.mma.cta_group::2 (M = 256, N = 256): each CTA holds 128
+// of the weight rows (its half of A, converted from NF4 by its own warps
+// into its shared memory) and two fp32 accumulators of 128 rows x 256 tokens
+// in tensor memory (all 512 columns); each accumulator's 256 tokens are
+// staged half in each CTA (B, by TMA in the 128-byte swizzled K-major
+// layout), so every MMA instruction is the full 128 x 256 x 16 per SM.
+//
+// The converted weight is written into shared memory in the 128-byte
+// swizzled layout the tensor cores read: K-major in the forward (a row n
+// holds 64 consecutive k), MN-major in the backward (a row holds 64
+// consecutive k of one contraction index n, two 64-wide blocks per CTA).
+// Both read the NF4 codes in their natural row-major layout (a 64-weight
+// run of one row shares one block constant), so the backward needs no
+// transposed copy of the weight.  The rank-r LoRA term continues the same
+// contraction over ceil(r/64) extra 64-wide slabs whose A operand (B
+// forward, A^T backward) and B operand (T forward, U backward) both come
+// by TMA.
+//
+// Codes are expanded through a 64 KiB table mapping a code byte to both of
+// its fp32 codebook values (one 8-byte copy per lane: no bank conflicts);
+// two weights cost one byte permute, one shared load, two multiplies by the
+// block constant (exactly RN(q * c2')) and one pack to bf16x2.
+//
+// Warp roles (448 threads per CTA, persistent over the pair's tiles):
+//   warp 0      TMA producer (both CTAs, into their own shared memory; the
+//               completion bytes count on the even CTA's barrier)
+//   warp 1      MMA issuer (one thread of the even CTA only)
+//   warps 2-13  converters: warp w handles the stages kb with kb % 3 ==
+//               (w - 2) / 4 (always ring slot kb % 3), 32 of the stage's 128
+//               64-weight runs; then the epilogue of its TMEM lane quarter
+//               w % 4: tcgen05.ld, bf16, stores coalesced along the
+//               weight-row index.
+// Every wait is bounded; a timeout records QLORA_ERR_TIMEOUT in a sticky
+// device word and ends the role.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+#include "tma_host.h"
+
+namespace qlora {
+
+__device__ int g_pair_error = 0;  // sticky: QLORA_ERR_TIMEOUT if a wait gave up
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kRowsCta = 128;                       // weight rows per CTA
+constexpr int kRowsPair = 2 * kRowsCta;             // MMA M
+constexpr int kSubTok = 256;                        // MMA N: tokens per accumulator
+constexpr int kSubs = 2;                            // accumulators
+constexpr int kTileTok = kSubs * kSubTok;           // tokens per tile
+constexpr int kHalfTok = kSubTok / 2;               // one accumulator's tokens staged by one CTA
+constexpr int kBK = 64;                             // contraction per stage
+constexpr int kStages = 3;
+constexpr int kABytes = kRowsCta * kBK * 2;         // 16 KiB
+constexpr int kBHalfBytes = kHalfTok * kBK * 2;     // 16 KiB
+constexpr int kStageBytes = kABytes + kSubs * kBHalfBytes;
+constexpr int kDqWarps = 12;
+constexpr int kParts = kDqWarps / 4;
+static_assert(kParts == kStages, "a part's stages must always use the same ring slot");
+constexpr int kPrefetch = 2;                        // own stages of codes in flight per converter lane
+constexpr int kThreads = 32 * (2 + kDqWarps);       // 448: 128 registers a thread
+constexpr int kLutBytes = 256 * 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kChunks = kSubs * kSubTok / 16;       // epilogue chunks of 16 columns
+constexpr int kBarOff = kStages * kStageBytes;
+constexpr int kLutOff = kBarOff + 1024;
+constexpr int kSmemBytes = 1024 /* alignment slack */ + kLutOff + kLutBytes;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+constexpr uint16_t kPairMask = 0x3;                 // both CTAs of the cluster
+// completion bytes of one stage over the pair: B halves of both CTAs, plus
+// (LoRA slabs) the A operand of both CTAs
+constexpr uint32_t kTxWeight = 2u * kSubs * kBHalfBytes;
+constexpr uint32_t kTxLora = kTxWeight + 2u * kABytes;
+
+struct PairParams {
+    const uint8_t* codes;   // W codes, N x K/2 (row-major, two k per byte)
+    const uint8_t* c2_fp8;  // N x K/64
+    const float* c1;
+    const float* mean;
+    uint16_t* out;          // forward: Y (M x N); backward: dX (M x K)
+    int M;                  // tokens
+    int rows;               // output rows of the product: N forward, K backward
+    int ctr;                // contraction over the weight: K forward, N backward
+    int N, K, r;
+    int kb_w;               // weight stages: ceil(ctr / 64)
+    int kb_total;           // + LoRA slabs
+    int num_t;              // token tiles
+    int num_tiles;          // tiles (pair units)
+    float q[16];
+};
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+struct Pipe {
+    uint8_t* smem;      // stage s at smem + s * kStageBytes: A (16 KiB), then B halves of the two accumulators
+    uint32_t bar0;      // full_b[S], full_a[S], empty[S], acc_full, acc_empty, drain (this CTA)
+    uint32_t tmem;
+    uint32_t rank;      // 0: the even CTA (issues the MMAs), 1: its peer
+    int pair, num_pairs;
+    __device__ uint32_t full_b(int s) const { return bar0 + 8u * s; }
+    __device__ uint32_t full_a(int s) const { return bar0 + 8u * (kStages + s); }
+    __device__ uint32_t empty(int s) const { return bar0 + 8u * (2 * kStages + s); }
+    __device__ uint32_t acc_full() const { return bar0 + 8u * (3 * kStages); }
+    __device__ uint32_t acc_empty() const { return bar0 + 8u * (3 * kStages + 1); }
+    __device__ uint32_t drain() const { return bar0 + 8u * (3 * kStages + 2); }
+    __device__ uint32_t sA(int s) const { return smem_u32(smem + s * kStageBytes); }
+    __device__ uint32_t sB(int s, int sub) const { return sA(s) + kABytes + sub * kBHalfBytes; }
+};
+
+// Use count of ring slot kb % kStages before stage kb of this pair's tile
+// number tcount: its parity is the phase every role waits on.
+__device__ __forceinline__ uint32_t slot_use(int kb, uint32_t tcount, int kb_total) {
+    const int s = kb % kStages;
+    const uint32_t uses_per_tile = static_cast<uint32_t>((kb_total - s + kStages - 1) / kStages);
+    return tcount * uses_per_tile + static_cast<uint32_t>(kb / kStages);
+}
+
+// First token and first weight row (of the pair) of tile `tile`.  The
+// forward walks the token tiles fastest (X is shared by every weight tile
+// and stays in L2); the backward walks the weight tiles fastest, so the
+// pairs working at the same time share a few token tiles of dY.
+template <bool kBwd>
+__device__ __forceinline__ void tile_coords(const PairParams& p, int tile, int& t0, int& row0) {
+    if (kBwd) {
+        const int num_w = p.num_tiles / p.num_t;
+        t0 = (tile / num_w) * kTileTok;
+        row0 = (tile % num_w) * kRowsPair;
+    } else {
+        t0 = (tile % p.num_t) * kTileTok;
+        row0 = (tile / p.num_t) * kRowsPair;
+    }
+}
+
+// warp 0, one thread, both CTAs: the activation halves of every stage (and
+// the LoRA slabs' A operand) into this CTA's ring; the even CTA also arms
+// the stage's completion byte count for the pair.
+template <bool kBwd>
+__device__ void role_tma(const Pipe& P, const PairParams& p, const CUtensorMap* tm_act, const CUtensorMap* tm_lact,
+                         const CUtensorMap* tm_lw, int* err) {
+    uint32_t tcount = 0;
+    for (int tile = P.pair; tile < p.num_tiles; tile += P.num_pairs, ++tcount) {
+        int t0, row0;
+        tile_coords<kBwd>(p, tile, t0, row0);
+        const int my_row0 = row0 + static_cast<int>(P.rank) * kRowsCta;
+        for (int kb = 0; kb < p.kb_total; ++kb) {
+            const int s = kb % kStages;
+            const uint32_t ph = slot_use(kb, tcount, p.kb_total) & 1u;
+            if (!mbar_wait(P.empty(s), ph ^ 1u, err)) return;
+            const uint32_t bar = cluster_map(P.full_b(s), 0);
+            const bool lora = kb >= p.kb_w;
+            if (P.rank == 0) mbar_arrive_expect_tx(P.full_b(s), lora ? kTxLora : kTxWeight);
+            const CUtensorMap* act = lora ? tm_lact : tm_act;
+            const int x = lora ? (kb - p.kb_w) * kBK : kb * kBK;
+            for (int sub = 0; sub < kSubs; ++sub)
+                tma_load_2d_pair(P.sB(s, sub), act, bar, x, t0 + sub * kSubTok + static_cast<int>(P.rank) * kHalfTok);
+            if (lora) {
+                const int j0 = (kb - p.kb_w) * kBK;
+                if (kBwd) {  // A^T rows k (MN-major): two 64-wide k blocks of A[j0 .. j0+63][k]
+                    tma_load_2d_pair(P.sA(s), tm_lw, bar, my_row0, j0);
+                    tma_load_2d_pair(P.sA(s) + 8192, tm_lw, bar, my_row0 + 64, j0);
+                } else {     // B rows n (K-major): B[n][j0 .. j0+63]
+                    tma_load_2d_pair(P.sA(s), tm_lw, bar, j0, my_row0);
+                }
+            }
+        }
+    }
+}
+
+// warp 1, one thread of the even CTA: per stage, for each 16-wide
+// contraction step, one pair MMA into each accumulator in turn.
+template <bool kBwd>
+__device__ void role_mma(const Pipe& P, const PairParams& p, int* err) {
+    constexpr uint32_t idesc = idesc_bf16(kRowsPair, kSubTok, kBwd ? 1 : 0, 0);
+    uint32_t tcount = 0;
+    for (int tile = P.pair; tile < p.num_tiles; tile += P.num_pairs, ++tcount) {
+        if (!mbar_wait_cluster(P.acc_empty(), (tcount & 1u) ^ 1u, err)) return;
+        tc_fence_after();
+        for (int kb = 0; kb < p.kb_total; ++kb) {
+            const int s = kb % kStages;
+            const uint32_t ph = slot_use(kb, tcount, p.kb_total) & 1u;
+            if (!mbar_wait_cluster(P.full_b(s), ph, err)) return;
+            if (!mbar_wait_cluster(P.full_a(s), ph, err)) return;
+            tc_fence_after();
+            const uint32_t sa = P.sA(s);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+                // 16 contraction steps: +32 bytes along a K-major row, +16 rows of 128 bytes MN-major
+                const uint64_t ad = kBwd ? sdesc_mnmajor_sw128(sa + kk * 2048, 8192)
+                                         : sdesc_kmajor_sw128(sa) + static_cast<uint64_t>(kk * 2);
+#pragma unroll
+                for (int sub = 0; sub < kSubs; ++sub) {
+                    const uint64_t bd = sdesc_kmajor_sw128(P.sB(s, sub)) + static_cast<uint64_t>(kk * 2);
+                    mma_bf16_ss_pair(P.tmem + sub * kSubTok, ad, bd, idesc, (kb | kk) != 0);
+                }
+            }
+            tc_commit_pair_mc(P.empty(s), kPairMask);
+        }
+        tc_commit_pair_mc(P.acc_full(), kPairMask);
+    }
+}
+
+// Lane 0 of the calling warp waits; the result is broadcast so the warp
+// proceeds (or gives up) together.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* err, int lane) {
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(bar, parity, err) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+// The two codebook values (q[high nibble], q[low nibble]) of one code byte
+// from the lane's own copy of the 256-entry table: entry b, lane l at byte
+// 256 b + 8 l; the byte and the lane offset form the address in one permute.
+__device__ __forceinline__ float2 lut_pair(const uint8_t* lut, uint32_t word, uint32_t lane_off, int byte) {
+    const uint32_t addr = __byte_perm(word, lane_off, 0x5504u | (static_cast<uint32_t>(byte) << 4));
+    return *reinterpret_cast<const float2*>(lut + addr);
+}
+
+// One 64-weight run (32 code bytes, element 2t in the high nibble of byte
+// t) times its block constant, as 32 bf16 pairs (the even element in the
+// low half, i.e. at the lower address).
+__device__ __forceinline__ void convert_run(const uint4& c0, const uint4& c1, float sc, const uint8_t* lut,
+                                            uint32_t lane_off, uint32_t (&v)[32]) {
+    const uint32_t w8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 q2 = lut_pair(lut, w8[h], lane_off, j);
+            v[4 * h + j] = pack_bf16x2(__fmul_rn(q2.x, sc), __fmul_rn(q2.y, sc));
+        }
+    }
+}
+
+// Writes one 128-byte row (64 bf16) of an operand tile in the 128-byte
+// swizzled layout: 16-byte chunk c of row `row` goes to chunk c ^ (row & 7).
+__device__ __forceinline__ void store_swizzled_row(uint8_t* row_base, int row, const uint32_t (&v)[32]) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(row_base + ((c ^ (row & 7)) << 4)) =
+            make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+}
+
+// A position in one part's sequence of stages over all of this pair's
+// tiles: the stages kb == part (mod 3) of tile 0, then of tile 1, ...
+struct Cursor {
+    int tile;
+    uint32_t tcount;
+    int kb;
+    int t0, row0;
+};
+
+template <bool kBwd>
+__device__ __forceinline__ void cursor_start(Cursor& c, const Pipe& P, const PairParams& p, int part) {
+    c.tile = P.pair;
+    c.tcount = 0;
+    c.kb = part;
+    if (c.tile < p.num_tiles) tile_coords<kBwd>(p, c.tile, c.t0, c.row0);
+}
+
+template <bool kBwd>
+__device__ __forceinline__ void cursor_next(Cursor& c, const Pipe& P, const PairParams& p, int part) {
+    c.kb += kParts;
+    if (c.kb >= p.kb_total) {
+        c.kb = part;
+        c.tile += P.num_pairs;
+        ++c.tcount;
+        if (c.tile < p.num_tiles) tile_coords<kBwd>(p, c.tile, c.t0, c.row0);
+    }
+}
+
+// The 64-weight run that lane task `t` (0..127) of a weight stage converts:
+// its weight row n and first column kcol in W (valid = inside W), and where
+// it goes in this CTA's A tile (row `arow` of 128 bytes at byte offset
+// `aoff`).  Forward: task t is weight row row0 + t, columns 64 kb ...
+// Backward: task t is contraction index n = 64 kb + (t & 63) and the k block
+// (t >> 6) of this CTA's 128 output rows.
+template <bool kBwd>
+__device__ __forceinline__ bool task_of(const PairParams& p, int kb, int my_row0, int t, int64_t& n, int64_t& kcol,
+                                        int& arow, int& aoff) {
+    if (kBwd) {
+        const int i = t & 63, b = t >> 6;
+        n = static_cast<int64_t>(kb) * kBK + i;
+        kcol = my_row0 + 64 * b;
+        arow = i;
+        aoff = b * 8192 + i * 128;
+    } else {
+        n = my_row0 + t;
+        kcol = static_cast<int64_t>(kb) * kBK;
+        arow = t;
+        aoff = t * 128;
+    }
+    return n < p.N && kcol < p.K;
+}
+
+// Epilogue of this pair's tile number tcount: this warp's TMEM lane quarter
+// (this CTA's weight rows my_row0 + 32 quarter ...), the 16-column chunks
+// part, part + 3, ...; the accumulators are released (on the even CTA's
+// barrier) after the warp's last load.
+__device__ __forceinline__ void tile_epilogue(const Pipe& P, const PairParams& p, uint32_t tcount, int t0,
+                                              int my_row0, int part, int quarter, int lane, int* err, bool& ok) {
+    if (!warp_wait(P.acc_full(), tcount & 1u, err, lane)) {
+        ok = false;
+        return;
+    }
+    tc_fence_after();
+    const int grow = my_row0 + quarter * 32 + lane;
+    const bool lane_ok = grow < p.rows;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+#pragma unroll 1
+    for (int c = part; c < kChunks; c += kParts) {
+        const int col = c * 16;  // accumulator c / 16, its columns 16 (c % 16) ..: tokens t0 + col ..
+        uint32_t acc[16];
+        tmem_ld_32x32b_x16(P.tmem + lane_base + col, acc);
+        tmem_wait_ld();
+        if (c + kParts >= kChunks) {  // this warp's last chunk
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(cluster_map(P.acc_empty(), 0));
+        }
+        if (lane_ok) {
+            uint16_t* o = p.out + static_cast<int64_t>(t0 + col) * p.rows + grow;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (t0 + col + j < p.M) o[static_cast<int64_t>(j) * p.rows] = f32_to_bf16_bits(__uint_as_float(acc[j]));
+        }
+    }
+}
+
+// warps 2..13 of both CTAs: each converts every third stage's weight runs
+// (32 of the stage's 128) into this CTA's A tile and then arrives on the
+// even CTA's full_a barrier; for LoRA slabs (loaded by TMA) it only
+// arrives.  After storing its first stage of the next tile it writes its
+// share of the previous tile's outputs.
+template <bool kBwd>
+__device__ __forceinline__ void role_convert(const Pipe& P, const PairParams& p, const uint8_t* lut, int warp,
+                                             int lane, int* err) {
+    const uint32_t lane_off = static_cast<uint32_t>(lane) * 8;
+    const int quarter = warp & 3;
+    const int part = (warp - 2) >> 2;
+    const int t = quarter * 32 + lane;  // this lane's run within a stage
+    const float mu = *p.mean;
+    const uint32_t full_a_leader0 = cluster_map(P.full_a(0), 0);
+    bool ok = true;
+
+    if (part >= p.kb_total) {  // no stages for this part: epilogues only
+        uint32_t tcount = 0;
+        for (int tile = P.pair; tile < p.num_tiles && ok; tile += P.num_pairs, ++tcount) {
+            int t0, row0;
+            tile_coords<kBwd>(p, tile, t0, row0);
+            tile_epilogue(P, p, tcount, t0, row0 + static_cast<int>(P.rank) * kRowsCta, part, quarter, lane, err, ok);
+        }
+        return;
+    }
+
+    uint4 cb0[kPrefetch], cb1[kPrefetch];
+    uint32_t sbyte[kPrefetch];
+    float sc1[kPrefetch];
+    auto issue = [&](const Cursor& c, int u) {
+        cb0[u] = make_uint4(0u, 0u, 0u, 0u);
+        cb1[u] = cb0[u];
+        sbyte[u] = 0u;
+        sc1[u] = 0.0f;
+        if (c.tile >= p.num_tiles || c.kb >= p.kb_w) return;
+        int64_t n, kcol;
+        int arow, aoff;
+        if (!task_of<kBwd>(p, c.kb, c.row0 + static_cast<int>(P.rank) * kRowsCta, t, n, kcol, arow, aoff)) return;
+        const uint8_t* src = p.codes + n * (p.K / 2) + kcol / 2;
+        cb0[u] = ldg_nc_v4(src);
+        cb1[u] = ldg_nc_v4(src + 16);
+        const int64_t blk = n * (p.K / kBK) + kcol / kBK;
+        sbyte[u] = __ldg(p.c2_fp8 + blk);
+        sc1[u] = __ldg(p.c1 + (blk >> 8));
+    };
+
+    Cursor ci, cc;  // the next stage to load, the next stage to convert
+    cursor_start<kBwd>(ci, P, p, part);
+    cursor_start<kBwd>(cc, P, p, part);
+#pragma unroll
+    for (int u = 0; u < kPrefetch; ++u) {
+        issue(ci, u);
+        cursor_next<kBwd>(ci, P, p, part);
+    }
+    int prev_t0 = 0, prev_row0 = 0;  // the tile whose epilogue is pending
+    while (cc.tile < p.num_tiles) {
+#pragma unroll
+        for (int u = 0; u < kPrefetch; ++u) {
+            if (cc.tile >= p.num_tiles) break;
+            const int kb = cc.kb;
+            const int s = part;  // == kb % kStages
+            const uint32_t ph = slot_use(kb, cc.tcount, p.kb_total) & 1u;
+            const int my_row0 = cc.row0 + static_cast<int>(P.rank) * kRowsCta;
+            uint32_t v[32];
+            int64_t n = 0, kcol = 0;
+            int arow = 0, aoff = 0;
+            const bool weight = kb < p.kb_w;
+            if (weight) {
+                const bool valid = task_of<kBwd>(p, kb, my_row0, t, n, kcol, arow, aoff);
+                // runs outside W are zero (in the backward they are part of the contraction)
+                const float sc = valid ? dq_constant(static_cast<uint8_t>(sbyte[u]), sc1[u], mu) : 0.0f;
+                convert_run(cb0[u], cb1[u], sc, lut, lane_off, v);
+            }
+            issue(ci, u);
+            cursor_next<kBwd>(ci, P, p, part);
+            if (!warp_wait(P.empty(s), ph ^ 1u, err, lane)) return;
+            if (weight) {
+                store_swizzled_row(P.smem + s * kStageBytes + aoff, arow, v);
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(full_a_leader0 + 8u * s);
+            if (kb == part && cc.tcount > 0) {  // first own stage of a tile: end the previous one
+                tile_epilogue(P, p, cc.tcount - 1, prev_t0, prev_row0 + static_cast<int>(P.rank) * kRowsCta, part,
+                              quarter, lane, err, ok);
+                if (!ok) return;
+            }
+            prev_t0 = cc.t0;
+            prev_row0 = cc.row0;
+            cursor_next<kBwd>(cc, P, p, part);
+        }
+    }
+    // the pair's last tile
+    tile_epilogue(P, p, cc.tcount - 1, prev_t0, prev_row0 + static_cast<int>(P.rank) * kRowsCta, part, quarter, lane,
+                  err, ok);
+}
+
+template <bool kBwd>
+__global__ void __launch_bounds__(kThreads, 1)
+k_nf4_gemm_pair(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_lact,
+                const __grid_constant__ CUtensorMap tm_lw, const __grid_constant__ PairParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte aligned base (the swizzle atoms), by pointer arithmetic so
+    // every access below stays a 32-bit shared-memory access; the offset is
+    // the same in both CTAs of the pair
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 3);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    Pipe P;
+    P.smem = smem;
+    P.bar0 = smem_u32(bars);
+    P.rank = cluster_ctarank();
+    P.pair = static_cast<int>(blockIdx.x >> 1);
+    P.num_pairs = static_cast<int>(gridDim.x >> 1);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(P.full_b(s), 1);          // the even CTA's expect_tx arrival (+ both CTAs' bytes)
+            mbar_init(P.full_a(s), 2 * 4);      // the part's four warps in each CTA
+            mbar_init(P.empty(s), 1);           // the pair MMA's commit
+        }
+        mbar_init(P.acc_full(), 1);
+        mbar_init(P.acc_empty(), 2 * kDqWarps);  // every converter warp of both CTAs
+        mbar_init(P.drain(), 1);
+        fence_barrier_init();
+    }
+    uint8_t* lut = smem + kLutOff;
+    for (int i = threadIdx.x; i < 256 * 32; i += kThreads)
+        reinterpret_cast<float2*>(lut)[i] = make_float2(p.q[i >> 9], p.q[(i >> 5) & 15]);
+    if (warp == 0) {
+        tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish_pair();
+    }
+    if (warp == 1 && lane == 0) {
+        tma_prefetch_desc(&tm_act);
+        tma_prefetch_desc(&tm_lact);
+        tma_prefetch_desc(&tm_lw);
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_arrive();  // both CTAs' barriers are initialised before any remote arrive
+    cluster_wait();
+    tc_fence_after();
+    P.tmem = *tmem_slot;
+    int* err = &g_pair_error;
+
+    if (warp == 0) {
+        if (lane == 0) role_tma<kBwd>(P, p, &tm_act, &tm_lact, &tm_lw, err);
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0 && P.rank == 0) {
+            role_mma<kBwd>(P, p, err);
+            // every pair MMA issued (also on an early exit) has completed
+            // before the tensor memory can be freed
+            tc_commit_pair_mc(P.drain(), 1);
+            mbar_wait(P.drain(), 0u, err);
+        }
+        __syncwarp();
+    } else {
+        role_convert<kBwd>(P, p, lut, warp, lane, err);
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_arrive();  // neither CTA frees its tensor memory or leaves while the pair may still use it
+    cluster_wait();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc_pair(P.tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host
+// Row-major bf16 matrix (outer x inner), 128-byte swizzled boxes of
+// box_inner (<= 64) x box_outer elements, zero fill outside.
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                   uint32_t box_outer) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Clusters of two kernels that can be resident at once, asked once per
+// context.
+template <bool kBwd>
+int max_pairs() {
+    static ContextMemo<int> memo;
+    uint64_t ctx = 0;
+    if (!current_context_id(&ctx)) return 0;
+    int n = 0;
+    memo.get(ctx, &n, [](int* v) {
+        cudaLaunchConfig_t cfg{};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * static_cast<unsigned>(num_sms()));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = kSmemBytes;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int c = 0;
+        if (cudaOccupancyMaxActiveClusters(&c, k_nf4_gemm_pair<kBwd>, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            c = 0;
+        }
+        *v = c;
+        return true;
+    });
+    return n;
+}
+
+template <bool kBwd>
+cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& ml, const CUtensorMap& mw, PairParams p,
+                        cudaStream_t st) {
+    static ContextMemo<int> attr_memo;
+    cudaError_t e = ensure_smem_limit(attr_memo, k_nf4_gemm_pair<kBwd>, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int maxp = max_pairs<kBwd>();
+    if (maxp <= 0) return cudaErrorNotSupported;
+    for (int i = 0; i < 16; ++i) p.q[i] = tables().q[i];
+    const int pairs = p.num_tiles < maxp ? p.num_tiles : maxp;
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * static_cast<unsigned>(pairs));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_nf4_gemm_pair<kBwd>, ma, ml, mw, p);
+    note_launches(1);
+    return e;
+}
+
+PairParams base_params(const Nf4Weight& w, int64_t M, int r, uint16_t* out, bool bwd) {
+    PairParams p{};
+    p.codes = w.codes;
+    p.c2_fp8 = w.c2_fp8;
+    p.c1 = w.c1;
+    p.mean = w.mean;
+    p.out = out;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(w.N);
+    p.K = static_cast<int>(w.K);
+    p.r = r;
+    p.rows = bwd ? p.K : p.N;
+    p.ctr = bwd ? p.N : p.K;
+    p.kb_w = static_cast<int>(ceil_div(p.ctr, kBK));
+    p.kb_total = p.kb_w + static_cast<int>(ceil_div(r, kBK));
+    p.num_t = static_cast<int>(ceil_div(M, kTileTok));
+    p.num_tiles = p.num_t * static_cast<int>(ceil_div(p.rows, kRowsPair));
+    return p;
+}
+
+}  // namespace
+
+bool pair_gemm_supported(int64_t M, const Nf4Weight& w, int r, bool bwd) {
+    // TMA row strides: X / dY / T / U / A / B rows a multiple of 16 bytes
+    return M >= 1 && M < (int64_t(1) << 31) && w.K >= kBK && w.K % kBK == 0 && w.N >= 1 &&
+           w.N < (int64_t(1) << 31) && w.K < (int64_t(1) << 31) && r >= 8 && r % 8 == 0 && r <= 256 &&
+           (!bwd || w.N % 8 == 0) && tensor_map_encoder() != nullptr;
+}
+
+cudaError_t launch_fwd_gemm_pair(const uint16_t* X, const Nf4Weight& w, const uint16_t* T, const uint16_t* B,
+                                 int64_t M, int r, uint16_t* Y, cudaStream_t st) {
+    PairParams p = base_params(w, M, r, Y, false);
+    CUtensorMap ma, ml, mw;
+    if (!make_map_bf16(&ma, X, static_cast<uint64_t>(w.K), static_cast<uint64_t>(M), kBK, kHalfTok) ||
+        !make_map_bf16(&ml, T, static_cast<uint64_t>(r), static_cast<uint64_t>(M), kBK, kHalfTok) ||
+        !make_map_bf16(&mw, B, static_cast<uint64_t>(r), static_cast<uint64_t>(w.N), kBK, kRowsCta))
+        return cudaErrorInvalidValue;
+    return launch_pair<false>(ma, ml, mw, p, st);
+}
+
+cudaError_t launch_bwd_dx_gemm_pair(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U, const uint16_t* A,
+                                    int64_t M, int r, uint16_t* dX, cudaStream_t st) {
+    PairParams p = base_params(w, M, r, dX, true);
+    CUtensorMap ma, ml, mw;
+    if (!make_map_bf16(&ma, dY, static_cast<uint64_t>(w.N), static_cast<uint64_t>(M), kBK, kHalfTok) ||
+        !make_map_bf16(&ml, U, static_cast<uint64_t>(r), static_cast<uint64_t>(M), kBK, kHalfTok) ||
+        !make_map_bf16(&mw, A, static_cast<uint64_t>(w.K), static_cast<uint64_t>(r), 64, kBK))
+        return cudaErrorInvalidValue;
+    return launch_pair<true>(ma, ml, mw, p, st);
+}
+
+int pair_device_error(int reset) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_pair_error, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (reset && v) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_pair_error, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    }
+    return v;
+}
+
+}  // namespace qlora

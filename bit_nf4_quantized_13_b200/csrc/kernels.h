@@ -76,6 +76,18 @@ size_t dx_tc_workspace(const Nf4Weight& w, int r);
 cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U, const uint16_t* A,
                                   int64_t M, int r, uint16_t* dX, void* ws, cudaStream_t stream);
 
+// gemm_pair_sm100.cu -- the same two GEMMs on pairs of SMs (cta_group::2,
+// 256 weight rows x 512 tokens per tile, the converted weight staged in
+// shared memory); no workspace: the backward reads the row-major codes.
+// Returns cudaErrorNotSupported (nothing launched) when no pair of CTAs
+// fits the device.
+bool pair_gemm_supported(int64_t M, const Nf4Weight& w, int r, bool bwd);
+cudaError_t launch_fwd_gemm_pair(const uint16_t* X, const Nf4Weight& w, const uint16_t* T, const uint16_t* B,
+                                 int64_t M, int r, uint16_t* Y, cudaStream_t stream);
+cudaError_t launch_bwd_dx_gemm_pair(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U, const uint16_t* A,
+                                    int64_t M, int r, uint16_t* dX, cudaStream_t stream);
+int pair_device_error(int reset);
+
 // gemv_sm100.cu -- the small-batch forward (1 <= M <= 16): T and Y in one
 // kernel that streams the weight once; T is written to T_save when it is not
 // null.  Returns cudaErrorNotSupported (nothing launched) when no cluster
