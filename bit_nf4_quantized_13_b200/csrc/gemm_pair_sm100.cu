@@ -31,10 +31,10 @@
 // forward, A^T backward) and B operand (T forward, U backward) both come
 // by TMA.
 //
-// Codes are expanded through a 64 KiB table mapping a code byte to both of
-// its fp32 codebook values (one 8-byte copy per lane: no bank conflicts);
-// two weights cost one byte permute, one shared load, two multiplies by the
-// block constant (exactly RN(q * c2')) and one pack to bf16x2.
+// Codes are expanded without a table in memory: each 64-weight run forms
+// its block's 16 possible bf16 values in registers and picks four weights
+// at a time with byte permutes (convert_run), so the conversion adds no
+// shared-memory traffic beside the converted tile itself.
 //
 // Warp roles (448 threads per CTA, persistent over the pair's tiles):
 //   warp 0      TMA producer (both CTAs, into their own shared memory; the
@@ -78,12 +78,10 @@ constexpr int kParts = kDqWarps / 4;
 static_assert(kParts == kStages, "a part's stages must always use the same ring slot");
 constexpr int kPrefetch = 2;                        // own stages of codes in flight per converter lane
 constexpr int kThreads = 32 * (2 + kDqWarps);       // 448: 128 registers a thread
-constexpr int kLutBytes = 256 * 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kChunks = kSubs * kSubTok / 16;       // epilogue chunks of 16 columns
 constexpr int kBarOff = kStages * kStageBytes;
-constexpr int kLutOff = kBarOff + 1024;
-constexpr int kSmemBytes = 1024 /* alignment slack */ + kLutOff + kLutBytes;
+constexpr int kSmemBytes = 1024 /* alignment slack */ + kBarOff + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 constexpr uint16_t kPairMask = 0x3;                 // both CTAs of the cluster
 // completion bytes of one stage over the pair: B halves of both CTAs, plus
@@ -198,13 +196,13 @@ __device__ void role_mma(const Pipe& P, const PairParams& p, int* err) {
     constexpr uint32_t idesc = idesc_bf16(kRowsPair, kSubTok, kBwd ? 1 : 0, 0);
     uint32_t tcount = 0;
     for (int tile = P.pair; tile < p.num_tiles; tile += P.num_pairs, ++tcount) {
-        if (!mbar_wait_cluster(P.acc_empty(), (tcount & 1u) ^ 1u, err)) return;
+        if (!mbar_wait(P.acc_empty(), (tcount & 1u) ^ 1u, err)) return;
         tc_fence_after();
         for (int kb = 0; kb < p.kb_total; ++kb) {
             const int s = kb % kStages;
             const uint32_t ph = slot_use(kb, tcount, p.kb_total) & 1u;
-            if (!mbar_wait_cluster(P.full_b(s), ph, err)) return;
-            if (!mbar_wait_cluster(P.full_a(s), ph, err)) return;
+            if (!mbar_wait(P.full_b(s), ph, err)) return;
+            if (!mbar_wait(P.full_a(s), ph, err)) return;
             tc_fence_after();
             const uint32_t sa = P.sA(s);
 #pragma unroll
@@ -234,37 +232,65 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* er
     return ok != 0;
 }
 
-// The two codebook values (q[high nibble], q[low nibble]) of one code byte
-// from the lane's own copy of the 256-entry table: entry b, lane l at byte
-// 256 b + 8 l; the byte and the lane offset form the address in one permute.
-__device__ __forceinline__ float2 lut_pair(const uint8_t* lut, uint32_t word, uint32_t lane_off, int byte) {
-    const uint32_t addr = __byte_perm(word, lane_off, 0x5504u | (static_cast<uint32_t>(byte) << 4));
-    return *reinterpret_cast<const float2*>(lut + addr);
-}
-
 // One 64-weight run (32 code bytes, element 2t in the high nibble of byte
 // t) times its block constant, as 32 bf16 pairs (the even element in the
-// low half, i.e. at the lower address).
-__device__ __forceinline__ void convert_run(const uint4& c0, const uint4& c1, float sc, const uint8_t* lut,
-                                            uint32_t lane_off, uint32_t (&v)[32]) {
+// low half, i.e. at the lower address), without any table in memory.
+//
+// The run's 16 possible values p_i = bf16(RN32(q_i * c2')) are formed once
+// (16 multiplies, 8 packs) and split into a low-byte plane L and a
+// high-byte plane H of 16 bytes each (4 registers each).  For four weights
+// (two code bytes w, nibbles n0..n3 from the least significant end, i.e.
+// weights 1, 0, 3, 2) one byte permute per plane and half of the table
+// picks byte (n_j & 7) for result byte j from entries 0-7 and another from
+// entries 8-15; bit 3 of each nibble, spread to a byte mask by a
+// sign-replicating permute, chooses between them; two more permutes
+// interleave the planes into the two bf16 pairs.  Every value is exactly
+// bf16(RN32(q[code] * c2')).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+__device__ __forceinline__ uint32_t lop_select(uint32_t a, uint32_t b, uint32_t m) {
+    return (a & ~m) | (b & m);  // one LOP3
+}
+
+__device__ __forceinline__ void convert_run(const uint4& c0, const uint4& c1, float sc, const float (&q)[16],
+                                            uint32_t (&v)[32]) {
+    uint32_t L[4], H[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t t0 = pack_bf16x2(__fmul_rn(q[4 * k], sc), __fmul_rn(q[4 * k + 1], sc));
+        const uint32_t t1 = pack_bf16x2(__fmul_rn(q[4 * k + 2], sc), __fmul_rn(q[4 * k + 3], sc));
+        L[k] = prmt(t0, t1, 0x6420u);  // low bytes of p_4k .. p_4k+3
+        H[k] = prmt(t0, t1, 0x7531u);  // high bytes
+    }
     const uint32_t w8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float2 q2 = lut_pair(lut, w8[h], lane_off, j);
-            v[4 * h + j] = pack_bf16x2(__fmul_rn(q2.x, sc), __fmul_rn(q2.y, sc));
+        for (int half = 0; half < 2; ++half) {
+            const uint32_t w = (w8[h] >> (16 * half)) & 0xffffu;  // code bytes 2 half, 2 half + 1
+            const uint32_t sel = w & 0x7777u;
+            const uint32_t m = prmt(w << 4, w, 0xD9C8u);        // byte j: 0xff iff bit 3 of nibble j
+            const uint32_t lo = lop_select(prmt(L[0], L[1], sel), prmt(L[2], L[3], sel), m);
+            const uint32_t hi = lop_select(prmt(H[0], H[1], sel), prmt(H[2], H[3], sel), m);
+            // lo/hi bytes hold weights (1, 0, 3, 2) of the four
+            v[4 * h + 2 * half] = prmt(lo, hi, 0x4051u);      // (w0, w1)
+            v[4 * h + 2 * half + 1] = prmt(lo, hi, 0x6273u);  // (w2, w3)
         }
     }
 }
 
 // Writes one 128-byte row (64 bf16) of an operand tile in the 128-byte
 // swizzled layout: 16-byte chunk c of row `row` goes to chunk c ^ (row & 7).
-__device__ __forceinline__ void store_swizzled_row(uint8_t* row_base, int row, const uint32_t (&v)[32]) {
+// `row_base` is a shared-memory address.
+__device__ __forceinline__ void store_swizzled_row(uint32_t row_base, int row, const uint32_t (&v)[32]) {
 #pragma unroll
     for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(row_base + ((c ^ (row & 7)) << 4)) =
-            make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_base + ((c ^ (row & 7)) << 4)),
+                     "r"(v[4 * c]), "r"(v[4 * c + 1]), "r"(v[4 * c + 2]), "r"(v[4 * c + 3])
+                     : "memory");
 }
 
 // A position in one part's sequence of stages over all of this pair's
@@ -342,7 +368,7 @@ __device__ __forceinline__ void tile_epilogue(const Pipe& P, const PairParams& p
         if (c + kParts >= kChunks) {  // this warp's last chunk
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(cluster_map(P.acc_empty(), 0));
+            if (lane == 0) mbar_arrive_remote(cluster_map(P.acc_empty(), 0));
         }
         if (lane_ok) {
             uint16_t* o = p.out + static_cast<int64_t>(t0 + col) * p.rows + grow;
@@ -359,9 +385,7 @@ __device__ __forceinline__ void tile_epilogue(const Pipe& P, const PairParams& p
 // arrives.  After storing its first stage of the next tile it writes its
 // share of the previous tile's outputs.
 template <bool kBwd>
-__device__ __forceinline__ void role_convert(const Pipe& P, const PairParams& p, const uint8_t* lut, int warp,
-                                             int lane, int* err) {
-    const uint32_t lane_off = static_cast<uint32_t>(lane) * 8;
+__device__ __forceinline__ void role_convert(const Pipe& P, const PairParams& p, int warp, int lane, int* err) {
     const int quarter = warp & 3;
     const int part = (warp - 2) >> 2;
     const int t = quarter * 32 + lane;  // this lane's run within a stage
@@ -424,17 +448,19 @@ __device__ __forceinline__ void role_convert(const Pipe& P, const PairParams& p,
                 const bool valid = task_of<kBwd>(p, kb, my_row0, t, n, kcol, arow, aoff);
                 // runs outside W are zero (in the backward they are part of the contraction)
                 const float sc = valid ? dq_constant(static_cast<uint8_t>(sbyte[u]), sc1[u], mu) : 0.0f;
-                convert_run(cb0[u], cb1[u], sc, lut, lane_off, v);
+                convert_run(cb0[u], cb1[u], sc, p.q, v);
             }
-            issue(ci, u);
-            cursor_next<kBwd>(ci, P, p, part);
             if (!warp_wait(P.empty(s), ph ^ 1u, err, lane)) return;
             if (weight) {
-                store_swizzled_row(P.smem + s * kStageBytes + aoff, arow, v);
+                store_swizzled_row(P.sA(s) + static_cast<uint32_t>(aoff), arow, v);
                 fence_proxy_async_smem();
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(full_a_leader0 + 8u * s);
+            if (lane == 0) mbar_arrive_remote(full_a_leader0 + 8u * s);
+            // the loads of a later stage go out after the hand-off, so that
+            // nothing above waits for them
+            issue(ci, u);
+            cursor_next<kBwd>(ci, P, p, part);
             if (kb == part && cc.tcount > 0) {  // first own stage of a tile: end the previous one
                 tile_epilogue(P, p, cc.tcount - 1, prev_t0, prev_row0 + static_cast<int>(P.rank) * kRowsCta, part,
                               quarter, lane, err, ok);
@@ -480,9 +506,6 @@ k_nf4_gemm_pair(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
         mbar_init(P.drain(), 1);
         fence_barrier_init();
     }
-    uint8_t* lut = smem + kLutOff;
-    for (int i = threadIdx.x; i < 256 * 32; i += kThreads)
-        reinterpret_cast<float2*>(lut)[i] = make_float2(p.q[i >> 9], p.q[(i >> 5) & 15]);
     if (warp == 0) {
         tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish_pair();
@@ -513,7 +536,7 @@ k_nf4_gemm_pair(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
         }
         __syncwarp();
     } else {
-        role_convert<kBwd>(P, p, lut, warp, lane, err);
+        role_convert<kBwd>(P, p, warp, lane, err);
     }
     tc_fence_before();
     __syncthreads();

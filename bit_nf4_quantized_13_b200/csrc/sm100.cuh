@@ -355,6 +355,13 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
+// Arrives on an mbarrier of another CTA of the cluster (`addr` from
+// cluster_map) with the default release semantics at CTA scope: what this
+// thread wrote before (and, after a proxy fence, made visible to the async
+// proxy) is ordered before the arrival, without a cluster-wide fence.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
 // Asynchronous 16-byte store into the shared memory of a CTA of the cluster;
 // completes (complete_tx, 16 bytes) on that CTA's mbarrier `bar` (both
 // addresses from cluster_map).
