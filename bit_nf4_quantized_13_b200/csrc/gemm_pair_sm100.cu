@@ -36,12 +36,12 @@
 // at a time with byte permutes (convert_run), so the conversion adds no
 // shared-memory traffic beside the converted tile itself.
 //
-// Warp roles (448 threads per CTA, persistent over the pair's tiles):
+// Warp roles (576 threads per CTA, persistent over the pair's tiles):
 //   warp 0      TMA producer (both CTAs, into their own shared memory; the
 //               completion bytes count on the even CTA's barrier)
 //   warp 1      MMA issuer (one thread of the even CTA only)
-//   warps 2-13  converters: warp w handles the stages kb with kb % 3 ==
-//               (w - 2) / 4 (always ring slot kb % 3), 32 of the stage's 128
+//   warps 2-17  converters: warp w handles the stages kb with kb % 4 ==
+//               (w - 2) / 4 (always ring slot kb % 4), 32 of the stage's 128
 //               64-weight runs; then the epilogue of its TMEM lane quarter
 //               w % 4: tcgen05.ld, bf16, stores coalesced along the
 //               weight-row index.
@@ -69,15 +69,15 @@ constexpr int kSubs = 2;                            // accumulators
 constexpr int kTileTok = kSubs * kSubTok;           // tokens per tile
 constexpr int kHalfTok = kSubTok / 2;               // one accumulator's tokens staged by one CTA
 constexpr int kBK = 64;                             // contraction per stage
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kABytes = kRowsCta * kBK * 2;         // 16 KiB
 constexpr int kBHalfBytes = kHalfTok * kBK * 2;     // 16 KiB
 constexpr int kStageBytes = kABytes + kSubs * kBHalfBytes;
-constexpr int kDqWarps = 12;
+constexpr int kDqWarps = 16;
 constexpr int kParts = kDqWarps / 4;
 static_assert(kParts == kStages, "a part's stages must always use the same ring slot");
-constexpr int kPrefetch = 2;                        // own stages of codes in flight per converter lane
-constexpr int kThreads = 32 * (2 + kDqWarps);       // 448: 128 registers a thread
+constexpr int kPrefetch = 1;                        // own stages of codes in flight per converter lane
+constexpr int kThreads = 32 * (2 + kDqWarps);       // 576: 112 registers a thread
 constexpr uint32_t kTmemCols = 512;
 constexpr int kChunks = kSubs * kSubTok / 16;       // epilogue chunks of 16 columns
 constexpr int kBarOff = kStages * kStageBytes;
@@ -139,18 +139,26 @@ __device__ __forceinline__ uint32_t slot_use(int kb, uint32_t tcount, int kb_tot
 }
 
 // First token and first weight row (of the pair) of tile `tile`.  The
-// forward walks the token tiles fastest (X is shared by every weight tile
-// and stays in L2); the backward walks the weight tiles fastest, so the
-// pairs working at the same time share a few token tiles of dY.
+// forward takes the weight rows in bands of kBand row tiles and, inside a
+// band, the token tiles slowest: the pairs working at the same time then
+// cover a compact block of a few token tiles of X and a few weight row
+// tiles, which stays in L2 even when X does not.  The backward walks the
+// weight tiles fastest, so the pairs working at the same time share a few
+// token tiles of dY while the weight's codes are reused from L2.
+constexpr int kBand = 8;
+
 template <bool kBwd>
 __device__ __forceinline__ void tile_coords(const PairParams& p, int tile, int& t0, int& row0) {
+    const int num_w = p.num_tiles / p.num_t;
     if (kBwd) {
-        const int num_w = p.num_tiles / p.num_t;
         t0 = (tile / num_w) * kTileTok;
         row0 = (tile % num_w) * kRowsPair;
     } else {
-        t0 = (tile % p.num_t) * kTileTok;
-        row0 = (tile / p.num_t) * kRowsPair;
+        const int band_tiles = kBand * p.num_t;  // tiles in a full band
+        const int band = tile / band_tiles, in = tile % band_tiles;
+        const int rows_in_band = min(kBand, num_w - band * kBand);
+        t0 = (in / rows_in_band) * kTileTok;
+        row0 = (band * kBand + in % rows_in_band) * kRowsPair;
     }
 }
 
