@@ -39,10 +39,9 @@ WORKLOAD = "llama7b_linears_w4096x4096_w11008x4096_m4096_r64_alpha16_quantize_fw
 M_TOKENS, RANK, ALPHA = 4096, 64, 16.0
 L2_FLUSH_BYTES = 256 << 20
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) per call of the dX path (k_prep_bwd + k_nf4_gemm_tc<1>), mean over
-# the two linears (57.5 MB and 217.4 MB), from one ncu capture of the kernels as they are now
-# (profiles/k_nf4_gemm_tc_llama7b_m4096.md); None when the kernels have changed since then.
-DX_TRAFFIC_BYTES = 137.45e6
+# DRAM bytes (read + write) per call of the dX GEMM, mean over the two linears, from one ncu
+# capture of the kernel as it is now (profiles/); None when the kernel has changed since then.
+DX_TRAFFIC_BYTES = None
 
 
 def linear_flops(M, N, K, r):
@@ -450,9 +449,9 @@ def run_native(args, world, rank, local):
                 dq32_bytes += dequant_bytes(n, 4)
     del w32buf
 
-    # the dominant kernel: the backward's dX path (the transposed-weight prep
-    # and the NF4 GEMM dX = dY W' + U A), timed live as the backward with dX
-    # minus the backward without it, per call, L2 flushed before each
+    # the dominant kernel: the backward's dX GEMM (dX = dY W' + U A), timed
+    # live as the backward with dX minus the backward without it, per call,
+    # L2 flushed before each
     dx_ms, dx_flops, dx_reps = 0.0, 0.0, max(5, args.steps // 4)
     for rep in range(dx_reps + 2):
         for b in bufs:
@@ -505,7 +504,7 @@ def run_native(args, world, rank, local):
             v["frac_hbm"] = v["gbs"] / peaks["hbm_gbs"]
             v["graph_frac_hbm"] = v["graph_gbs"] / peaks["hbm_gbs"]
     dx_tflops = dx_flops / (dx_ms * 1e-3) / 1e12
-    roofline = {"kernel": "k_nf4_gemm_tc<1> with k_prep_bwd: dX = dY W'^T' + U A of qlora_linear_bwd "
+    roofline = {"kernel": "k_nf4_gemm_pair<1>: dX = dY W' + U A of qlora_linear_bwd "
                           "(largest share of the step in the ncu launch list)",
                 "bound": "tensor", "achieved": dx_tflops, "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": dx_tflops / tc_peak, "traffic": DX_TRAFFIC_BYTES, "peak_source": peak_src,

@@ -29,22 +29,22 @@ int num_sms() {
 }
 
 cudaError_t launch_fwd_gemm(const uint16_t* X, const Nf4Weight& w, const uint16_t* T,
-                            const uint16_t* B, int64_t M, int r, uint16_t* Y, cudaStream_t st) {
+                            const uint16_t* B, int64_t M, int r, uint16_t* Y, void* ws, size_t ws_bytes,
+                            cudaStream_t st) {
     if (pair_gemm_supported(M, w, r, false)) {
-        const cudaError_t e = launch_fwd_gemm_pair(X, w, T, B, M, r, Y, st);
+        const cudaError_t e = launch_fwd_gemm_pair(X, w, T, B, M, r, Y, ws, ws_bytes, st);
         if (e != cudaErrorNotSupported) return e;
     }
-    if (fwd_tc_supported(M, w, r)) return launch_fwd_gemm_tc(X, w, T, B, M, r, Y, st);
     return launch_fwd_gemm_simt(X, w, T, B, M, r, Y, st);
 }
 
 cudaError_t launch_bwd_dx_gemm(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U,
-                               const uint16_t* A, int64_t M, int r, uint16_t* dX, void* ws, cudaStream_t st) {
+                               const uint16_t* A, int64_t M, int r, uint16_t* dX, void* ws, size_t ws_bytes,
+                               cudaStream_t st) {
     if (pair_gemm_supported(M, w, r, true)) {
-        const cudaError_t e = launch_bwd_dx_gemm_pair(dY, w, U, A, M, r, dX, st);
+        const cudaError_t e = launch_bwd_dx_gemm_pair(dY, w, U, A, M, r, dX, ws, ws_bytes, st);
         if (e != cudaErrorNotSupported) return e;
     }
-    if (dx_tc_supported(M, w, r)) return launch_bwd_dx_gemm_tc(dY, w, U, A, M, r, dX, ws, st);
     return launch_bwd_dx_gemm_simt(dY, w, U, A, M, r, dX, st);
 }
 
@@ -135,16 +135,15 @@ int qlora_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c
 
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
     if (check_linear(M, N, K, r) != QLORA_OK) return 0;
-    // T (used when T_save is NULL)
-    return align256(static_cast<size_t>(M) * r * 2);
+    // T (used when T_save is NULL), then the GEMM's split-tile scratch
+    return align256(static_cast<size_t>(M) * r * 2) + pair_gemm_workspace();
 }
 
 size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
     if (check_linear(M, N, K, r) != QLORA_OK) return 0;
     const size_t mr = align256(static_cast<size_t>(M) * r * 2);
-    // U, T (when T is NULL), the transposed weight of the dX GEMM
-    Nf4Weight w{nullptr, nullptr, nullptr, nullptr, N, K};
-    return 2 * mr + align256(dx_tc_workspace(w, r));
+    // U, T (when T is NULL), then the dX GEMM's split-tile scratch
+    return 2 * mr + pair_gemm_workspace();
 }
 
 int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
@@ -160,6 +159,9 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     if (!ws || !aligned16(ws) || ws_bytes < qlora_linear_fwd_workspace_size(M, N, K, r))
         return QLORA_ERR_WORKSPACE;
     uint16_t* T = T_save ? T_save : reinterpret_cast<uint16_t*>(ws);
+    const size_t t_bytes = align256(static_cast<size_t>(M) * r * 2);
+    void* gws = reinterpret_cast<char*>(ws) + t_bytes;
+    const size_t gws_bytes = ws_bytes - t_bytes;
     cudaStream_t cs = as_stream(stream);
     Nf4Weight w{codes, c2_fp8, c1, mean, N, K};
     if (gemv_supported(M, N, K, r)) {  // a few tokens: one stream over the weight
@@ -167,7 +169,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
         if (g != cudaErrorNotSupported) return cuda_status(g);  // else: no cluster shape fits
     }
     cudaError_t e = lora_xat(X, A, M, N, K, r, s, T, cs);
-    if (e == cudaSuccess) e = launch_fwd_gemm(X, w, T, B, M, r, Y, cs);
+    if (e == cudaSuccess) e = launch_fwd_gemm(X, w, T, B, M, r, Y, gws, gws_bytes, cs);
     return cuda_status(e);
 }
 
@@ -195,23 +197,23 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N
     uint16_t* Tw = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + mr);
     Nf4Weight w{codes, c2_fp8, c1, mean, N, K};
     void* dxws = reinterpret_cast<char*>(ws) + 2 * mr;
+    const size_t dxws_bytes = ws_bytes - 2 * mr;
     cudaError_t e = cudaSuccess;
     if (!T) {
         e = lora_xat(X, A, M, N, K, r, s, Tw, cs);
         T = Tw;
     }
     if (e == cudaSuccess) e = lora_dyb(dY, B, M, N, K, r, s, U, cs);
-    if (e == cudaSuccess && dX) e = launch_bwd_dx_gemm(dY, w, U, A, M, r, dX, dxws, cs);
+    if (e == cudaSuccess && dX) e = launch_bwd_dx_gemm(dY, w, U, A, M, r, dX, dxws, dxws_bytes, cs);
     if (e == cudaSuccess) e = lora_grads(dY, X, T, U, M, N, K, r, dA, dB, cs);
     return cuda_status(e);
 }
 
 int qlora_device_error(int reset) {
-    const int a = gemm_device_error(reset);
+    const int a = pair_device_error(reset);
     const int b = lora_device_error(reset);
     const int c = gemv_device_error(reset);
-    const int d = pair_device_error(reset);
-    return a != QLORA_OK ? a : b != QLORA_OK ? b : c != QLORA_OK ? c : d;
+    return a != QLORA_OK ? a : b != QLORA_OK ? b : c;
 }
 
 int qlora_debug_wait_timeout(uint64_t limit_ns, void* stream) {

@@ -45,8 +45,7 @@ cudaError_t launch_lora_da_tc(const uint16_t* X, const uint16_t* U, int64_t M, i
 cudaError_t launch_lora_db_tc(const uint16_t* dY, const uint16_t* T, int64_t M, int64_t N, int r, uint16_t* dB,
                               cudaStream_t stream);
 int lora_device_error(int reset);
-int gemm_device_error(int reset);  // gemm_nf4_sm100.cu
-// gemm_nf4_sm100.cu: a kernel whose one bounded wait is never satisfied
+// gemm_pair_sm100.cu: a kernel whose one bounded wait is never satisfied
 // (records QLORA_ERR_TIMEOUT after limit_ns)
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
 // gemm_simt.cu: CUDA-core versions (any shape)
@@ -65,27 +64,21 @@ cudaError_t launch_bwd_dx_gemm_simt(const uint16_t* dY, const Nf4Weight& w, cons
                                     const uint16_t* A, int64_t M, int r, uint16_t* dX,
                                     cudaStream_t stream);
 
-// gemm_nf4_sm100.cu -- tcgen05 forward and backward-dX (r % 8 == 0; the
-// backward also needs N % 8 == 0)
-bool fwd_tc_supported(int64_t M, const Nf4Weight& w, int r);
-bool dx_tc_supported(int64_t M, const Nf4Weight& w, int r);
-cudaError_t launch_fwd_gemm_tc(const uint16_t* X, const Nf4Weight& w, const uint16_t* T, const uint16_t* B,
-                               int64_t M, int r, uint16_t* Y, cudaStream_t stream);
-// The backward needs dx_tc_workspace bytes for the transposed weight copy.
-size_t dx_tc_workspace(const Nf4Weight& w, int r);
-cudaError_t launch_bwd_dx_gemm_tc(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U, const uint16_t* A,
-                                  int64_t M, int r, uint16_t* dX, void* ws, cudaStream_t stream);
-
-// gemm_pair_sm100.cu -- the same two GEMMs on pairs of SMs (cta_group::2,
-// 256 weight rows x 512 tokens per tile, the converted weight staged in
-// shared memory); no workspace: the backward reads the row-major codes.
-// Returns cudaErrorNotSupported (nothing launched) when no pair of CTAs
-// fits the device.
+// gemm_pair_sm100.cu -- the frozen-weight GEMMs on the tensor cores, on
+// pairs of SMs (cta_group::2, 256 weight rows x 512 tokens per tile, the
+// converted weight staged in shared memory; the backward reads the
+// row-major codes).  The tiles' contraction stages are shared out evenly
+// over the pairs; a tile split between pairs is finished through the
+// workspace (pair_gemm_workspace bytes, 256-byte aligned).  Returns
+// cudaErrorNotSupported (nothing launched) when no pair of CTAs fits the
+// device.
 bool pair_gemm_supported(int64_t M, const Nf4Weight& w, int r, bool bwd);
+size_t pair_gemm_workspace();
 cudaError_t launch_fwd_gemm_pair(const uint16_t* X, const Nf4Weight& w, const uint16_t* T, const uint16_t* B,
-                                 int64_t M, int r, uint16_t* Y, cudaStream_t stream);
+                                 int64_t M, int r, uint16_t* Y, void* ws, size_t ws_bytes, cudaStream_t stream);
 cudaError_t launch_bwd_dx_gemm_pair(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U, const uint16_t* A,
-                                    int64_t M, int r, uint16_t* dX, cudaStream_t stream);
+                                    int64_t M, int r, uint16_t* dX, void* ws, size_t ws_bytes,
+                                    cudaStream_t stream);
 int pair_device_error(int reset);
 
 // gemv_sm100.cu -- the small-batch forward (1 <= M <= 16): T and Y in one
@@ -97,13 +90,15 @@ cudaError_t launch_fwd_gemv(const uint16_t* X, const Nf4Weight& w, const uint16_
                             int r, float s, uint16_t* Y, uint16_t* T_save, cudaStream_t stream);
 int gemv_device_error(int reset);
 
-// gemm_*.cu -- the frozen-weight GEMMs with the LoRA slab fused in
+// abi.cu -- the frozen-weight GEMMs with the LoRA slab fused in, on the
+// tensor cores where the shapes allow, else on the CUDA cores
 //   Y  = bf16(X W'^T + T B^T)      (M x N)
 //   dX = bf16(dY W' + U A)         (M x K)
 cudaError_t launch_fwd_gemm(const uint16_t* X, const Nf4Weight& w, const uint16_t* T,
-                            const uint16_t* B, int64_t M, int r, uint16_t* Y, cudaStream_t stream);
+                            const uint16_t* B, int64_t M, int r, uint16_t* Y, void* ws, size_t ws_bytes,
+                            cudaStream_t stream);
 cudaError_t launch_bwd_dx_gemm(const uint16_t* dY, const Nf4Weight& w, const uint16_t* U,
-                               const uint16_t* A, int64_t M, int r, uint16_t* dX, void* ws,
+                               const uint16_t* A, int64_t M, int r, uint16_t* dX, void* ws, size_t ws_bytes,
                                cudaStream_t stream);
 
 }  // namespace qlora
