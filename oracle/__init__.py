@@ -76,6 +76,8 @@ def lib():
                                             i64, vp, vp, vp]
             L.oracle_int8_quant.argtypes = [vp, i64, vp, vp]
             L.oracle_int8_dequant.argtypes = [vp, i64, flt, vp]
+            L.oracle_int8_quant_blocks.argtypes = [vp, i64, i64, vp, vp]
+            L.oracle_int8_dequant_blocks.argtypes = [vp, i64, i64, vp, vp]
             L.oracle_set_threads.argtypes = [i32]
             L.oracle_get_threads.restype = i32
             _lib = L
@@ -246,4 +248,23 @@ def int8_dequant(xq, c):
     xq = np.ascontiguousarray(xq, np.int8)
     out = np.zeros(xq.size, np.float32)
     lib().oracle_int8_dequant(_p(xq), xq.size, ctypes.c_float(c), _p(out))
+    return out
+
+
+def int8_quant_blocks(x, block: int = 64):
+    """Eq. (1) on consecutive blocks: (codes int8[n], c fp32[ceil(n/block)])."""
+    x = _f32(x).reshape(-1)
+    nb = (x.size + block - 1) // block
+    out = np.zeros(x.size, np.int8)
+    c = np.zeros(max(nb, 1), np.float32)
+    lib().oracle_int8_quant_blocks(_p(x), x.size, block, _p(out), _p(c))
+    return out, c[:nb]
+
+
+def int8_dequant_blocks(xq, c, block: int = 64):
+    """Eq. (2) on consecutive blocks."""
+    xq = np.ascontiguousarray(xq, np.int8).reshape(-1)
+    c = _f32(c)
+    out = np.zeros(xq.size, np.float32)
+    lib().oracle_int8_dequant_blocks(_p(xq), xq.size, block, _p(c), _p(out))
     return out

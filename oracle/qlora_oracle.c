@@ -638,11 +638,13 @@ int oracle_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t 
 }
 
 /* ------------------------------------------------------------------------ */
-/* Block-wise Int8 absmax quantization, [notes] 3.1 eq. 1 and eq. 2.  Not   */
-/* on the NF4 path; kept to anchor the pages' worked example.               */
+/* Block-wise Int8 absmax quantization, [notes] 3.1 eq. 1 and eq. 2 (the    */
+/* 8-bit baseline the NF4 type is compared with).                           */
 /*   c = 127 / absmax(X),  X_int8 = round(c X),  dequant = X_int8 / c       */
 /* round() is the pages' "round half away from zero" (C's round()).  The    */
-/* arithmetic is fp32 throughout.                                            */
+/* arithmetic is fp32 throughout.  A block whose absmax is 0 stores c = 0   */
+/* and codes 0 and dequantizes to 0 (eq. 2 would divide by 0; the pages do  */
+/* not treat that case).                                                     */
 /* ------------------------------------------------------------------------ */
 
 void oracle_int8_quant(const float* x, int64_t n, int8_t* out, float* c)
@@ -659,5 +661,23 @@ void oracle_int8_quant(const float* x, int64_t n, int8_t* out, float* c)
 
 void oracle_int8_dequant(const int8_t* xq, int64_t n, float c, float* out)
 {
-    for (int64_t i = 0; i < n; ++i) out[i] = (float)xq[i] / c;
+    for (int64_t i = 0; i < n; ++i) out[i] = c != 0.0f ? (float)xq[i] / c : 0.0f;
+}
+
+/* The same over consecutive blocks of `block` elements of a flattened    */
+/* tensor (the last block may be partial): one constant c per block.      */
+void oracle_int8_quant_blocks(const float* x, int64_t n, int64_t block, int8_t* out, float* c)
+{
+    for (int64_t b0 = 0, j = 0; b0 < n; b0 += block, ++j) {
+        int64_t len = n - b0 < block ? n - b0 : block;
+        oracle_int8_quant(x + b0, len, out + b0, c + j);
+    }
+}
+
+void oracle_int8_dequant_blocks(const int8_t* xq, int64_t n, int64_t block, const float* c, float* out)
+{
+    for (int64_t b0 = 0, j = 0; b0 < n; b0 += block, ++j) {
+        int64_t len = n - b0 < block ? n - b0 : block;
+        oracle_int8_dequant(xq + b0, len, c[j], out + b0);
+    }
 }

@@ -487,3 +487,40 @@ def test_int8_absmax_worked_example():
     assert codes.tolist() == [int(v) for v in g["codes"]]
     deq = oracle.int8_dequant(codes, c)
     np.testing.assert_allclose(deq, g["dequant"], rtol=0, atol=2e-6)
+
+
+def test_int8_blocks_follow_the_definition():
+    """Block-wise eq. (1)/(2): every block gets c = RN32(127 / absmax) and
+    codes round-half-away(RN32(c x)) -- checked against a numpy restatement
+    element by element; the absmax element maps to +-127; |codes| <= 127;
+    a zero block has c = 0, codes 0 and dequantizes to exact zeros; the
+    round trip is within half a step (absmax / 254) plus fp32 rounding."""
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal(64 * 37 + 13) * 0.02).astype(np.float32)
+    x[64 * 5:64 * 6] = 0.0                      # a zero block
+    x[64 * 9 + 3] = 0.5                          # an outlier
+    codes, c = oracle.int8_quant_blocks(x, 64)
+    nb = -(-x.size // 64)
+    assert c.size == nb
+    for j in range(nb):
+        blk = x[64 * j:64 * j + 64]
+        a = np.float32(np.max(np.abs(blk)))
+        if a == 0:
+            assert c[j] == 0 and not codes[64 * j:64 * j + 64].any()
+            continue
+        cj = np.float32(np.float32(127.0) / a)
+        assert c[j] == cj
+        t = (cj * blk).astype(np.float32)   # RN32(c x)
+        t64 = t.astype(np.float64)          # half away from zero, exactly, in fp64
+        ref = np.sign(t64) * np.floor(np.abs(t64) + 0.5)
+        np.testing.assert_array_equal(codes[64 * j:64 * j + blk.size].astype(np.float64), ref)
+        k = int(np.argmax(np.abs(blk)))
+        assert abs(int(codes[64 * j + k])) == 127
+    assert np.abs(codes.astype(np.int32)).max() <= 127
+    deq = oracle.int8_dequant_blocks(codes, c, 64)
+    assert not deq[64 * 5:64 * 6].any()
+    for j in range(nb):
+        blk = x[64 * j:64 * j + 64]
+        a = float(np.max(np.abs(blk)))
+        err = np.abs(deq[64 * j:64 * j + blk.size].astype(np.float64) - blk)
+        assert np.all(err <= a / 254 * (1 + 1e-5) + 1e-12)
