@@ -64,6 +64,8 @@ def _load() -> ctypes.CDLL:
         "qlora_device_error": (i32, [i32]),
         "qlora_quantize_nf4_dq_noalloc": (i32, [vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]),
         "qlora_debug_wait_timeout": (i32, [ctypes.c_uint64, vp]),
+        "qlora_int8_quantize": (i32, [vp, i64, i32, vp, vp, vp, vp]),
+        "qlora_int8_dequantize": (i32, [vp, vp, i64, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -338,6 +340,47 @@ def qlora_device_error(reset: bool = False) -> int:
     """Sticky error word of the tensor-core kernels (0 = none, 6 = a bounded
     in-kernel wait timed out)."""
     return int(_get_lib().qlora_device_error(1 if reset else 0))
+
+
+def qlora_int8_quantize(x, block: int = 64, codes=None, c=None, status=None, stream=None):
+    """Block-wise Int8 absmax quantization (eq. 1): returns (codes int8, c fp32)."""
+    torch = _torch()
+    _need_dtype(torch.float32, x=x)
+    n = x.numel()
+    nb = -(-n // block)
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    if c is None:
+        c = torch.empty(max(nb, 1), dtype=torch.float32, device=x.device)
+    _need_dtype(torch.int8, codes=codes)
+    _need_dtype(torch.float32, c=c)
+    if codes.numel() < n or c.numel() < nb:
+        raise ValueError("codes / c too small")
+    if status is not None:
+        _need_dtype(torch.int32, status=status)
+    _need_cuda(x, codes, c, status)
+    _check("qlora_int8_quantize", _get_lib().qlora_int8_quantize(_ptr(x), n, int(block), _ptr(codes), _ptr(c),
+                                                                 _ptr(status), _stream(stream)))
+    return codes, c
+
+
+def qlora_int8_dequantize(codes, c, block: int = 64, out=None, stream=None):
+    """Eq. (2): fp32 values from Int8 codes and the per-block constants."""
+    torch = _torch()
+    _need_dtype(torch.int8, codes=codes)
+    _need_dtype(torch.float32, c=c)
+    n = codes.numel()
+    if c.numel() < -(-n // block):
+        raise ValueError("c too small")
+    if out is None:
+        out = torch.empty(codes.shape, dtype=torch.float32, device=codes.device)
+    _need_dtype(torch.float32, out=out)
+    if out.numel() < n:
+        raise ValueError("out too small")
+    _need_cuda(codes, c, out)
+    _check("qlora_int8_dequantize", _get_lib().qlora_int8_dequantize(_ptr(codes), _ptr(c), n, int(block),
+                                                                     _ptr(out), _stream(stream)))
+    return out
 
 
 def qlora_debug_wait_timeout(limit_ns: int, stream=None) -> None:

@@ -216,6 +216,26 @@ int qlora_device_error(int reset) {
     return a != QLORA_OK ? a : b != QLORA_OK ? b : c;
 }
 
+int qlora_int8_quantize(const float* x, int64_t numel, int block, int8_t* codes, float* c, int32_t* status,
+                        void* stream) {
+    if (numel < 0) return QLORA_ERR_INVALID_ARG;
+    if (!int8_block_supported(block)) return QLORA_ERR_UNSUPPORTED;
+    if (numel >= kMaxNumel) return QLORA_ERR_UNSUPPORTED;
+    if (numel == 0) return QLORA_OK;
+    if (!ok_ptr(x) || !ok_ptr(codes) || !ok_ptr(c)) return QLORA_ERR_INVALID_ARG;
+    if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return QLORA_ERR_INVALID_ARG;
+    return cuda_status(launch_int8_quantize(x, numel, block, codes, c, status, as_stream(stream)));
+}
+
+int qlora_int8_dequantize(const int8_t* codes, const float* c, int64_t numel, int block, float* out, void* stream) {
+    if (numel < 0) return QLORA_ERR_INVALID_ARG;
+    if (!int8_block_supported(block)) return QLORA_ERR_UNSUPPORTED;
+    if (numel >= kMaxNumel) return QLORA_ERR_UNSUPPORTED;
+    if (numel == 0) return QLORA_OK;
+    if (!ok_ptr(codes) || !ok_ptr(c) || !ok_ptr(out)) return QLORA_ERR_INVALID_ARG;
+    return cuda_status(launch_int8_dequantize(codes, c, numel, block, out, as_stream(stream)));
+}
+
 int qlora_debug_wait_timeout(uint64_t limit_ns, void* stream) {
     if (limit_ns == 0 || limit_ns > kMaxSelftestWaitNs) return QLORA_ERR_INVALID_ARG;
     return cuda_status(launch_wait_selftest(limit_ns, as_stream(stream)));

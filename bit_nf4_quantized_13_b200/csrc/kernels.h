@@ -19,6 +19,14 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const
                               const float* mean, int64_t numel, void* out, int out_dtype,
                               cudaStream_t stream);
 
+// int8.cu -- block-wise Int8 absmax quantization (eq. 1) and dequantization
+// (eq. 2), block in {32, 64, 128, 256}
+bool int8_block_supported(int block);
+cudaError_t launch_int8_quantize(const float* x, int64_t numel, int block, int8_t* codes, float* c,
+                                 int32_t* status, cudaStream_t stream);
+cudaError_t launch_int8_dequantize(const int8_t* codes, const float* c, int64_t numel, int block, float* out,
+                                   cudaStream_t stream);
+
 // The frozen NF4 weight W (N x K row-major) as the GEMM kernels see it.
 struct Nf4Weight {
     const uint8_t* codes;   // N*K/2 bytes

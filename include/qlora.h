@@ -206,6 +206,29 @@ int qlora_fp8_e4m3_encode(const float* x, uint8_t* out, int64_t n, void* stream)
 int qlora_device_error(int reset);
 
 /*
+ * qlora_int8_quantize -- block-wise Int8 absmax quantization, the 8-bit
+ * baseline of section 3.1, eq. (1), applied to consecutive blocks of
+ * `block` elements of the flattened tensor (block in {32, 64, 128, 256};
+ * the last block may be partial):
+ *   c[j]    = RN32(127 / absmax(block j))           (0 for an all-zero block)
+ *   code[i] = round_half_away_from_zero(RN32(c[j] * x[i]))   in [-127, 127]
+ *   x       in : numel fp32;  codes out: numel int8;  c out: ceil(numel/block) fp32
+ *   status  out: nullable device int32, cleared to QLORA_OK then set to
+ *                QLORA_ERR_NONFINITE if a block holds a NaN or Inf (or its
+ *                constant overflows fp32); the outputs are then unspecified.
+ * Pointers 16-byte aligned.  numel == 0 enqueues nothing.
+ */
+int qlora_int8_quantize(const float* x, int64_t numel, int block, int8_t* codes, float* c,
+                        int32_t* status, void* stream);
+
+/*
+ * qlora_int8_dequantize -- eq. (2): x'[i] = RN32(code[i] / c[j]), 0 where
+ * c[j] == 0.  Same layout as qlora_int8_quantize; out: numel fp32.
+ */
+int qlora_int8_dequantize(const int8_t* codes, const float* c, int64_t numel, int block, float* out,
+                          void* stream);
+
+/*
  * qlora_debug_wait_timeout -- failure-detection self-test (no counterpart
  * in the paper).  Launches one single-thread kernel on `stream` whose
  * bounded wait (the same wait every pipeline stage of the tensor-core

@@ -88,6 +88,13 @@ def test_argument_validation_on_host(q):
                               1 << 20, None) == 1
     assert L.qlora_fp8_e4m3_encode(P, P, -1, None) == 1
     assert L.qlora_fp8_e4m3_encode(None, None, 0, None) == 0
+    # Int8: block sizes, negative sizes, pointers
+    assert L.qlora_int8_quantize(P, 64, 48, P, P, None, None) == 2
+    assert L.qlora_int8_quantize(P, -1, 64, P, P, None, None) == 1
+    assert L.qlora_int8_quantize(None, 64, 64, P, P, None, None) == 1
+    assert L.qlora_int8_quantize(P, 0, 64, None, None, None, None) == 0
+    assert L.qlora_int8_dequantize(P, P, 64, 512, P, None) == 2
+    assert L.qlora_int8_dequantize(P, P, 64, 64, P + 8, None) == 1
     # the failure-detection self-test refuses limits outside (0, 1 s]
     assert L.qlora_debug_wait_timeout(0, None) == 1
     assert L.qlora_debug_wait_timeout(2_000_000_000, None) == 1
