@@ -55,6 +55,10 @@ def lib():
             L.oracle_nf4_delta.restype = dbl
             L.oracle_nf4_delta.argtypes = []
             L.oracle_nf4_codebook.argtypes = [vp]
+            L.oracle_fp4_codebook.argtypes = [vp]
+            L.oracle_int4_codebook.argtypes = [vp]
+            L.oracle_e2m1_decode.restype = dbl
+            L.oracle_e2m1_decode.argtypes = [i32]
             L.oracle_quantize_nf4.restype = i32
             L.oracle_quantize_nf4.argtypes = [vp, i64, i32, vp, vp, vp]
             L.oracle_mean_exact.restype = i32
@@ -115,15 +119,32 @@ def nf4_codebook() -> np.ndarray:
     return q
 
 
+QTYPES = ("nf4", "fp4", "int4")
+
+
+def e2m1_decode(bits: int) -> float:
+    return float(lib().oracle_e2m1_decode(int(bits)))
+
+
+def codebook(qtype: str = "nf4") -> np.ndarray:
+    """The 16-entry table of a 4-bit type: "nf4", "fp4" (OCP E2M1 / 6) or
+    "int4" (k / 7)."""
+    q = np.zeros(16, np.float32)
+    fn = {"nf4": lib().oracle_nf4_codebook, "fp4": lib().oracle_fp4_codebook,
+          "int4": lib().oracle_int4_codebook}[qtype]
+    fn(_p(q))
+    return q
+
+
 # -- a2, a3 ----------------------------------------------------------------
-def quantize_nf4(w, block: int = 64):
+def quantize_nf4(w, block: int = 64, qtype: str = "nf4"):
     """Returns (codes uint8[ceil(n/2)], c2 fp32[ceil(n/64)], status)."""
     w = _f32(w).reshape(-1)
     n = w.size
     nb = (n + block - 1) // block
     codes = np.zeros((n + 1) // 2, np.uint8)
     c2 = np.zeros(nb, np.float32)
-    q = nf4_codebook()
+    q = codebook(qtype)
     st = lib().oracle_quantize_nf4(_p(w), n, block, _p(q), _p(codes), _p(c2))
     return codes, c2, int(st)
 
@@ -170,11 +191,11 @@ def double_quant(c2, mu, block2: int = 256):
     return b, c1
 
 
-def quantize_nf4_dq(w, block: int = 64, block2: int = 256):
+def quantize_nf4_dq(w, block: int = 64, block2: int = 256, qtype: str = "nf4"):
     """The full quantization of one frozen weight: a2-a5.
 
     Returns a dict with codes, c2_fp8, c1, mean, and the intermediate c2."""
-    codes, c2, st = quantize_nf4(w, block)
+    codes, c2, st = quantize_nf4(w, block, qtype)
     mu, _, st2 = mean_exact(c2)
     b, c1 = double_quant(c2, mu, block2)
     return {"codes": codes, "c2_fp8": b, "c1": c1, "mean": np.float32(mu), "c2": c2,
@@ -190,11 +211,11 @@ def dequant_constants(c2_fp8, c1, mu, block2: int = 256) -> np.ndarray:
     return out
 
 
-def dequantize(codes, c2_fp8, c1, mu, numel: int, block: int = 64, block2: int = 256):
+def dequantize(codes, c2_fp8, c1, mu, numel: int, block: int = 64, block2: int = 256, qtype: str = "nf4"):
     codes = np.ascontiguousarray(codes, np.uint8)
     b = np.ascontiguousarray(c2_fp8, np.uint8)
     c1 = _f32(c1)
-    q = nf4_codebook()
+    q = codebook(qtype)
     out = np.zeros(numel, np.float32)
     lib().oracle_dequantize(_p(codes), _p(b), _p(c1), ctypes.c_float(mu), numel, block, block2,
                             _p(q), _p(out))

@@ -178,6 +178,51 @@ void oracle_nf4_codebook(float q[16])
 /* absmax is 0 stores c2 = 0 and the zero code (index 7) everywhere.        */
 /* ------------------------------------------------------------------------ */
 
+/* ------------------------------------------------------------------------ */
+/* The 4-bit types NF4 is compared with ([notes] 5.1.2, Table 2): FP4 read  */
+/* as OCP E2M1 and Int4 as eq. 1 at 4 bits.  Both are 16-entry tables in   */
+/* [-1, 1] used exactly like the NF4 table (absmax scaling, nearest value,  */
+/* ties to the lower index); a value that repeats is listed twice (the      */
+/* second copy is never the nearest).                                       */
+/* ------------------------------------------------------------------------ */
+
+/* E2M1 bit pattern -> value: sign bit 3, exponent bits 2..1 (bias 1),      */
+/* mantissa bit 0; exponent 0 is subnormal (0 or 0.5).                      */
+double oracle_e2m1_decode(int bits)
+{
+    int sgn = (bits >> 3) & 1, e = (bits >> 1) & 3, m = bits & 1;
+    double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sgn ? -mag : mag;
+}
+
+/* FP4: the distinct E2M1 values in ascending order, divided by the largest */
+/* (6); the top value is repeated to fill 16 entries.                       */
+void oracle_fp4_codebook(float q[16])
+{
+    double v[16];
+    int n = 0;
+    for (int b = 0; b < 16; ++b) {
+        double x = oracle_e2m1_decode(b);
+        int dup = 0;
+        for (int i = 0; i < n; ++i) if (v[i] == x) dup = 1;   /* -0 == +0 */
+        if (!dup) v[n++] = x;
+    }
+    for (int i = 1; i < n; ++i)                                /* insertion sort */
+        for (int j = i; j > 0 && v[j - 1] > v[j]; --j) { double t = v[j]; v[j] = v[j - 1]; v[j - 1] = t; }
+    double top = v[n - 1];
+    for (int i = 0; i < 16; ++i) q[i] = (float)(v[i < n ? i : n - 1] / top);
+}
+
+/* Int4: eq. 1 with 2^(4-1) - 1 = 7 levels per side: k / 7, k = -7..7, the  */
+/* top value repeated at index 15.                                          */
+void oracle_int4_codebook(float q[16])
+{
+    for (int i = 0; i < 16; ++i) {
+        int k = i < 15 ? i - 7 : 7;
+        q[i] = (float)((double)k / 7.0);
+    }
+}
+
 static int nearest_code(float n, const float q[16])
 {
     int best = 0;

@@ -524,3 +524,47 @@ def test_int8_blocks_follow_the_definition():
         a = float(np.max(np.abs(blk)))
         err = np.abs(deq[64 * j:64 * j + blk.size].astype(np.float64) - blk)
         assert np.all(err <= a / 254 * (1 + 1e-5) + 1e-12)
+
+
+# ------------------------------------------- the FP4 / Int4 comparison types
+
+def test_e2m1_decode_matches_the_format():
+    """OCP E2M1: sign, 2-bit exponent (bias 1), 1-bit mantissa; exponent 0 is
+    subnormal.  The 16 patterns give +-{0, 0.5, 1, 1.5, 2, 3, 4, 6}."""
+    import math
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for b in range(16):
+        v = oracle.e2m1_decode(b)
+        assert abs(v) == mags[b & 7]
+        assert (math.copysign(1.0, v) < 0) == (b >= 8)  # the sign bit, -0 included
+
+
+def test_fp4_and_int4_tables():
+    f = oracle.codebook("fp4")
+    ref = np.array(sorted({s * m for s in (-1, 1) for m in (0, 0.5, 1, 1.5, 2, 3, 4, 6)}), np.float64) / 6.0
+    assert ref.size == 15
+    np.testing.assert_array_equal(f[:15], ref.astype(np.float32))
+    assert f[15] == f[14] == 1.0 and f[0] == -1.0 and np.all(np.diff(f[:15]) > 0)
+    i4 = oracle.codebook("int4")
+    np.testing.assert_array_equal(i4[:15], (np.arange(-7, 8) / 7.0).astype(np.float32))
+    assert i4[15] == i4[14] == 1.0 and np.all(i4[:15] == -i4[14::-1])
+
+
+@pytest.mark.parametrize("qtype", ["fp4", "int4"])
+def test_other_types_encode_by_brute_force(qtype):
+    """Codes are the argmin over the type's table (ties to the lower index):
+    the repeated top value is never chosen; block maxima map to the ends."""
+    q = oracle.codebook(qtype)
+    rng = np.random.default_rng(11)
+    w = (rng.standard_normal(64 * 20 + 9) * 0.02).astype(np.float32)
+    codes, c2, st = oracle.quantize_nf4(w, 64, qtype)
+    assert st == 0
+    allc = np.empty(w.size, np.int64)
+    allc[0::2] = codes >> 4
+    allc[1::2] = (codes & 15)[: w.size // 2]
+    for j in range(c2.size):
+        blk = w[64 * j:64 * j + 64]
+        n = (blk / c2[j]).astype(np.float32)
+        d = np.abs(n[:, None] - q[None, :]).astype(np.float32)
+        np.testing.assert_array_equal(allc[64 * j:64 * j + blk.size], np.argmin(d, axis=1))
+    assert not np.any(allc == 15)
