@@ -34,6 +34,8 @@ STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPO
                 3: "QLORA_ERR_WORKSPACE", 4: "QLORA_ERR_CUDA", 5: "QLORA_ERR_NONFINITE",
                 6: "QLORA_ERR_TIMEOUT"}
 BLOCK, BLOCK2, MAX_RANK = 64, 256, 256
+TYPE_NF4, TYPE_FP4, TYPE_INT4 = 0, 1, 2
+QTYPES = {"nf4": TYPE_NF4, "fp4": TYPE_FP4, "int4": TYPE_INT4}
 
 
 class QloraError(RuntimeError):
@@ -50,6 +52,13 @@ def _load() -> ctypes.CDLL:
     i64, i32, vp, sz, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
     sig = {
         "qlora_nf4_codebook": (i32, [vp]),
+        "qlora_codebook": (i32, [i32, vp]),
+        "qlora_quantize_4bit_dq": (i32, [i32, vp, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp]),
+        "qlora_dequantize_4bit": (i32, [i32, vp, vp, vp, vp, i64, i32, i32, vp, i32, vp]),
+        "qlora_linear_fwd_4bit": (i32, [i32, vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp, vp,
+                                        sz, vp]),
+        "qlora_linear_bwd_4bit": (i32, [i32, vp, vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp,
+                                        vp, vp, vp, sz, vp]),
         "qlora_quantize_workspace_size": (sz, [i64]),
         "qlora_quantize_nf4_dq": (i32, [vp, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp]),
         "qlora_dequantize": (i32, [vp, vp, vp, vp, i64, i32, i32, vp, i32, vp]),
@@ -185,6 +194,13 @@ def qlora_nf4_codebook() -> np.ndarray:
     return out
 
 
+def qlora_codebook(qtype: int = TYPE_NF4) -> np.ndarray:
+    """The 16 values of a 4-bit data type (TYPE_NF4, TYPE_FP4, TYPE_INT4)."""
+    out = np.zeros(16, np.float32)
+    _check("qlora_codebook", _get_lib().qlora_codebook(int(qtype), out.ctypes.data_as(ctypes.c_void_p)))
+    return out
+
+
 # ----------------------------------------------------------------- quantize
 
 @dataclass
@@ -195,6 +211,7 @@ class Nf4Weight:
     c1: object      # float32 [ceil(numel/16384)]
     mean: object    # float32 [1]
     shape: tuple
+    qtype: int = 0  # the 4-bit data type the codes index (TYPE_NF4 / TYPE_FP4 / TYPE_INT4)
 
     @property
     def numel(self) -> int:
@@ -211,7 +228,7 @@ def qlora_quantize_workspace_size(numel: int) -> int:
     return int(_get_lib().qlora_quantize_workspace_size(int(numel)))
 
 
-def alloc_nf4_weight(shape, device) -> Nf4Weight:
+def alloc_nf4_weight(shape, device, qtype: int = TYPE_NF4) -> Nf4Weight:
     torch = _torch()
     n = 1
     for d in shape:
@@ -220,28 +237,31 @@ def alloc_nf4_weight(shape, device) -> Nf4Weight:
     return Nf4Weight(torch.empty((n + 1) // 2, dtype=torch.uint8, device=device),
                      torch.empty(max(nb, 1), dtype=torch.uint8, device=device),
                      torch.empty(max(-(-nb // BLOCK2), 1), dtype=torch.float32, device=device),
-                     torch.zeros(1, dtype=torch.float32, device=device), tuple(int(d) for d in shape))
+                     torch.zeros(1, dtype=torch.float32, device=device), tuple(int(d) for d in shape),
+                     int(qtype))
 
 
 def qlora_quantize_nf4_dq(W, out: Nf4Weight | None = None, ws=None, status=None,
-                          stream=None) -> Nf4Weight:
-    """NF4 + double quantization of an fp32 CUDA tensor (any shape, flattened)."""
+                          stream=None, qtype: int = TYPE_NF4) -> Nf4Weight:
+    """4-bit (NF4 by default) + double quantization of an fp32 CUDA tensor
+    (any shape, flattened)."""
     torch = _torch()
     _need_cuda(W)
     if W.dtype != torch.float32:
         raise ValueError("W must be float32")
     n = W.numel()
-    w = out if out is not None else alloc_nf4_weight(tuple(W.shape), W.device)
+    w = out if out is not None else alloc_nf4_weight(tuple(W.shape), W.device, qtype)
+    w.qtype = int(qtype)
     _need_weight(w, n)
     _need_cuda(W, w.codes, w.c2_fp8, w.c1, w.mean, ws, status)
     if status is not None:
         _need_dtype(torch.int32, status=status)
     if ws is None:
         ws = _workspace(qlora_quantize_workspace_size(n), W.device)
-    st = _get_lib().qlora_quantize_nf4_dq(_ptr(W), n, BLOCK, BLOCK2, _ptr(w.codes), _ptr(w.c2_fp8),
-                                   _ptr(w.c1), _ptr(w.mean), _ptr(ws), ws.numel(), _ptr(status),
-                                   _stream(stream))
-    _check("qlora_quantize_nf4_dq", st)
+    st = _get_lib().qlora_quantize_4bit_dq(int(qtype), _ptr(W), n, BLOCK, BLOCK2, _ptr(w.codes), _ptr(w.c2_fp8),
+                                           _ptr(w.c1), _ptr(w.mean), _ptr(ws), ws.numel(), _ptr(status),
+                                           _stream(stream))
+    _check("qlora_quantize_4bit_dq", st)
     return w
 
 
@@ -256,9 +276,9 @@ def qlora_dequantize(w: Nf4Weight, out_dtype=None, out=None, stream=None):
     if out.numel() < w.numel:
         raise ValueError(f"out holds {out.numel()} elements, {w.numel} needed")
     _need_cuda(w.codes, w.c2_fp8, w.c1, w.mean, out)
-    st = _get_lib().qlora_dequantize(_ptr(w.codes), _ptr(w.c2_fp8), _ptr(w.c1), _ptr(w.mean), w.numel,
-                              BLOCK, BLOCK2, _ptr(out), code, _stream(stream))
-    _check("qlora_dequantize", st)
+    st = _get_lib().qlora_dequantize_4bit(int(w.qtype), _ptr(w.codes), _ptr(w.c2_fp8), _ptr(w.c1), _ptr(w.mean),
+                                          w.numel, BLOCK, BLOCK2, _ptr(out), code, _stream(stream))
+    _check("qlora_dequantize_4bit", st)
     return out
 
 
@@ -286,10 +306,10 @@ def qlora_linear_fwd(X, w: Nf4Weight, A, B, s: float, Y=None, T_save=None, ws=No
         T_save = torch.empty((M, r), dtype=torch.bfloat16, device=X.device)
     if ws is None:
         ws = _workspace(qlora_linear_fwd_workspace_size(M, N, K, r), X.device)
-    st = _get_lib().qlora_linear_fwd(_ptr(X), M, N, K, _ptr(w.codes), _ptr(w.c2_fp8), _ptr(w.c1),
-                              _ptr(w.mean), _ptr(A), _ptr(B), r, float(s), _ptr(Y), _ptr(T_save),
-                              _ptr(ws), ws.numel(), _stream(stream))
-    _check("qlora_linear_fwd", st)
+    st = _get_lib().qlora_linear_fwd_4bit(int(w.qtype), _ptr(X), M, N, K, _ptr(w.codes), _ptr(w.c2_fp8),
+                                          _ptr(w.c1), _ptr(w.mean), _ptr(A), _ptr(B), r, float(s), _ptr(Y),
+                                          _ptr(T_save), _ptr(ws), ws.numel(), _stream(stream))
+    _check("qlora_linear_fwd_4bit", st)
     return Y, T_save
 
 
@@ -313,11 +333,11 @@ def qlora_linear_bwd(dY, X, w: Nf4Weight, A, B, s: float, T=None, dX=None, dA=No
         dB = torch.empty((N, r), dtype=torch.bfloat16, device=X.device)
     if ws is None:
         ws = _workspace(qlora_linear_bwd_workspace_size(M, N, K, r), X.device)
-    st = _get_lib().qlora_linear_bwd(_ptr(dY), _ptr(X), M, N, K, _ptr(w.codes), _ptr(w.c2_fp8),
-                              _ptr(w.c1), _ptr(w.mean), _ptr(A), _ptr(B), r, float(s), _ptr(T),
-                              _ptr(dX if want_dx else None), _ptr(dA), _ptr(dB), _ptr(ws),
-                              ws.numel(), _stream(stream))
-    _check("qlora_linear_bwd", st)
+    st = _get_lib().qlora_linear_bwd_4bit(int(w.qtype), _ptr(dY), _ptr(X), M, N, K, _ptr(w.codes),
+                                          _ptr(w.c2_fp8), _ptr(w.c1), _ptr(w.mean), _ptr(A), _ptr(B), r,
+                                          float(s), _ptr(T), _ptr(dX if want_dx else None), _ptr(dA), _ptr(dB),
+                                          _ptr(ws), ws.numel(), _stream(stream))
+    _check("qlora_linear_bwd_4bit", st)
     return dX, dA, dB
 
 

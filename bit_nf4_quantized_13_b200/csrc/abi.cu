@@ -109,10 +109,10 @@ size_t qlora_quantize_workspace_size(int64_t numel) {
     return static_cast<size_t>(kBinBytes + kFlagBytes + round_up(nb * 4, 16));
 }
 
-int qlora_quantize_nf4_dq(const float* W, int64_t numel, int block, int block2, uint8_t* codes,
-                          uint8_t* c2_fp8, float* c1, float* mean, void* ws, size_t ws_bytes,
-                          int32_t* status, void* stream) {
-    if (numel < 0) return QLORA_ERR_INVALID_ARG;
+int qlora_quantize_4bit_dq(int qtype, const float* W, int64_t numel, int block, int block2, uint8_t* codes,
+                           uint8_t* c2_fp8, float* c1, float* mean, void* ws, size_t ws_bytes,
+                           int32_t* status, void* stream) {
+    if (numel < 0 || !valid_qtype(qtype)) return QLORA_ERR_INVALID_ARG;
     if (block != QLORA_BLOCK || block2 != QLORA_BLOCK2) return QLORA_ERR_UNSUPPORTED;
     if (numel >= kMaxNumel) return QLORA_ERR_UNSUPPORTED;
     if (numel == 0) return QLORA_OK;
@@ -120,17 +120,32 @@ int qlora_quantize_nf4_dq(const float* W, int64_t numel, int block, int block2, 
         return QLORA_ERR_INVALID_ARG;
     if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return QLORA_ERR_INVALID_ARG;
     if (!ws || !aligned16(ws) || ws_bytes < qlora_quantize_workspace_size(numel)) return QLORA_ERR_WORKSPACE;
-    return cuda_status(launch_quantize_nf4_dq(W, numel, codes, c2_fp8, c1, mean, ws, status, as_stream(stream)));
+    return cuda_status(
+        launch_quantize_nf4_dq(W, numel, codes, c2_fp8, c1, mean, ws, status, as_stream(stream), qtype));
 }
 
-int qlora_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c1, const float* mean,
-                     int64_t numel, int block, int block2, void* out, int out_dtype, void* stream) {
-    if (numel < 0 || (out_dtype != 0 && out_dtype != 1)) return QLORA_ERR_INVALID_ARG;
+int qlora_quantize_nf4_dq(const float* W, int64_t numel, int block, int block2, uint8_t* codes,
+                          uint8_t* c2_fp8, float* c1, float* mean, void* ws, size_t ws_bytes,
+                          int32_t* status, void* stream) {
+    return qlora_quantize_4bit_dq(QLORA_TYPE_NF4, W, numel, block, block2, codes, c2_fp8, c1, mean, ws, ws_bytes,
+                                  status, stream);
+}
+
+int qlora_dequantize_4bit(int qtype, const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,
+                          const float* mean, int64_t numel, int block, int block2, void* out, int out_dtype,
+                          void* stream) {
+    if (numel < 0 || (out_dtype != 0 && out_dtype != 1) || !valid_qtype(qtype)) return QLORA_ERR_INVALID_ARG;
     if (block != QLORA_BLOCK || block2 != QLORA_BLOCK2) return QLORA_ERR_UNSUPPORTED;
     if (numel >= kMaxNumel) return QLORA_ERR_UNSUPPORTED;
     if (numel == 0) return QLORA_OK;
     if (check_weight(codes, c2_fp8, c1, mean) != QLORA_OK || !ok_ptr(out)) return QLORA_ERR_INVALID_ARG;
-    return cuda_status(launch_dequantize(codes, c2_fp8, c1, mean, numel, out, out_dtype, as_stream(stream)));
+    return cuda_status(launch_dequantize(codes, c2_fp8, c1, mean, numel, out, out_dtype, as_stream(stream), qtype));
+}
+
+int qlora_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c1, const float* mean,
+                     int64_t numel, int block, int block2, void* out, int out_dtype, void* stream) {
+    return qlora_dequantize_4bit(QLORA_TYPE_NF4, codes, c2_fp8, c1, mean, numel, block, block2, out, out_dtype,
+                                 stream);
 }
 
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
@@ -146,10 +161,11 @@ size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r) {
     return 2 * mr + pair_gemm_workspace();
 }
 
-int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
-                     const uint8_t* c2_fp8, const float* c1, const float* mean, const uint16_t* A,
-                     const uint16_t* B, int r, float s, uint16_t* Y, uint16_t* T_save, void* ws,
-                     size_t ws_bytes, void* stream) {
+int qlora_linear_fwd_4bit(int qtype, const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
+                          const uint8_t* c2_fp8, const float* c1, const float* mean, const uint16_t* A,
+                          const uint16_t* B, int r, float s, uint16_t* Y, uint16_t* T_save, void* ws,
+                          size_t ws_bytes, void* stream) {
+    if (!valid_qtype(qtype)) return QLORA_ERR_INVALID_ARG;
     int st = check_linear(M, N, K, r);
     if (st != QLORA_OK) return st;
     if (check_weight(codes, c2_fp8, c1, mean) != QLORA_OK) return QLORA_ERR_INVALID_ARG;
@@ -163,7 +179,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     void* gws = reinterpret_cast<char*>(ws) + t_bytes;
     const size_t gws_bytes = ws_bytes - t_bytes;
     cudaStream_t cs = as_stream(stream);
-    Nf4Weight w{codes, c2_fp8, c1, mean, N, K};
+    Nf4Weight w{codes, c2_fp8, c1, mean, N, K, qtype};
     if (gemv_supported(M, N, K, r)) {  // a few tokens: one stream over the weight
         const cudaError_t g = launch_fwd_gemv(X, w, A, B, M, r, s, Y, T_save, cs);
         if (g != cudaErrorNotSupported) return cuda_status(g);  // else: no cluster shape fits
@@ -173,11 +189,20 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     return cuda_status(e);
 }
 
-int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N, int64_t K,
-                     const uint8_t* codes, const uint8_t* c2_fp8, const float* c1, const float* mean,
-                     const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* T,
-                     uint16_t* dX, uint16_t* dA, uint16_t* dB, void* ws, size_t ws_bytes,
-                     void* stream) {
+int qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
+                     const uint8_t* c2_fp8, const float* c1, const float* mean, const uint16_t* A,
+                     const uint16_t* B, int r, float s, uint16_t* Y, uint16_t* T_save, void* ws,
+                     size_t ws_bytes, void* stream) {
+    return qlora_linear_fwd_4bit(QLORA_TYPE_NF4, X, M, N, K, codes, c2_fp8, c1, mean, A, B, r, s, Y, T_save, ws,
+                                 ws_bytes, stream);
+}
+
+int qlora_linear_bwd_4bit(int qtype, const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                          const uint8_t* codes, const uint8_t* c2_fp8, const float* c1, const float* mean,
+                          const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* T,
+                          uint16_t* dX, uint16_t* dA, uint16_t* dB, void* ws, size_t ws_bytes,
+                          void* stream) {
+    if (!valid_qtype(qtype)) return QLORA_ERR_INVALID_ARG;
     int st = check_linear(M, N, K, r);
     if (st != QLORA_OK) return st;
     if (check_weight(codes, c2_fp8, c1, mean) != QLORA_OK) return QLORA_ERR_INVALID_ARG;
@@ -195,7 +220,7 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N
     const size_t mr = align256(static_cast<size_t>(M) * r * 2);
     uint16_t* U = reinterpret_cast<uint16_t*>(ws);
     uint16_t* Tw = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + mr);
-    Nf4Weight w{codes, c2_fp8, c1, mean, N, K};
+    Nf4Weight w{codes, c2_fp8, c1, mean, N, K, qtype};
     void* dxws = reinterpret_cast<char*>(ws) + 2 * mr;
     const size_t dxws_bytes = ws_bytes - 2 * mr;
     cudaError_t e = cudaSuccess;
@@ -207,6 +232,15 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N
     if (e == cudaSuccess && dX) e = launch_bwd_dx_gemm(dY, w, U, A, M, r, dX, dxws, dxws_bytes, cs);
     if (e == cudaSuccess) e = lora_grads(dY, X, T, U, M, N, K, r, dA, dB, cs);
     return cuda_status(e);
+}
+
+int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                     const uint8_t* codes, const uint8_t* c2_fp8, const float* c1, const float* mean,
+                     const uint16_t* A, const uint16_t* B, int r, float s, const uint16_t* T,
+                     uint16_t* dX, uint16_t* dA, uint16_t* dB, void* ws, size_t ws_bytes,
+                     void* stream) {
+    return qlora_linear_bwd_4bit(QLORA_TYPE_NF4, dY, X, M, N, K, codes, c2_fp8, c1, mean, A, B, r, s, T, dX, dA, dB,
+                                 ws, ws_bytes, stream);
 }
 
 int qlora_device_error(int reset) {

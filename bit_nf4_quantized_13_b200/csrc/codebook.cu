@@ -1,4 +1,5 @@
-// codebook.cu -- host construction of the NF4 type and of the encoder tables.
+// codebook.cu -- host construction of the 4-bit data types (NF4, and FP4 and
+// Int4 for comparison) and of their encoder tables.
 //
 // The NF4 values follow the QLoRA study notes (gitcode.csdn.net), section 3.2:
 // quantiles of N(0,1), 2^(k-1) for the negative half and 2^(k-1)+1 for the
@@ -46,7 +47,7 @@ double normal_quantile(double p) {
     return p < 0.5 ? -x : x;
 }
 
-void build_codebook(float q[16]) {
+void build_nf4(float q[16]) {
     const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
     const double top = normal_quantile(delta);
     double v[16];
@@ -56,6 +57,25 @@ void build_codebook(float q[16]) {
     // positive half: probabilities 1/2 + (delta - 1/2) * i / 8, i = 1..8
     for (int i = 1; i <= 8; ++i) v[7 + i] = normal_quantile(0.5 + (delta - 0.5) * i / 8.0);
     for (int i = 0; i < 16; ++i) q[i] = static_cast<float>(v[i] / top);
+}
+
+// FP4 as OCP E2M1 (1 sign, 2 exponent, 1 mantissa bit): magnitudes 0, 0.5,
+// 1, 1.5, 2, 3, 4, 6, normalised by the largest so that absmax maps to +-1.
+// The 15 distinct signed values in ascending order (the two zeros of the
+// format are one value), the top one repeated at index 15.
+void build_fp4(float q[16]) {
+    const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    for (int i = 7; i >= 1; --i) q[7 - i] = static_cast<float>(-mag[i] / 6.0);
+    q[7] = 0.0f;
+    for (int i = 1; i <= 7; ++i) q[7 + i] = static_cast<float>(mag[i] / 6.0);
+    q[15] = q[14];
+}
+
+// Int4 as the 4-bit case of the absmax integer quantization of eq. (1): the
+// symmetric levels k / 7, k = -7 .. 7, the top one repeated at index 15.
+void build_int4(float q[16]) {
+    for (int k = -7; k <= 7; ++k) q[k + 7] = static_cast<float>(static_cast<double>(k) / 7.0);
+    q[15] = q[14];
 }
 
 // fp32 total order on bit patterns (for bisection over representable values)
@@ -100,11 +120,18 @@ int bin_of(float n) {
     return static_cast<int>(u >> 18) - 0x1000;
 }
 
-Nf4Tables build_tables() {
+Nf4Tables build_tables(int qtype) {
     Nf4Tables t;
-    build_codebook(t.q);
+    if (qtype == QLORA_TYPE_FP4)
+        build_fp4(t.q);
+    else if (qtype == QLORA_TYPE_INT4)
+        build_int4(t.q);
+    else
+        build_nf4(t.q);
+    // a repeated value never wins (ties go to the lower index): its threshold
+    // lies beyond the range of n
     float thr[15];
-    for (int j = 0; j < 15; ++j) thr[j] = threshold(t.q[j], t.q[j + 1]);
+    for (int j = 0; j < 15; ++j) thr[j] = t.q[j] == t.q[j + 1] ? 2.0f : threshold(t.q[j], t.q[j + 1]);
     auto code_of = [&](float n) {
         int c = 0;
         for (int j = 0; j < 15; ++j) c += (n >= thr[j]);
@@ -132,28 +159,35 @@ Nf4Tables build_tables() {
         for (int j = 0; j < 15; ++j)
             if (thr[j] > first && thr[j] <= last) { t.thr[b] = thr[j]; ++inside; }
         if (inside > 1 || code_of(last) != t.base[b] + inside) {
-            // cannot happen for the NF4 type (thresholds are >= 0.08 apart,
-            // bins are 1/16 wide); keep the failure loud
+            // cannot happen for the three types (their thresholds are at
+            // least 0.08 apart, the bins 1/16 wide); keep the failure loud
             t.base[b] = -1000;
         }
     }
     return t;
 }
 
-std::once_flag g_once;
-Nf4Tables g_tables;
+std::once_flag g_once[3];
+Nf4Tables g_tables[3];
 
 }  // namespace
 
-const Nf4Tables& tables() {
-    std::call_once(g_once, [] { g_tables = build_tables(); });
-    return g_tables;
+const Nf4Tables& tables(int qtype) {
+    const int t = (qtype == QLORA_TYPE_FP4 || qtype == QLORA_TYPE_INT4) ? qtype : QLORA_TYPE_NF4;
+    std::call_once(g_once[t], [t] { g_tables[t] = build_tables(t); });
+    return g_tables[t];
+}
+
+bool valid_qtype(int qtype) {
+    return qtype == QLORA_TYPE_NF4 || qtype == QLORA_TYPE_FP4 || qtype == QLORA_TYPE_INT4;
 }
 
 }  // namespace qlora
 
-extern "C" int qlora_nf4_codebook(float out_host[16]) {
-    if (!out_host) return QLORA_ERR_INVALID_ARG;
-    memcpy(out_host, qlora::tables().q, sizeof(float) * 16);
+extern "C" int qlora_codebook(int qtype, float out_host[16]) {
+    if (!out_host || !qlora::valid_qtype(qtype)) return QLORA_ERR_INVALID_ARG;
+    memcpy(out_host, qlora::tables(qtype).q, sizeof(float) * 16);
     return QLORA_OK;
 }
+
+extern "C" int qlora_nf4_codebook(float out_host[16]) { return qlora_codebook(QLORA_TYPE_NF4, out_host); }

@@ -27,7 +27,9 @@ struct Nf4Tables {
     int base[33];
 };
 
-const Nf4Tables& tables();  // host: lazily built, immutable
+// host: lazily built per data type (QLORA_TYPE_*), immutable
+const Nf4Tables& tables(int qtype = QLORA_TYPE_NF4);
+bool valid_qtype(int qtype);
 
 // ---------------------------------------------------------------- bf16 bits
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {

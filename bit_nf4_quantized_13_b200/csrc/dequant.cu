@@ -138,7 +138,7 @@ k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,
                               const float* mean, int64_t numel, void* out, int out_dtype,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, int qtype) {
     static ContextMemo<int> memo_bf16, memo_f32;
     const cudaError_t attr = out_dtype == 1 ? ensure_smem_limit(memo_bf16, k_dequant<true>, kLutBytes)
                                             : ensure_smem_limit(memo_f32, k_dequant<false>, kLutBytes);
@@ -147,9 +147,9 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const
     const int64_t want = ceil_div(chunks, kThreads / 32);
     const int grid = static_cast<int>(want < num_sms() * 3LL ? (want > 0 ? want : 1) : num_sms() * 3LL);
     if (out_dtype == 1)
-        k_dequant<true><<<grid, kThreads, kLutBytes, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables());
+        k_dequant<true><<<grid, kThreads, kLutBytes, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables(qtype));
     else
-        k_dequant<false><<<grid, kThreads, kLutBytes, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables());
+        k_dequant<false><<<grid, kThreads, kLutBytes, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables(qtype));
     note_launches(1);
     return cudaGetLastError();
 }

@@ -828,7 +828,6 @@ cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& ml, const CUte
     if (e != cudaSuccess) return e;
     int pairs = max_pairs<kBwd>();
     if (pairs <= 0) return cudaErrorNotSupported;
-    for (int i = 0; i < 16; ++i) p.q[i] = tables().q[i];
     // no more pairs than the workspace has slots for, and at least a few
     // stages for each
     while (pairs > 1 && (ws == nullptr || ws_bytes < ws_bytes_for(pairs))) --pairs;
@@ -881,6 +880,7 @@ PairParams base_params(const Nf4Weight& w, int64_t M, int r, uint16_t* out, bool
     p.num_t = static_cast<int>(ceil_div(M, kTileTok));
     p.num_tiles = p.num_t * static_cast<int>(ceil_div(p.rows, kRowsPair));
     p.iters = static_cast<int64_t>(p.num_tiles) * p.kb_total;
+    for (int i = 0; i < 16; ++i) p.q[i] = tables(w.qtype).q[i];
     return p;
 }
 

@@ -104,7 +104,8 @@ cudaError_t gemm(int64_t Mo, int64_t No, const Opnd& a1, const Opnd& b1, int64_t
                  const Opnd& b2, int64_t K2, float alpha, uint16_t* C, int64_t ldc, cudaStream_t st) {
     if (Mo == 0 || No == 0) return cudaSuccess;
     dim3 grid(static_cast<unsigned>(ceil_div(No, BN)), static_cast<unsigned>(ceil_div(Mo, BM)));
-    k_gemm_simt<<<grid, kThreads, 0, st>>>(Mo, No, a1, b1, K1, a2, b2, K2, alpha, C, ldc, tables());
+    const int qtype = a1.kind != 0 ? a1.w.qtype : (b1.kind != 0 ? b1.w.qtype : QLORA_TYPE_NF4);
+    k_gemm_simt<<<grid, kThreads, 0, st>>>(Mo, No, a1, b1, K1, a2, b2, K2, alpha, C, ldc, tables(qtype));
     note_launches(1);
     return cudaGetLastError();
 }

@@ -27,19 +27,22 @@
 //    bf16(RN(q[code] * c2')); both are one bf16 rounding from w').
 //  * X fragments stay in registers for the whole kernel: a warp always owns
 //    the same K-blocks of its CTA's slice.
-//  * Split-K across the cluster: each CTA reduces its warps' partials in
-//    shared memory, then CTA rank 0 sums the C partials in rank order
-//    (deterministic), adds T B^T with one more MMA per 16 ranks and stores
-//    Y.
+//  * Split-K across the cluster, reduced once: every unit's partials go
+//    from the compute warps into one of two reduction slots; the producer
+//    warp sums a slot's warps in warp order into this CTA's own per-unit
+//    sums (kept in its shared memory for the whole kernel) and frees the
+//    slot.  No warp waits on another's per-unit work unless it runs two
+//    units ahead of the reduction.  At the end, after one cluster barrier,
+//    CTA rank c finishes the units c, c + C, ...: it adds the C CTAs' sums
+//    in rank order (distributed shared memory; deterministic), adds T B^T
+//    with one more MMA per 16 ranks and stores Y.
 //  * T = bf16(s X A^T) is formed in the same kernel from the register
 //    resident X fragments (the rows of A take the MMA's A operand in the
-//    permuted k order), reduced over the cluster like the unit partials.
-//  * 14 decode warps per CTA run free of one another; a 15th warp issues
-//    the copies and sums their partials (named-barrier hand-off) and pushes
-//    the CTA's partial into rank 0's shared memory with st.async (completing
-//    on an mbarrier); in rank 0 a 16th warp finishes the units as their
-//    partials land and hands the slot buffers (up to 4) back with remote
-//    arrives, so no warp's per-unit work serialises behind another's.
+//    permuted k order), reduced like the unit partials; every CTA forms the
+//    same T from the cluster's sums.
+//  * 14 compute warps stream the units; a 15th issues the copies and
+//    reduces the slots; a 16th pulls the constants and the rows of B into
+//    L2 early; all 16 finish the units at the end.
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -65,12 +68,10 @@ constexpr int kMaxBw = 3;                    // 64-blocks per warp per unit
 constexpr int kMaxCtaBlocks = kWarps * kMaxBw;
 constexpr int kMaxCl = 8;                    // CTAs per cluster
 constexpr int kStages = 6;                   // most stages a launch uses
-constexpr int kSlotBufs = 4;                 // most units a CTA may run ahead of rank 0's epilogue
 constexpr int kLutBytes = 256 * 256;         // 256 entries x 64 words (32 used)
 constexpr int kMaxRankTiles = 4;             // r <= 64
 constexpr int kTStride = 16 * kMaxRankTiles; // T staging row (ranks), bf16
-constexpr int kBarRedFull = 1;               // named barrier: partials written (compute warps arrive)
-constexpr int kBarRedFree = 2;               // named barrier: partials read (producer arrives)
+constexpr int kRedSlots = 2;                 // reduction slots (units in flight between compute and reduce)
 
 struct GemvParams {
     const uint8_t* codes;
@@ -90,22 +91,24 @@ struct GemvParams {
     int row_stride;         // bytes between rows of a stage
     int stage_bytes;
     int nstages;            // ring depth, <= kStages
-    int nslot;              // slot buffers: 2 or kSlotBufs
+    int nmax;               // most units a cluster owns (the per-unit sums kept in shared memory)
     float q[16];
 };
 
 struct GemvSmem {
-    size_t red_off, slot_off, tslot_off, tbuf_off, bar_off, total;
+    size_t red_off, part_off, tpart_off, tbuf_off, bar_off, total;
 };
 
-__host__ __device__ constexpr GemvSmem gemv_smem(int NT, int stage_bytes, int nstages, int cl, int rt, int nslot) {
+// LUT | stages | reduction slots [2][kWarps][NT][32] | this CTA's unit sums
+// [nmax][NT][32] | its T sums [rt][NT][32] | T (bf16) | barriers
+__host__ __device__ constexpr GemvSmem gemv_smem(int NT, int stage_bytes, int nstages, int nmax, int rt) {
     GemvSmem m{};
     m.red_off = kLutBytes + static_cast<size_t>(nstages) * stage_bytes;
-    m.slot_off = m.red_off + kWarps * NT * 32 * 16;
-    m.tslot_off = m.slot_off + static_cast<size_t>(nslot) * cl * NT * 32 * 16;
-    m.tbuf_off = m.tslot_off + static_cast<size_t>(cl) * rt * NT * 32 * 16;
+    m.part_off = m.red_off + static_cast<size_t>(kRedSlots) * kWarps * NT * 32 * 16;
+    m.tpart_off = m.part_off + static_cast<size_t>(nmax) * NT * 32 * 16;
+    m.tbuf_off = m.tpart_off + static_cast<size_t>(rt) * NT * 32 * 16;
     m.bar_off = m.tbuf_off + 16 * kTStride * 2;
-    m.total = m.bar_off + (kStages + 2 * kSlotBufs + 1) * 8;
+    m.total = m.bar_off + (2 * kStages + 2 * kRedSlots) * 8;
     return m;
 }
 
@@ -114,17 +117,6 @@ __host__ __device__ constexpr GemvSmem gemv_smem(int NT, int stage_bytes, int ns
 __device__ __forceinline__ uint32_t lut_pair(const uint8_t* lut, uint32_t word, uint32_t lane_off, int byte) {
     const uint32_t addr = __byte_perm(word, lane_off, 0x5504u | (static_cast<uint32_t>(byte) << 4));
     return *reinterpret_cast<const uint32_t*>(lut + addr);
-}
-
-// Named-barrier hand-off between the compute warps and the producer warp;
-// the warp is reconverged first (the barriers are warp-aligned).
-__device__ __forceinline__ void bar_arrive(int id) {
-    __syncwarp();
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(kBarThreads) : "memory");
-}
-__device__ __forceinline__ void bar_wait(int id) {
-    __syncwarp();
-    named_bar_sync(id, kBarThreads);
 }
 
 // Issues the copy of unit `u` into `stage`, completing on `bar`: one
@@ -153,151 +145,119 @@ __device__ __forceinline__ void load_b_rows(const GemvParams& p, int u, int g, i
     }
 }
 
-// Sum of the 15 compute warps' partials (fragment layout), warp order.
-template <int NT>
-__device__ __forceinline__ void sum_partials(const float4* red, int lane, float4 (&v)[NT]) {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        float4 sum = red[nt * 32 + lane];
-#pragma unroll
-        for (int w = 1; w < kWarps; ++w) {
-            const float4 x = red[(w * NT + nt) * 32 + lane];
-            sum.x += x.x; sum.y += x.y; sum.z += x.z; sum.w += x.w;
-        }
-        v[nt] = sum;
-    }
-}
+// The barriers: full[s] (TMA bytes of stage s), empty[s] (every compute
+// lane has read stage s), red_full[b] (every compute lane has written slot
+// b), red_empty[b] (the reducer has read slot b).
+struct GemvBars {
+    uint64_t* full;
+    uint64_t* empty;
+    uint64_t* red_full;
+    uint64_t* red_empty;
+};
 
-// The producer warp of every CTA: issues the stage copies, reduces the
-// compute warps' partials and pushes the CTA's partial of T and of every
-// unit into rank 0's shared memory (st.async).
+// The producer warp of every CTA: refills the stages and reduces the
+// compute warps' partials, slot after slot (T's rank tiles first, then the
+// units), into this CTA's own sums in shared memory.
 template <int NT>
-__device__ __forceinline__ void producer_warp(const CUtensorMap* map, const GemvParams& p, uint8_t* smem, const GemvSmem& L, uint64_t* full,
-                                              uint64_t* slot_full, uint64_t* slot_empty, uint64_t* t_full,
-                                              uint32_t crank, int cid, int ncl, int n_local,
-                                              int b0, int nblk, int lane) {
-    const int g = lane >> 2, qd = lane & 3;
+__device__ __forceinline__ void producer_warp(const CUtensorMap* map, const GemvParams& p, uint8_t* smem,
+                                              const GemvSmem& L, const GemvBars& B, int cid, int ncl, int n_local,
+                                              int b0, int lane) {
     const int RT = (p.r + 15) >> 4;
     const int nst = p.nstages;
     uint8_t* stages = smem + kLutBytes;
     const float4* red = reinterpret_cast<const float4*>(smem + L.red_off);
-    const float4* slot = reinterpret_cast<const float4*>(smem + L.slot_off);
-    const float4* tslot = reinterpret_cast<const float4*>(smem + L.tslot_off);
+    float4* part = reinterpret_cast<float4*>(smem + L.part_off);
+    float4* tpart = reinterpret_cast<float4*>(smem + L.tpart_off);
 
-    if (lane == 0) {
-        const int pre = n_local < nst ? n_local : nst;
-        for (int i = 0; i < pre; ++i) issue_unit(map, p, cid + i * ncl, stages + i * p.stage_bytes, &full[i], b0);
-    }
-    const uint32_t tslot_r0 = cluster_map(smem_u32(smem + L.tslot_off), 0);
-    const uint32_t t_full_r0 = cluster_map(smem_u32(t_full), 0);
-    const uint32_t slot_r0 = cluster_map(smem_u32(smem + L.slot_off), 0);
-    const uint32_t slot_full_r0 = cluster_map(smem_u32(slot_full), 0);
-
-    // this CTA's part of X A^T, one 16-rank tile per round
-    for (int rt = 0; rt < RT; ++rt) {
-        bar_wait(kBarRedFull);
-        float4 v[NT];
-        sum_partials<NT>(red, lane, v);
-        bar_arrive(kBarRedFree);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-            st_async_f4(tslot_r0 + static_cast<uint32_t>((((crank * RT + rt) * NT + nt) * 32 + lane) * 16), v[nt],
-                        t_full_r0);
-    }
-
+    const int nq = RT + n_local;
 #pragma unroll 1
-    for (int i = 0; i < n_local; ++i) {
-        bar_wait(kBarRedFull);  // unit i's partials are written: its stage is free too
-        if (lane == 0 && i + nst < n_local)
-            issue_unit(map, p, cid + (i + nst) * ncl, stages + (i % nst) * p.stage_bytes, &full[i % nst], b0);
-        float4 v[NT];
-        sum_partials<NT>(red, lane, v);
-        bar_arrive(kBarRedFree);
-        const int b = i % p.nslot, k = i / p.nslot;
-        if (k >= 1) mbar_wait(smem_u32(&slot_empty[b]), (k - 1) & 1, &g_gemv_error);
+    for (int q = 0; q < nq; ++q) {
+        const int b = q % kRedSlots;
+        const int i = q - RT;  // unit (>= 0) or rank tile (< 0)
+        if (i >= 0 && lane == 0 && i + nst < n_local) {
+            // unit i has been read from its stage: refill the stage with unit i + nst
+            const int s = i % nst;
+            if (mbar_wait(smem_u32(&B.empty[s]), (i / nst) & 1, &g_gemv_error))
+                issue_unit(map, p, cid + (i + nst) * ncl, stages + s * p.stage_bytes, &B.full[s], b0);
+        }
+        mbar_wait(smem_u32(&B.red_full[b]), (q / kRedSlots) & 1, &g_gemv_error);
+        float4* dst = i >= 0 ? part + static_cast<size_t>(i) * NT * 32 : tpart + static_cast<size_t>(q) * NT * 32;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-            st_async_f4(slot_r0 + static_cast<uint32_t>((((b * p.cl + crank) * NT + nt) * 32 + lane) * 16), v[nt],
-                        slot_full_r0 + static_cast<uint32_t>(b * 8));
+        for (int nt = 0; nt < NT; ++nt) {
+            float4 sum = red[((b * kWarps + 0) * NT + nt) * 32 + lane];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) {  // warp order: deterministic
+                const float4 x = red[((b * kWarps + w) * NT + nt) * 32 + lane];
+                sum.x += x.x; sum.y += x.y; sum.z += x.z; sum.w += x.w;
+            }
+            dst[nt * 32 + lane] = sum;
+        }
+        mbar_arrive(smem_u32(&B.red_empty[b]));
     }
 }
 
-// Rank 0's epilogue warp, one unit behind the partials: T = bf16(s * sum of
-// the T partials in rank order) once, then per unit the C partials summed in
-// rank order, the slot buffer handed back to every CTA, T B^T added with one
-// MMA per 16 ranks and Y stored.
+// Every warp of every CTA, after the cluster barrier: T = bf16(s * the
+// cluster's T sums in rank order) into tbuf (warp 0; rank 0 of cluster 0
+// also stores T_save), then the units c, c + C, ... of this CTA (rank c):
+// the C CTAs' sums in rank order, plus T B^T, stored as Y.
 template <int NT>
-__device__ __forceinline__ void epilogue_warp(const GemvParams& p, uint8_t* smem, const GemvSmem& L,
-                                              uint64_t* slot_full, uint64_t* slot_empty, uint64_t* t_full, int cid,
-                                              int ncl, int n_local, int lane) {
+__device__ __forceinline__ void final_epilogue(const GemvParams& p, uint8_t* smem, const GemvSmem& L, uint32_t crank,
+                                               int cid, int ncl, int n_local, int warp, int lane) {
     const int g = lane >> 2, qd = lane & 3;
     const int RT = (p.r + 15) >> 4;
-    const float4* slot = reinterpret_cast<const float4*>(smem + L.slot_off);
-    const float4* tslot = reinterpret_cast<const float4*>(smem + L.tslot_off);
     uint16_t* tbuf = reinterpret_cast<uint16_t*>(smem + L.tbuf_off);  // [16 tokens][kTStride]
-    const uint32_t slot_bytes = static_cast<uint32_t>(p.cl) * NT * 32 * 16;
-    if (lane == 0) {
-        mbar_arrive_expect_tx(smem_u32(t_full), static_cast<uint32_t>(p.cl) * RT * NT * 32 * 16);
-        for (int b = 0; b < p.nslot; ++b) mbar_arrive_expect_tx(smem_u32(&slot_full[b]), slot_bytes);
-    }
-    uint32_t ba[kMaxRankTiles][4];  // B rows of the next unit to finish
-    if (n_local > 0) load_b_rows(p, cid, g, qd, ba);
-    uint32_t tf[NT][kMaxRankTiles][2];
-    bool t_ready = false;
-#pragma unroll 1
-    for (int i = 0; i < n_local; ++i) {
-        if (!t_ready) {  // T: lane holds (rank 16 rt + g (+8), token 8 nt + 2 qd (+1)) of every tile
-            mbar_wait(smem_u32(t_full), 0, &g_gemv_error);
-            for (int rt = 0; rt < RT; ++rt) {
+    const uint32_t part0 = smem_u32(smem + L.part_off);
+    const uint32_t tpart0 = smem_u32(smem + L.tpart_off);
+    if (warp == 0) {
+        for (int rt = 0; rt < RT; ++rt) {
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    float4 v = tslot[((0 * RT + rt) * NT + nt) * 32 + lane];
-                    for (int rk = 1; rk < p.cl; ++rk) {
-                        const float4 w = tslot[((rk * RT + rt) * NT + nt) * 32 + lane];
-                        v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
-                    }
-                    const float e4[4] = {v.x, v.y, v.z, v.w};
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint32_t off = static_cast<uint32_t>(((rt * NT + nt) * 32 + lane) * 16);
+                float4 v = ld_cluster_f4(cluster_map(tpart0 + off, 0));
+                for (int rk = 1; rk < p.cl; ++rk) {
+                    const float4 w = ld_cluster_f4(cluster_map(tpart0 + off, static_cast<uint32_t>(rk)));
+                    v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+                }
+                const float e4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = 16 * rt + g + 8 * (e >> 1);
-                        const int tok = 8 * nt + 2 * qd + (e & 1);
-                        const uint16_t tb = f32_to_bf16_bits(e4[e] * p.s);
-                        tbuf[tok * kTStride + j] = tb;
-                        if (p.T_save && cid == 0 && tok < p.M && j < p.r)
-                            p.T_save[static_cast<int64_t>(tok) * p.r + j] = tb;
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 16 * rt + g + 8 * (e >> 1);
+                    const int tok = 8 * nt + 2 * qd + (e & 1);
+                    const uint16_t tb = f32_to_bf16_bits(e4[e] * p.s);
+                    tbuf[tok * kTStride + j] = tb;
+                    if (p.T_save && cid == 0 && crank == 0 && tok < p.M && j < p.r)
+                        p.T_save[static_cast<int64_t>(tok) * p.r + j] = tb;
                 }
             }
-            __syncwarp();
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int st = 0; st < kMaxRankTiles; ++st)
-#pragma unroll
-                    for (int hf = 0; hf < 2; ++hf)  // T as the B operand of the LoRA MMA: (k = rank, n = token)
-                        tf[nt][st][hf] = (16 * st < p.r) ? *reinterpret_cast<const uint32_t*>(
-                                                               &tbuf[(8 * nt + g) * kTStride + 16 * st + 2 * qd + 8 * hf])
-                                                         : 0u;
-            t_ready = true;
         }
-        const int b = i % p.nslot, k = i / p.nslot;
+    }
+    __syncthreads();
+    uint32_t tf[NT][kMaxRankTiles][2];  // T as the B operand of the LoRA MMA: (k = rank, n = token)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int st = 0; st < kMaxRankTiles; ++st)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+                tf[nt][st][hf] = (16 * st < p.r)
+                                     ? *reinterpret_cast<const uint32_t*>(&tbuf[(8 * nt + g) * kTStride + 16 * st + 2 * qd + 8 * hf])
+                                     : 0u;
+    const int nw = kThreads / 32;
+#pragma unroll 1
+    for (int i = static_cast<int>(crank) + p.cl * warp; i < n_local; i += p.cl * nw) {
         const int n0 = (cid + i * ncl) * kRows;
-        mbar_wait(smem_u32(&slot_full[b]), k & 1, &g_gemv_error);
+        uint32_t ba[kMaxRankTiles][4];
+        load_b_rows(p, cid + i * ncl, g, qd, ba);
         float acc[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            float4 sum = slot[((b * p.cl + 0) * NT + nt) * 32 + lane];
+            const uint32_t off = static_cast<uint32_t>(((i * NT + nt) * 32 + lane) * 16);
+            float4 sum = ld_cluster_f4(cluster_map(part0 + off, 0));
             for (int rk = 1; rk < p.cl; ++rk) {
-                const float4 v = slot[((b * p.cl + rk) * NT + nt) * 32 + lane];
+                const float4 v = ld_cluster_f4(cluster_map(part0 + off, static_cast<uint32_t>(rk)));
                 sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
             }
             acc[nt][0] = sum.x; acc[nt][1] = sum.y; acc[nt][2] = sum.z; acc[nt][3] = sum.w;
-        }
-        __syncwarp();
-        if (i + p.nslot < n_local) {  // the buffer's next use: arm it, then release it to every CTA
-            if (lane == 0) mbar_arrive_expect_tx(smem_u32(&slot_full[b]), slot_bytes);
-            __syncwarp();
-            if (lane < p.cl) mbar_arrive_cluster(cluster_map(smem_u32(&slot_empty[b]), lane));
         }
 #pragma unroll
         for (int st = 0; st < kMaxRankTiles; ++st) {
@@ -306,7 +266,6 @@ __device__ __forceinline__ void epilogue_warp(const GemvParams& p, uint8_t* smem
             for (int nt = 0; nt < NT; ++nt)  // A: a0a1 row g, a2a3 row g+8, a4..a7 the same 8 ranks further
                 mma_16816(acc[nt], ba[st][0], ba[st][1], ba[st][2], ba[st][3], tf[nt][st][0], tf[nt][st][1]);
         }
-        if (i + 1 < n_local) load_b_rows(p, cid + (i + 1) * ncl, g, qd, ba);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -317,7 +276,6 @@ __device__ __forceinline__ void epilogue_warp(const GemvParams& p, uint8_t* smem
             }
         }
     }
-
 }
 
 // X fragments of warp `warp`'s blocks: block jloc = warp + kWarps * jj.
@@ -347,8 +305,38 @@ __device__ __forceinline__ void load_x_frags(const GemvParams& p, int b0, int nb
     }
 }
 
+// The 16th warp of every CTA pulls into L2 what the other warps will load
+// later: the units' FP8 constants and c1, and the rows of B the epilogue
+// needs.
+__device__ __forceinline__ void prefetch_warp(const GemvParams& p, int cid, int ncl, int n_local, int b0, int nblk,
+                                              int lane) {
+    for (int i = 0; i < n_local; ++i) {
+        const int64_t row0 = static_cast<int64_t>(cid + i * ncl) * kRows;
+        if (lane < kRows) {  // row lane of the unit: its FP8 bytes of this slice, and its c1 words
+            const int64_t blk0 = (row0 + lane) * p.KB + b0;
+            for (int j = 0; j < nblk; j += 128)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p.c2_fp8 + blk0 + j));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.c1 + (blk0 >> 8)));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.B + (row0 + lane) * p.r));
+        }
+    }
+}
+
+// Writes this warp's partial of slot sequence number q into reduction slot
+// q % 2 (after the reducer has freed it) and arrives on the slot.
 template <int NT>
-__device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem, const GemvSmem& L, uint64_t* full,
+__device__ __forceinline__ void put_partial(uint8_t* smem, const GemvSmem& L, const GemvBars& B, int q, int warp,
+                                            int lane, const float (&v)[NT][4]) {
+    const int b = q % kRedSlots;
+    if (q >= kRedSlots) mbar_wait(smem_u32(&B.red_empty[b]), ((q / kRedSlots) - 1) & 1, &g_gemv_error);
+    float4* red = reinterpret_cast<float4*>(smem + L.red_off) + (b * kWarps + warp) * NT * 32;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) red[nt * 32 + lane] = make_float4(v[nt][0], v[nt][1], v[nt][2], v[nt][3]);
+    mbar_arrive(smem_u32(&B.red_full[b]));
+}
+
+template <int NT>
+__device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem, const GemvSmem& L, const GemvBars& B,
                                              int cid, int ncl, int n_local, int b0, int nblk, int warp, int lane,
                                              const uint32_t (&xf)[kMaxBw][NT][8]) {
     const int g = lane >> 2, qd = lane & 3;
@@ -356,7 +344,6 @@ __device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem,
     const int nst = p.nstages;
     const uint8_t* lut = smem;
     const uint8_t* stages = smem + kLutBytes;
-    float4* red = reinterpret_cast<float4*>(smem + L.red_off) + warp * NT * 32;  // this warp's [NT][32]
 
     // This CTA's part of X A^T, one 16-rank tile at a time: the rows of A
     // are the MMA's A operand in the same permuted k order as the codes.
@@ -392,10 +379,7 @@ __device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem,
                                   xf[jj][nt][2 * t + 1]);
             }
         }
-        if (rt > 0) bar_wait(kBarRedFree);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) red[nt * 32 + lane] = make_float4(ta[nt][0], ta[nt][1], ta[nt][2], ta[nt][3]);
-        bar_arrive(kBarRedFull);
+        put_partial<NT>(smem, L, B, rt, warp, lane, ta);
     }
 
     const float mean = __ldg(p.mean);
@@ -423,7 +407,7 @@ __device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem,
     for (int i = 0; i < n_local; ++i) {
         const int s = i % nst;
         load_consts(i + 1, c1n, fbn);  // the next unit's: the loads overlap this unit
-        mbar_wait(smem_u32(&full[s]), (i / nst) & 1, &g_gemv_error);
+        mbar_wait(smem_u32(&B.full[s]), (i / nst) & 1, &g_gemv_error);
         const uint8_t* stg = stages + s * p.stage_bytes;
 
         float acc[NT][4];
@@ -466,17 +450,14 @@ __device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem,
                 }
             }
         }
+        mbar_arrive(smem_u32(&B.empty[s]));  // this lane has read the stage
 #pragma unroll
         for (int jj = 0; jj < kMaxBw; ++jj) {
             c1c[jj] = c1n[jj];
             fbc[jj] = fbn[jj];
         }
-        bar_wait(kBarRedFree);  // the producer has read the previous partials
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) red[nt * 32 + lane] = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
-        bar_arrive(kBarRedFull);
+        put_partial<NT>(smem, L, B, RT + i, warp, lane, acc);
     }
-    bar_wait(kBarRedFree);  // pairs with the producer's last release
 }
 
 template <int NT>
@@ -484,11 +465,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemv_nf4(const __grid_constant_
                                                            const __grid_constant__ GemvParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int RT = (p.r + 15) >> 4;
-    const GemvSmem L = gemv_smem(NT, p.stage_bytes, p.nstages, p.cl, RT, p.nslot);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-    uint64_t* slot_full = full + kStages;          // rank 0: a unit's partials have all landed
-    uint64_t* slot_empty = slot_full + kSlotBufs;  // every rank: rank 0 has read the buffer
-    uint64_t* t_full = slot_empty + kSlotBufs;     // rank 0: the T partials have all landed
+    const GemvSmem L = gemv_smem(NT, p.stage_bytes, p.nstages, p.nmax, RT);
+    GemvBars B;
+    B.full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+    B.empty = B.full + kStages;
+    B.red_full = B.empty + kStages;
+    B.red_empty = B.red_full + kRedSlots;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t crank = cluster_ctarank();
@@ -498,13 +480,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemv_nf4(const __grid_constant_
     const int nblk = static_cast<int>(static_cast<int64_t>(crank + 1) * p.KB / p.cl) - b0;
     const int n_local = cid < p.units ? (p.units - 1 - cid) / ncl + 1 : 0;
 
-    // the compute warps' X fragments first: their loads fly during the set-up
+    // the producer arms the barriers and sends off the first copies at once;
+    // the compute warps' X fragment loads fly during the rest of the set-up
+    if (warp == kWarps && lane == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(smem_u32(&B.full[i]), 1);
+            mbar_init(smem_u32(&B.empty[i]), kCompute);   // every compute lane
+        }
+        for (int i = 0; i < kRedSlots; ++i) {
+            mbar_init(smem_u32(&B.red_full[i]), kCompute);
+            mbar_init(smem_u32(&B.red_empty[i]), 32);     // every reducer lane
+        }
+        fence_barrier_init();
+        const int pre = n_local < p.nstages ? n_local : p.nstages;
+        for (int i = 0; i < pre; ++i)
+            issue_unit(&map_codes, p, cid + i * ncl, smem + kLutBytes + i * p.stage_bytes, &B.full[i], b0);
+    }
     uint32_t xf[kMaxBw][NT][8];
     if (warp < kWarps) load_x_frags<NT>(p, b0, nblk, warp, lane, xf);
-    if (tid == 0) {
-        for (int i = 0; i < kStages + 2 * kSlotBufs + 1; ++i) mbar_init(smem_u32(&full[i]), 1);
-        fence_barrier_init();
-    }
     if (tid < 256) {  // the decode table: entry v replicated into words 0..31 of row v
         const uint32_t e = pack_bf16x2(p.q[tid >> 4], p.q[tid & 15]);
         uint4* row = reinterpret_cast<uint4*>(smem + tid * 256);
@@ -512,22 +505,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemv_nf4(const __grid_constant_
         for (int i = 0; i < 8; ++i) row[i] = make_uint4(e, e, e, e);
     }
     __syncthreads();
-    cluster_arrive();  // every CTA's barriers are initialised before any remote traffic
-    cluster_wait();
 
     if (warp == kWarps)
-        producer_warp<NT>(&map_codes, p, smem, L, full, slot_full, slot_empty, t_full, crank, cid, ncl, n_local, b0,
-                          nblk, lane);
-    else if (warp == kWarps + 1) {
-        if (crank == 0) epilogue_warp<NT>(p, smem, L, slot_full, slot_empty, t_full, cid, ncl, n_local, lane);
-    } else
-        compute_warp<NT>(p, smem, L, full, cid, ncl, n_local, b0, nblk, warp, lane, xf);
-    cluster_arrive();  // no CTA leaves while cluster peers may still address its shared memory
+        producer_warp<NT>(&map_codes, p, smem, L, B, cid, ncl, n_local, b0, lane);
+    else if (warp < kWarps)
+        compute_warp<NT>(p, smem, L, B, cid, ncl, n_local, b0, nblk, warp, lane, xf);
+    else
+        prefetch_warp(p, cid, ncl, n_local, b0, nblk, lane);
+    __syncthreads();   // this CTA's sums are complete
+    cluster_arrive();  // ... and every CTA's
+    cluster_wait();
+    final_epilogue<NT>(p, smem, L, crank, cid, ncl, n_local, warp, lane);
+    cluster_arrive();  // no CTA leaves while cluster peers may still read its shared memory
     cluster_wait();
 }
 
 struct Plan {
-    int cl, clusters, row_stride, stage_bytes, nstages, nslot;
+    int cl, clusters, row_stride, stage_bytes, nstages, nmax;
     size_t smem;
 };
 
@@ -583,17 +577,24 @@ bool make_plan(int64_t N, int64_t K, int r, Plan& best) {
         pl.row_stride = static_cast<int>(round_up(maxblk * 32, 128) + 32);  // = 32 mod 128: no bank conflicts
         if (pl.row_stride / 8 > 256) continue;                                 // tensor-map box width
         pl.stage_bytes = static_cast<int>(round_up(kRows * pl.row_stride, 128));
+        // the units of a cluster, for the largest cluster count this size allows
+        const int cl_max = sms / cl;
+        const int nmax_est = static_cast<int>(ceil_div(units, units < cl_max ? units : cl_max));
         pl.nstages = 0;
-        for (int nslot = kSlotBufs; nslot >= 2 && !pl.nstages; nslot /= 2) {
-            for (int ns = kStages; ns >= 3 && !pl.nstages; --ns)
-                if (gemv_smem(NT, pl.stage_bytes, ns, cl, RT, nslot).total <= 227 * 1024) pl.nstages = ns;
-            pl.nslot = nslot;
-        }
+        for (int ns = kStages; ns >= 3 && !pl.nstages; --ns)
+            if (gemv_smem(NT, pl.stage_bytes, ns, nmax_est, RT).total <= 227 * 1024) pl.nstages = ns;
         if (!pl.nstages) continue;
-        pl.smem = gemv_smem(NT, pl.stage_bytes, pl.nstages, cl, RT, pl.nslot).total;
+        pl.nmax = nmax_est;
+        pl.smem = gemv_smem(NT, pl.stage_bytes, pl.nstages, pl.nmax, RT).total;
         const int maxc = max_clusters<NT>(cl, pl.smem);
         if (maxc <= 0) continue;
         pl.clusters = units < maxc ? units : maxc;
+        // fewer clusters fit than assumed: more units each, fewer stages if need be
+        pl.nmax = static_cast<int>(ceil_div(units, pl.clusters));
+        while (pl.nstages >= 3 && gemv_smem(NT, pl.stage_bytes, pl.nstages, pl.nmax, RT).total > 227 * 1024)
+            --pl.nstages;
+        if (pl.nstages < 3) continue;
+        pl.smem = gemv_smem(NT, pl.stage_bytes, pl.nstages, pl.nmax, RT).total;
         const int per = static_cast<int>(ceil_div(units, pl.clusters));
         const double eff = static_cast<double>(units) / (static_cast<double>(pl.clusters) * per) *
                            (static_cast<double>(pl.clusters) * cl / sms);
@@ -677,8 +678,8 @@ cudaError_t launch_fwd_gemv(const uint16_t* X, const Nf4Weight& w, const uint16_
     p.row_stride = pl.row_stride;
     p.stage_bytes = pl.stage_bytes;
     p.nstages = pl.nstages;
-    p.nslot = pl.nslot;
-    const float* q = tables().q;
+    p.nmax = pl.nmax;
+    const float* q = tables(w.qtype).q;
     for (int i = 0; i < 16; ++i) p.q[i] = q[i];
     return two ? launch_gemv<2>(p, pl, st) : launch_gemv<1>(p, pl, st);
 }

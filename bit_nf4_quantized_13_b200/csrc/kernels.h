@@ -6,18 +6,20 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/qlora.h"
+
 namespace qlora {
 
 // quantize.cu
 cudaError_t launch_quantize_nf4_dq(const float* W, int64_t numel, uint8_t* codes, uint8_t* c2_fp8,
                                    float* c1, float* mean, void* ws, int32_t* status,
-                                   cudaStream_t stream);
+                                   cudaStream_t stream, int qtype = QLORA_TYPE_NF4);
 cudaError_t launch_e4m3_encode(const float* x, uint8_t* out, int64_t n, cudaStream_t stream);
 
 // dequant.cu
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,
                               const float* mean, int64_t numel, void* out, int out_dtype,
-                              cudaStream_t stream);
+                              cudaStream_t stream, int qtype = QLORA_TYPE_NF4);
 
 // int8.cu -- block-wise Int8 absmax quantization (eq. 1) and dequantization
 // (eq. 2), block in {32, 64, 128, 256}
@@ -34,6 +36,7 @@ struct Nf4Weight {
     const float* c1;        // N*K/16384 floats (rounded up)
     const float* mean;      // 1 float
     int64_t N, K;
+    int qtype = QLORA_TYPE_NF4;  // the 4-bit data type the codes index
 };
 
 // The skinny rank-r products of the LoRA path

@@ -372,7 +372,7 @@ __global__ void k_e4m3_encode(const float* __restrict__ x, uint8_t* __restrict__
 
 cudaError_t launch_quantize_nf4_dq(const float* W, int64_t numel, uint8_t* codes, uint8_t* c2_fp8,
                                    float* c1, float* mean, void* ws, int32_t* status,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, int qtype) {
     const int64_t nb = ceil_div(numel, kBlock);
     auto* bins = reinterpret_cast<unsigned long long*>(ws);
     int* flag = reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + kBinBytes);
@@ -396,7 +396,7 @@ cudaError_t launch_quantize_nf4_dq(const float* W, int64_t numel, uint8_t* codes
         });
     const int64_t cap = static_cast<int64_t>(num_sms()) * resident;
     const int grid1 = static_cast<int>(want < cap ? want : cap);
-    k_nf4_quantize<<<grid1, kQuantThreads, 0, stream>>>(W, numel, codes, c2, bins, flag, tables());
+    k_nf4_quantize<<<grid1, kQuantThreads, 0, stream>>>(W, numel, codes, c2, bins, flag, tables(qtype));
     note_launches(1);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;

@@ -47,6 +47,13 @@ typedef enum qlora_status {
     QLORA_ERR_TIMEOUT = 6      /* from qlora_device_error: a device-side wait gave up  */
 } qlora_status;
 
+/* The 4-bit data types (section 3.2 builds NF4; FP4 and Int4 are the types
+ * it is compared with): the codes are indices into a sorted table of 16
+ * values in [-1, 1], scaled by the block constant. */
+#define QLORA_TYPE_NF4 0   /* NormalFloat: eq. (4), the default everywhere    */
+#define QLORA_TYPE_FP4 1   /* OCP E2M1 values / 6: 15 distinct, top repeated   */
+#define QLORA_TYPE_INT4 2  /* eq. (1) at 4 bits: k / 7, k = -7..7, top repeated */
+
 #define QLORA_BLOCK 64       /* first-level block: elements per absmax constant  */
 #define QLORA_BLOCK2 256     /* second-level block: constants per FP8 scale       */
 #define QLORA_MAX_RANK 256   /* largest LoRA rank r                              */
@@ -62,6 +69,18 @@ typedef enum qlora_status {
  * Returns QLORA_ERR_INVALID_ARG for a NULL pointer.
  */
 int qlora_nf4_codebook(float out_host[16]);
+
+/*
+ * qlora_codebook -- the 16 values of a 4-bit data type (QLORA_TYPE_*),
+ * ascending, into the HOST array out_host.  NF4 as qlora_nf4_codebook.
+ * FP4: the OCP E2M1 magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6} with both signs,
+ * divided by 6 (15 distinct values; its two zeros are one value), the top
+ * value repeated at index 15.  Int4: k / 7 for k = -7 .. 7, the top value
+ * repeated at index 15.  A repeated value is never chosen by the nearest-
+ * value rule (ties go to the lower index).  QLORA_ERR_INVALID_ARG for a NULL
+ * pointer or an unknown type.
+ */
+int qlora_codebook(int qtype, float out_host[16]);
 
 /*
  * Workspace bytes that qlora_quantize_nf4_dq needs for `numel` weights:
@@ -97,6 +116,33 @@ size_t qlora_quantize_workspace_size(int64_t numel);
 int qlora_quantize_nf4_dq(const float* W, int64_t numel, int block, int block2,
                           uint8_t* codes, uint8_t* c2_fp8, float* c1, float* mean,
                           void* ws, size_t ws_bytes, int32_t* status, void* stream);
+
+/*
+ * qlora_quantize_4bit_dq, qlora_dequantize_4bit, qlora_linear_fwd_4bit,
+ * qlora_linear_bwd_4bit -- the same calls for any of the 4-bit data types:
+ * `qtype` (QLORA_TYPE_*) first, then exactly the arguments of
+ * qlora_quantize_nf4_dq, qlora_dequantize, qlora_linear_fwd and
+ * qlora_linear_bwd, with the same definitions with q_i the type's table
+ * (qlora_codebook).  The NF4 calls are these with QLORA_TYPE_NF4.  An
+ * unknown type returns QLORA_ERR_INVALID_ARG.
+ */
+int qlora_quantize_4bit_dq(int qtype, const float* W, int64_t numel, int block, int block2,
+                           uint8_t* codes, uint8_t* c2_fp8, float* c1, float* mean,
+                           void* ws, size_t ws_bytes, int32_t* status, void* stream);
+int qlora_dequantize_4bit(int qtype, const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,
+                          const float* mean, int64_t numel, int block, int block2,
+                          void* out, int out_dtype, void* stream);
+int qlora_linear_fwd_4bit(int qtype, const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                          const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,
+                          const float* mean, const uint16_t* A, const uint16_t* B, int r,
+                          float s, uint16_t* Y, uint16_t* T_save, void* ws, size_t ws_bytes,
+                          void* stream);
+int qlora_linear_bwd_4bit(int qtype, const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N,
+                          int64_t K, const uint8_t* codes, const uint8_t* c2_fp8,
+                          const float* c1, const float* mean, const uint16_t* A,
+                          const uint16_t* B, int r, float s, const uint16_t* T,
+                          uint16_t* dX, uint16_t* dA, uint16_t* dB, void* ws,
+                          size_t ws_bytes, void* stream);
 
 /*
  * qlora_quantize_nf4_dq_noalloc -- the same quantization as

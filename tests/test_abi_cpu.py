@@ -46,6 +46,8 @@ def test_codebook_matches_oracle_bit_exact(q):
     ref = oracle.nf4_codebook()
     np.testing.assert_array_equal(got.view(np.uint32), ref.view(np.uint32))
     assert q.lib.qlora_nf4_codebook(None) == 1
+    for name, qt in (("nf4", q.TYPE_NF4), ("fp4", q.TYPE_FP4), ("int4", q.TYPE_INT4)):
+        np.testing.assert_array_equal(q.qlora_codebook(qt).view(np.uint32), oracle.codebook(name).view(np.uint32))
 
 
 def test_workspace_sizes(q):
@@ -95,6 +97,12 @@ def test_argument_validation_on_host(q):
     assert L.qlora_int8_quantize(P, 0, 64, None, None, None, None) == 0
     assert L.qlora_int8_dequantize(P, P, 64, 512, P, None) == 2
     assert L.qlora_int8_dequantize(P, P, 64, 64, P + 8, None) == 1
+    # the typed 4-bit entry points refuse unknown types
+    assert L.qlora_quantize_4bit_dq(3, P, 64, 64, 256, P, P, P, P, P, 4096, None, None) == 1
+    assert L.qlora_dequantize_4bit(-1, P, P, P, P, 64, 64, 256, P, 0, None) == 1
+    assert L.qlora_linear_fwd_4bit(9, P, 16, 64, 128, P, P, P, P, P, P, 8, f32(1), P, P, P, 1 << 20, None) == 1
+    assert L.qlora_linear_bwd_4bit(9, P, P, 16, 64, 128, P, P, P, P, P, P, 8, f32(1), None, P, P, P, P, 1 << 20,
+                                   None) == 1
     # the failure-detection self-test refuses limits outside (0, 1 s]
     assert L.qlora_debug_wait_timeout(0, None) == 1
     assert L.qlora_debug_wait_timeout(2_000_000_000, None) == 1

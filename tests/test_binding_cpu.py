@@ -47,12 +47,14 @@ def test_consistent_operands_reach_the_library(fake, M, N, K, r):
     w = weight(N, K)
     Y, T = q.qlora_linear_fwd(bf16(M, K), w, bf16(r, K), bf16(N, r), 0.25)
     assert Y.shape == (M, N) and T.shape == (M, r)
-    name, args = fake.calls[-1]
-    assert name == "qlora_linear_fwd" and args[1:4] == (M, N, K) and args[10] == r
+    name, args = fake.calls[-1]  # the typed entry point: the data type first
+    assert name == "qlora_linear_fwd_4bit" and args[0] == q.TYPE_NF4
+    assert args[2:5] == (M, N, K) and args[11] == r
     dX, dA, dB = q.qlora_linear_bwd(bf16(M, N), bf16(M, K), w, bf16(r, K), bf16(N, r), 0.25, T=T)
     assert dX.shape == (M, K) and dA.shape == (r, K) and dB.shape == (N, r)
     name, args = fake.calls[-1]
-    assert name == "qlora_linear_bwd" and args[2:5] == (M, N, K) and args[11] == r
+    assert name == "qlora_linear_bwd_4bit" and args[0] == q.TYPE_NF4
+    assert args[3:6] == (M, N, K) and args[12] == r
 
 
 def test_disagreeing_operands_are_refused(fake):
@@ -94,7 +96,12 @@ def test_library_status_becomes_an_exception(fake):
 def test_quantize_and_dequantize_buffers_are_checked(fake):
     W = torch.zeros((64, 128), dtype=torch.float32)
     w = q.qlora_quantize_nf4_dq(W)
-    assert fake.calls[-1][0] == "qlora_quantize_nf4_dq" and fake.calls[-1][1][1] == W.numel()
+    assert fake.calls[-1][0] == "qlora_quantize_4bit_dq" and fake.calls[-1][1][0] == q.TYPE_NF4
+    assert fake.calls[-1][1][2] == W.numel()
+    wf = q.qlora_quantize_nf4_dq(W, qtype=q.TYPE_FP4)  # the data type reaches the library and stays with the weight
+    assert fake.calls[-1][1][0] == q.TYPE_FP4 and wf.qtype == q.TYPE_FP4
+    q.qlora_dequantize(wf, torch.float32)
+    assert fake.calls[-1][0] == "qlora_dequantize_4bit" and fake.calls[-1][1][0] == q.TYPE_FP4
     small = q.Nf4Weight(w.codes[:100], w.c2_fp8, w.c1, w.mean, (64, 128))
     with pytest.raises(ValueError):
         q.qlora_quantize_nf4_dq(W, out=small)
