@@ -155,9 +155,9 @@ struct GemvBars {
     uint64_t* red_empty;
 };
 
-// The producer warp of every CTA: refills the stages and reduces the
-// compute warps' partials, slot after slot (T's rank tiles first, then the
-// units), into this CTA's own sums in shared memory.
+// The producer warp of every CTA: issues and refills the stages and reduces
+// the compute warps' partials, slot after slot (the units, then T's rank
+// tiles), into this CTA's own sums in shared memory.
 template <int NT>
 __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const GemvParams& p, uint8_t* smem,
                                               const GemvSmem& L, const GemvBars& B, int cid, int ncl, int n_local,
@@ -168,12 +168,16 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const Gemv
     const float4* red = reinterpret_cast<const float4*>(smem + L.red_off);
     float4* part = reinterpret_cast<float4*>(smem + L.part_off);
     float4* tpart = reinterpret_cast<float4*>(smem + L.tpart_off);
+    if (lane == 0) {
+        const int pre = n_local < nst ? n_local : nst;
+        for (int i = 0; i < pre; ++i) issue_unit(map, p, cid + i * ncl, stages + i * p.stage_bytes, &B.full[i], b0);
+    }
 
-    const int nq = RT + n_local;
+    const int nq = n_local + RT;
 #pragma unroll 1
     for (int q = 0; q < nq; ++q) {
         const int b = q % kRedSlots;
-        const int i = q - RT;  // unit (>= 0) or rank tile (< 0)
+        const int i = q < n_local ? q : -1;  // unit, or one of T's rank tiles after the units
         if (i >= 0 && lane == 0 && i + nst < n_local) {
             // unit i has been read from its stage: refill the stage with unit i + nst
             const int s = i % nst;
@@ -181,7 +185,8 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap* map, const Gemv
                 issue_unit(map, p, cid + (i + nst) * ncl, stages + s * p.stage_bytes, &B.full[s], b0);
         }
         mbar_wait(smem_u32(&B.red_full[b]), (q / kRedSlots) & 1, &g_gemv_error);
-        float4* dst = i >= 0 ? part + static_cast<size_t>(i) * NT * 32 : tpart + static_cast<size_t>(q) * NT * 32;
+        float4* dst = i >= 0 ? part + static_cast<size_t>(i) * NT * 32
+                             : tpart + static_cast<size_t>(q - n_local) * NT * 32;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             float4 sum = red[((b * kWarps + 0) * NT + nt) * 32 + lane];
@@ -306,8 +311,8 @@ __device__ __forceinline__ void load_x_frags(const GemvParams& p, int b0, int nb
 }
 
 // The 16th warp of every CTA pulls into L2 what the other warps will load
-// later: the units' FP8 constants and c1, and the rows of B the epilogue
-// needs.
+// later: the units' FP8 constants and c1, the rows of B the epilogue needs
+// and the rows of A over this CTA's K-slice.
 __device__ __forceinline__ void prefetch_warp(const GemvParams& p, int cid, int ncl, int n_local, int b0, int nblk,
                                               int lane) {
     for (int i = 0; i < n_local; ++i) {
@@ -320,6 +325,11 @@ __device__ __forceinline__ void prefetch_warp(const GemvParams& p, int cid, int 
             asm volatile("prefetch.global.L2 [%0];" ::"l"(p.B + (row0 + lane) * p.r));
         }
     }
+    // the rows of A over this CTA's K-slice (for X A^T after the units)
+    const int64_t k0 = static_cast<int64_t>(b0) * 64, kn = static_cast<int64_t>(nblk) * 64;
+    for (int j = 0; j < p.r; ++j)
+        for (int64_t k = 64 * lane; k < kn; k += 64 * 32)  // one 128-byte line per lane
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.A + j * static_cast<int64_t>(p.K) + k0 + k));
 }
 
 // Writes this warp's partial of slot sequence number q into reduction slot
@@ -344,43 +354,6 @@ __device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem,
     const int nst = p.nstages;
     const uint8_t* lut = smem;
     const uint8_t* stages = smem + kLutBytes;
-
-    // This CTA's part of X A^T, one 16-rank tile at a time: the rows of A
-    // are the MMA's A operand in the same permuted k order as the codes.
-    for (int rt = 0; rt < RT; ++rt) {
-        float ta[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) ta[nt][0] = ta[nt][1] = ta[nt][2] = ta[nt][3] = 0.0f;
-#pragma unroll
-        for (int jj = 0; jj < kMaxBw; ++jj) {
-            const int jloc = warp + kWarps * jj;
-            if (jloc < nblk) {
-                uint4 ra[2][2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int j = 16 * rt + g + 8 * h;
-                    ra[h][0] = ra[h][1] = make_uint4(0, 0, 0, 0);
-                    if (j < p.r) {
-                        const uint4* src = reinterpret_cast<const uint4*>(
-                            p.A + static_cast<int64_t>(j) * p.K + static_cast<int64_t>(b0 + jloc) * 64 + 16 * qd);
-                        ra[h][0] = __ldg(src);
-                        ra[h][1] = __ldg(src + 1);
-                    }
-                }
-                const uint32_t wg[8] = {ra[0][0].x, ra[0][0].y, ra[0][0].z, ra[0][0].w,
-                                        ra[0][1].x, ra[0][1].y, ra[0][1].z, ra[0][1].w};
-                const uint32_t wh[8] = {ra[1][0].x, ra[1][0].y, ra[1][0].z, ra[1][0].w,
-                                        ra[1][1].x, ra[1][1].y, ra[1][1].z, ra[1][1].w};
-#pragma unroll
-                for (int t = 0; t < 4; ++t)
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-                        mma_16816(ta[nt], wg[2 * t], wh[2 * t], wg[2 * t + 1], wh[2 * t + 1], xf[jj][nt][2 * t],
-                                  xf[jj][nt][2 * t + 1]);
-            }
-        }
-        put_partial<NT>(smem, L, B, rt, warp, lane, ta);
-    }
 
     const float mean = __ldg(p.mean);
     const uint32_t lane_off = static_cast<uint32_t>(lane) * 4;
@@ -456,8 +429,46 @@ __device__ __forceinline__ void compute_warp(const GemvParams& p, uint8_t* smem,
             c1c[jj] = c1n[jj];
             fbc[jj] = fbn[jj];
         }
-        put_partial<NT>(smem, L, B, RT + i, warp, lane, acc);
+        put_partial<NT>(smem, L, B, i, warp, lane, acc);
     }
+    // This CTA's part of X A^T, one 16-rank tile at a time, after the units
+    // (the rows of A were pulled into L2 meanwhile): the rows of A are the
+    // MMA's A operand in the same permuted k order as the codes.
+    for (int rt = 0; rt < RT; ++rt) {
+        float ta[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) ta[nt][0] = ta[nt][1] = ta[nt][2] = ta[nt][3] = 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < kMaxBw; ++jj) {
+            const int jloc = warp + kWarps * jj;
+            if (jloc < nblk) {
+                uint4 ra[2][2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int j = 16 * rt + g + 8 * h;
+                    ra[h][0] = ra[h][1] = make_uint4(0, 0, 0, 0);
+                    if (j < p.r) {
+                        const uint4* src = reinterpret_cast<const uint4*>(
+                            p.A + static_cast<int64_t>(j) * p.K + static_cast<int64_t>(b0 + jloc) * 64 + 16 * qd);
+                        ra[h][0] = __ldg(src);
+                        ra[h][1] = __ldg(src + 1);
+                    }
+                }
+                const uint32_t wg[8] = {ra[0][0].x, ra[0][0].y, ra[0][0].z, ra[0][0].w,
+                                        ra[0][1].x, ra[0][1].y, ra[0][1].z, ra[0][1].w};
+                const uint32_t wh[8] = {ra[1][0].x, ra[1][0].y, ra[1][0].z, ra[1][0].w,
+                                        ra[1][1].x, ra[1][1].y, ra[1][1].z, ra[1][1].w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_16816(ta[nt], wg[2 * t], wh[2 * t], wg[2 * t + 1], wh[2 * t + 1], xf[jj][nt][2 * t],
+                                  xf[jj][nt][2 * t + 1]);
+            }
+        }
+        put_partial<NT>(smem, L, B, n_local + rt, warp, lane, ta);
+    }
+
 }
 
 template <int NT>
@@ -492,9 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemv_nf4(const __grid_constant_
             mbar_init(smem_u32(&B.red_empty[i]), 32);     // every reducer lane
         }
         fence_barrier_init();
-        const int pre = n_local < p.nstages ? n_local : p.nstages;
-        for (int i = 0; i < pre; ++i)
-            issue_unit(&map_codes, p, cid + i * ncl, smem + kLutBytes + i * p.stage_bytes, &B.full[i], b0);
+        tma_prefetch_desc(&map_codes);
     }
     uint32_t xf[kMaxBw][NT][8];
     if (warp < kWarps) load_x_frags<NT>(p, b0, nblk, warp, lane, xf);
