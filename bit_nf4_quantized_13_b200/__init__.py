@@ -75,6 +75,11 @@ def _load() -> ctypes.CDLL:
         "qlora_debug_wait_timeout": (i32, [ctypes.c_uint64, vp]),
         "qlora_int8_quantize": (i32, [vp, i64, i32, vp, vp, vp, vp]),
         "qlora_int8_dequantize": (i32, [vp, vp, i64, i32, vp, vp]),
+        "qlora_linear_group_fwd_workspace_size": (sz, [i64, i32, i32]),
+        "qlora_linear_group_bwd_workspace_size": (sz, [i64, i32, i32]),
+        "qlora_linear_group_fwd": (i32, [i32, vp, i64, i64, vp, i32, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
+        "qlora_linear_group_bwd": (i32, [i32, vp, vp, i64, i64, vp, i32, vp, vp, i32, f32, vp, vp, vp, vp,
+                                         vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -339,6 +344,102 @@ def qlora_linear_bwd(dY, X, w: Nf4Weight, A, B, s: float, T=None, dX=None, dA=No
                                           _ptr(ws), ws.numel(), _stream(stream))
     _check("qlora_linear_bwd_4bit", st)
     return dX, dA, dB
+
+
+class _Weight4bit(ctypes.Structure):
+    """The C struct qlora_weight_4bit."""
+    _fields_ = [("codes", ctypes.c_void_p), ("c2_fp8", ctypes.c_void_p), ("c1", ctypes.c_void_p),
+                ("mean", ctypes.c_void_p), ("N", ctypes.c_int64)]
+
+
+def _group_dims(X, ws_, A_cat, B_cat):
+    """(M, K, r, [N_g], descriptor array) of a group call."""
+    torch = _torch()
+    if not 1 <= len(ws_) <= 4:
+        raise ValueError(f"a group holds 1 to 4 linears, got {len(ws_)}")
+    if X.dim() != 2 or A_cat.dim() != 2 or B_cat.dim() != 2:
+        raise ValueError("X, A_cat and B_cat must be 2-D")
+    M, K = (int(d) for d in X.shape)
+    qtype = int(ws_[0].qtype)
+    ns = []
+    for w in ws_:
+        if len(w.shape) != 2 or int(w.shape[1]) != K:
+            raise ValueError(f"every weight must be N_g x {K}, got {w.shape}")
+        if int(w.qtype) != qtype:
+            raise ValueError("the weights of a group share one 4-bit type")
+        _need_weight(w, int(w.shape[0]) * K)
+        ns.append(int(w.shape[0]))
+    G = len(ws_)
+    if int(A_cat.shape[0]) % G:
+        raise ValueError(f"A_cat has {A_cat.shape[0]} rows, not a multiple of {G}")
+    r = int(A_cat.shape[0]) // G
+    _need_shape("A_cat", A_cat, (G * r, K))
+    _need_shape("B_cat", B_cat, (sum(ns), r))
+    _need_dtype(torch.bfloat16, X=X, A_cat=A_cat, B_cat=B_cat)
+    desc = (_Weight4bit * G)(*[_Weight4bit(w.codes.data_ptr(), w.c2_fp8.data_ptr(), w.c1.data_ptr(),
+                                           w.mean.data_ptr(), n) for w, n in zip(ws_, ns)])
+    return M, K, r, ns, qtype, desc
+
+
+def qlora_linear_group_fwd_workspace_size(M, G, r) -> int:
+    return int(_get_lib().qlora_linear_group_fwd_workspace_size(int(M), int(G), int(r)))
+
+
+def qlora_linear_group_bwd_workspace_size(M, G, r) -> int:
+    return int(_get_lib().qlora_linear_group_bwd_workspace_size(int(M), int(G), int(r)))
+
+
+def qlora_linear_group_fwd(X, weights, A_cat, B_cat, s: float, Y=None, T_save=None, ws=None, stream=None):
+    """G linears on the same input (q/k/v, gate/up) as one: Y = [Y_1 .. Y_G]
+    (M x sum N_g) with Y_g = X W_g'^T + s (X A_g^T) B_g^T; A_cat = [A_1; ..],
+    B_cat = [B_1; ..].  Returns (Y, T) with T = [T_1 .. T_G] (M x G r)."""
+    torch = _torch()
+    M, K, r, ns, qtype, desc = _group_dims(X, weights, A_cat, B_cat)
+    G, n_all = len(ns), sum(ns)
+    _need_shape("Y", Y, (M, n_all))
+    _need_shape("T_save", T_save, (M, G * r))
+    _need_dtype(torch.bfloat16, Y=Y, T_save=T_save)
+    _need_cuda(X, A_cat, B_cat, Y, T_save, ws, *[t for w in weights for t in (w.codes, w.c2_fp8, w.c1, w.mean)])
+    if Y is None:
+        Y = torch.empty((M, n_all), dtype=torch.bfloat16, device=X.device)
+    if T_save is None:
+        T_save = torch.empty((M, G * r), dtype=torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = _workspace(qlora_linear_group_fwd_workspace_size(M, G, r), X.device)
+    st = _get_lib().qlora_linear_group_fwd(qtype, _ptr(X), M, K, desc, G, _ptr(A_cat), _ptr(B_cat), r, float(s),
+                                           _ptr(Y), _ptr(T_save), _ptr(ws), ws.numel(), _stream(stream))
+    _check("qlora_linear_group_fwd", st)
+    return Y, T_save
+
+
+def qlora_linear_group_bwd(dY, X, weights, A_cat, B_cat, s: float, T=None, dX=None, dA_cat=None, dB_cat=None,
+                           ws=None, want_dx: bool = True, stream=None):
+    """Gradients of qlora_linear_group_fwd: dX = sum_g dY_g W_g' + U_g A_g,
+    dA_cat = [dA_1; ..], dB_cat = [dB_1; ..]; no gradient for the weights."""
+    torch = _torch()
+    M, K, r, ns, qtype, desc = _group_dims(X, weights, A_cat, B_cat)
+    G, n_all = len(ns), sum(ns)
+    _need_shape("dY", dY, (M, n_all))
+    _need_shape("T", T, (M, G * r))
+    _need_shape("dX", dX, (M, K))
+    _need_shape("dA_cat", dA_cat, (G * r, K))
+    _need_shape("dB_cat", dB_cat, (n_all, r))
+    _need_dtype(torch.bfloat16, dY=dY, T=T, dX=dX, dA_cat=dA_cat, dB_cat=dB_cat)
+    _need_cuda(dY, X, A_cat, B_cat, T, dX, dA_cat, dB_cat, ws,
+               *[t for w in weights for t in (w.codes, w.c2_fp8, w.c1, w.mean)])
+    if want_dx and dX is None:
+        dX = torch.empty((M, K), dtype=torch.bfloat16, device=X.device)
+    if dA_cat is None:
+        dA_cat = torch.empty((G * r, K), dtype=torch.bfloat16, device=X.device)
+    if dB_cat is None:
+        dB_cat = torch.empty((n_all, r), dtype=torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = _workspace(qlora_linear_group_bwd_workspace_size(M, G, r), X.device)
+    st = _get_lib().qlora_linear_group_bwd(qtype, _ptr(dY), _ptr(X), M, K, desc, G, _ptr(A_cat), _ptr(B_cat), r,
+                                           float(s), _ptr(T), _ptr(dX if want_dx else None), _ptr(dA_cat),
+                                           _ptr(dB_cat), _ptr(ws), ws.numel(), _stream(stream))
+    _check("qlora_linear_group_bwd", st)
+    return dX, dA_cat, dB_cat
 
 
 def qlora_fp8_e4m3_encode(x, out=None, stream=None):

@@ -243,6 +243,121 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N
                                  ws, ws_bytes, stream);
 }
 
+size_t qlora_linear_group_fwd_workspace_size(int64_t M, int G, int r) {
+    if (M < 0 || G < 1 || G > kMaxGroupLinears || r < 1 || static_cast<int64_t>(G) * r > QLORA_MAX_RANK) return 0;
+    return align256(static_cast<size_t>(M) * G * r * 2) + pair_gemm_workspace();
+}
+
+size_t qlora_linear_group_bwd_workspace_size(int64_t M, int G, int r) {
+    if (M < 0 || G < 1 || G > kMaxGroupLinears || r < 1 || static_cast<int64_t>(G) * r > QLORA_MAX_RANK) return 0;
+    return 2 * align256(static_cast<size_t>(M) * G * r * 2) + pair_gemm_workspace();
+}
+
+}  // extern "C"
+
+namespace {
+
+// Validates a group's descriptors and fills `g`; QLORA_OK or the error.
+int check_group(int qtype, int64_t M, int64_t K, const qlora_weight_4bit* W, int G, int r, Nf4Group* g) {
+    if (!valid_qtype(qtype) || !W || M < 0 || K < 1 || r < 1 || G < 1) return QLORA_ERR_INVALID_ARG;
+    if (G > kMaxGroupLinears || static_cast<int64_t>(G) * r > QLORA_MAX_RANK || K % QLORA_BLOCK != 0 || r % 8 != 0)
+        return QLORA_ERR_UNSUPPORTED;
+    g->G = G;
+    for (int i = 0; i < G; ++i) {
+        if (check_weight(W[i].codes, W[i].c2_fp8, W[i].c1, W[i].mean) != QLORA_OK || W[i].N < 1)
+            return QLORA_ERR_INVALID_ARG;
+        if (check_linear(M, W[i].N, K, r) != QLORA_OK) return QLORA_ERR_UNSUPPORTED;
+        g->w[i] = Nf4Weight{W[i].codes, W[i].c2_fp8, W[i].c1, W[i].mean, W[i].N, K, qtype};
+    }
+    int64_t n_all = 0;
+    for (int i = 0; i < G; ++i) n_all += W[i].N;
+    if (M > 0 && (!pair_group_supported(M, *g, r) || !lora_tc_supported(M, n_all, K, G * r)))
+        return QLORA_ERR_UNSUPPORTED;
+    return QLORA_OK;
+}
+
+int64_t group_n(const Nf4Group& g) {
+    int64_t n = 0;
+    for (int i = 0; i < g.G; ++i) n += g.w[i].N;
+    return n;
+}
+
+int pair_status(cudaError_t e) { return e == cudaErrorNotSupported ? QLORA_ERR_UNSUPPORTED : cuda_status(e); }
+
+}  // namespace
+
+extern "C" {
+
+int qlora_linear_group_fwd(int qtype, const uint16_t* X, int64_t M, int64_t K, const qlora_weight_4bit* W, int G,
+                           const uint16_t* A_cat, const uint16_t* B_cat, int r, float s, uint16_t* Y,
+                           uint16_t* T_save, void* ws, size_t ws_bytes, void* stream) {
+    Nf4Group g{};
+    const int st = check_group(qtype, M, K, W, G, r, &g);
+    if (st != QLORA_OK) return st;
+    if (!ok_ptr(A_cat) || !ok_ptr(B_cat) || (M > 0 && (!ok_ptr(X) || !ok_ptr(Y)))) return QLORA_ERR_INVALID_ARG;
+    if (T_save && !aligned16(T_save)) return QLORA_ERR_INVALID_ARG;
+    if (M == 0) return QLORA_OK;
+    if (!ws || !aligned16(ws) || ws_bytes < qlora_linear_group_fwd_workspace_size(M, G, r)) return QLORA_ERR_WORKSPACE;
+    const int rc = G * r;
+    const size_t t_bytes = align256(static_cast<size_t>(M) * rc * 2);
+    uint16_t* T = T_save ? T_save : reinterpret_cast<uint16_t*>(ws);
+    cudaStream_t cs = as_stream(stream);
+    // every adapter's T in one rank-(G r) product: column g r + j is s X A_g[j]^T
+    cudaError_t e = lora_xat(X, A_cat, M, group_n(g), K, rc, s, T, cs);
+    if (e != cudaSuccess) return cuda_status(e);
+    return pair_status(launch_fwd_gemm_pair_group(X, g, T, B_cat, M, r, Y, reinterpret_cast<char*>(ws) + t_bytes,
+                                                  ws_bytes - t_bytes, cs));
+}
+
+int qlora_linear_group_bwd(int qtype, const uint16_t* dY, const uint16_t* X, int64_t M, int64_t K,
+                           const qlora_weight_4bit* W, int G, const uint16_t* A_cat, const uint16_t* B_cat, int r,
+                           float s, const uint16_t* T, uint16_t* dX, uint16_t* dA_cat, uint16_t* dB_cat, void* ws,
+                           size_t ws_bytes, void* stream) {
+    Nf4Group g{};
+    const int st = check_group(qtype, M, K, W, G, r, &g);
+    if (st != QLORA_OK) return st;
+    if (!ok_ptr(A_cat) || !ok_ptr(B_cat) || !ok_ptr(dA_cat) || !ok_ptr(dB_cat)) return QLORA_ERR_INVALID_ARG;
+    if (M > 0 && (!ok_ptr(dY) || !ok_ptr(X))) return QLORA_ERR_INVALID_ARG;
+    if ((T && !aligned16(T)) || (dX && !aligned16(dX))) return QLORA_ERR_INVALID_ARG;
+    const int rc = G * r;
+    const int64_t n_all = group_n(g);
+    cudaStream_t cs = as_stream(stream);
+    if (M == 0) {  // empty batch: the adapter gradients are zero
+        cudaError_t e = cudaMemsetAsync(dA_cat, 0, static_cast<size_t>(rc) * K * 2, cs);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dB_cat, 0, static_cast<size_t>(n_all) * r * 2, cs);
+        return cuda_status(e);
+    }
+    if (!ws || !aligned16(ws) || ws_bytes < qlora_linear_group_bwd_workspace_size(M, G, r)) return QLORA_ERR_WORKSPACE;
+    const size_t mr = align256(static_cast<size_t>(M) * rc * 2);
+    uint16_t* U = reinterpret_cast<uint16_t*>(ws);
+    uint16_t* Tw = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + mr);
+    cudaError_t e = cudaSuccess;
+    if (!T) {
+        e = lora_xat(X, A_cat, M, n_all, K, rc, s, Tw, cs);
+        T = Tw;
+    }
+    // U_g = s dY_g B_g into columns g r .. of U; dY_g is a column block of dY
+    int64_t n0 = 0;
+    for (int i = 0; i < G && e == cudaSuccess; ++i) {
+        e = launch_lora_dyb_tc(dY + n0, B_cat + n0 * r, M, g.w[i].N, r, s, U + static_cast<int64_t>(i) * r, cs, n_all,
+                               rc);
+        n0 += g.w[i].N;
+    }
+    if (e == cudaSuccess && dX) {
+        e = launch_bwd_dx_gemm_pair_group(dY, g, U, A_cat, M, r, dX, reinterpret_cast<char*>(ws) + 2 * mr,
+                                          ws_bytes - 2 * mr, cs);
+        if (e == cudaErrorNotSupported) return QLORA_ERR_UNSUPPORTED;
+    }
+    // dA_g = U_g^T X for all g at once (rows of dA_cat); dB_g = dY_g^T T_g
+    if (e == cudaSuccess) e = launch_lora_da_tc(X, U, M, K, rc, dA_cat, cs);
+    n0 = 0;
+    for (int i = 0; i < G && e == cudaSuccess; ++i) {
+        e = launch_lora_db_tc(dY + n0, T + static_cast<int64_t>(i) * r, M, g.w[i].N, r, dB_cat + n0 * r, cs, n_all, rc);
+        n0 += g.w[i].N;
+    }
+    return cuda_status(e);
+}
+
 int qlora_device_error(int reset) {
     const int a = pair_device_error(reset);
     const int b = lora_device_error(reset);

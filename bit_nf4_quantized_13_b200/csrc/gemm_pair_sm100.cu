@@ -93,11 +93,20 @@ constexpr int kSlotFloats = kRowsPair * kTileTok;
 constexpr int kFlagCount = 2 * kDqWarps;            // warps of both CTAs that store a slot
 constexpr int kMinStagesPerPair = 8;
 
+constexpr int kMaxGroups = 4;  // linears sharing one input, stacked along N
+
 struct PairParams {
-    const uint8_t* codes;   // W codes, N x K/2 (row-major, two k per byte)
-    const uint8_t* c2_fp8;  // N x K/64
-    const float* c1;
-    const float* mean;
+    // the frozen weights: G linears stacked along N (rows gstart[g] ..
+    // gstart[g+1] - 1 of the product belong to linear g), each its own four
+    // NF4 buffers (codes N_g x K/2 row-major, two k per byte; N_g x K/64
+    // FP8 constants; c1; mean)
+    const uint8_t* codes[kMaxGroups];
+    const uint8_t* c2_fp8[kMaxGroups];
+    const float* c1[kMaxGroups];
+    const float* mean[kMaxGroups];
+    int gstart[kMaxGroups + 1];
+    int G;
+    int r_lora_off;         // forward: T columns of linear g start at g * r_lora_off
     uint16_t* out;          // forward: Y (M x N); backward: dX (M x K)
     int M;                  // tokens
     int rows;               // output rows of the product: N forward, K backward
@@ -120,6 +129,15 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
+}
+
+// The linear holding row n of the stacked weights.
+__device__ __forceinline__ int group_of(const PairParams& p, int64_t n) {
+    int g = 0;
+#pragma unroll
+    for (int i = 1; i < kMaxGroups; ++i)
+        if (i < p.G && n >= p.gstart[i]) g = i;
+    return g;
 }
 
 struct Pipe {
@@ -267,7 +285,9 @@ __device__ void role_tma(const Pipe& P, const PairParams& p, const Range& R, con
             const bool lora = kb >= p.kb_w;
             if (P.rank == 0) mbar_arrive_expect_tx(P.full_b(s), lora ? kTxLora : kTxWeight);
             const CUtensorMap* act = lora ? tm_lact : tm_act;
-            const int x = lora ? (kb - p.kb_w) * kBK : kb * kBK;
+            // forward: the tile's linear picks its own columns of T
+            const int t_off = (!kBwd && lora) ? group_of(p, sg.row0) * p.r_lora_off : 0;
+            const int x = lora ? t_off + (kb - p.kb_w) * kBK : kb * kBK;
             for (int sub = 0; sub < kSubs; ++sub)
                 tma_load_2d_pair(P.sB(s, sub), act, bar, x,
                                  sg.t0 + sub * kSubTok + static_cast<int>(P.rank) * kHalfTok);
@@ -602,12 +622,11 @@ __device__ __forceinline__ void seg_epilogue(const Pipe& P, const PairParams& p,
 // outputs of every earlier segment not yet done, so the MMAs of the next
 // segment find the first stages ready once the accumulators are free.
 template <bool kBwd>
-__device__ __forceinline__ void role_convert(const Pipe& P, const PairParams& p, const Range& R, int warp, int lane,
-                                             int /*unused*/ = 0) {
+__device__ __forceinline__ void role_convert(const Pipe& P, const PairParams& p, const Range& R, int warp,
+                                             int lane) {
     const int quarter = warp & 3;
     const int part = (warp - 2) >> 2;
     const int t = quarter * 32 + lane;  // this lane's run within a stage
-    const float mu = *p.mean;
     const uint32_t full_a_leader0 = cluster_map(P.full_a(0), 0);
     const int n_local = pair_stages(p, R);
     bool ok = true;
@@ -633,12 +652,13 @@ __device__ __forceinline__ void role_convert(const Pipe& P, const PairParams& p,
     SegCache cload, cconv;
     uint4 cb0 = make_uint4(0u, 0u, 0u, 0u), cb1 = cb0;
     uint32_t sbyte = 0u;
-    float sc1 = 0.0f;
+    float sc1 = 0.0f, smu = 0.0f;
     auto issue = [&](int local) {
         cb0 = make_uint4(0u, 0u, 0u, 0u);
         cb1 = cb0;
         sbyte = 0u;
         sc1 = 0.0f;
+        smu = 0.0f;
         if (local >= n_local) return;
         int kb;
         seg_for(cload, local, kb);
@@ -646,12 +666,15 @@ __device__ __forceinline__ void role_convert(const Pipe& P, const PairParams& p,
         int64_t n, kcol;
         int arow, aoff;
         if (!task_of<kBwd>(p, kb, cload.my_row0, t, n, kcol, arow, aoff)) return;
-        const uint8_t* src = p.codes + n * (p.K / 2) + kcol / 2;
+        const int g = group_of(p, n);
+        const int64_t nl = n - p.gstart[g];  // the row within linear g
+        const uint8_t* src = p.codes[g] + nl * (p.K / 2) + kcol / 2;
         cb0 = ldg_nc_v4(src);
         cb1 = ldg_nc_v4(src + 16);
-        const int64_t blk = n * (p.K / kBK) + kcol / kBK;
-        sbyte = __ldg(p.c2_fp8 + blk);
-        sc1 = __ldg(p.c1 + (blk >> 8));
+        const int64_t blk = nl * (p.K / kBK) + kcol / kBK;
+        sbyte = __ldg(p.c2_fp8[g] + blk);
+        sc1 = __ldg(p.c1[g] + (blk >> 8));
+        smu = __ldg(p.mean[g]);
     };
 
     issue(part);
@@ -667,7 +690,7 @@ __device__ __forceinline__ void role_convert(const Pipe& P, const PairParams& p,
         if (weight) {
             const bool valid = task_of<kBwd>(p, kb, cconv.my_row0, t, n, kcol, arow, aoff);
             // runs outside W are zero (in the backward they are part of the contraction)
-            const float sc = valid ? dq_constant(static_cast<uint8_t>(sbyte), sc1, mu) : 0.0f;
+            const float sc = valid ? dq_constant(static_cast<uint8_t>(sbyte), sc1, smu) : 0.0f;
             convert_run(cb0, cb1, sc, p.q, v);
         }
         if (!warp_wait(P.empty(s), ph ^ 1u, lane)) return;
@@ -864,10 +887,14 @@ cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& ml, const CUte
 
 PairParams base_params(const Nf4Weight& w, int64_t M, int r, uint16_t* out, bool bwd) {
     PairParams p{};
-    p.codes = w.codes;
-    p.c2_fp8 = w.c2_fp8;
-    p.c1 = w.c1;
-    p.mean = w.mean;
+    p.G = 1;
+    p.codes[0] = w.codes;
+    p.c2_fp8[0] = w.c2_fp8;
+    p.c1[0] = w.c1;
+    p.mean[0] = w.mean;
+    p.gstart[0] = 0;
+    p.gstart[1] = static_cast<int>(w.N);
+    p.r_lora_off = 0;
     p.out = out;
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(w.N);
@@ -935,6 +962,67 @@ cudaError_t launch_bwd_dx_gemm_pair(const uint16_t* dY, const Nf4Weight& w, cons
     if (!make_map_bf16(&ma, dY, static_cast<uint64_t>(w.N), static_cast<uint64_t>(M), kBK, kHalfTok) ||
         !make_map_bf16(&ml, U, static_cast<uint64_t>(r), static_cast<uint64_t>(M), kBK, kHalfTok) ||
         !make_map_bf16(&mw, A, static_cast<uint64_t>(w.K), static_cast<uint64_t>(r), 64, kBK))
+        return cudaErrorInvalidValue;
+    return launch_pair<true>(ma, ml, mw, p, ws, ws_bytes, st);
+}
+
+bool pair_group_supported(int64_t M, const Nf4Group& g, int r) {
+    if (g.G < 1 || g.G > kMaxGroups || r < 8 || r % 8 != 0 || g.G * r > 256) return false;
+    int64_t n = 0;
+    for (int i = 0; i < g.G; ++i) {
+        if (g.w[i].N < 1 || g.w[i].N % kRowsPair != 0 || g.w[i].K != g.w[0].K || g.w[i].qtype != g.w[0].qtype)
+            return false;
+        n += g.w[i].N;
+    }
+    Nf4Weight all = g.w[0];
+    all.N = n;
+    return n < (int64_t(1) << 31) && pair_gemm_supported(M, all, g.G * r, true);
+}
+
+// The stacked weight: rows gstart[i] .. of the product are linear i's.
+PairParams group_params(const Nf4Group& g, int64_t M, int r_slabs, uint16_t* out, bool bwd) {
+    Nf4Weight all = g.w[0];
+    int64_t n = 0;
+    for (int i = 0; i < g.G; ++i) n += g.w[i].N;
+    all.N = n;
+    PairParams p = base_params(all, M, r_slabs, out, bwd);
+    p.G = g.G;
+    int64_t start = 0;
+    for (int i = 0; i < g.G; ++i) {
+        p.codes[i] = g.w[i].codes;
+        p.c2_fp8[i] = g.w[i].c2_fp8;
+        p.c1[i] = g.w[i].c1;
+        p.mean[i] = g.w[i].mean;
+        p.gstart[i] = static_cast<int>(start);
+        start += g.w[i].N;
+    }
+    p.gstart[g.G] = static_cast<int>(start);
+    return p;
+}
+
+cudaError_t launch_fwd_gemm_pair_group(const uint16_t* X, const Nf4Group& g, const uint16_t* T, const uint16_t* B_cat,
+                                       int64_t M, int r, uint16_t* Y, void* ws, size_t ws_bytes, cudaStream_t st) {
+    PairParams p = group_params(g, M, r, Y, false);
+    p.r_lora_off = r;
+    const int64_t K = g.w[0].K;
+    CUtensorMap ma, ml, mw;
+    if (!make_map_bf16(&ma, X, static_cast<uint64_t>(K), static_cast<uint64_t>(M), kBK, kHalfTok) ||
+        !make_map_bf16(&ml, T, static_cast<uint64_t>(g.G) * r, static_cast<uint64_t>(M), kBK, kHalfTok) ||
+        !make_map_bf16(&mw, B_cat, static_cast<uint64_t>(r), static_cast<uint64_t>(p.N), kBK, kRowsCta))
+        return cudaErrorInvalidValue;
+    return launch_pair<false>(ma, ml, mw, p, ws, ws_bytes, st);
+}
+
+cudaError_t launch_bwd_dx_gemm_pair_group(const uint16_t* dY, const Nf4Group& g, const uint16_t* U,
+                                          const uint16_t* A_cat, int64_t M, int r, uint16_t* dX, void* ws,
+                                          size_t ws_bytes, cudaStream_t st) {
+    const int rc = g.G * r;  // the LoRA contraction: every linear's rank
+    PairParams p = group_params(g, M, rc, dX, true);
+    const int64_t K = g.w[0].K;
+    CUtensorMap ma, ml, mw;
+    if (!make_map_bf16(&ma, dY, static_cast<uint64_t>(p.N), static_cast<uint64_t>(M), kBK, kHalfTok) ||
+        !make_map_bf16(&ml, U, static_cast<uint64_t>(rc), static_cast<uint64_t>(M), kBK, kHalfTok) ||
+        !make_map_bf16(&mw, A_cat, static_cast<uint64_t>(K), static_cast<uint64_t>(rc), 64, kBK))
         return cudaErrorInvalidValue;
     return launch_pair<true>(ma, ml, mw, p, ws, ws_bytes, st);
 }

@@ -50,11 +50,11 @@ bool lora_tc_supported(int64_t M, int64_t N, int64_t K, int r);
 cudaError_t launch_lora_xat_tc(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, float s,
                                uint16_t* T, cudaStream_t stream);
 cudaError_t launch_lora_dyb_tc(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t N, int r, float s,
-                               uint16_t* U, cudaStream_t stream);
+                               uint16_t* U, cudaStream_t stream, int64_t ld_dy = 0, int ld_u = 0);
 cudaError_t launch_lora_da_tc(const uint16_t* X, const uint16_t* U, int64_t M, int64_t K, int r, uint16_t* dA,
                               cudaStream_t stream);
 cudaError_t launch_lora_db_tc(const uint16_t* dY, const uint16_t* T, int64_t M, int64_t N, int r, uint16_t* dB,
-                              cudaStream_t stream);
+                              cudaStream_t stream, int64_t ld_dy = 0, int64_t ld_t = 0);
 int lora_device_error(int reset);
 // gemm_pair_sm100.cu: a kernel whose one bounded wait is never satisfied
 // (records QLORA_ERR_TIMEOUT after limit_ns)
@@ -91,6 +91,23 @@ cudaError_t launch_bwd_dx_gemm_pair(const uint16_t* dY, const Nf4Weight& w, cons
                                     int64_t M, int r, uint16_t* dX, void* ws, size_t ws_bytes,
                                     cudaStream_t stream);
 int pair_device_error(int reset);
+
+// Linears that read the same input (q/k/v, gate/up), stacked along N: the
+// forward and the dX GEMM of the whole group in one launch each.  Every
+// N_g a multiple of 256, at most 4 linears, G * r <= 256.
+//   forward:  Y[:, n_g ..] = X W_g'^T + T[:, g r ..] B_g^T     (T: M x G r)
+//   backward: dX = sum_g dY[:, n_g ..] W_g' + U A_cat          (U: M x G r)
+constexpr int kMaxGroupLinears = 4;
+struct Nf4Group {
+    Nf4Weight w[kMaxGroupLinears];
+    int G;
+};
+bool pair_group_supported(int64_t M, const Nf4Group& g, int r);
+cudaError_t launch_fwd_gemm_pair_group(const uint16_t* X, const Nf4Group& g, const uint16_t* T, const uint16_t* B_cat,
+                                       int64_t M, int r, uint16_t* Y, void* ws, size_t ws_bytes, cudaStream_t stream);
+cudaError_t launch_bwd_dx_gemm_pair_group(const uint16_t* dY, const Nf4Group& g, const uint16_t* U,
+                                          const uint16_t* A_cat, int64_t M, int r, uint16_t* dX, void* ws,
+                                          size_t ws_bytes, cudaStream_t stream);
 
 // gemv_sm100.cu -- the small-batch forward (1 <= M <= 16): T and Y in one
 // kernel that streams the weight once; T is written to T_save when it is not

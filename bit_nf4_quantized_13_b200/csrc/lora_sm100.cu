@@ -46,7 +46,8 @@ constexpr int kABytes = kRows * kBK * 2;  // 16 KiB
 constexpr int kMaxSmem = 200 * 1024;
 
 struct SkinnyParams {
-    uint16_t* out;  // rows x r bf16, or r x rows when transposed
+    uint16_t* out;  // rows x r bf16 (row pitch ldo), or r x rows when transposed
+    int ldo;
     float scale;
     int transposed;
     int rows;      // output rows
@@ -201,7 +202,7 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                     o[2 * static_cast<int64_t>(p.rows)] = static_cast<uint16_t>(hi & 0xffffu);
                     o[3 * static_cast<int64_t>(p.rows)] = static_cast<uint16_t>(hi >> 16);
                 } else {
-                    *reinterpret_cast<uint2*>(p.out + static_cast<int64_t>(row) * p.r + c) = make_uint2(lo, hi);
+                    *reinterpret_cast<uint2*>(p.out + static_cast<int64_t>(row) * p.ldo + c) = make_uint2(lo, hi);
                 }
             }
         }
@@ -217,12 +218,14 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
 // ------------------------------------------------------------------ host
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() { return tensor_map_encoder(); }
 
+// Row-major bf16 matrix (outer x inner, rows `pitch` elements apart; 0 =
+// inner), 128-byte swizzled boxes of box_inner x box_outer.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-              uint32_t box_outer) {
+              uint32_t box_outer, uint64_t pitch = 0) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {inner * 2};
+    cuuint64_t strides[1] = {(pitch ? pitch : inner) * 2};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
@@ -262,12 +265,13 @@ Plan plan(int64_t rows, int64_t ctr, int r, bool b_mn) {
 
 template <bool A_MN, bool B_MN>
 cudaError_t run(const Plan& pl, const CUtensorMap& ma, const CUtensorMap& mb, int64_t rows, int r, float scale,
-                uint16_t* out, bool transposed, cudaStream_t st) {
+                uint16_t* out, bool transposed, cudaStream_t st, int ldo = 0) {
     static ContextMemo<int> attr_memo;
     const cudaError_t attr = ensure_smem_limit(attr_memo, k_lora_tc<A_MN, B_MN>, kMaxSmem + 2048);
     if (attr != cudaSuccess) return attr;
     SkinnyParams p;
     p.out = out;
+    p.ldo = ldo ? ldo : r;
     p.scale = scale;
     p.transposed = transposed ? 1 : 0;
     p.rows = static_cast<int>(rows);
@@ -312,12 +316,14 @@ cudaError_t launch_lora_xat_tc(const uint16_t* X, const uint16_t* A, int64_t M, 
 }
 
 // U = bf16(s dY B): A operand dY (K-major over n), B operand B^T (MN-major).
+// dY and U may be column blocks of wider matrices (row pitches ld_dy, ld_u).
 cudaError_t launch_lora_dyb_tc(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t N, int r, float s,
-                               uint16_t* U, cudaStream_t st) {
+                               uint16_t* U, cudaStream_t st, int64_t ld_dy, int ld_u) {
     const Plan pl = plan(M, N, r, true);
     CUtensorMap ma, mb;
-    if (!make_map(&ma, dY, N, M, kBK, kRows) || !make_map(&mb, B, r, N, 64, kBK)) return cudaErrorInvalidValue;
-    return run<false, true>(pl, ma, mb, M, r, s, U, false, st);
+    if (!make_map(&ma, dY, N, M, kBK, kRows, static_cast<uint64_t>(ld_dy)) || !make_map(&mb, B, r, N, 64, kBK))
+        return cudaErrorInvalidValue;
+    return run<false, true>(pl, ma, mb, M, r, s, U, false, st, ld_u);
 }
 
 // dA = bf16(U^T X) computed as dA^T[k][j] = sum_m X[m][k] U[m][j]: both MN-major.
@@ -330,11 +336,14 @@ cudaError_t launch_lora_da_tc(const uint16_t* X, const uint16_t* U, int64_t M, i
 }
 
 // dB = bf16(dY^T T), dB[n][j] = sum_m dY[m][n] T[m][j]: both MN-major.
+// dY and T may be column blocks of wider matrices (row pitches ld_dy, ld_t).
 cudaError_t launch_lora_db_tc(const uint16_t* dY, const uint16_t* T, int64_t M, int64_t N, int r, uint16_t* dB,
-                              cudaStream_t st) {
+                              cudaStream_t st, int64_t ld_dy, int64_t ld_t) {
     const Plan pl = plan(N, M, r, true);
     CUtensorMap ma, mb;
-    if (!make_map(&ma, dY, N, M, 64, kBK) || !make_map(&mb, T, r, M, 64, kBK)) return cudaErrorInvalidValue;
+    if (!make_map(&ma, dY, N, M, 64, kBK, static_cast<uint64_t>(ld_dy)) ||
+        !make_map(&mb, T, r, M, 64, kBK, static_cast<uint64_t>(ld_t)))
+        return cudaErrorInvalidValue;
     return run<true, true>(pl, ma, mb, N, r, 1.0f, dB, false, st);
 }
 

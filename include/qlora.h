@@ -189,9 +189,10 @@ int qlora_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c
 /*
  * Workspace bytes for qlora_linear_fwd / qlora_linear_bwd.  The forward
  * needs M*r*2 bytes for T (used when T_save is NULL); the backward needs U
- * and T (M*r*2 bytes each, 256-byte aligned) plus, for dX, the transposed
- * copy of the weight its GEMM reads (about 1.1 bytes per weight).  A
- * workspace of the larger size serves both.
+ * and T (M*r*2 bytes each, 256-byte aligned).  Both add the GEMM's scratch
+ * for output tiles whose contraction is split between SM pairs: one 512 KiB
+ * fp32 slot per pair of SMs of the current device plus a few flags (about
+ * 37 MiB on a 148-SM part).  A workspace of the larger size serves both.
  */
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int r);
 size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r);
@@ -234,6 +235,56 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, int64_t N
                      const uint16_t* B, int r, float s, const uint16_t* T,
                      uint16_t* dX, uint16_t* dA, uint16_t* dB, void* ws,
                      size_t ws_bytes, void* stream);
+
+/*
+ * The frozen 4-bit weight of one linear: the four device buffers
+ * qlora_quantize_4bit_dq writes for an N x K row-major weight.
+ */
+typedef struct qlora_weight_4bit {
+    const uint8_t* codes;  /* N*K/2 bytes      */
+    const uint8_t* c2_fp8; /* N*K/64 bytes     */
+    const float* c1;       /* ceil(N*K/16384)  */
+    const float* mean;     /* 1 float          */
+    int64_t N;             /* output features  */
+} qlora_weight_4bit;
+
+/*
+ * qlora_linear_group_fwd / qlora_linear_group_bwd -- G QLoRA linears that
+ * read the same input (an attention block's q, k and v projections; an MLP's
+ * gate and up projections), each with its own frozen weight W_g (N_g x K,
+ * all of one 4-bit type) and its own rank-r adapter (A_g, B_g), run as one:
+ * the products are exactly those of G qlora_linear_fwd / _bwd calls (same
+ * definitions, same rounding points), stacked.  Buffers:
+ *   W      in : host array of G descriptors (device buffers inside).
+ *   A_cat  in : (G r) x K bf16, A_1 .. A_G stacked by rows.
+ *   B_cat  in : (sum N_g) x r bf16, B_1 .. B_G stacked by rows.
+ *   Y     out : M x (sum N_g) bf16, Y_g in columns n_g .. n_g + N_g - 1
+ *               (n_g = N_1 + .. + N_{g-1}).
+ *   T_save / T: M x (G r) bf16, T_g in columns g r .. (nullable as in the
+ *               single calls).
+ *   dY     in : M x (sum N_g), laid out like Y.
+ *   dX    out : M x K = sum_g dY_g W_g' + U_g A_g, one bf16 rounding of the
+ *               fp32 sum (nullable: skipped).
+ *   dA_cat out: (G r) x K, dA_g stacked like A_cat.
+ *   dB_cat out: (sum N_g) x r, dB_g stacked like B_cat.
+ * Requires 1 <= G <= 4, every N_g a multiple of 256, K % 64 == 0, r % 8 == 0
+ * and G r <= 256 (else QLORA_ERR_UNSUPPORTED; use the single calls), M >= 0.
+ * The frozen-weight GEMM of the group is one kernel over the stacked weight,
+ * its dX GEMM one kernel whose contraction runs over all G weights and the
+ * G r adapter columns.  Workspace: the _workspace_size functions (fwd: T;
+ * bwd: U and T, each M x G r bf16; both plus the GEMM scratch).
+ */
+size_t qlora_linear_group_fwd_workspace_size(int64_t M, int G, int r);
+size_t qlora_linear_group_bwd_workspace_size(int64_t M, int G, int r);
+int qlora_linear_group_fwd(int qtype, const uint16_t* X, int64_t M, int64_t K,
+                           const qlora_weight_4bit* W, int G, const uint16_t* A_cat,
+                           const uint16_t* B_cat, int r, float s, uint16_t* Y,
+                           uint16_t* T_save, void* ws, size_t ws_bytes, void* stream);
+int qlora_linear_group_bwd(int qtype, const uint16_t* dY, const uint16_t* X, int64_t M,
+                           int64_t K, const qlora_weight_4bit* W, int G,
+                           const uint16_t* A_cat, const uint16_t* B_cat, int r, float s,
+                           const uint16_t* T, uint16_t* dX, uint16_t* dA_cat,
+                           uint16_t* dB_cat, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * qlora_fp8_e4m3_encode -- the FP8 encoder the double quantization uses

@@ -57,6 +57,10 @@ def test_workspace_sizes(q):
     assert q.qlora_linear_fwd_workspace_size(4096, 4096, 4096, 64) >= 4096 * 64 * 2
     assert q.qlora_linear_bwd_workspace_size(4096, 4096, 4096, 64) >= 2 * 4096 * 64 * 2
     assert q.qlora_linear_fwd_workspace_size(16, 100, 100, 8) == 0  # K % 64 != 0
+    assert q.qlora_linear_group_fwd_workspace_size(4096, 3, 64) >= 4096 * 192 * 2
+    assert q.qlora_linear_group_bwd_workspace_size(4096, 3, 64) >= 2 * 4096 * 192 * 2
+    assert q.qlora_linear_group_fwd_workspace_size(16, 5, 8) == 0      # more than 4 linears
+    assert q.qlora_linear_group_bwd_workspace_size(16, 2, 256) == 0    # G r > 256
 
 
 def test_argument_validation_on_host(q):
@@ -103,6 +107,24 @@ def test_argument_validation_on_host(q):
     assert L.qlora_linear_fwd_4bit(9, P, 16, 64, 128, P, P, P, P, P, P, 8, f32(1), P, P, P, 1 << 20, None) == 1
     assert L.qlora_linear_bwd_4bit(9, P, P, 16, 64, 128, P, P, P, P, P, P, 8, f32(1), None, P, P, P, P, 1 << 20,
                                    None) == 1
+    # grouped linears: group size, total rank, weight descriptors, type
+    W = (q._Weight4bit * 5)(*[q._Weight4bit(P, P, P, P, 256) for _ in range(5)])
+    gf = L.qlora_linear_group_fwd
+    assert gf(0, P, 0, 128, W, 3, P, P, 8, f32(1), P, None, None, 0, None) == 0   # M == 0: nothing to do
+    assert gf(0, P, 0, 128, W, 5, P, P, 8, f32(1), P, None, None, 0, None) == 2   # G > 4
+    assert gf(0, P, 0, 128, W, 0, P, P, 8, f32(1), P, None, None, 0, None) == 1   # G < 1
+    assert gf(0, P, 0, 128, None, 2, P, P, 8, f32(1), P, None, None, 0, None) == 1
+    assert gf(0, P, 0, 128, W, 3, P, P, 128, f32(1), P, None, None, 0, None) == 2  # G r > 256
+    assert gf(0, P, 0, 128, W, 2, P, P, 12, f32(1), P, None, None, 0, None) == 2   # r % 8
+    assert gf(0, P, 0, 100, W, 2, P, P, 8, f32(1), P, None, None, 0, None) == 2    # K % 64
+    assert gf(9, P, 0, 128, W, 2, P, P, 8, f32(1), P, None, None, 0, None) == 1    # unknown type
+    assert gf(0, P, 0, 128, W, 2, None, P, 8, f32(1), P, None, None, 0, None) == 1
+    Wn = (q._Weight4bit * 2)(q._Weight4bit(P, P, P, P, 256), q._Weight4bit(P, None, P, P, 256))
+    assert gf(0, P, 0, 128, Wn, 2, P, P, 8, f32(1), P, None, None, 0, None) == 1
+    Wr = (q._Weight4bit * 2)(q._Weight4bit(P, P, P, P, 256), q._Weight4bit(P, P, P, P, 100))
+    assert gf(0, P, 16, 128, Wr, 2, P, P, 8, f32(1), P, None, None, 0, None) == 2  # N_g % 256
+    assert L.qlora_linear_group_bwd(0, P, P, 0, 128, W, 2, P, P, 8, f32(1), None, P, None, P, None, 0,
+                                    None) == 1  # dA_cat NULL
     # the failure-detection self-test refuses limits outside (0, 1 s]
     assert L.qlora_debug_wait_timeout(0, None) == 1
     assert L.qlora_debug_wait_timeout(2_000_000_000, None) == 1
