@@ -448,6 +448,28 @@ def run_native(args, world, rank, local):
                 dq32_ms += e0.elapsed_time(e1)
                 dq32_bytes += dequant_bytes(n, 4)
     del w32buf
+    # the DRAM write ceiling these outputs meet: a plain fill (torch's own
+    # kernel) of a 2 GiB buffer, 16x the L2, so that the cache absorbs a
+    # negligible part of the writes
+    fill_buf = torch.empty(1 << 29, dtype=torch.float32, device=dev)
+    fill_ms, fill_bytes = 0.0, 0
+    for rep in range(5):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fill_buf.fill_(1.0)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if rep >= 2:
+            fill_ms += e0.elapsed_time(e1)
+            fill_bytes += 4 * fill_buf.numel()
+    del fill_buf
+    fill_gbs = fill_bytes / (fill_ms * 1e-3) / 1e9
+    # time the output bytes alone take at that rate, over the dequant's time
+    dq32_write_frac = (sum(4 * b["case"].W.size for b in bufs) / (fill_gbs * 1e9)) / \
+        (dq32_ms * 1e-3 / (max(3, args.steps // 4))) if dq32_ms else None
+    dq16_write_frac = (sum(2 * b["case"].W.size for b in bufs) / (fill_gbs * 1e9)) / \
+        (dq_ms * 1e-3 / (max(3, args.steps // 4))) if dq_ms else None
 
     # the dominant kernel: the backward's dX GEMM (dX = dY W' + U A), timed
     # live as the backward with dX minus the backward without it, per call,
@@ -576,6 +598,19 @@ def run_native(args, world, rank, local):
                 "dequant_bf16_frac_hbm": (dq_bytes / (dq_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]) if dq_ms else None,
                 "dequant_fp32_gbs": dq32_bytes / (dq32_ms * 1e-3) / 1e9 if dq32_ms else None,
                 "dequant_fp32_frac_hbm": (dq32_bytes / (dq32_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]) if dq32_ms else None,
+                "write_only_fill_gbs": fill_gbs,
+                "dequant_fp32_frac_write_ceiling": dq32_write_frac,
+                "dequant_bf16_frac_write_ceiling": dq16_write_frac,
+                "full_set_dequant_fp32_frac_write_ceiling": (
+                    (4.0 * full7b["params"] / (fill_gbs * 1e9)) / (full7b["dequant_fp32_ms"] * 1e-3)
+                    if full7b else None),
+                "full_set_dequant_bf16_frac_write_ceiling": (
+                    (2.0 * full7b["params"] / (fill_gbs * 1e9)) / (full7b["dequant_bf16_ms"] * 1e-3)
+                    if full7b else None),
+                "write_ceiling_note": ("output bytes / (fill GB/s) over the dequant's time; the fill is "
+                                       "torch fill_ of a 2 GiB fp32 buffer (L2 flushed), writes only; the "
+                                       "dequant also reads 0.52 B per weight, and part of its 67-180 MB "
+                                       "output can stay in the 126 MB L2 when the call ends"),
                 "fwd_tflops": fwd_tflops, "fwd_frac_tensor": fwd_tflops / tc_peak,
                 "bwd_tflops": bflops / (bt * 1e-3) / 1e12, "dx_path_tflops": dx_tflops,
                 "unfused_fwd_tflops": k9_tflops,
@@ -676,6 +711,7 @@ def run_llama65b_layer(q, torch, dev, stream, flush, peaks, args):
     reps = max(3, min(10, args.steps // 5))
     out = {}
     tc_b, tc_s = peaks["bf16_tflops"], peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    sampler = clock_sampler(dev.index if dev.index is not None else 0)  # clocks of these long dense runs
     for M in synth.LLAMA65B_TOKENS:
         lin = []
         for i, (nm, n, k) in enumerate(layer):
@@ -707,6 +743,7 @@ def run_llama65b_layer(q, torch, dev, stream, flush, peaks, args):
 
         layer_pass()
         torch.cuda.synchronize()
+        tw0 = time.time()
         fwd_ms = [0.0] * len(layer)
         bwd_ms = [0.0] * len(layer)
         tot_ms = 0.0
@@ -728,10 +765,60 @@ def run_llama65b_layer(q, torch, dev, stream, flush, peaks, args):
                         "fwd_tflops": ff / (fwd_ms[i] * 1e-3) / 1e12, "bwd_tflops": fb / (bwd_ms[i] * 1e-3) / 1e12,
                         "fwd_bwd_tflops": (ff + fb) / ((fwd_ms[i] + bwd_ms[i]) * 1e-3) / 1e12})
         tf = fl_tot / (tot_ms * 1e-3) / 1e12
+        tw1 = time.time()
+        grouped = grouped_layer(q, torch, dev, stream, flush, lin, wqs, M, reps, fl_tot, tot_ms)
+        tw2 = time.time()
         out[f"m{M}"] = {"layer_ms": tot_ms, "layer_flops": fl_tot, "layer_tflops": tf,
-                        "frac_burst": tf / tc_b, "frac_sustained": tf / tc_s, "linears": per}
+                        "frac_burst": tf / tc_b, "frac_sustained": tf / tc_s, "linears": per,
+                        "clocks": sampler.summary(tw0, tw1), "grouped": grouped}
+        out[f"m{M}"]["grouped"]["clocks"] = sampler.summary(tw1, tw2)
         del lin
+    sampler.stop()
     return out
+
+
+def grouped_layer(q, torch, dev, stream, flush, lin, wqs, M, reps, fl_tot, per_linear_ms):
+    """The same layer as a decoder block runs it: q, k, v read one input and
+    run as one grouped linear, gate and up likewise; o and down alone.  Same
+    FLOPs as the seven separate linears; timed over the whole pass."""
+    s_lora = ALPHA / RANK
+    parts = []
+    for idx in ((0, 1, 2), (3,), (4, 5), (6,)):
+        ds = [lin[i] for i in idx]
+        n_all, k = sum(d["N"] for d in ds), ds[0]["K"]
+        G = len(idx)
+        g = {"w": [wqs[i] for i in idx], "X": ds[0]["X"],
+             "A": torch.cat([d["A"] for d in ds]).contiguous(), "B": torch.cat([d["B"] for d in ds]).contiguous(),
+             "dY": torch.cat([d["dY"] for d in ds], dim=1).contiguous(),
+             "Y": torch.empty((M, n_all), dtype=torch.bfloat16, device=dev),
+             "T": torch.empty((M, G * RANK), dtype=torch.bfloat16, device=dev),
+             "dX": torch.empty((M, k), dtype=torch.bfloat16, device=dev),
+             "dA": torch.empty((G * RANK, k), dtype=torch.bfloat16, device=dev),
+             "dB": torch.empty((n_all, RANK), dtype=torch.bfloat16, device=dev)}
+        g["ws"] = torch.empty(q.qlora_linear_group_bwd_workspace_size(M, G, RANK), dtype=torch.uint8, device=dev)
+        parts.append(g)
+
+    def block_pass():
+        for g in parts:
+            q.qlora_linear_group_fwd(g["X"], g["w"], g["A"], g["B"], s_lora, Y=g["Y"], T_save=g["T"], ws=g["ws"])
+        for g in reversed(parts):
+            q.qlora_linear_group_bwd(g["dY"], g["X"], g["w"], g["A"], g["B"], s_lora, T=g["T"], dX=g["dX"],
+                                     dA_cat=g["dA"], dB_cat=g["dB"], ws=g["ws"])
+
+    block_pass()
+    torch.cuda.synchronize()
+    ms = 0.0
+    for _ in range(reps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        block_pass()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms += a.elapsed_time(b) / reps
+    del parts
+    return {"layer_ms": ms, "layer_tflops": fl_tot / (ms * 1e-3) / 1e12, "vs_per_linear": per_linear_ms / ms,
+            "groups": "qkv, o, gate+up, down"}
 
 
 def decode_bytes(M, N, K, r):

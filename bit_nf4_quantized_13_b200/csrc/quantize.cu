@@ -229,6 +229,8 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
         }
         finish_chunk(base, mb);
     }
+    // the double-quant kernel may now be scheduled onto SMs this grid frees
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (bad) sbad = 1;
     __syncthreads();
     for (int i = threadIdx.x; i < 256; i += blockDim.x) {
@@ -329,6 +331,9 @@ k_double_quant(const float* __restrict__ c2, int64_t nb, const unsigned long lon
     __shared__ unsigned long long sv[64];
     __shared__ float smu;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // launched as a programmatic dependent of k_nf4_quantize: wait for that
+    // grid's completion (and its bins, c2 and flag) before reading anything
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (warp == 0) {
         const float mu = mean_from_bins(bins, nb, sv);
         if (lane == 0) smu = mu;
@@ -403,9 +408,22 @@ cudaError_t launch_quantize_nf4_dq(const float* W, int64_t numel, uint8_t* codes
     const int64_t ng = ceil_div(nb, kBlock2);
     const int64_t want2 = ceil_div(ng, kDqThreads / 32);
     const int grid2 = static_cast<int>(want2 < num_sms() * 4LL ? want2 : num_sms() * 4LL);
-    k_double_quant<<<grid2, kDqThreads, 0, stream>>>(c2, nb, bins, flag, c2_fp8, c1, mean, status);
+    // programmatic stream serialization: its launch overlaps the quantize
+    // kernel's tail; griddepcontrol.wait inside orders every read after it
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid2));
+    cfg.blockDim = dim3(kDqThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, k_double_quant, static_cast<const float*>(c2), nb,
+                             static_cast<const unsigned long long*>(bins), static_cast<const int*>(flag), c2_fp8, c1,
+                             mean, status);
     note_launches(1);
-    return cudaGetLastError();
+    return err;
 }
 
 cudaError_t launch_e4m3_encode(const float* x, uint8_t* out, int64_t n, cudaStream_t stream) {
