@@ -40,8 +40,10 @@ M_TOKENS, RANK, ALPHA = 4096, 64, 16.0
 L2_FLUSH_BYTES = 256 << 20
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) per call of the dX GEMM, mean over the two linears, from one ncu
-# capture of the kernel as it is now (profiles/); None when the kernel has changed since then.
-DX_TRAFFIC_BYTES = None
+# capture of the kernel as it is now (profiles/k_nf4_gemm_pair_llama7b_m4096.md: 43.73 MB for
+# the 4096x4096 linear, whose 33.5 MB dX is still in L2 when the launch ends, and 174.99 MB for
+# the 11008x4096 one); None when the kernel has changed since then.
+DX_TRAFFIC_BYTES = 109.36e6
 
 
 def linear_flops(M, N, K, r):

@@ -19,6 +19,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kChunk = 1024;  // weights per warp per step
+constexpr int kDepth = 3;     // chunks whose codes and constants a warp has in flight
 constexpr int kLutBytes = 256 * 256;
 
 // (q[high nibble], q[low nibble]) of one code byte from the lane's copy
@@ -73,34 +74,38 @@ k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
     int64_t c = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
 
-    // the lane's four groups of chunk c: codes and the constants' inputs
-    uint32_t cw[4], fb[4];
-    float s1[4];
-    auto load = [&](int64_t ch, uint32_t (&w)[4], uint32_t (&b)[4], float (&x)[4]) {
+    // the lane's four groups of a chunk: codes and the constants' inputs,
+    // kDepth chunks in flight per warp (a register ring)
+    struct Chunk {
+        uint32_t cw[4], fb[4];
+        float s1[4];
+    };
+    auto load = [&](int64_t ch, Chunk& k) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int64_t e = ch * kChunk + 8 * lane + 256 * i;
-            w[i] = ld_nc_u32(codes + (e >> 1));
-            b[i] = __ldg(c2_fp8 + (e >> 6));
-            x[i] = __ldg(c1 + (e >> 14));
+            k.cw[i] = ld_nc_u32(codes + (e >> 1));
+            k.fb[i] = __ldg(c2_fp8 + (e >> 6));
+            k.s1[i] = __ldg(c1 + (e >> 14));
         }
     };
-    if (c < nfull) load(c, cw, fb, s1);
-    for (; c < nfull; c += nwarps) {
-        uint32_t ncw[4] = {cw[0], cw[1], cw[2], cw[3]}, nfb[4] = {fb[0], fb[1], fb[2], fb[3]};
-        float ns1[4] = {s1[0], s1[1], s1[2], s1[3]};
-        if (c + nwarps < nfull) load(c + nwarps, ncw, nfb, ns1);
+    Chunk ring[kDepth];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float w[8];
-            expand8(cw[i], dq_constant(static_cast<uint8_t>(fb[i]), s1[i], mu), lut, lane_off, w);
-            store8<OUT_BF16>(out, c * kChunk + 8 * lane + 256 * i, w);
-        }
+    for (int k = 0; k < kDepth; ++k)
+        if (c + k * nwarps < nfull) load(c + k * nwarps, ring[k]);
+    for (int64_t base = c; base < nfull; base += kDepth * nwarps) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            cw[i] = ncw[i];
-            fb[i] = nfb[i];
-            s1[i] = ns1[i];
+        for (int k = 0; k < kDepth; ++k) {
+            const int64_t ch = base + k * nwarps;
+            if (ch >= nfull) break;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float w[8];
+                expand8(ring[k].cw[i], dq_constant(static_cast<uint8_t>(ring[k].fb[i]), ring[k].s1[i], mu), lut,
+                        lane_off, w);
+                store8<OUT_BF16>(out, ch * kChunk + 8 * lane + 256 * i, w);
+            }
+            if (ch + kDepth * nwarps < nfull) load(ch + kDepth * nwarps, ring[k]);
         }
     }
     // the ragged last chunk (< 1024 weights), by one warp: whole 8-weight
