@@ -5,9 +5,9 @@
 //
 // HBM-bound: 0.5 + 1/64 + 1/16384 bytes read and 4 (fp32) or 2 (bf16) bytes
 // written per weight, the writes dominating.  A warp expands 1024 weights
-// per step; lane l takes the four 8-weight groups at 8 l + 256 i, so each
-// load instruction reads one contiguous 128-byte run of codes and each
-// bf16 store instruction writes one contiguous 512-byte run (whole sectors).
+// per step, and every store instruction writes one contiguous 512-byte run
+// (whole sectors): for bf16 output lane l takes the four 8-weight groups at
+// 8 l + 256 i, for fp32 output the eight 4-weight groups at 4 l + 128 i.
 // A code byte becomes both of its fp32 codebook values through a 256-entry
 // table with one copy per lane (no bank conflicts): one byte permute and
 // one shared load per two weights.
@@ -19,7 +19,8 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kChunk = 1024;  // weights per warp per step
-constexpr int kDepth = 3;     // chunks whose codes and constants a warp has in flight
+constexpr int kDepthBf16 = 3;  // chunks whose codes and constants a warp has in flight
+constexpr int kDepthF32 = 2;   // (fewer for fp32 output: twice the parts per chunk)
 constexpr int kLutBytes = 256 * 256;
 
 // (q[high nibble], q[low nibble]) of one code byte from the lane's copy
@@ -31,6 +32,12 @@ __device__ __forceinline__ float2 lut_pair(const uint8_t* lut, uint32_t word, ui
 __device__ __forceinline__ uint32_t ld_nc_u32(const uint8_t* p) {
     uint32_t v;
     asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_nc_u16(const uint8_t* p) {
+    uint16_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
     return v;
 }
 
@@ -74,19 +81,28 @@ k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
     int64_t c = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
 
-    // the lane's four groups of a chunk: codes and the constants' inputs,
-    // kDepth chunks in flight per warp (a register ring)
+    // The lane's parts of a chunk.  bf16 output: part p is the 8 weights at
+    // 256 p + 8 lane (4 code bytes; one 16-byte store, 512 contiguous bytes
+    // per warp).  fp32 output: part p is the 4 weights at 128 p + 4 lane
+    // (2 code bytes; one 16-byte store, again 512 contiguous bytes per warp,
+    // so every store instruction writes whole sectors).  kDepth chunks of
+    // codes and constants are in flight per warp (a register ring).
+    constexpr int kParts = OUT_BF16 ? 4 : 8;
+    constexpr int kDepth = OUT_BF16 ? kDepthBf16 : kDepthF32;
     struct Chunk {
-        uint32_t cw[4], fb[4];
-        float s1[4];
+        uint32_t cw[kParts], fb[kParts];
+        float s1[kParts];
+    };
+    auto first = [&](int64_t ch, int p) -> int64_t {
+        return ch * kChunk + (OUT_BF16 ? 256 * p + 8 * lane : 128 * p + 4 * lane);
     };
     auto load = [&](int64_t ch, Chunk& k) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int64_t e = ch * kChunk + 8 * lane + 256 * i;
-            k.cw[i] = ld_nc_u32(codes + (e >> 1));
-            k.fb[i] = __ldg(c2_fp8 + (e >> 6));
-            k.s1[i] = __ldg(c1 + (e >> 14));
+        for (int p = 0; p < kParts; ++p) {
+            const int64_t e = first(ch, p);
+            k.cw[p] = OUT_BF16 ? ld_nc_u32(codes + (e >> 1)) : ld_nc_u16(codes + (e >> 1));
+            k.fb[p] = __ldg(c2_fp8 + (e >> 6));
+            k.s1[p] = __ldg(c1 + (e >> 14));
         }
     };
     Chunk ring[kDepth];
@@ -99,11 +115,20 @@ k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
             const int64_t ch = base + k * nwarps;
             if (ch >= nfull) break;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float w[8];
-                expand8(ring[k].cw[i], dq_constant(static_cast<uint8_t>(ring[k].fb[i]), ring[k].s1[i], mu), lut,
-                        lane_off, w);
-                store8<OUT_BF16>(out, ch * kChunk + 8 * lane + 256 * i, w);
+            for (int p = 0; p < kParts; ++p) {
+                const float cp = dq_constant(static_cast<uint8_t>(ring[k].fb[p]), ring[k].s1[p], mu);
+                const int64_t e = first(ch, p);
+                if (OUT_BF16) {
+                    float w[8];
+                    expand8(ring[k].cw[p], cp, lut, lane_off, w);
+                    store8<true>(out, e, w);
+                } else {
+                    const float2 a = lut_pair(lut, ring[k].cw[p], lane_off, 0);
+                    const float2 b = lut_pair(lut, ring[k].cw[p], lane_off, 1);
+                    __stcs(reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + e),
+                           make_float4(__fmul_rn(a.x, cp), __fmul_rn(a.y, cp), __fmul_rn(b.x, cp),
+                                       __fmul_rn(b.y, cp)));
+                }
             }
             if (ch + kDepth * nwarps < nfull) load(ch + kDepth * nwarps, ring[k]);
         }
