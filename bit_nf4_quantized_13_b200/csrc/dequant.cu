@@ -8,9 +8,10 @@
 // per step, and every store instruction writes one contiguous 512-byte run
 // (whole sectors): for bf16 output lane l takes the four 8-weight groups at
 // 8 l + 256 i, for fp32 output the eight 4-weight groups at 4 l + 128 i.
-// A code byte becomes both of its fp32 codebook values through a 256-entry
-// table with one copy per lane (no bank conflicts): one byte permute and
-// one shared load per two weights.
+// The 16 codebook values live one per lane (lanes i and i + 16 hold q[i]),
+// and a warp shuffle indexed by the 4-bit code fetches each weight's value:
+// no shared memory, so the launch needs no carve-out change and no table
+// set-up, which is most of the fixed cost at the sizes of one linear.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -21,12 +22,12 @@ constexpr int kThreads = 256;
 constexpr int kChunk = 1024;  // weights per warp per step
 constexpr int kDepthBf16 = 3;  // chunks whose codes and constants a warp has in flight
 constexpr int kDepthF32 = 2;   // (fewer for fp32 output: twice the parts per chunk)
-constexpr int kLutBytes = 256 * 256;
 
-// (q[high nibble], q[low nibble]) of one code byte from the lane's copy
-__device__ __forceinline__ float2 lut_pair(const uint8_t* lut, uint32_t word, uint32_t lane_off, int byte) {
-    const uint32_t addr = __byte_perm(word, lane_off, 0x5504u | (static_cast<uint32_t>(byte) << 4));
-    return *reinterpret_cast<const float2*>(lut + addr);
+// (q[high nibble], q[low nibble]) of byte `byte` of `word`; qv is q[lane % 16]
+__device__ __forceinline__ float2 q_pair(float qv, uint32_t word, int byte) {
+    const uint32_t b = (word >> (8 * byte)) & 0xFFu;
+    return make_float2(__shfl_sync(0xffffffffu, qv, static_cast<int>(b >> 4)),
+                       __shfl_sync(0xffffffffu, qv, static_cast<int>(b & 15u)));
 }
 
 __device__ __forceinline__ uint32_t ld_nc_u32(const uint8_t* p) {
@@ -42,11 +43,12 @@ __device__ __forceinline__ uint32_t ld_nc_u16(const uint8_t* p) {
 }
 
 // 8 weights of one group (4 code bytes, element 2t the high nibble of byte
-// t) scaled by the block constant: w[i] = RN32(q[code_i] * c2').
-__device__ __forceinline__ void expand8(uint32_t cw, float cp, const uint8_t* lut, uint32_t lane_off, float (&w)[8]) {
+// t) scaled by the block constant: w[i] = RN32(q[code_i] * c2').  All 32
+// lanes must take part (warp shuffles).
+__device__ __forceinline__ void expand8(uint32_t cw, float cp, float qv, float (&w)[8]) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const float2 q2 = lut_pair(lut, cw, lane_off, j);
+        const float2 q2 = q_pair(qv, cw, j);
         w[2 * j] = __fmul_rn(q2.x, cp);
         w[2 * j + 1] = __fmul_rn(q2.y, cp);
     }
@@ -70,12 +72,8 @@ __global__ void __launch_bounds__(kThreads)
 k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
           const float* __restrict__ c1, const float* __restrict__ mean, int64_t numel,
           void* __restrict__ out, Nf4Tables tabs) {
-    extern __shared__ __align__(16) uint8_t lut[];  // entry b, lane l at 256 b + 8 l
-    for (int i = threadIdx.x; i < 256 * 32; i += kThreads)
-        reinterpret_cast<float2*>(lut)[i] = make_float2(tabs.q[i >> 9], tabs.q[(i >> 5) & 15]);
-    __syncthreads();
     const int lane = threadIdx.x & 31;
-    const uint32_t lane_off = static_cast<uint32_t>(lane) * 8;
+    const float qv = tabs.q[lane & 15];
     const float mu = *mean;
     const int64_t nfull = numel / kChunk;  // whole 1024-weight chunks
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
@@ -120,11 +118,11 @@ k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
                 const int64_t e = first(ch, p);
                 if (OUT_BF16) {
                     float w[8];
-                    expand8(ring[k].cw[p], cp, lut, lane_off, w);
+                    expand8(ring[k].cw[p], cp, qv, w);
                     store8<true>(out, e, w);
                 } else {
-                    const float2 a = lut_pair(lut, ring[k].cw[p], lane_off, 0);
-                    const float2 b = lut_pair(lut, ring[k].cw[p], lane_off, 1);
+                    const float2 a = q_pair(qv, ring[k].cw[p], 0);
+                    const float2 b = q_pair(qv, ring[k].cw[p], 1);
                     __stcs(reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + e),
                            make_float4(__fmul_rn(a.x, cp), __fmul_rn(a.y, cp), __fmul_rn(b.x, cp),
                                        __fmul_rn(b.y, cp)));
@@ -133,8 +131,9 @@ k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
             if (ch + kDepth * nwarps < nfull) load(ch + kDepth * nwarps, ring[k]);
         }
     }
-    // the ragged last chunk (< 1024 weights), by one warp: whole 8-weight
-    // groups vectorized, the last partial group element by element
+    // the ragged last chunk (< 1024 weights), by one warp, lanes diverging:
+    // direct table reads, whole 8-weight groups stored as vectors, the last
+    // partial group element by element
     const int64_t wid = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     if (nfull * kChunk < numel && wid == nfull % nwarps) {
 #pragma unroll 1
@@ -147,7 +146,11 @@ k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
                                     (static_cast<uint32_t>(codes[(e >> 1) + 2]) << 16) |
                                     (static_cast<uint32_t>(codes[(e >> 1) + 3]) << 24);
                 float w[8];
-                expand8(w4, cp, lut, lane_off, w);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t b = (w4 >> (8 * (j >> 1))) & 0xFFu;
+                    w[j] = __fmul_rn(tabs.q[(j & 1) ? (b & 15u) : (b >> 4)], cp);
+                }
                 store8<OUT_BF16>(out, e, w);
             } else {
                 for (int64_t k = e; k < numel; ++k) {
@@ -169,17 +172,13 @@ k_dequant(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ c2_fp8,
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const float* c1,
                               const float* mean, int64_t numel, void* out, int out_dtype,
                               cudaStream_t stream, int qtype) {
-    static ContextMemo<int> memo_bf16, memo_f32;
-    const cudaError_t attr = out_dtype == 1 ? ensure_smem_limit(memo_bf16, k_dequant<true>, kLutBytes)
-                                            : ensure_smem_limit(memo_f32, k_dequant<false>, kLutBytes);
-    if (attr != cudaSuccess) return attr;
     const int64_t chunks = ceil_div(numel, kChunk);
     const int64_t want = ceil_div(chunks, kThreads / 32);
     const int grid = static_cast<int>(want < num_sms() * 3LL ? (want > 0 ? want : 1) : num_sms() * 3LL);
     if (out_dtype == 1)
-        k_dequant<true><<<grid, kThreads, kLutBytes, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables(qtype));
+        k_dequant<true><<<grid, kThreads, 0, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables(qtype));
     else
-        k_dequant<false><<<grid, kThreads, kLutBytes, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables(qtype));
+        k_dequant<false><<<grid, kThreads, 0, stream>>>(codes, c2_fp8, c1, mean, numel, out, tables(qtype));
     note_launches(1);
     return cudaGetLastError();
 }
