@@ -450,23 +450,29 @@ def run_native(args, world, rank, local):
                 dq32_ms += e0.elapsed_time(e1)
                 dq32_bytes += dequant_bytes(n, 4)
     del w32buf
-    # the DRAM write ceiling these outputs meet: a plain fill (torch's own
-    # kernel) of a 2 GiB buffer, 16x the L2, so that the cache absorbs a
-    # negligible part of the writes
-    fill_buf = torch.empty(1 << 29, dtype=torch.float32, device=dev)
-    fill_ms, fill_bytes = 0.0, 0
-    for rep in range(5):
-        flush()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        fill_buf.fill_(1.0)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        if rep >= 2:
-            fill_ms += e0.elapsed_time(e1)
-            fill_bytes += 4 * fill_buf.numel()
-    del fill_buf
-    fill_gbs = fill_bytes / (fill_ms * 1e-3) / 1e9
+    # the DRAM ceilings these kernels meet, from the library's own probe
+    # kernels (16-byte streaming stores / loads) over a 2 GiB buffer, 16x the
+    # L2, so that the cache absorbs a negligible part; torch's fill beside
+    ceil_buf = torch.empty(1 << 29, dtype=torch.float32, device=dev)
+    ceil_sink = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def ceiling_gbs(fn):
+        ms = 0.0
+        for rep in range(5):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 2:
+                ms += e0.elapsed_time(e1)
+        return 3 * 4 * ceil_buf.numel() / (ms * 1e-3) / 1e9
+
+    fill_gbs = ceiling_gbs(lambda: q.qlora_debug_fill(ceil_buf, 0x3F800000))
+    read_gbs = ceiling_gbs(lambda: q.qlora_debug_read(ceil_buf, ceil_sink))
+    torch_fill_gbs = ceiling_gbs(lambda: ceil_buf.fill_(1.0))
+    del ceil_buf, ceil_sink
     # time the output bytes alone take at that rate, over the dequant's time
     dq32_write_frac = (sum(4 * b["case"].W.size for b in bufs) / (fill_gbs * 1e9)) / \
         (dq32_ms * 1e-3 / (max(3, args.steps // 4))) if dq32_ms else None
@@ -600,7 +606,11 @@ def run_native(args, world, rank, local):
                 "dequant_bf16_frac_hbm": (dq_bytes / (dq_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]) if dq_ms else None,
                 "dequant_fp32_gbs": dq32_bytes / (dq32_ms * 1e-3) / 1e9 if dq32_ms else None,
                 "dequant_fp32_frac_hbm": (dq32_bytes / (dq32_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]) if dq32_ms else None,
-                "write_only_fill_gbs": fill_gbs,
+                "write_ceiling_gbs": fill_gbs,
+                "read_ceiling_gbs": read_gbs,
+                "torch_fill_gbs": torch_fill_gbs,
+                "quantize_frac_read_ceiling": (sum(4.0 * c.W.size for c in cases) * args.steps / (read_gbs * 1e9))
+                / (qt * 1e-3),
                 "dequant_fp32_frac_write_ceiling": dq32_write_frac,
                 "dequant_bf16_frac_write_ceiling": dq16_write_frac,
                 "full_set_dequant_fp32_frac_write_ceiling": (
@@ -609,10 +619,10 @@ def run_native(args, world, rank, local):
                 "full_set_dequant_bf16_frac_write_ceiling": (
                     (2.0 * full7b["params"] / (fill_gbs * 1e9)) / (full7b["dequant_bf16_ms"] * 1e-3)
                     if full7b else None),
-                "write_ceiling_note": ("output bytes / (fill GB/s) over the dequant's time; the fill is "
-                                       "torch fill_ of a 2 GiB fp32 buffer (L2 flushed), writes only; the "
-                                       "dequant also reads 0.52 B per weight, and part of its 67-180 MB "
-                                       "output can stay in the 126 MB L2 when the call ends"),
+                "ceiling_note": ("ceilings: qlora_debug_fill / qlora_debug_read over a 2 GiB buffer, L2 "
+                                 "flushed; frac_write_ceiling = output bytes at the write ceiling over the "
+                                 "dequant's time (it also reads 0.52 B per weight), frac_read_ceiling = the "
+                                 "4 B per weight read at the read ceiling over the quantize time"),
                 "fwd_tflops": fwd_tflops, "fwd_frac_tensor": fwd_tflops / tc_peak,
                 "bwd_tflops": bflops / (bt * 1e-3) / 1e12, "dx_path_tflops": dx_tflops,
                 "unfused_fwd_tflops": k9_tflops,

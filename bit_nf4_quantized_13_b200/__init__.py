@@ -75,6 +75,8 @@ def _load() -> ctypes.CDLL:
         "qlora_debug_wait_timeout": (i32, [ctypes.c_uint64, vp]),
         "qlora_int8_quantize": (i32, [vp, i64, i32, vp, vp, vp, vp]),
         "qlora_int8_dequantize": (i32, [vp, vp, i64, i32, vp, vp]),
+        "qlora_debug_fill": (i32, [vp, i64, ctypes.c_uint32, vp]),
+        "qlora_debug_read": (i32, [vp, i64, ctypes.c_uint32, vp, vp]),
         "qlora_linear_group_fwd_workspace_size": (sz, [i64, i32, i32]),
         "qlora_linear_group_bwd_workspace_size": (sz, [i64, i32, i32]),
         "qlora_linear_group_fwd": (i32, [i32, vp, i64, i64, vp, i32, vp, vp, i32, f32, vp, vp, vp, sz, vp]),
@@ -455,6 +457,29 @@ def qlora_fp8_e4m3_encode(x, out=None, stream=None):
     _check("qlora_fp8_e4m3_encode",
            _get_lib().qlora_fp8_e4m3_encode(_ptr(x), _ptr(out), x.numel(), _stream(stream)))
     return out
+
+
+def qlora_debug_fill(dst, value: int = 0, stream=None):
+    """Measurement aid: the DRAM write ceiling (a 16-byte streaming fill of
+    a contiguous CUDA tensor whose size is a multiple of 16 bytes)."""
+    _need_cuda(dst)
+    nbytes = dst.numel() * dst.element_size()
+    if nbytes % 16:
+        raise ValueError("the buffer must be a multiple of 16 bytes")
+    _check("qlora_debug_fill", _get_lib().qlora_debug_fill(_ptr(dst), nbytes // 4, int(value) & 0xffffffff,
+                                                           _stream(stream)))
+
+
+def qlora_debug_read(src, sink, never: int = 0x9E3779B9, stream=None):
+    """Measurement aid: the DRAM read ceiling (a 16-byte streaming read of a
+    contiguous CUDA tensor; `sink` is a 4-byte CUDA tensor written only if
+    the data folds to `never`)."""
+    _need_cuda(src, sink)
+    nbytes = src.numel() * src.element_size()
+    if nbytes % 16:
+        raise ValueError("the buffer must be a multiple of 16 bytes")
+    _check("qlora_debug_read", _get_lib().qlora_debug_read(_ptr(src), nbytes // 4, int(never) & 0xffffffff,
+                                                           _ptr(sink), _stream(stream)))
 
 
 def qlora_device_error(reset: bool = False) -> int:

@@ -390,6 +390,16 @@ int qlora_debug_wait_timeout(uint64_t limit_ns, void* stream) {
     return cuda_status(launch_wait_selftest(limit_ns, as_stream(stream)));
 }
 
+int qlora_debug_fill(uint32_t* dst, int64_t n_words, uint32_t value, void* stream) {
+    if (n_words < 0 || n_words % 4 != 0 || (n_words > 0 && !ok_ptr(dst))) return QLORA_ERR_INVALID_ARG;
+    return cuda_status(launch_probe_fill(dst, n_words, value, as_stream(stream)));
+}
+
+int qlora_debug_read(const uint32_t* src, int64_t n_words, uint32_t never, uint32_t* sink, void* stream) {
+    if (n_words < 0 || n_words % 4 != 0 || (n_words > 0 && (!ok_ptr(src) || !sink))) return QLORA_ERR_INVALID_ARG;
+    return cuda_status(launch_probe_read(src, n_words, never, sink, as_stream(stream)));
+}
+
 uint64_t qlora_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int qlora_fp8_e4m3_encode(const float* x, uint8_t* out, int64_t n, void* stream) {

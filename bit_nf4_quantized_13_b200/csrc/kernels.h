@@ -21,6 +21,12 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* c2_fp8, const
                               const float* mean, int64_t numel, void* out, int out_dtype,
                               cudaStream_t stream, int qtype = QLORA_TYPE_NF4);
 
+// probe.cu -- the DRAM ceilings: a write-only fill and a read-only pass
+// (16-byte accesses; n_words a multiple of 4, pointers 16-byte aligned)
+cudaError_t launch_probe_fill(uint32_t* dst, int64_t n_words, uint32_t value, cudaStream_t stream);
+cudaError_t launch_probe_read(const uint32_t* src, int64_t n_words, uint32_t never, uint32_t* sink,
+                              cudaStream_t stream);
+
 // int8.cu -- block-wise Int8 absmax quantization (eq. 1) and dequantization
 // (eq. 2), block in {32, 64, 128, 256}
 bool int8_block_supported(int block);

@@ -303,6 +303,21 @@ int qlora_fp8_e4m3_encode(const float* x, uint8_t* out, int64_t n, void* stream)
 int qlora_device_error(int reset);
 
 /*
+ * qlora_debug_fill / qlora_debug_read -- measurement aids, not part of the
+ * method: the DRAM write and read ceilings that the HBM-bound kernels
+ * (quantize, dequantize, the small-batch forward) are compared with.
+ * qlora_debug_fill writes `value` to n_words 32-bit words at dst;
+ * qlora_debug_read reads n_words words at src and writes their XOR-fold to
+ * *sink only if it equals `never` (so the reads are kept; pass a value the
+ * data cannot fold to, and the call writes nothing).  Both use 16-byte
+ * accesses in whole 512-byte warp runs.  n_words must be a
+ * multiple of 4 and the pointers 16-byte aligned (device memory), else
+ * QLORA_ERR_INVALID_ARG; n_words == 0 launches nothing.
+ */
+int qlora_debug_fill(uint32_t* dst, int64_t n_words, uint32_t value, void* stream);
+int qlora_debug_read(const uint32_t* src, int64_t n_words, uint32_t never, uint32_t* sink, void* stream);
+
+/*
  * qlora_int8_quantize -- block-wise Int8 absmax quantization, the 8-bit
  * baseline of section 3.1, eq. (1), applied to consecutive blocks of
  * `block` elements of the flattened tensor (block in {32, 64, 128, 256};

@@ -125,6 +125,13 @@ def test_argument_validation_on_host(q):
     assert gf(0, P, 16, 128, Wr, 2, P, P, 8, f32(1), P, None, None, 0, None) == 2  # N_g % 256
     assert L.qlora_linear_group_bwd(0, P, P, 0, 128, W, 2, P, P, 8, f32(1), None, P, None, P, None, 0,
                                     None) == 1  # dA_cat NULL
+    # the ceiling probes: word counts that are not whole 16-byte runs, NULL pointers
+    assert L.qlora_debug_fill(P, 3, 0, None) == 1
+    assert L.qlora_debug_fill(None, 4, 0, None) == 1
+    assert L.qlora_debug_fill(P + 4, 4, 0, None) == 1
+    assert L.qlora_debug_fill(None, 0, 0, None) == 0       # nothing to write, nothing launched
+    assert L.qlora_debug_read(P, 4, 0, None, None) == 1    # no sink
+    assert L.qlora_debug_read(P, -4, 0, P, None) == 1
     # the failure-detection self-test refuses limits outside (0, 1 s]
     assert L.qlora_debug_wait_timeout(0, None) == 1
     assert L.qlora_debug_wait_timeout(2_000_000_000, None) == 1
