@@ -65,9 +65,7 @@ cudaError_t lora_dyb(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t N
 cudaError_t lora_grads(const uint16_t* dY, const uint16_t* X, const uint16_t* T, const uint16_t* U, int64_t M,
                        int64_t N, int64_t K, int r, uint16_t* dA, uint16_t* dB, cudaStream_t st) {
     if (!lora_tc_supported(M, N, K, r)) return launch_lora_grads_simt(dY, X, T, U, M, N, K, r, dA, dB, st);
-    cudaError_t e = launch_lora_da_tc(X, U, M, K, r, dA, st);
-    if (e != cudaSuccess) return e;
-    return launch_lora_db_tc(dY, T, M, N, r, dB, st);
+    return launch_lora_grads_tc(X, U, dY, T, M, N, K, r, dA, dB, st);
 }
 
 }  // namespace qlora

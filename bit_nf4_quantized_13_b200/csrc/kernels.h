@@ -61,6 +61,10 @@ cudaError_t launch_lora_da_tc(const uint16_t* X, const uint16_t* U, int64_t M, i
                               cudaStream_t stream);
 cudaError_t launch_lora_db_tc(const uint16_t* dY, const uint16_t* T, int64_t M, int64_t N, int r, uint16_t* dB,
                               cudaStream_t stream, int64_t ld_dy = 0, int64_t ld_t = 0);
+// dA and dB in one launch
+cudaError_t launch_lora_grads_tc(const uint16_t* X, const uint16_t* U, const uint16_t* dY, const uint16_t* T,
+                                 int64_t M, int64_t N, int64_t K, int r, uint16_t* dA, uint16_t* dB,
+                                 cudaStream_t stream);
 int lora_device_error(int reset);
 // gemm_pair_sm100.cu: a kernel whose one bounded wait is never satisfied
 // (records QLORA_ERR_TIMEOUT after limit_ns)

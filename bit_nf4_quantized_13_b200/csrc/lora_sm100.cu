@@ -45,12 +45,22 @@ constexpr int kThreads = 128;
 constexpr int kABytes = kRows * kBK * 2;  // 16 KiB
 constexpr int kMaxSmem = 200 * 1024;
 
-struct SkinnyParams {
-    uint16_t* out;  // rows x r bf16 (row pitch ldo), or r x rows when transposed
+// One product's output: rows x r bf16 (row pitch ldo), or r x rows when
+// transposed, scaled by `scale` before the rounding.
+struct SkinnyOut {
+    uint16_t* out;
     int ldo;
     float scale;
     int transposed;
     int rows;      // output rows
+};
+
+// A launch computes one product, or two of the same kind (the same operand
+// majorness, rank and contraction length: dA and dB), CTAs with blockIdx.x
+// below tiles0 taking the first and the rest the second.
+struct SkinnyParams {
+    SkinnyOut o[2];
+    int tiles0;    // row tiles of the first product
     int r;
     int nt;        // r rounded up to 16 (MMA N)
     int kb_total;  // 64-wide contraction blocks
@@ -62,7 +72,8 @@ struct SkinnyParams {
 
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kThreads)
-k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, const SkinnyParams p) {
+k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+          const __grid_constant__ CUtensorMap ta2, const __grid_constant__ CUtensorMap tb2, const SkinnyParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int stage_bytes = kABytes + p.b_bytes;
@@ -74,7 +85,11 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
     auto empty = [&](int s) { return bar0 + 8u * (p.stages + s); };
     const uint32_t done = bar0 + 8u * (2 * p.stages);
 
-    const int row0 = blockIdx.x * kRows;
+    const bool second = static_cast<int>(blockIdx.x) >= p.tiles0;
+    const SkinnyOut o = second ? p.o[1] : p.o[0];
+    const CUtensorMap* mapa = second ? &ta2 : &ta;
+    const CUtensorMap* mapb = second ? &tb2 : &tb;
+    const int row0 = (static_cast<int>(blockIdx.x) - (second ? p.tiles0 : 0)) * kRows;
     const int split = static_cast<int>(cluster_ctarank());  // == blockIdx.y: the cluster spans the splits
     const int kb_begin = static_cast<int>(static_cast<int64_t>(split) * p.kb_total / p.splits);
     const int kb_end = static_cast<int>(static_cast<int64_t>(split + 1) * p.kb_total / p.splits);
@@ -99,8 +114,8 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
     bool ok = true;
 
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&ta);
-        tma_prefetch_desc(&tb);
+        tma_prefetch_desc(mapa);
+        tma_prefetch_desc(mapb);
         for (int kb = kb_begin, it = 0; kb < kb_end; ++kb, ++it) {
             const int s = it % p.stages;
             const uint32_t ph = (it / p.stages) & 1u;
@@ -109,15 +124,15 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
             const uint32_t sa = smem_u32(smem + s * stage_bytes);
             const uint32_t sb = sa + kABytes;
             if (A_MN) {  // 128 MN-contiguous rows as two 64-wide boxes, 64 contraction rows each
-                tma_load_2d(sa, &ta, full(s), row0, kb * kBK);
-                tma_load_2d(sa + 8192, &ta, full(s), row0 + 64, kb * kBK);
+                tma_load_2d(sa, mapa, full(s), row0, kb * kBK);
+                tma_load_2d(sa + 8192, mapa, full(s), row0 + 64, kb * kBK);
             } else {
-                tma_load_2d(sa, &ta, full(s), kb * kBK, row0);
+                tma_load_2d(sa, mapa, full(s), kb * kBK, row0);
             }
             if (B_MN) {
-                for (int b = 0; b * 64 < p.nt; ++b) tma_load_2d(sb + b * 8192, &tb, full(s), b * 64, kb * kBK);
+                for (int b = 0; b * 64 < p.nt; ++b) tma_load_2d(sb + b * 8192, mapb, full(s), b * 64, kb * kBK);
             } else {
-                tma_load_2d(sb, &tb, full(s), kb * kBK, 0);
+                tma_load_2d(sb, mapb, full(s), kb * kBK, 0);
             }
         }
     } else if (warp == 1 && lane == 0) {
@@ -176,8 +191,11 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
         const int q4 = p.nt / 4;
         const uint32_t acc_s = smem_u32(acc);
         for (int idx = threadIdx.x; idx < rows_per * q4; idx += kThreads) {
-            const int lr = split * rows_per + idx / q4;
-            const int c = (idx % q4) * 4;
+            // consecutive threads take consecutive columns of one row, or (a
+            // transposed output, whose rows are the columns in memory)
+            // consecutive rows of one column group: coalesced stores either way
+            const int lr = split * rows_per + (o.transposed ? idx % rows_per : idx / q4);
+            const int c = (o.transposed ? idx / rows_per : idx % q4) * 4;
             const uint32_t off = static_cast<uint32_t>((lr * ld + c) * 4);
             // all ranks' values in flight together, then summed in rank order
             float4 v[8];
@@ -192,17 +210,17 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
                 }
             }
             const int row = row0 + lr;
-            if (row < p.rows && c < p.r) {
-                const uint32_t lo = pack_bf16x2(sum.x * p.scale, sum.y * p.scale);
-                const uint32_t hi = pack_bf16x2(sum.z * p.scale, sum.w * p.scale);
-                if (p.transposed) {
-                    uint16_t* o = p.out + static_cast<int64_t>(c) * p.rows + row;
-                    o[0] = static_cast<uint16_t>(lo & 0xffffu);
-                    o[p.rows] = static_cast<uint16_t>(lo >> 16);
-                    o[2 * static_cast<int64_t>(p.rows)] = static_cast<uint16_t>(hi & 0xffffu);
-                    o[3 * static_cast<int64_t>(p.rows)] = static_cast<uint16_t>(hi >> 16);
+            if (row < o.rows && c < p.r) {
+                const uint32_t lo = pack_bf16x2(sum.x * o.scale, sum.y * o.scale);
+                const uint32_t hi = pack_bf16x2(sum.z * o.scale, sum.w * o.scale);
+                if (o.transposed) {
+                    uint16_t* dst = o.out + static_cast<int64_t>(c) * o.rows + row;
+                    dst[0] = static_cast<uint16_t>(lo & 0xffffu);
+                    dst[o.rows] = static_cast<uint16_t>(lo >> 16);
+                    dst[2 * static_cast<int64_t>(o.rows)] = static_cast<uint16_t>(hi & 0xffffu);
+                    dst[3 * static_cast<int64_t>(o.rows)] = static_cast<uint16_t>(hi >> 16);
                 } else {
-                    *reinterpret_cast<uint2*>(p.out + static_cast<int64_t>(row) * p.ldo + c) = make_uint2(lo, hi);
+                    *reinterpret_cast<uint2*>(o.out + static_cast<int64_t>(row) * o.ldo + c) = make_uint2(lo, hi);
                 }
             }
         }
@@ -263,18 +281,29 @@ Plan plan(int64_t rows, int64_t ctr, int r, bool b_mn) {
     return pl;
 }
 
+SkinnyOut out_desc(uint16_t* out, int64_t rows, int r, float scale, bool transposed, int ldo) {
+    SkinnyOut o;
+    o.out = out;
+    o.ldo = ldo ? ldo : r;
+    o.scale = scale;
+    o.transposed = transposed ? 1 : 0;
+    o.rows = static_cast<int>(rows);
+    return o;
+}
+
+// Launches one product (tiles1 == 0) or two of the same kind in one grid:
+// the first product's pl.tiles row tiles, then tiles1 of the second.
 template <bool A_MN, bool B_MN>
-cudaError_t run(const Plan& pl, const CUtensorMap& ma, const CUtensorMap& mb, int64_t rows, int r, float scale,
-                uint16_t* out, bool transposed, cudaStream_t st, int ldo = 0) {
+cudaError_t launch_skinny(const Plan& pl, const CUtensorMap& ma, const CUtensorMap& mb, const SkinnyOut& o0,
+                          const CUtensorMap& ma2, const CUtensorMap& mb2, const SkinnyOut& o1, int64_t tiles1,
+                          int r, cudaStream_t st) {
     static ContextMemo<int> attr_memo;
     const cudaError_t attr = ensure_smem_limit(attr_memo, k_lora_tc<A_MN, B_MN>, kMaxSmem + 2048);
     if (attr != cudaSuccess) return attr;
     SkinnyParams p;
-    p.out = out;
-    p.ldo = ldo ? ldo : r;
-    p.scale = scale;
-    p.transposed = transposed ? 1 : 0;
-    p.rows = static_cast<int>(rows);
+    p.o[0] = o0;
+    p.o[1] = o1;
+    p.tiles0 = static_cast<int>(pl.tiles);
     p.r = r;
     p.nt = pl.nt;
     p.kb_total = pl.kb_total;
@@ -288,15 +317,22 @@ cudaError_t run(const Plan& pl, const CUtensorMap& ma, const CUtensorMap& mb, in
     attr_c[0].val.clusterDim.x = 1;
     attr_c[0].val.clusterDim.y = static_cast<unsigned>(pl.splits);
     attr_c[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(static_cast<unsigned>(pl.tiles), static_cast<unsigned>(pl.splits));
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.tiles + tiles1), static_cast<unsigned>(pl.splits));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = static_cast<size_t>(pl.smem);
     cfg.stream = st;
     cfg.attrs = attr_c;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_lora_tc<A_MN, B_MN>, ma, mb, p);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_lora_tc<A_MN, B_MN>, ma, mb, ma2, mb2, p);
     note_launches(1);
     return e;
+}
+
+template <bool A_MN, bool B_MN>
+cudaError_t run(const Plan& pl, const CUtensorMap& ma, const CUtensorMap& mb, int64_t rows, int r, float scale,
+                uint16_t* out, bool transposed, cudaStream_t st, int ldo = 0) {
+    const SkinnyOut o = out_desc(out, rows, r, scale, transposed, ldo);
+    return launch_skinny<A_MN, B_MN>(pl, ma, mb, o, ma, mb, o, 0, r, st);
 }
 
 }  // namespace
@@ -345,6 +381,23 @@ cudaError_t launch_lora_db_tc(const uint16_t* dY, const uint16_t* T, int64_t M, 
         !make_map(&mb, T, r, M, 64, kBK, static_cast<uint64_t>(ld_t)))
         return cudaErrorInvalidValue;
     return run<true, true>(pl, ma, mb, N, r, 1.0f, dB, false, st);
+}
+
+// dA and dB of one linear in one launch: both read their operands across
+// the contraction (MN-major) over the same M tokens; the split count is
+// planned for their row tiles together.
+cudaError_t launch_lora_grads_tc(const uint16_t* X, const uint16_t* U, const uint16_t* dY, const uint16_t* T,
+                                 int64_t M, int64_t N, int64_t K, int r, uint16_t* dA, uint16_t* dB,
+                                 cudaStream_t st) {
+    Plan pl = plan(K + N, M, r, true);
+    const int64_t tiles_a = ceil_div(K, kRows), tiles_b = ceil_div(N, kRows);
+    pl.tiles = tiles_a;
+    CUtensorMap ma, mb, mc, md;
+    if (!make_map(&ma, X, K, M, 64, kBK) || !make_map(&mb, U, r, M, 64, kBK) || !make_map(&mc, dY, N, M, 64, kBK) ||
+        !make_map(&md, T, r, M, 64, kBK))
+        return cudaErrorInvalidValue;
+    return launch_skinny<true, true>(pl, ma, mb, out_desc(dA, K, r, 1.0f, true, 0), mc, md,
+                                     out_desc(dB, N, r, 1.0f, false, 0), tiles_b, r, st);
 }
 
 int lora_device_error(int reset) {
