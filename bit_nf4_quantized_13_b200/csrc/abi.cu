@@ -334,25 +334,18 @@ int qlora_linear_group_bwd(int qtype, const uint16_t* dY, const uint16_t* X, int
         e = lora_xat(X, A_cat, M, n_all, K, rc, s, Tw, cs);
         T = Tw;
     }
-    // U_g = s dY_g B_g into columns g r .. of U; dY_g is a column block of dY
-    int64_t n0 = 0;
-    for (int i = 0; i < G && e == cudaSuccess; ++i) {
-        e = launch_lora_dyb_tc(dY + n0, B_cat + n0 * r, M, g.w[i].N, r, s, U + static_cast<int64_t>(i) * r, cs, n_all,
-                               rc);
-        n0 += g.w[i].N;
-    }
+    // U_g = s dY_g B_g into columns g r .. of U (dY_g a column block of dY), one launch
+    int64_t Ns[kMaxGroupLinears];
+    for (int i = 0; i < G; ++i) Ns[i] = g.w[i].N;
+    if (e == cudaSuccess) e = launch_lora_dyb_group(dY, B_cat, M, Ns, G, r, s, U, cs);
     if (e == cudaSuccess && dX) {
         e = launch_bwd_dx_gemm_pair_group(dY, g, U, A_cat, M, r, dX, reinterpret_cast<char*>(ws) + 2 * mr,
                                           ws_bytes - 2 * mr, cs);
         if (e == cudaErrorNotSupported) return QLORA_ERR_UNSUPPORTED;
     }
-    // dA_g = U_g^T X for all g at once (rows of dA_cat); dB_g = dY_g^T T_g
+    // dA_g = U_g^T X for all g at once (rows of dA_cat); dB_g = dY_g^T T_g, one launch
     if (e == cudaSuccess) e = launch_lora_da_tc(X, U, M, K, rc, dA_cat, cs);
-    n0 = 0;
-    for (int i = 0; i < G && e == cudaSuccess; ++i) {
-        e = launch_lora_db_tc(dY + n0, T + static_cast<int64_t>(i) * r, M, g.w[i].N, r, dB_cat + n0 * r, cs, n_all, rc);
-        n0 += g.w[i].N;
-    }
+    if (e == cudaSuccess) e = launch_lora_db_group(dY, T, M, Ns, G, r, dB_cat, cs);
     return cuda_status(e);
 }
 

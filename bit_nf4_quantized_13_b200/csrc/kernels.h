@@ -61,6 +61,12 @@ cudaError_t launch_lora_da_tc(const uint16_t* X, const uint16_t* U, int64_t M, i
                               cudaStream_t stream);
 cudaError_t launch_lora_db_tc(const uint16_t* dY, const uint16_t* T, int64_t M, int64_t N, int r, uint16_t* dB,
                               cudaStream_t stream, int64_t ld_dy = 0, int64_t ld_t = 0);
+// the G linears of a group in one launch each: U_g (columns g r .. of U,
+// row pitch G r) and dB_g (rows n_g .. of dB_cat); dY is M x sum(Ns)
+cudaError_t launch_lora_dyb_group(const uint16_t* dY, const uint16_t* B_cat, int64_t M, const int64_t* Ns, int G,
+                                  int r, float s, uint16_t* U, cudaStream_t stream);
+cudaError_t launch_lora_db_group(const uint16_t* dY, const uint16_t* T, int64_t M, const int64_t* Ns, int G, int r,
+                                 uint16_t* dB_cat, cudaStream_t stream);
 // dA and dB in one launch
 cudaError_t launch_lora_grads_tc(const uint16_t* X, const uint16_t* U, const uint16_t* dY, const uint16_t* T,
                                  int64_t M, int64_t N, int64_t K, int r, uint16_t* dA, uint16_t* dB,

@@ -45,25 +45,29 @@ constexpr int kThreads = 128;
 constexpr int kABytes = kRows * kBK * 2;  // 16 KiB
 constexpr int kMaxSmem = 200 * 1024;
 
-// One product's output: rows x r bf16 (row pitch ldo), or r x rows when
-// transposed, scaled by `scale` before the rounding.
+// One product of a launch: its output, rows x r bf16 (row pitch ldo), or
+// r x rows when transposed, scaled by `scale` before the rounding; its
+// contraction length; its first row tile in the grid.
 struct SkinnyOut {
     uint16_t* out;
     int ldo;
     float scale;
     int transposed;
     int rows;      // output rows
+    int kb_total;  // 64-wide contraction blocks
+    int tile0;     // grid x of its first row tile
 };
 
-// A launch computes one product, or two of the same kind (the same operand
-// majorness, rank and contraction length: dA and dB), CTAs with blockIdx.x
-// below tiles0 taking the first and the rest the second.
+// A launch computes up to kMaxProducts products of one kind (the same
+// operand majorness and rank: dA with dB, or the U or dB of the linears of a
+// group), CTA column blockIdx.x belonging to the last product whose tile0
+// it has reached.
+constexpr int kMaxProducts = 4;
 struct SkinnyParams {
-    SkinnyOut o[2];
-    int tiles0;    // row tiles of the first product
+    SkinnyOut o[kMaxProducts];
+    int nprod;
     int r;
     int nt;        // r rounded up to 16 (MMA N)
-    int kb_total;  // 64-wide contraction blocks
     int splits;    // CTAs per cluster, a power of two
     int stages;
     int b_bytes;   // bytes of one B stage
@@ -72,8 +76,10 @@ struct SkinnyParams {
 
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kThreads)
-k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
-          const __grid_constant__ CUtensorMap ta2, const __grid_constant__ CUtensorMap tb2, const SkinnyParams p) {
+k_lora_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
+          const __grid_constant__ CUtensorMap ta1, const __grid_constant__ CUtensorMap tb1,
+          const __grid_constant__ CUtensorMap ta2, const __grid_constant__ CUtensorMap tb2,
+          const __grid_constant__ CUtensorMap ta3, const __grid_constant__ CUtensorMap tb3, const SkinnyParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int stage_bytes = kABytes + p.b_bytes;
@@ -85,14 +91,16 @@ k_lora_tc(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtens
     auto empty = [&](int s) { return bar0 + 8u * (p.stages + s); };
     const uint32_t done = bar0 + 8u * (2 * p.stages);
 
-    const bool second = static_cast<int>(blockIdx.x) >= p.tiles0;
-    const SkinnyOut o = second ? p.o[1] : p.o[0];
-    const CUtensorMap* mapa = second ? &ta2 : &ta;
-    const CUtensorMap* mapb = second ? &tb2 : &tb;
-    const int row0 = (static_cast<int>(blockIdx.x) - (second ? p.tiles0 : 0)) * kRows;
+    const int bx = static_cast<int>(blockIdx.x);
+    const int prod = (p.nprod > 1 && bx >= p.o[1].tile0 ? 1 : 0) + (p.nprod > 2 && bx >= p.o[2].tile0 ? 1 : 0) +
+                     (p.nprod > 3 && bx >= p.o[3].tile0 ? 1 : 0);
+    const SkinnyOut o = prod == 0 ? p.o[0] : prod == 1 ? p.o[1] : prod == 2 ? p.o[2] : p.o[3];
+    const CUtensorMap* mapa = prod == 0 ? &ta0 : prod == 1 ? &ta1 : prod == 2 ? &ta2 : &ta3;
+    const CUtensorMap* mapb = prod == 0 ? &tb0 : prod == 1 ? &tb1 : prod == 2 ? &tb2 : &tb3;
+    const int row0 = (bx - o.tile0) * kRows;
     const int split = static_cast<int>(cluster_ctarank());  // == blockIdx.y: the cluster spans the splits
-    const int kb_begin = static_cast<int>(static_cast<int64_t>(split) * p.kb_total / p.splits);
-    const int kb_end = static_cast<int>(static_cast<int64_t>(split + 1) * p.kb_total / p.splits);
+    const int kb_begin = static_cast<int>(static_cast<int64_t>(split) * o.kb_total / p.splits);
+    const int kb_end = static_cast<int>(static_cast<int64_t>(split + 1) * o.kb_total / p.splits);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
@@ -281,49 +289,58 @@ Plan plan(int64_t rows, int64_t ctr, int r, bool b_mn) {
     return pl;
 }
 
-SkinnyOut out_desc(uint16_t* out, int64_t rows, int r, float scale, bool transposed, int ldo) {
+SkinnyOut out_desc(uint16_t* out, int64_t rows, int r, float scale, bool transposed, int ldo, int kb_total) {
     SkinnyOut o;
     o.out = out;
     o.ldo = ldo ? ldo : r;
     o.scale = scale;
     o.transposed = transposed ? 1 : 0;
     o.rows = static_cast<int>(rows);
+    o.kb_total = kb_total;
+    o.tile0 = 0;
     return o;
 }
 
-// Launches one product (tiles1 == 0) or two of the same kind in one grid:
-// the first product's pl.tiles row tiles, then tiles1 of the second.
+// Launches n (1 .. kMaxProducts) products of one kind in one grid: product
+// i's ceil(rows / 128) row tiles after those of the products before it.
+// pl supplies the shared shape (rank, stages, shared memory, splits).
 template <bool A_MN, bool B_MN>
-cudaError_t launch_skinny(const Plan& pl, const CUtensorMap& ma, const CUtensorMap& mb, const SkinnyOut& o0,
-                          const CUtensorMap& ma2, const CUtensorMap& mb2, const SkinnyOut& o1, int64_t tiles1,
+cudaError_t launch_skinny(const Plan& pl, int n, const CUtensorMap* ma, const CUtensorMap* mb, const SkinnyOut* o,
                           int r, cudaStream_t st) {
     static ContextMemo<int> attr_memo;
     const cudaError_t attr = ensure_smem_limit(attr_memo, k_lora_tc<A_MN, B_MN>, kMaxSmem + 2048);
     if (attr != cudaSuccess) return attr;
-    SkinnyParams p;
-    p.o[0] = o0;
-    p.o[1] = o1;
-    p.tiles0 = static_cast<int>(pl.tiles);
+    if (n < 1 || n > kMaxProducts) return cudaErrorInvalidValue;
+    SkinnyParams p{};
+    int64_t tiles = 0;
+    for (int i = 0; i < kMaxProducts; ++i) {
+        p.o[i] = o[i < n ? i : 0];
+        p.o[i].tile0 = static_cast<int>(tiles);
+        if (i < n) tiles += ceil_div(o[i].rows > 0 ? o[i].rows : 1, kRows);
+    }
+    p.nprod = n;
     p.r = r;
     p.nt = pl.nt;
-    p.kb_total = pl.kb_total;
     p.splits = pl.splits;
     p.stages = pl.stages;
     p.b_bytes = pl.b_bytes;
     p.tmem_cols = pl.tmem_cols;
+    if (tiles >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr_c[1];
     attr_c[0].id = cudaLaunchAttributeClusterDimension;
     attr_c[0].val.clusterDim.x = 1;
     attr_c[0].val.clusterDim.y = static_cast<unsigned>(pl.splits);
     attr_c[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(static_cast<unsigned>(pl.tiles + tiles1), static_cast<unsigned>(pl.splits));
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(pl.splits));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = static_cast<size_t>(pl.smem);
     cfg.stream = st;
     cfg.attrs = attr_c;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_lora_tc<A_MN, B_MN>, ma, mb, ma2, mb2, p);
+    auto m = [&](const CUtensorMap* v, int i) -> const CUtensorMap& { return v[i < n ? i : 0]; };
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_lora_tc<A_MN, B_MN>, m(ma, 0), m(mb, 0), m(ma, 1), m(mb, 1),
+                                             m(ma, 2), m(mb, 2), m(ma, 3), m(mb, 3), p);
     note_launches(1);
     return e;
 }
@@ -331,8 +348,8 @@ cudaError_t launch_skinny(const Plan& pl, const CUtensorMap& ma, const CUtensorM
 template <bool A_MN, bool B_MN>
 cudaError_t run(const Plan& pl, const CUtensorMap& ma, const CUtensorMap& mb, int64_t rows, int r, float scale,
                 uint16_t* out, bool transposed, cudaStream_t st, int ldo = 0) {
-    const SkinnyOut o = out_desc(out, rows, r, scale, transposed, ldo);
-    return launch_skinny<A_MN, B_MN>(pl, ma, mb, o, ma, mb, o, 0, r, st);
+    const SkinnyOut o = out_desc(out, rows, r, scale, transposed, ldo, pl.kb_total);
+    return launch_skinny<A_MN, B_MN>(pl, 1, &ma, &mb, &o, r, st);
 }
 
 }  // namespace
@@ -384,20 +401,88 @@ cudaError_t launch_lora_db_tc(const uint16_t* dY, const uint16_t* T, int64_t M, 
 }
 
 // dA and dB of one linear in one launch: both read their operands across
-// the contraction (MN-major) over the same M tokens; the split count is
-// planned for their row tiles together.
+// the contraction (MN-major) over the same M tokens.  The split count is
+// the largest (<= 8) that keeps both products' row tiles x splits within
+// two CTAs per SM: measured on the 7B and 65B shapes, more splits only add
+// waves of clusters (and their fixed cost), fewer leave SMs idle.
 cudaError_t launch_lora_grads_tc(const uint16_t* X, const uint16_t* U, const uint16_t* dY, const uint16_t* T,
                                  int64_t M, int64_t N, int64_t K, int r, uint16_t* dA, uint16_t* dB,
                                  cudaStream_t st) {
     Plan pl = plan(K + N, M, r, true);
     const int64_t tiles_a = ceil_div(K, kRows), tiles_b = ceil_div(N, kRows);
-    pl.tiles = tiles_a;
-    CUtensorMap ma, mb, mc, md;
-    if (!make_map(&ma, X, K, M, 64, kBK) || !make_map(&mb, U, r, M, 64, kBK) || !make_map(&mc, dY, N, M, 64, kBK) ||
-        !make_map(&md, T, r, M, 64, kBK))
+    int splits = 1;
+    while (splits * 2 <= 8 && splits * 2 <= pl.kb_total && (tiles_a + tiles_b) * splits * 2 <= 2LL * num_sms())
+        splits *= 2;
+    pl.splits = splits;
+    CUtensorMap ma[2], mb[2];
+    if (!make_map(&ma[0], X, K, M, 64, kBK) || !make_map(&mb[0], U, r, M, 64, kBK) ||
+        !make_map(&ma[1], dY, N, M, 64, kBK) || !make_map(&mb[1], T, r, M, 64, kBK))
         return cudaErrorInvalidValue;
-    return launch_skinny<true, true>(pl, ma, mb, out_desc(dA, K, r, 1.0f, true, 0), mc, md,
-                                     out_desc(dB, N, r, 1.0f, false, 0), tiles_b, r, st);
+    const SkinnyOut o[2] = {out_desc(dA, K, r, 1.0f, true, 0, pl.kb_total), out_desc(dB, N, r, 1.0f, false, 0, pl.kb_total)};
+    return launch_skinny<true, true>(pl, 2, ma, mb, o, r, st);
+}
+
+namespace {
+
+// Largest split count (<= 8, <= kb) whose CTAs (tiles x splits) stay within
+// two per SM.
+int group_splits(int64_t tiles, int kb) {
+    int splits = 1;
+    while (splits * 2 <= 8 && splits * 2 <= kb && tiles * splits * 2 <= 2LL * num_sms()) splits *= 2;
+    return splits;
+}
+
+}  // namespace
+
+// U_g = bf16(s dY_g B_g) for the G linears of a group in one launch: dY_g is
+// the column block n_g .. of dY (row pitch n_all), B_g the rows n_g .. of
+// B_cat, U_g the columns g r .. of U (row pitch G r).
+cudaError_t launch_lora_dyb_group(const uint16_t* dY, const uint16_t* B_cat, int64_t M, const int64_t* Ns, int G,
+                                  int r, float s, uint16_t* U, cudaStream_t st) {
+    if (G < 1 || G > kMaxProducts) return cudaErrorInvalidValue;
+    int64_t n_all = 0, n_max = 0, n_min = -1;
+    for (int g = 0; g < G; ++g) {
+        n_all += Ns[g];
+        n_max = Ns[g] > n_max ? Ns[g] : n_max;
+        n_min = (n_min < 0 || Ns[g] < n_min) ? Ns[g] : n_min;
+    }
+    Plan pl = plan(M * G, n_max, r, true);
+    pl.splits = group_splits(G * ceil_div(M, kRows), static_cast<int>(ceil_div(n_min, kBK)));
+    CUtensorMap ma[kMaxProducts], mb[kMaxProducts];
+    SkinnyOut o[kMaxProducts];
+    int64_t n0 = 0;
+    for (int g = 0; g < G; ++g) {
+        if (!make_map(&ma[g], dY + n0, Ns[g], M, kBK, kRows, static_cast<uint64_t>(n_all)) ||
+            !make_map(&mb[g], B_cat + n0 * r, r, Ns[g], 64, kBK))
+            return cudaErrorInvalidValue;
+        o[g] = out_desc(U + static_cast<int64_t>(g) * r, M, r, s, false, G * r, static_cast<int>(ceil_div(Ns[g], kBK)));
+        n0 += Ns[g];
+    }
+    return launch_skinny<false, true>(pl, G, ma, mb, o, r, st);
+}
+
+// dB_g = bf16(dY_g^T T_g) for the G linears of a group in one launch (dB_g
+// the rows n_g .. of dB_cat; T_g the columns g r .. of T, row pitch G r).
+cudaError_t launch_lora_db_group(const uint16_t* dY, const uint16_t* T, int64_t M, const int64_t* Ns, int G, int r,
+                                 uint16_t* dB_cat, cudaStream_t st) {
+    if (G < 1 || G > kMaxProducts) return cudaErrorInvalidValue;
+    int64_t n_all = 0;
+    for (int g = 0; g < G; ++g) n_all += Ns[g];
+    Plan pl = plan(n_all, M, r, true);
+    int64_t tiles = 0;
+    for (int g = 0; g < G; ++g) tiles += ceil_div(Ns[g], kRows);
+    pl.splits = group_splits(tiles, pl.kb_total);
+    CUtensorMap ma[kMaxProducts], mb[kMaxProducts];
+    SkinnyOut o[kMaxProducts];
+    int64_t n0 = 0;
+    for (int g = 0; g < G; ++g) {
+        if (!make_map(&ma[g], dY + n0, Ns[g], M, 64, kBK, static_cast<uint64_t>(n_all)) ||
+            !make_map(&mb[g], T + static_cast<int64_t>(g) * r, r, M, 64, kBK, static_cast<uint64_t>(G) * r))
+            return cudaErrorInvalidValue;
+        o[g] = out_desc(dB_cat + n0 * r, Ns[g], r, 1.0f, false, 0, pl.kb_total);
+        n0 += Ns[g];
+    }
+    return launch_skinny<true, true>(pl, G, ma, mb, o, r, st);
 }
 
 int lora_device_error(int reset) {
