@@ -753,12 +753,16 @@ def run_llama65b_layer(q, torch, dev, stream, flush, peaks, args):
                 if ev is not None:
                     ev[i][2].record(stream)
 
+        block_pass, parts = grouped_block(q, torch, dev, lin, wqs, M)
         layer_pass()
+        block_pass()
         torch.cuda.synchronize()
         tw0 = time.time()
         fwd_ms = [0.0] * len(layer)
         bwd_ms = [0.0] * len(layer)
-        tot_ms = 0.0
+        tot_ms, blk_ms = 0.0, 0.0
+        # the layer linear by linear and as a grouped block, in turn, so that
+        # both meet the same clock and power state
         for _ in range(reps):
             flush()
             ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in layer]
@@ -768,6 +772,14 @@ def run_llama65b_layer(q, torch, dev, stream, flush, peaks, args):
                 fwd_ms[i] += ev[i][0].elapsed_time(ev[i][1]) / reps
                 bwd_ms[i] += ev[i][1].elapsed_time(ev[i][2]) / reps
             tot_ms += ev[0][0].elapsed_time(ev[-1][2]) / reps
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            block_pass()
+            b.record(stream)
+            torch.cuda.synchronize()
+            blk_ms += a.elapsed_time(b) / reps
+        del parts
         per = []
         fl_tot = 0.0
         for i, (nm, n, k) in enumerate(layer):
@@ -778,21 +790,20 @@ def run_llama65b_layer(q, torch, dev, stream, flush, peaks, args):
                         "fwd_bwd_tflops": (ff + fb) / ((fwd_ms[i] + bwd_ms[i]) * 1e-3) / 1e12})
         tf = fl_tot / (tot_ms * 1e-3) / 1e12
         tw1 = time.time()
-        grouped = grouped_layer(q, torch, dev, stream, flush, lin, wqs, M, reps, fl_tot, tot_ms)
-        tw2 = time.time()
+        grouped = {"layer_ms": blk_ms, "layer_tflops": fl_tot / (blk_ms * 1e-3) / 1e12,
+                   "vs_per_linear": tot_ms / blk_ms, "groups": "qkv, o, gate+up, down"}
         out[f"m{M}"] = {"layer_ms": tot_ms, "layer_flops": fl_tot, "layer_tflops": tf,
                         "frac_burst": tf / tc_b, "frac_sustained": tf / tc_s, "linears": per,
                         "clocks": sampler.summary(tw0, tw1), "grouped": grouped}
-        out[f"m{M}"]["grouped"]["clocks"] = sampler.summary(tw1, tw2)
         del lin
     sampler.stop()
     return out
 
 
-def grouped_layer(q, torch, dev, stream, flush, lin, wqs, M, reps, fl_tot, per_linear_ms):
+def grouped_block(q, torch, dev, lin, wqs, M):
     """The same layer as a decoder block runs it: q, k, v read one input and
     run as one grouped linear, gate and up likewise; o and down alone.  Same
-    FLOPs as the seven separate linears; timed over the whole pass."""
+    FLOPs as the seven separate linears.  Returns the pass and its buffers."""
     s_lora = ALPHA / RANK
     parts = []
     for idx in ((0, 1, 2), (3,), (4, 5), (6,)):
@@ -817,20 +828,7 @@ def grouped_layer(q, torch, dev, stream, flush, lin, wqs, M, reps, fl_tot, per_l
             q.qlora_linear_group_bwd(g["dY"], g["X"], g["w"], g["A"], g["B"], s_lora, T=g["T"], dX=g["dX"],
                                      dA_cat=g["dA"], dB_cat=g["dB"], ws=g["ws"])
 
-    block_pass()
-    torch.cuda.synchronize()
-    ms = 0.0
-    for _ in range(reps):
-        flush()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        block_pass()
-        b.record(stream)
-        torch.cuda.synchronize()
-        ms += a.elapsed_time(b) / reps
-    del parts
-    return {"layer_ms": ms, "layer_tflops": fl_tot / (ms * 1e-3) / 1e12, "vs_per_linear": per_linear_ms / ms,
-            "groups": "qkv, o, gate+up, down"}
+    return block_pass, parts
 
 
 def decode_bytes(M, N, K, r):
