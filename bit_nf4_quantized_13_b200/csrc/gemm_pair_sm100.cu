@@ -373,40 +373,6 @@ __device__ __forceinline__ uint32_t lop_select(uint32_t a, uint32_t b, uint32_t 
     return (a & ~m) | (b & m);  // one LOP3
 }
 
-// Converts one 64-weight run and writes it as row `row` (128 bytes at
-// shared address `row_base`) of an operand tile in the 128-byte swizzled
-// layout: the 16-byte chunk of weights 8h .. 8h + 7 goes to chunk
-// h ^ (row & 7).  Each chunk is stored as soon as it is formed.
-__device__ __forceinline__ void convert_store_run(const uint4& c0, const uint4& c1, float sc, const float (&q)[16],
-                                                  uint32_t row_base, int row) {
-    uint32_t L[4], H[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const uint32_t t0 = pack_bf16x2(__fmul_rn(q[4 * k], sc), __fmul_rn(q[4 * k + 1], sc));
-        const uint32_t t1 = pack_bf16x2(__fmul_rn(q[4 * k + 2], sc), __fmul_rn(q[4 * k + 3], sc));
-        L[k] = prmt(t0, t1, 0x6420u);  // low bytes of p_4k .. p_4k+3
-        H[k] = prmt(t0, t1, 0x7531u);  // high bytes
-    }
-    const uint32_t w8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-    for (int h = 0; h < 8; ++h) {
-        uint32_t v[4];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const uint32_t w = (w8[h] >> (16 * half)) & 0xffffu;  // code bytes 2 half, 2 half + 1
-            const uint32_t sel = w & 0x7777u;
-            const uint32_t m = prmt(w << 4, w, 0xD9C8u);        // byte j: 0xff iff bit 3 of nibble j
-            const uint32_t lo = lop_select(prmt(L[0], L[1], sel), prmt(L[2], L[3], sel), m);
-            const uint32_t hi = lop_select(prmt(H[0], H[1], sel), prmt(H[2], H[3], sel), m);
-            // lo/hi bytes hold weights (1, 0, 3, 2) of the four
-            v[2 * half] = prmt(lo, hi, 0x4051u);      // (w0, w1)
-            v[2 * half + 1] = prmt(lo, hi, 0x6273u);  // (w2, w3)
-        }
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_base + ((h ^ (row & 7)) << 4)), "r"(v[0]),
-                     "r"(v[1]), "r"(v[2]), "r"(v[3])
-                     : "memory");
-    }
-}
 
 // The same conversion into registers (32 bf16 pairs, even element in the
 // low half), for a store after the ring slot is free.
@@ -446,12 +412,6 @@ __device__ __forceinline__ void store_swizzled_row(uint32_t row_base, int row, c
                      : "memory");
 }
 
-// A row of zeros (a run outside W, part of the contraction in the backward).
-__device__ __forceinline__ void store_zero_row(uint32_t row_base) {
-#pragma unroll
-    for (int h = 0; h < 8; ++h)
-        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(row_base + (h << 4)), "r"(0u) : "memory");
-}
 
 // The 64-weight run that lane task `t` (0..127) of a weight stage converts:
 // its weight row n and first column kcol in W (valid = inside W), and where
