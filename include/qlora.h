@@ -206,7 +206,7 @@ size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int r);
  * the four buffers of qlora_quantize_nf4_dq for an N x K row-major weight.
  * Requires K % 64 == 0, 1 <= r <= 256, M >= 0, N >= 1.
  * Small batches (1 <= M <= 16 with N % 16 == 0, 8 <= r <= 64, r % 8 == 0,
- * K <= 23040) take a single weight-streaming kernel that applies each
+ * K <= 21504) take a single weight-streaming kernel that applies each
  * 64-block's constant c2' to the block's partial dot product, i.e. the
  * weight enters as bf16(q[code]) * c2' rather than bf16(q[code] * c2'):
  * the same value up to one bf16 rounding, within the forward's tolerance.
