@@ -75,12 +75,13 @@ def test_tile_spanning_shape():
 
 @pytest.mark.parametrize("M,N,K", [(830, 4864, 128), (1001, 4864, 128), (1090, 4864, 128), (1200, 4864, 128),
                                    (830, 128, 4864), (1001, 128, 4864), (1090, 128, 4864), (1200, 128, 4864)])
-def test_every_token_tile_width(M, N, K):
-    """The GEMMs pick a token-tile width of 256, 320, 352, 384 or 416 per
-    problem from the tile count per CTA round (148 CTAs): these shapes
-    select 320, 352, 384 and 416 in the forward (weight rows N = 4864) and
-    in the dX product (rows K = 4864), each with a ragged token tail; 64
-    sampled rows."""
+def test_partial_rounds_and_split_tiles(M, N, K):
+    """Tile counts that leave the GEMMs' last round of tiles partly empty:
+    the forward with 19 weight-row tiles (N = 4864) x 2-3 token tiles of
+    512, and the dX product with 19 row tiles (K = 4864) over a contraction
+    of only two 64-blocks plus the LoRA slab, each with a ragged token tail,
+    so the last round's stages are split between SM pairs and finished
+    through the workspace; 64 sampled rows."""
     case = synth.linear_case(f"w{M}n{N}k{K}", M, N, K, 16, 16.0, seed=21, outlier_frac=0.001)
     rows = np.sort(synth.rng(0, 121).choice(M, 64, replace=False)).astype(np.int64)
     _run_case(case, rows=rows)
