@@ -450,6 +450,7 @@ def run_native(args, world, rank, local):
                 dq32_ms += e0.elapsed_time(e1)
                 dq32_bytes += dequant_bytes(n, 4)
     del w32buf
+    other_types = run_other_types(q, torch, dev, stream, flush, bufs, peaks_hbm=load_peaks()[0]["hbm_gbs"])
     # the DRAM ceilings these kernels meet, from the library's own probe
     # kernels (16-byte streaming stores / loads) over a 2 GiB buffer, 16x the
     # L2, so that the cache absorbs a negligible part; torch's fill beside
@@ -626,6 +627,7 @@ def run_native(args, world, rank, local):
                 "fwd_tflops": fwd_tflops, "fwd_frac_tensor": fwd_tflops / tc_peak,
                 "bwd_tflops": bflops / (bt * 1e-3) / 1e12, "dx_path_tflops": dx_tflops,
                 "unfused_fwd_tflops": k9_tflops,
+                "other_types": other_types,
                 "decode": decode,
                 "full_llama7b_weight_set": full7b,
                 "llama65b_layer": l65b,
@@ -797,6 +799,50 @@ def run_llama65b_layer(q, torch, dev, stream, flush, peaks, args):
                         "clocks": sampler.summary(tw0, tw1), "grouped": grouped}
         del lin
     sampler.stop()
+    return out
+
+
+def run_other_types(q, torch, dev, stream, flush, bufs, peaks_hbm):
+    """The comparison types on the same two 7B-shaped weights: quantization
+    to FP4 (E2M1) and Int4 with the NF4 path's kernels (the type's table),
+    and block-wise Int8 (block 64) quantize and dequantize; per call, L2
+    flushed, mean over 3 timed rounds after 2."""
+    def timed(fn):
+        ms = 0.0
+        for rep in range(5):
+            for b in bufs:
+                flush()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn(b)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if rep >= 2:
+                    ms += e0.elapsed_time(e1)
+        return ms / 3
+    out = {}
+    nbytes_q = sum(quant_bytes(b["case"].W.size) for b in bufs)
+    for name, qt in (("fp4", q.TYPE_FP4), ("int4", q.TYPE_INT4)):
+        ws_ = [q.alloc_nf4_weight(b["case"].W.shape, dev, qt) for b in bufs]
+        idx = {id(b): i for i, b in enumerate(bufs)}
+        ms = timed(lambda b: q.qlora_quantize_nf4_dq(b["W"], out=ws_[idx[id(b)]], ws=b["qws"], qtype=qt))
+        out[f"{name}_quantize_gbs"] = nbytes_q / (ms * 1e-3) / 1e9
+        out[f"{name}_quantize_frac_hbm"] = out[f"{name}_quantize_gbs"] / peaks_hbm
+        del ws_
+    n_all = sum(b["case"].W.size for b in bufs)
+    i8 = [(torch.empty(b["case"].W.size, dtype=torch.int8, device=dev),
+           torch.empty(-(-b["case"].W.size // 64), dtype=torch.float32, device=dev),
+           torch.empty(b["case"].W.size, dtype=torch.float32, device=dev)) for b in bufs]
+    idx = {id(b): i for i, b in enumerate(bufs)}
+    int8_bytes = n_all * (4 + 1) + 4 * sum(-(-b["case"].W.size // 64) for b in bufs)
+    ms = timed(lambda b: q.qlora_int8_quantize(b["W"].view(-1), 64, codes=i8[idx[id(b)]][0], c=i8[idx[id(b)]][1]))
+    out["int8_quantize_gbs"] = int8_bytes / (ms * 1e-3) / 1e9
+    ms = timed(lambda b: q.qlora_int8_dequantize(i8[idx[id(b)]][0], i8[idx[id(b)]][1], 64, out=i8[idx[id(b)]][2]))
+    out["int8_dequant_gbs"] = int8_bytes / (ms * 1e-3) / 1e9
+    out["int8_quantize_frac_hbm"] = out["int8_quantize_gbs"] / peaks_hbm
+    out["int8_dequant_frac_hbm"] = out["int8_dequant_gbs"] / peaks_hbm
+    out["note"] = "both 7B-shaped weights per round; Int8 bytes: 4 B fp32 + 1 B code per element + 4 B per 64-block"
+    del i8
     return out
 
 

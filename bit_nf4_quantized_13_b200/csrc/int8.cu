@@ -6,10 +6,11 @@
 //   x' = RN32(code / c)             (a block with absmax 0: c = 0, x' = 0)
 //
 // HBM-bound: 4 bytes read and 1 + 4/block written per element to quantize,
-// 1 + 4/block read and 4 written to dequantize.  A warp takes one block of
-// `kB` consecutive elements at a time; lane l holds elements kB/32 * l ...
-// (contiguous), so loads and stores are single vector accesses per lane
-// and whole warps read and write contiguous runs.
+// 1 + 4/block read and 4 written to dequantize.  A warp takes blocks of
+// `kB` consecutive elements, two to four at a time (all their loads issued
+// before any is used); lane l holds elements kB/32 * l ... of a block
+// (contiguous), so loads and stores are vector accesses per lane and whole
+// warps read and write contiguous runs.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -81,29 +82,39 @@ __global__ void __launch_bounds__(kThreads)
 k_int8_quantize(const float* __restrict__ x, int64_t nfull, int8_t* __restrict__ codes, float* __restrict__ c,
                 int* __restrict__ bad_flag) {
     constexpr int kPer = kB / 32;
+    constexpr int kU = kPer >= 8 ? 2 : 4;  // blocks a warp has in flight
     const int lane = threadIdx.x & 31;
     const int64_t nw = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
     bool bad = false;
-    for (int64_t b = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5; b < nfull; b += nw) {
-        const int64_t e = b * kB + static_cast<int64_t>(lane) * kPer;
-        float v[kPer];
-        Vec<kPer>::load(x + e, v);
-        float a = 0.0f;
+    for (int64_t b0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5; b0 < nfull; b0 += nw * kU) {
+        float v[kU][kPer];
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) a = fmaxf(a, fabsf(v[i]));
-        bool nonfinite = false;
+        for (int u = 0; u < kU; ++u) {
+            const int64_t b = b0 + u * nw;
+            if (b < nfull) Vec<kPer>::load(x + b * kB + static_cast<int64_t>(lane) * kPer, v[u]);
+        }
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) nonfinite |= !isfinite(v[i]);
+        for (int u = 0; u < kU; ++u) {
+            const int64_t b = b0 + u * nw;
+            if (b >= nfull) break;
+            const int64_t e = b * kB + static_cast<int64_t>(lane) * kPer;
+            float a = 0.0f;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-        const float cc = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
-        nonfinite |= !isfinite(cc);
-        bad |= nonfinite;
-        int q[kPer];
+            for (int i = 0; i < kPer; ++i) a = fmaxf(a, fabsf(v[u][i]));
+            bool nonfinite = false;
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) q[i] = isfinite(cc) ? static_cast<int>(roundf(__fmul_rn(cc, v[i]))) : 0;
-        store_codes<kPer>(codes + e, q);
-        if (lane == 0) c[b] = cc;
+            for (int i = 0; i < kPer; ++i) nonfinite |= !isfinite(v[u][i]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            const float cc = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+            nonfinite |= !isfinite(cc);
+            bad |= nonfinite;
+            int q[kPer];
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) q[i] = isfinite(cc) ? static_cast<int>(roundf(__fmul_rn(cc, v[u][i]))) : 0;
+            store_codes<kPer>(codes + e, q);
+            if (lane == 0) c[b] = cc;
+        }
     }
     if (bad && bad_flag) atomicExch(bad_flag, QLORA_ERR_NONFINITE);
 }
@@ -152,34 +163,48 @@ __global__ void __launch_bounds__(kThreads)
 k_int8_dequantize(const int8_t* __restrict__ codes, const float* __restrict__ c, int64_t numel,
                   float* __restrict__ out) {
     constexpr int kPer = kB / 32;
+    constexpr int kU = kPer >= 8 ? 2 : 4;  // blocks a warp has in flight
     const int lane = threadIdx.x & 31;
     const int64_t nw = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
     const int64_t nfull = numel / kB;
-    for (int64_t b = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5; b < nfull; b += nw) {
-        const int64_t e = b * kB + static_cast<int64_t>(lane) * kPer;
-        int q[kPer];
-        load_codes<kPer>(codes + e, q);
-        const float cc = __ldg(c + b);
-        float v[kPer];
+    for (int64_t b0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5; b0 < nfull; b0 += nw * kU) {
+        int q[kU][kPer];
+        float cc[kU];
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) v[i] = cc != 0.0f ? __fdiv_rn(static_cast<float>(q[i]), cc) : 0.0f;
+        for (int u = 0; u < kU; ++u) {
+            const int64_t b = b0 + u * nw;
+            if (b < nfull) {
+                load_codes<kPer>(codes + b * kB + static_cast<int64_t>(lane) * kPer, q[u]);
+                cc[u] = __ldg(c + b);
+            }
+        }
 #pragma unroll
-        for (int i = 0; i < kPer; i += (kPer >= 4 ? 4 : kPer)) {
-            if (kPer >= 4)
-                __stcs(reinterpret_cast<float4*>(out + e + i), make_float4(v[i], v[(i + 1) % kPer], v[(i + 2) % kPer],
-                                                                           v[(i + 3) % kPer]));
-            else if (kPer == 2)
-                __stcs(reinterpret_cast<float2*>(out + e), make_float2(v[0], v[1 % kPer]));
-            else
-                __stcs(out + e, v[0]);
+        for (int u = 0; u < kU; ++u) {
+            const int64_t b = b0 + u * nw;
+            if (b >= nfull) break;
+            const int64_t e = b * kB + static_cast<int64_t>(lane) * kPer;
+            float v[kPer];
+#pragma unroll
+            for (int i = 0; i < kPer; ++i)
+                v[i] = cc[u] != 0.0f ? __fdiv_rn(static_cast<float>(q[u][i]), cc[u]) : 0.0f;
+#pragma unroll
+            for (int i = 0; i < kPer; i += (kPer >= 4 ? 4 : kPer)) {
+                if (kPer >= 4)
+                    __stcs(reinterpret_cast<float4*>(out + e + i), make_float4(v[i], v[(i + 1) % kPer], v[(i + 2) % kPer],
+                                                                               v[(i + 3) % kPer]));
+                else if (kPer == 2)
+                    __stcs(reinterpret_cast<float2*>(out + e), make_float2(v[0], v[1 % kPer]));
+                else
+                    __stcs(out + e, v[0]);
+            }
         }
     }
     // the ragged last block, by the warp whose turn it is
     const int64_t tail = numel - nfull * kB;
     if (tail > 0 && ((static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5) == nfull % nw) {
-        const float cc = c[nfull];
+        const float ct = c[nfull];
         for (int64_t i = nfull * kB + lane; i < numel; i += 32)
-            out[i] = cc != 0.0f ? __fdiv_rn(static_cast<float>(codes[i]), cc) : 0.0f;
+            out[i] = ct != 0.0f ? __fdiv_rn(static_cast<float>(codes[i]), ct) : 0.0f;
     }
 }
 
