@@ -123,3 +123,44 @@ def test_quantize_and_dequantize_buffers_are_checked(fake):
 def test_cpu_tensors_are_refused_without_the_fake():
     with pytest.raises(ValueError):
         q._need_cuda(torch.zeros(4))
+
+
+def test_group_operands_reach_the_library(fake):
+    M, K, r = 48, 256, 16
+    ws_ = [weight(512, K), weight(256, K), weight(256, K)]
+    A_cat, B_cat = bf16(3 * r, K), bf16(1024, r)
+    Y, T = q.qlora_linear_group_fwd(bf16(M, K), ws_, A_cat, B_cat, 0.5)
+    assert Y.shape == (M, 1024) and T.shape == (M, 3 * r)
+    name, args = fake.calls[-1]
+    assert name == "qlora_linear_group_fwd" and args[0] == q.TYPE_NF4
+    assert args[2:4] == (M, K) and args[5] == 3 and args[8] == r
+    desc = args[4]  # the host array of weight descriptors
+    assert [desc[i].N for i in range(3)] == [512, 256, 256]
+    assert desc[1].codes == ws_[1].codes.data_ptr()
+    dX, dA, dB = q.qlora_linear_group_bwd(bf16(M, 1024), bf16(M, K), ws_, A_cat, B_cat, 0.5, T=T)
+    assert dX.shape == (M, K) and dA.shape == (3 * r, K) and dB.shape == (1024, r)
+    name, args = fake.calls[-1]
+    assert name == "qlora_linear_group_bwd" and args[3:5] == (M, K) and args[6] == 3 and args[9] == r
+
+
+def test_group_disagreeing_operands_are_refused(fake):
+    M, K, r = 8, 128, 8
+    w1, w2 = weight(256, K), weight(256, K)
+    X, A_cat, B_cat = bf16(M, K), bf16(2 * r, K), bf16(512, r)
+    bad = [
+        (X, [w1, weight(256, K + 64)], A_cat, B_cat),        # the weights disagree on K
+        (X, [w1, w2], bf16(2 * r + 1, K), B_cat),            # A_cat rows not G r
+        (X, [w1, w2], A_cat, bf16(511, r)),                  # B_cat rows not sum N_g
+        (X, [w1, w2, w1, w2, w1], bf16(5 * r, K), bf16(1280, r)),  # more than four linears
+        (X, [], A_cat, B_cat),                               # no linear
+        (X.float(), [w1, w2], A_cat, B_cat),                 # dtype
+    ]
+    for args in bad:
+        with pytest.raises(ValueError):
+            q.qlora_linear_group_fwd(*args, 1.0)
+    w_fp4 = q.alloc_nf4_weight((256, K), "cpu", q.TYPE_FP4)
+    with pytest.raises(ValueError):  # one 4-bit type per group
+        q.qlora_linear_group_fwd(X, [w1, w_fp4], A_cat, B_cat, 1.0)
+    with pytest.raises(ValueError):
+        q.qlora_linear_group_bwd(bf16(M, 511), X, [w1, w2], A_cat, B_cat, 1.0)
+    assert fake.calls == [], "nothing may reach the library"
