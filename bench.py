@@ -699,6 +699,7 @@ def run_full_7b_set(q, torch, dev, stream, peaks):
     b16 = sum(dequant_bytes(n * k, 2) for _, n, k in shapes)
     del out32, out16, wqs
     hbm = peaks["hbm_gbs"]
+    one = run_one_large_tensor(q, torch, dev, stream, hbm, timed)
     return {"tensors": len(shapes), "params": params, "bits_per_param": 8.0 * stored / params,
             "stored_bytes": stored,
             "quantize_ms": tq, "quantize_gbs": qbytes / (tq * 1e-3) / 1e9,
@@ -707,7 +708,33 @@ def run_full_7b_set(q, torch, dev, stream, peaks):
             "dequant_fp32_frac_hbm": b32 / (t32 * 1e-3) / 1e9 / hbm,
             "dequant_bf16_ms": t16, "dequant_bf16_gbs": b16 / (t16 * 1e-3) / 1e9,
             "dequant_bf16_frac_hbm": b16 / (t16 * 1e-3) / 1e9 / hbm,
-            "inputs": "Student-t df=5 x 0.02/sqrt(5/3), generated on the GPU (synth.student_t_device, seed 0)"}
+            "inputs": "Student-t df=5 x 0.02/sqrt(5/3), generated on the GPU (synth.student_t_device, seed 0)",
+            "one_tensor_32768x32768": one}
+
+
+def run_one_large_tensor(q, torch, dev, stream, hbm, timed):
+    """One 32768 x 32768 weight (2^30 weights, Student-t as the 7B set, 4 GiB
+    of fp32 against a 126 MB L2): quantize, dequantize to fp32 and to bf16,
+    each timed alone, so that the per-call fixed cost (launches, the bins'
+    clearing, the double quantization) is small against the streaming."""
+    n = 1 << 30
+    W = synth.student_t_device(0, 5000, n, dev).view(32768, 32768)
+    wq = q.alloc_nf4_weight((32768, 32768), dev)
+    qws = torch.empty(q.qlora_quantize_workspace_size(n), dtype=torch.uint8, device=dev)
+    q.qlora_quantize_nf4_dq(W, out=wq, ws=qws)
+    tq = timed(lambda: q.qlora_quantize_nf4_dq(W, out=wq, ws=qws), reps=3)
+    del W
+    out = {"quantize_ms": tq, "quantize_gbs": quant_bytes(n) / (tq * 1e-3) / 1e9}
+    for name, dtype, nbytes in (("fp32", torch.float32, 4), ("bf16", torch.bfloat16, 2)):
+        o = torch.empty((32768, 32768), dtype=dtype, device=dev)
+        q.qlora_dequantize(wq, dtype, out=o)
+        t = timed(lambda: q.qlora_dequantize(wq, dtype, out=o), reps=3)
+        out[f"dequant_{name}_ms"] = t
+        out[f"dequant_{name}_gbs"] = dequant_bytes(n, nbytes) / (t * 1e-3) / 1e9
+        del o
+    for k in [k for k in out if k.endswith("_gbs")]:
+        out[k.replace("_gbs", "_frac_hbm")] = out[k] / hbm
+    return out
 
 
 def run_llama65b_layer(q, torch, dev, stream, flush, peaks, args):
