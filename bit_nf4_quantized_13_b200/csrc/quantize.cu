@@ -246,14 +246,16 @@ k_nf4_quantize(const float* __restrict__ W, int64_t numel, uint8_t* __restrict__
 // bins[E] * 2^(max(E,1) - 150).  As an integer multiple of 2^-149 the total
 // is sum_E bins[E] << (max(E,1) - 1).  Lane l folds its eight bins
 // E = 8l .. 8l+7 into one 128-bit value relative to 2^(max(8l,1) - 1)
-// (each term < 2^64 shifted by at most 7: the sum stays below 2^75); lane 0
-// adds the non-zero lane values into 32-bit digits, rounds the total once to
-// the nearest double (round bit and sticky bit), divides by nb in double
-// and rounds to fp32.
+// (each term < 2^64 shifted by at most 7: the sum stays below 2^75).  The
+// non-zero lane values (one or two for real weights, whose constants share
+// a few exponents) are then added, by every lane alike, into 32-bit digits
+// held in registers (only compile-time indices, so nothing goes to local
+// memory); the total is rounded once to the nearest double (round bit and
+// sticky bit, from the leading 64 bits), divided by nb in double and
+// rounded to fp32.  Called by one whole warp; every lane returns the mean.
 constexpr int kDigits = 12;
 
-__device__ float mean_from_bins(const unsigned long long* __restrict__ bins, int64_t nb,
-                                unsigned long long* sv /* shared, 64: lane values lo, hi */) {
+__device__ float mean_from_bins(const unsigned long long* __restrict__ bins, int64_t nb) {
     const int lane = threadIdx.x & 31;
     unsigned long long lo = 0, hi = 0;
     const int e0 = 8 * lane, base = e0 ? e0 : 1;  // exponent field whose bin shift is the lane's origin
@@ -266,60 +268,63 @@ __device__ float mean_from_bins(const unsigned long long* __restrict__ bins, int
         lo += vlo;
         hi += vhi + (lo < vlo ? 1ull : 0ull);
     }
-    sv[2 * lane] = lo;
-    sv[2 * lane + 1] = hi;
-    __syncwarp();
-    float mu = 0.0f;
-    if (lane == 0) {
-        uint32_t d[kDigits + 1];
+    uint32_t d[kDigits + 1];
 #pragma unroll
-        for (int i = 0; i <= kDigits; ++i) d[i] = 0u;
-        for (int l = 0; l < 32; ++l) {
-            const unsigned long long vlo = sv[2 * l], vhi = sv[2 * l + 1];
-            if ((vlo | vhi) == 0ull) continue;
-            const int sh = (l ? 8 * l : 1) - 1;  // bit position of the lane value's origin
-            const int d0 = sh >> 5, off = sh & 31;
-            // the value (< 2^75) as 32-bit words, shifted by off into 4 words
-            const uint32_t w[3] = {static_cast<uint32_t>(vlo), static_cast<uint32_t>(vlo >> 32),
-                                   static_cast<uint32_t>(vhi)};
-            uint32_t p[4];
-            p[0] = w[0] << off;
-            p[1] = off ? (w[1] << off) | (w[0] >> (32 - off)) : w[1];
-            p[2] = off ? (w[2] << off) | (w[1] >> (32 - off)) : w[2];
-            p[3] = off ? (w[2] >> (32 - off)) : 0u;
-            unsigned long long carry = 0;
-            for (int i = 0; d0 + i <= kDigits; ++i) {
-                const unsigned long long t = static_cast<unsigned long long>(d[d0 + i]) + (i < 4 ? p[i] : 0u) + carry;
-                d[d0 + i] = static_cast<uint32_t>(t);
-                carry = t >> 32;
-                if (i >= 3 && carry == 0) break;
-            }
+    for (int i = 0; i <= kDigits; ++i) d[i] = 0u;
+    // the same mask in every lane, so the loop is warp-uniform
+    unsigned rest = __ballot_sync(0xffffffffu, (lo | hi) != 0ull);
+    while (rest) {
+        const int l = __ffs(rest) - 1;
+        rest &= rest - 1u;
+        const unsigned long long vlo = __shfl_sync(0xffffffffu, lo, l), vhi = __shfl_sync(0xffffffffu, hi, l);
+        const int sh = (l ? 8 * l : 1) - 1;  // bit position of the lane value's origin, <= 247
+        const int d0 = sh >> 5, off = sh & 31;
+        // the value (< 2^75) as 32-bit words, shifted by off into 4 words at digits d0 .. d0+3
+        const uint32_t w0 = static_cast<uint32_t>(vlo), w1 = static_cast<uint32_t>(vlo >> 32),
+                       w2 = static_cast<uint32_t>(vhi);
+        const uint32_t p0 = w0 << off;
+        const uint32_t p1 = off ? (w1 << off) | (w0 >> (32 - off)) : w1;
+        const uint32_t p2 = off ? (w2 << off) | (w1 >> (32 - off)) : w2;
+        const uint32_t p3 = off ? (w2 >> (32 - off)) : 0u;
+        unsigned long long carry = 0;
+#pragma unroll
+        for (int i = 0; i <= kDigits; ++i) {
+            const int k = i - d0;
+            const uint32_t add = k == 0 ? p0 : k == 1 ? p1 : k == 2 ? p2 : k == 3 ? p3 : 0u;
+            const unsigned long long t = static_cast<unsigned long long>(d[i]) + add + carry;
+            d[i] = static_cast<uint32_t>(t);
+            carry = t >> 32;
         }
-        int top = -1;
-        for (int i = kDigits; i >= 0; --i)
-            if (d[i]) { top = i; break; }
-        double sum = 0.0;
-        if (top >= 0) {
-            // the leading 64 bits of the total (digits top, top-1, top-2), left aligned
-            const unsigned long long t0 = (static_cast<unsigned long long>(d[top]) << 32) | (top >= 1 ? d[top - 1] : 0u);
-            const uint32_t t1 = top >= 2 ? d[top - 2] : 0u;
-            const int lz = __clzll(t0);  // < 32: d[top] != 0
-            const unsigned long long lead = lz ? (t0 << lz) | (static_cast<unsigned long long>(t1) >> (32 - lz)) : t0;
-            // bit position (over the whole total) of the lead's lowest bit
-            const int lead_lsb = 32 * top + 32 - lz - 64;  // = msb - 63, may be negative
-            unsigned long long m = lead >> 11;              // 53 bits
-            const bool rnd = (lead >> 10) & 1ull;
-            bool sticky = (lead & 0x3ffull) != 0;
-            // bits below the lead: the low lz bits of t1 and the digits under it
-            const uint32_t t1_below = lz ? (t1 & ((1u << (32 - lz)) - 1u)) : t1;  // t1's bits under the lead
-            sticky |= t1_below != 0u;
-            for (int i = 0; i < top - 2 && !sticky; ++i) sticky = d[i] != 0u;
-            if (rnd && (sticky || (m & 1ull))) m += 1ull;  // 2^53 stays exact
-            sum = ldexp(static_cast<double>(m), lead_lsb + 11 - 149);
-        }
-        mu = __double2float_rn(__ddiv_rn(sum, static_cast<double>(nb)));
     }
-    return __shfl_sync(0xffffffffu, mu, 0);
+    // highest non-zero digit, the two under it, and whether any lower digit is non-zero
+    int top = -1;
+#pragma unroll
+    for (int i = 0; i <= kDigits; ++i)
+        if (d[i]) top = i;
+    if (top < 0) return 0.0f;
+    uint32_t dt = 0u, dt1 = 0u, dt2 = 0u;
+    bool sticky = false;
+#pragma unroll
+    for (int i = 0; i <= kDigits; ++i) {
+        dt = i == top ? d[i] : dt;
+        dt1 = i == top - 1 ? d[i] : dt1;
+        dt2 = i == top - 2 ? d[i] : dt2;
+        sticky |= i < top - 2 && d[i] != 0u;
+    }
+    // the leading 64 bits of the total (digits top, top-1, top-2), left aligned
+    const unsigned long long t0 = (static_cast<unsigned long long>(dt) << 32) | dt1;
+    const int lz = __clzll(t0);  // < 32: dt != 0
+    const unsigned long long lead = lz ? (t0 << lz) | (static_cast<unsigned long long>(dt2) >> (32 - lz)) : t0;
+    // bit position (over the whole total) of the lead's lowest bit
+    const int lead_lsb = 32 * top + 32 - lz - 64;  // = msb - 63, may be negative
+    unsigned long long m = lead >> 11;              // 53 bits
+    const bool rnd = (lead >> 10) & 1ull;
+    sticky |= (lead & 0x3ffull) != 0;
+    // dt2's bits under the lead
+    sticky |= (lz ? (dt2 & ((1u << (32 - lz)) - 1u)) : dt2) != 0u;
+    if (rnd && (sticky || (m & 1ull))) m += 1ull;  // 2^53 stays exact
+    const double sum = ldexp(static_cast<double>(m), lead_lsb + 11 - 149);
+    return __double2float_rn(__ddiv_rn(sum, static_cast<double>(nb)));
 }
 
 constexpr int kDqThreads = 256;  // 8 warps, one 256-group per warp at a time
@@ -328,14 +333,25 @@ __global__ void __launch_bounds__(kDqThreads)
 k_double_quant(const float* __restrict__ c2, int64_t nb, const unsigned long long* __restrict__ bins,
                const int* __restrict__ flag, uint8_t* __restrict__ c2_fp8, float* __restrict__ c1,
                float* __restrict__ mean_out, int32_t* __restrict__ status) {
-    __shared__ unsigned long long sv[64];
     __shared__ float smu;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t ng = ceil_div(nb, kBlock2);
+    const int64_t wpb = kDqThreads / 32;
+    const int64_t g0 = static_cast<int64_t>(blockIdx.x) * wpb + warp;
+    float y[kBlock2 / 32];  // the constants of this warp's current group
+    auto load_group = [&](int64_t g) {
+#pragma unroll
+        for (int i = 0; i < kBlock2 / 32; ++i) {
+            const int64_t j = g * kBlock2 + 32 * i + lane;
+            y[i] = j < nb ? c2[j] : 0.0f;
+        }
+    };
     // launched as a programmatic dependent of k_nf4_quantize: wait for that
     // grid's completion (and its bins, c2 and flag) before reading anything
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (g0 < ng) load_group(g0);  // in flight while warp 0 finds the mean
     if (warp == 0) {
-        const float mu = mean_from_bins(bins, nb, sv);
+        const float mu = mean_from_bins(bins, nb);
         if (lane == 0) smu = mu;
     }
     __syncthreads();
@@ -344,15 +360,13 @@ k_double_quant(const float* __restrict__ c2, int64_t nb, const unsigned long lon
         *mean_out = mu;
         if (status) *status = (*flag) ? QLORA_ERR_NONFINITE : QLORA_OK;
     }
-    const int64_t ng = ceil_div(nb, kBlock2);
-    const int64_t wpb = kDqThreads / 32;
-    for (int64_t g = static_cast<int64_t>(blockIdx.x) * wpb + warp; g < ng; g += static_cast<int64_t>(gridDim.x) * wpb) {
-        float y[kBlock2 / 32];
+    for (int64_t g = g0; g < ng; g += static_cast<int64_t>(gridDim.x) * wpb) {
+        if (g != g0) load_group(g);
         float a = 0.0f;
 #pragma unroll
         for (int i = 0; i < kBlock2 / 32; ++i) {
             const int64_t j = g * kBlock2 + 32 * i + lane;
-            y[i] = j < nb ? __fsub_rn(c2[j], mu) : 0.0f;
+            y[i] = j < nb ? __fsub_rn(y[i], mu) : 0.0f;
             a = fmaxf(a, fabsf(y[i]));
         }
 #pragma unroll
